@@ -1,0 +1,89 @@
+"""Seeded synthetic workloads shared by the tests, the smoke entry and the bench.
+
+This module only draws random inputs and names shapes; it contains none of the
+attention arithmetic, so the CUDA path and the CPU oracle can both be fed from
+it without sharing any of the method.
+
+Recipe (fixed so every run sees the same numbers): a torch CPU ``Generator``
+seeded with ``seed``; fp32 standard normals drawn in the order q, k, v, dO,
+each of shape [B, H, N, d]; q and k are multiplied by ``qk_gain`` (exact, a
+power of two) and then every tensor is rounded to the workload's dtype with
+round-to-nearest-even (``Tensor.to``).  The oracle runs on those rounded values.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    dtype: str           # "f32" or "bf16"
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    backward: bool
+    qk_gain: float = 1.0
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def flops_fwd(self) -> float:
+        """4*B*H*N^2*d, halved under the causal mask."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def flops_bwd(self) -> float:
+        return 2.5 * self.flops_fwd()
+
+
+# The five workloads the attention path is measured and checked on.
+WORKLOADS = {
+    "c1_f32_1x2x256x64": Workload("c1_f32_1x2x256x64", "f32", 1, 2, 256, 64, False, True, seed=1001),
+    "c2_bf16_16x16x512x64": Workload("c2_bf16_16x16x512x64", "bf16", 16, 16, 512, 64, False, False, seed=1002),
+    "c3_bf16_8x12x1024x64_causal": Workload("c3_bf16_8x12x1024x64_causal", "bf16", 8, 12, 1024, 64, True, True, seed=1003),
+    "c4_bf16_4x16x4096x128_causal": Workload("c4_bf16_4x16x4096x128_causal", "bf16", 4, 16, 4096, 128, True, True, seed=1004),
+    "c5_bf16_1x16x16384x128_causal_qk2": Workload("c5_bf16_1x16x16384x128_causal_qk2", "bf16", 1, 16, 16384, 128, True, True, qk_gain=2.0, seed=1005),
+}
+
+
+def make_inputs(w: Workload, seed: int | None = None, B: int | None = None, H: int | None = None,
+                N: int | None = None):
+    """Draw (q, k, v, dO) on the CPU for workload ``w`` (shape overrides allowed).
+
+    Returns a dict of CPU tensors in the workload's dtype.
+    """
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    N = w.N if N is None else N
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    shape = (B, H, N, w.d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    do = torch.randn(shape, generator=g, dtype=torch.float32)
+    if w.qk_gain != 1.0:
+        q = q * w.qk_gain
+        k = k * w.qk_gain
+    dt = w.torch_dtype
+    return {"q": q.to(dt), "k": k.to(dt), "v": v.to(dt), "do": do.to(dt)}
+
+
+def random_tensors(shape, dtype, seed: int, count: int = 4, gain: float = 1.0):
+    """``count`` seeded standard-normal tensors of ``shape`` (times ``gain``), rounded to ``dtype``."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return [(torch.randn(shape, generator=g, dtype=torch.float32) * gain).to(dtype)
+            for _ in range(count)]

@@ -1,0 +1,316 @@
+/*
+ * Exact attention oracle, fp64, CPU.  TEST INFRASTRUCTURE ONLY.
+ *
+ * This file is the checker for the CUDA path, not part of it.  Only the test
+ * suite, the smoke entry and the bench's CPU-baseline / reference arm may load
+ * it.  It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes is the plain definition of attention that the FlashAttention
+ * pages state the tiled method reproduces exactly ("Exact, not approximate",
+ * vibeengines.com/paper/flash-attention; "Guarantees versus empirical results",
+ * chorfi.xyz/research/papers/paper-flashattention):
+ *
+ *   s_ij = scale * <q_i, k_j>               (j allowed: all j, or j <= i if causal)
+ *   m_i  = max_j s_ij,  l_i = sum_j e^{s_ij - m_i}
+ *   P_ij = e^{s_ij - m_i} / l_i             (safe softmax, "The math, worked with
+ *                                            real numbers", first formula)
+ *   O_i  = sum_j P_ij v_j,  LSE_i = m_i + ln l_i
+ *
+ * The full score row is materialised, one row at a time (the pages'
+ * "standard attention" that writes every score, "The real bottleneck").
+ *
+ * The backward pass is not written out on the pages (they only say that the
+ * method recomputes attention in the backward pass).  It is the textbook
+ * softmax / matrix-product calculus for the scalar loss L = sum(O * dO):
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = <dO_i, v_j>
+ *   D_i   = sum_j P_ij dP_ij
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale * sum_j dS_ij k_j,   dK_j = scale * sum_i dS_ij q_i
+ *
+ * oracle_softmax_online / oracle_attn_fwd_tiled restate the pages' online
+ * softmax update rule ("The math, worked with real numbers", the three update
+ * lines for m_new, l_new, O_new; final answer O / l) with an arbitrary block
+ * size; they exist only to pin the "block size never changes the answer" and
+ * "online softmax == naive softmax" assertions ("Solve it yourself").
+ *
+ * Layout: every tensor is [BH][N][d] row-major fp64 (BH = batch * heads);
+ * lse is [BH][N].  Masking convention (not fixed by the pages): square,
+ * top-left aligned causal mask, key j allowed iff j <= i.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Safe softmax of one row: subtract the row max, exponentiate, divide by the sum. */
+void oracle_softmax_naive(const double* s, long n, double* w)
+{
+    double m = -INFINITY;
+    for (long j = 0; j < n; ++j)
+        if (s[j] > m) m = s[j];
+    double l = 0.0;
+    for (long j = 0; j < n; ++j) {
+        w[j] = exp(s[j] - m);
+        l += w[j];
+    }
+    for (long j = 0; j < n; ++j) w[j] /= l;
+}
+
+/*
+ * Online softmax: walk the row in blocks, keep a running max m and a running
+ * sum l; when a block raises the max, the old sum is multiplied by
+ * e^{m_old - m_new} before the block's terms are added.  m_trace / l_trace (may
+ * be NULL) receive m and l after each block.
+ */
+void oracle_softmax_online(const double* s, long n, long block, double* w,
+                           double* m_trace, double* l_trace)
+{
+    double m = -INFINITY, l = 0.0;
+    long nb = 0;
+    for (long b0 = 0; b0 < n; b0 += block) {
+        long b1 = b0 + block < n ? b0 + block : n;
+        double m_blk = -INFINITY;
+        for (long j = b0; j < b1; ++j)
+            if (s[j] > m_blk) m_blk = s[j];
+        double m_new = m > m_blk ? m : m_blk;
+        double add = 0.0;
+        for (long j = b0; j < b1; ++j) add += exp(s[j] - m_new);
+        l = (m == -INFINITY ? 0.0 : l * exp(m - m_new)) + add;
+        m = m_new;
+        if (m_trace) m_trace[nb] = m;
+        if (l_trace) l_trace[nb] = l;
+        ++nb;
+    }
+    for (long j = 0; j < n; ++j) w[j] = exp(s[j] - m) / l;
+}
+
+/* Number of keys row i may attend to. */
+static long n_allowed(long i, long N, int causal) { return causal ? i + 1 : N; }
+
+static double dot(const double* a, const double* b, long d)
+{
+    double acc = 0.0;
+    for (long t = 0; t < d; ++t) acc += a[t] * b[t];
+    return acc;
+}
+
+/*
+ * One query row of one head: materialise the score row into srow (length N),
+ * turn it into P in place, write O_i and LSE_i.
+ */
+static void fwd_row(const double* qi, const double* k, const double* v, double* oi,
+                    double* lse_i, long i, long N, long d, double scale, int causal,
+                    double* srow)
+{
+    long nk = n_allowed(i, N, causal);
+    double m = -INFINITY;
+    for (long j = 0; j < nk; ++j) {
+        srow[j] = scale * dot(qi, k + j * d, d);
+        if (srow[j] > m) m = srow[j];
+    }
+    double l = 0.0;
+    for (long j = 0; j < nk; ++j) {
+        srow[j] = exp(srow[j] - m);
+        l += srow[j];
+    }
+    for (long t = 0; t < d; ++t) oi[t] = 0.0;
+    for (long j = 0; j < nk; ++j) {
+        double p = srow[j] / l;
+        const double* vj = v + j * d;
+        for (long t = 0; t < d; ++t) oi[t] += p * vj[t];
+    }
+    *lse_i = m + log(l);
+}
+
+/* Forward over all heads and rows.  Returns 0, or -1 on bad sizes / no memory. */
+int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o,
+                    double* lse, long BH, long N, long d, double scale, int causal)
+{
+    if (BH < 0 || N < 0 || d < 1) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* srow = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+        if (!srow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 16) collapse(2)
+        for (long h = 0; h < BH; ++h)
+            for (long i = 0; i < N; ++i) {
+                if (!srow) continue;
+                const long base = h * N * d;
+                fwd_row(q + base + i * d, k + base, v + base, o + base + i * d,
+                        lse + h * N + i, i, N, d, scale, causal, srow);
+            }
+        free(srow);
+    }
+    return err;
+}
+
+/*
+ * Forward for rows [i0, i1) of ONE head (q, k, v point at that head's [N][d]
+ * block; o / lse receive i1 - i0 rows).  Used to check sampled rows of
+ * workloads too large to run whole.
+ */
+int oracle_attn_fwd_rows(const double* q, const double* k, const double* v, double* o,
+                         double* lse, long N, long d, long i0, long i1, double scale,
+                         int causal)
+{
+    if (N < 1 || d < 1 || i0 < 0 || i1 > N || i0 > i1) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* srow = (double*)malloc((size_t)N * sizeof(double));
+        if (!srow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (long i = i0; i < i1; ++i) {
+            if (!srow) continue;
+            fwd_row(q + i * d, k, v, o + (i - i0) * d, lse + (i - i0), i, N, d, scale,
+                    causal, srow);
+        }
+        free(srow);
+    }
+    return err;
+}
+
+/*
+ * The online (tiled) restatement: each row walks the keys in blocks of `block`,
+ * updating m, l and the output accumulator with the same factor e^{m_old-m_new},
+ * and divides by l at the end.
+ */
+int oracle_attn_fwd_tiled(const double* q, const double* k, const double* v, double* o,
+                          double* lse, long BH, long N, long d, double scale, int causal,
+                          long block)
+{
+    if (BH < 0 || N < 0 || d < 1 || block < 1) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* sblk = (double*)malloc((size_t)block * sizeof(double));
+        if (!sblk) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 16) collapse(2)
+        for (long h = 0; h < BH; ++h)
+            for (long i = 0; i < N; ++i) {
+                if (!sblk) continue;
+                const long base = h * N * d;
+                const double* qi = q + base + i * d;
+                double* oi = o + base + i * d;
+                long nk = n_allowed(i, N, causal);
+                double m = -INFINITY, l = 0.0;
+                for (long t = 0; t < d; ++t) oi[t] = 0.0;
+                for (long b0 = 0; b0 < nk; b0 += block) {
+                    long b1 = b0 + block < nk ? b0 + block : nk;
+                    double m_blk = -INFINITY;
+                    for (long j = b0; j < b1; ++j) {
+                        sblk[j - b0] = scale * dot(qi, k + base + j * d, d);
+                        if (sblk[j - b0] > m_blk) m_blk = sblk[j - b0];
+                    }
+                    double m_new = m > m_blk ? m : m_blk;
+                    double alpha = (m == -INFINITY) ? 0.0 : exp(m - m_new);
+                    l *= alpha;
+                    for (long t = 0; t < d; ++t) oi[t] *= alpha;
+                    for (long j = b0; j < b1; ++j) {
+                        double p = exp(sblk[j - b0] - m_new);
+                        l += p;
+                        const double* vj = v + base + j * d;
+                        for (long t = 0; t < d; ++t) oi[t] += p * vj[t];
+                    }
+                    m = m_new;
+                }
+                for (long t = 0; t < d; ++t) oi[t] /= l;
+                lse[h * N + i] = m + log(l);
+            }
+        free(sblk);
+    }
+    return err;
+}
+
+/*
+ * Backward for all heads (dq, dk, dv fully written).  Parallel over heads only,
+ * so each head's dK / dV sums run in one thread in row order.
+ */
+int oracle_attn_bwd(const double* q, const double* k, const double* v, const double* dO,
+                    double* dq, double* dk, double* dv, long BH, long N, long d,
+                    double scale, int causal)
+{
+    if (BH < 0 || N < 0 || d < 1) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* prow = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+        double* dprow = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+        if (!prow || !dprow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long h = 0; h < BH; ++h) {
+            if (!prow || !dprow) continue;
+            const long base = h * N * d;
+            const double *qh = q + base, *kh = k + base, *vh = v + base, *doh = dO + base;
+            double *dqh = dq + base, *dkh = dk + base, *dvh = dv + base;
+            memset(dkh, 0, (size_t)(N * d) * sizeof(double));
+            memset(dvh, 0, (size_t)(N * d) * sizeof(double));
+            for (long i = 0; i < N; ++i) {
+                const double* qi = qh + i * d;
+                const double* doi = doh + i * d;
+                long nk = n_allowed(i, N, causal);
+                /* P_i: the materialised, max-subtracted softmax row */
+                double m = -INFINITY;
+                for (long j = 0; j < nk; ++j) {
+                    prow[j] = scale * dot(qi, kh + j * d, d);
+                    if (prow[j] > m) m = prow[j];
+                }
+                double l = 0.0;
+                for (long j = 0; j < nk; ++j) {
+                    prow[j] = exp(prow[j] - m);
+                    l += prow[j];
+                }
+                for (long j = 0; j < nk; ++j) prow[j] /= l;
+                /* dP_i and D_i = sum_j P_ij dP_ij */
+                double D = 0.0;
+                for (long j = 0; j < nk; ++j) {
+                    dprow[j] = dot(doi, vh + j * d, d);
+                    D += prow[j] * dprow[j];
+                }
+                double* dqi = dqh + i * d;
+                for (long t = 0; t < d; ++t) dqi[t] = 0.0;
+                for (long j = 0; j < nk; ++j) {
+                    double ds = prow[j] * (dprow[j] - D);
+                    const double* kj = kh + j * d;
+                    double* dkj = dkh + j * d;
+                    double* dvj = dvh + j * d;
+                    for (long t = 0; t < d; ++t) {
+                        dqi[t] += ds * kj[t];
+                        dkj[t] += ds * qi[t];
+                        dvj[t] += prow[j] * doi[t];
+                    }
+                }
+                for (long t = 0; t < d; ++t) dqi[t] *= scale;
+            }
+            for (long e = 0; e < N * d; ++e) dkh[e] *= scale;
+        }
+        free(prow);
+        free(dprow);
+    }
+    return err;
+}

@@ -1,0 +1,151 @@
+"""Python access to the fp64 CPU attention oracle (``attn_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke entry and the bench's CPU
+baseline / reference arm use this module; the CUDA library never does.  It
+shares no code with the CUDA path.  The C source states what each function
+computes and which passage of the FlashAttention pages it follows.
+
+All arrays are float64, laid out [B, H, N, d] (lse: [B, H, N]).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` with gcc (OpenMP, no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+             "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        L = ctypes.c_long
+        D = ctypes.c_double
+        I = ctypes.c_int
+        lib.oracle_num_threads.restype = I
+        lib.oracle_softmax_naive.argtypes = [P, L, P]
+        lib.oracle_softmax_online.argtypes = [P, L, L, P, P, P]
+        lib.oracle_attn_fwd.argtypes = [P, P, P, P, P, L, L, L, D, I]
+        lib.oracle_attn_fwd.restype = I
+        lib.oracle_attn_fwd_rows.argtypes = [P, P, P, P, P, L, L, L, L, D, I]
+        lib.oracle_attn_fwd_rows.restype = I
+        lib.oracle_attn_fwd_tiled.argtypes = [P, P, P, P, P, L, L, L, D, I, L]
+        lib.oracle_attn_fwd_tiled.restype = I
+        lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, D, I]
+        lib.oracle_attn_bwd.restype = I
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Exact conversion of a numpy array or torch tensor (fp32 / bf16 / fp64) to C-contiguous fp64."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def softmax_naive(row):
+    s = _f64(row).ravel()
+    w = np.empty_like(s)
+    _load().oracle_softmax_naive(_ptr(s), s.size, _ptr(w))
+    return w
+
+
+def softmax_online(row, block: int):
+    """Returns (weights, m after each block, l after each block)."""
+    s = _f64(row).ravel()
+    nb = -(-s.size // block)
+    w = np.empty_like(s)
+    mt = np.empty(nb)
+    lt = np.empty(nb)
+    _load().oracle_softmax_online(_ptr(s), s.size, block, _ptr(w), _ptr(mt), _ptr(lt))
+    return w, mt, lt
+
+
+def _check4(q, k, v):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    assert q.ndim == 4 and q.shape == k.shape == v.shape, (q.shape, k.shape, v.shape)
+    return q, k, v
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool):
+    """Exact attention forward.  Returns (O [B,H,N,d], LSE [B,H,N])."""
+    q, k, v = _check4(q, k, v)
+    B, H, N, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, H, N))
+    rc = _load().oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                 B * H, N, d, float(scale), int(bool(causal)))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd failed (%d)" % rc)
+    return o, lse
+
+
+def attn_fwd_rows(q, k, v, i0: int, i1: int, scale: float, causal: bool):
+    """Rows [i0, i1) of ONE head; q, k, v are that head's [N, d] arrays."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N, d = q.shape
+    o = np.empty((i1 - i0, d))
+    lse = np.empty(i1 - i0)
+    rc = _load().oracle_attn_fwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                      N, d, i0, i1, float(scale), int(bool(causal)))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd_rows failed (%d)" % rc)
+    return o, lse
+
+
+def attn_fwd_tiled(q, k, v, scale: float, causal: bool, block: int):
+    """The online-softmax restatement with key block size ``block``."""
+    q, k, v = _check4(q, k, v)
+    B, H, N, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, H, N))
+    rc = _load().oracle_attn_fwd_tiled(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                       B * H, N, d, float(scale), int(bool(causal)), int(block))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd_tiled failed (%d)" % rc)
+    return o, lse
+
+
+def attn_bwd(q, k, v, do, scale: float, causal: bool):
+    """Exact attention backward for L = sum(O * dO).  Returns (dQ, dK, dV)."""
+    q, k, v = _check4(q, k, v)
+    do = _f64(do)
+    assert do.shape == q.shape
+    B, H, N, d = q.shape
+    dq = np.empty_like(q)
+    dk = np.empty_like(q)
+    dv = np.empty_like(q)
+    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), B * H, N, d, float(scale), int(bool(causal)))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_bwd failed (%d)" % rc)
+    return dq, dk, dv

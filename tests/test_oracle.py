@@ -1,0 +1,247 @@
+"""Pins for the fp64 CPU oracle (no GPU).
+
+Every check here compares the oracle against something other than itself:
+values the FlashAttention explainer page prints, closed forms, torch's own
+softmax / logsumexp / autograd on tiny inputs, central finite differences, and
+invariants that follow from rows of P summing to one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rand(shape, seed, gain=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * gain
+
+
+def _torch_attention(q, k, v, scale, causal):
+    """Library formulation: torch fp64 softmax over the full score matrix."""
+    q, k, v = (torch.from_numpy(np.asarray(x, dtype=np.float64)) for x in (q, k, v))
+    s = scale * q @ k.transpose(-1, -2)
+    if causal:
+        N = s.shape[-1]
+        mask = torch.ones(N, N, dtype=torch.bool).triu(1)
+        s = s.masked_fill(mask, float("-inf"))
+    return (torch.softmax(s, -1) @ v).numpy(), torch.logsumexp(s, -1).numpy()
+
+
+# ---------------------------------------------------------------- worked row
+
+
+def test_worked_row_online_trace_matches_page():
+    g = _golden("worked_row.json")
+    w, m_trace, l_trace = oracle.softmax_online(g["row"], g["block"])
+    nd = g["printed_decimals"]
+    assert list(m_trace) == g["m_after_block"]
+    assert round(l_trace[0], nd) == g["l_after_first_block"]
+    assert round(l_trace[-1], nd) == g["l_final"]
+    assert [round(x, nd) for x in w] == g["weights"]
+    # the same weights from the naive (whole-row) softmax
+    assert [round(x, nd) for x in oracle.softmax_naive(g["row"])] == g["weights"]
+    # the page's identity: the final sum equals e^-1 + e^-2 + e^0 + e^-3
+    assert abs(l_trace[-1] - (math.exp(-1) + math.exp(-2) + 1 + math.exp(-3))) < 1e-15
+
+
+def test_worked_row_rescale_step_is_exact_not_printed_rounding():
+    # the rescaled old sum is (e^0 + e^-1) * e^(2-3); the page prints 0.5033
+    # (rounding of a rounded number), exact is 0.503215...
+    row = [2.0, 1.0, 3.0, 0.0]
+    _, _, lt = oracle.softmax_online(row, 2)
+    rescaled = lt[0] * math.exp(2 - 3)
+    assert abs(rescaled - 0.5032147244) < 1e-9
+    assert abs(lt[1] - (rescaled + 1 + math.exp(-3))) < 1e-15
+
+
+@pytest.mark.parametrize("n", [1, 2, 5, 64, 257])
+@pytest.mark.parametrize("block", [1, 2, 3, 7, 64, None])
+def test_online_softmax_equals_naive_and_sums_to_one(n, block):
+    row = _rand(n, seed=n * 31 + (block or 0), gain=5.0)
+    naive = oracle.softmax_naive(row)
+    online, _, _ = oracle.softmax_online(row, block or n)
+    assert np.max(np.abs(online - naive)) < 1e-13
+    assert abs(online.sum() - 1.0) < 1e-13
+    # and both agree with the library softmax
+    ref = torch.softmax(torch.from_numpy(row), 0).numpy()
+    assert np.max(np.abs(naive - ref)) < 1e-13
+
+
+# ---------------------------------------------------------------- forward
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1), (1, 2, 5, 3), (2, 1, 8, 4), (1, 1, 7, 2)])
+def test_fwd_matches_library_bruteforce(shape, causal):
+    q, k, v = (_rand(shape, seed=s) for s in (1, 2, 3))
+    scale = 1 / math.sqrt(shape[-1])
+    o, lse = oracle.attn_fwd(q, k, v, scale, causal)
+    o_ref, lse_ref = _torch_attention(q, k, v, scale, causal)
+    assert np.max(np.abs(o - o_ref)) < 1e-13
+    assert np.max(np.abs(lse - lse_ref)) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("block", [1, 2, 3, 7, 64, 100])
+def test_block_size_never_changes_the_answer(block, causal):
+    shape = (1, 2, 100, 16)
+    q, k, v = (_rand(shape, seed=s, gain=2.0) for s in (11, 12, 13))
+    scale = 0.25
+    o, lse = oracle.attn_fwd(q, k, v, scale, causal)
+    ot, lset = oracle.attn_fwd_tiled(q, k, v, scale, causal, block)
+    assert np.max(np.abs(ot - o)) < 1e-13
+    assert np.max(np.abs(lset - lse)) < 1e-13
+
+
+def test_page_demo_tiled_equals_standard():
+    g = _golden("demo_qkv.json")
+    q, k, v = (np.array(g[x], dtype=np.float64)[None, None] for x in ("Q", "K", "V"))
+    scale = 1 / math.sqrt(q.shape[-1])
+    o, lse = oracle.attn_fwd(q, k, v, scale, False)
+    o_ref, lse_ref = _torch_attention(q, k, v, scale, False)
+    assert np.max(np.abs(o - o_ref)) <= g["max_abs_diff"]
+    for b in g["blocks"]:
+        ot, _ = oracle.attn_fwd_tiled(q, k, v, scale, False, b)
+        assert np.max(np.abs(ot - o)) <= g["max_abs_diff"]
+
+
+def test_fwd_rows_matches_full():
+    shape = (1, 1, 50, 8)
+    q, k, v = (_rand(shape, seed=s) for s in (21, 22, 23))
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, 0.3, causal)
+        orow, lrow = oracle.attn_fwd_rows(q[0, 0], k[0, 0], v[0, 0], 17, 33, 0.3, causal)
+        assert np.array_equal(orow, o[0, 0, 17:33])
+        assert np.array_equal(lrow, lse[0, 0, 17:33])
+
+
+# closed forms ------------------------------------------------------------
+
+
+def test_single_key_returns_its_value():
+    q, k, v = (_rand((2, 3, 1, 5), seed=s) for s in (31, 32, 33))
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, 0.7, causal)
+        assert np.max(np.abs(o - v)) < 1e-15
+        assert np.max(np.abs(lse - 0.7 * np.sum(q * k, -1))) < 1e-14
+
+
+def test_zero_queries_give_uniform_weights():
+    N, d = 9, 4
+    q = np.zeros((1, 1, N, d))
+    k, v = (_rand((1, 1, N, d), seed=s) for s in (41, 42))
+    o, lse = oracle.attn_fwd(q, k, v, 1.0, False)
+    assert np.max(np.abs(o[0, 0] - v[0, 0].mean(0))) < 1e-14
+    assert np.max(np.abs(lse - math.log(N))) < 1e-14
+    o, lse = oracle.attn_fwd(q, k, v, 1.0, True)
+    prefix_mean = np.cumsum(v[0, 0], 0) / np.arange(1, N + 1)[:, None]
+    assert np.max(np.abs(o[0, 0] - prefix_mean)) < 1e-14
+    assert np.max(np.abs(lse[0, 0] - np.log(np.arange(1, N + 1)))) < 1e-14
+
+
+def test_causal_first_row_is_first_value():
+    q, k, v = (_rand((1, 2, 6, 3), seed=s, gain=3.0) for s in (51, 52, 53))
+    o, _ = oracle.attn_fwd(q, k, v, 1.0, True)
+    assert np.max(np.abs(o[:, :, 0] - v[:, :, 0])) < 1e-15
+
+
+def test_identity_values_expose_the_weights_and_rows_sum_to_one():
+    N = 6
+    q, k = (_rand((1, 1, N, N), seed=s) for s in (61, 62))
+    v = np.eye(N)[None, None]
+    for causal in (False, True):
+        o, _ = oracle.attn_fwd(q, k, v, 0.5, causal)
+        s = 0.5 * q[0, 0] @ k[0, 0].T
+        for i in range(N):
+            n = i + 1 if causal else N
+            w = torch.softmax(torch.from_numpy(s[i, :n]), 0).numpy()
+            assert np.max(np.abs(o[0, 0, i, :n] - w)) < 1e-14
+            assert np.all(o[0, 0, i, n:] == 0.0)
+        assert np.max(np.abs(o.sum(-1) - 1.0)) < 1e-14
+
+
+def test_worked_row_as_an_attention_problem():
+    # q0 = e1, k_j = s_j * e1, scale 1, V = I: row 0 of O is the worked row's weights.
+    g = _golden("worked_row.json")
+    N = d = 4
+    q = np.zeros((1, 1, N, d))
+    k = np.zeros((1, 1, N, d))
+    q[0, 0, 0, 0] = 1.0
+    k[0, 0, :, 0] = g["row"]
+    v = np.eye(N)[None, None]
+    o, lse = oracle.attn_fwd(q, k, v, 1.0, False)
+    assert [round(x, 4) for x in o[0, 0, 0]] == g["weights"]
+    assert round(math.exp(lse[0, 0, 0] - 3.0), 4) == g["l_final"]
+
+
+# ---------------------------------------------------------------- backward
+
+
+def _loss(q, k, v, g, scale, causal):
+    o, _ = oracle.attn_fwd(q, k, v, scale, causal)
+    return float(np.sum(o * g))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_matches_central_finite_differences(causal):
+    shape = (1, 2, 5, 3)
+    q, k, v, g = (_rand(shape, seed=s) for s in (71, 72, 73, 74))
+    scale = 0.6
+    dq, dk, dv = oracle.attn_bwd(q, k, v, g, scale, causal)
+    h = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}; args_p[name] = xp
+            args_m = {"q": q, "k": k, "v": v}; args_m[name] = xm
+            num[idx] = (_loss(args_p["q"], args_p["k"], args_p["v"], g, scale, causal)
+                        - _loss(args_m["q"], args_m["k"], args_m["v"], g, scale, causal)) / (2 * h)
+        err = np.max(np.abs(num - grad)) / max(1.0, np.max(np.abs(grad)))
+        assert err < 1e-6, (name, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_matches_torch_autograd(causal):
+    shape = (2, 2, 11, 6)
+    q, k, v, g = (_rand(shape, seed=s) for s in (81, 82, 83, 84))
+    scale = 1 / math.sqrt(6)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, g, scale, causal)
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+    s = scale * tq @ tk.transpose(-1, -2)
+    if causal:
+        s = s.masked_fill(torch.ones(11, 11, dtype=torch.bool).triu(1), float("-inf"))
+    o = torch.softmax(s, -1) @ tv
+    (o * torch.from_numpy(g)).sum().backward()
+    for a, b in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.max(np.abs(a - b.numpy())) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_invariants(causal):
+    shape = (1, 3, 40, 8)
+    q, k, v, g = (_rand(shape, seed=s, gain=1.5) for s in (91, 92, 93, 94))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, g, 0.35, causal)
+    # rows of dS sum to zero  =>  sum_j dK_j = 0
+    assert np.max(np.abs(dk.sum(2))) < 1e-12
+    # rows of P sum to one    =>  sum_j dV_j = sum_i dO_i
+    assert np.max(np.abs(dv.sum(2) - g.sum(2))) < 1e-12
+    if causal:
+        # the last key is seen only by the last query: dV_{N-1} = P_{N-1,N-1} dO_{N-1}
+        o, lse = oracle.attn_fwd(q, k, v, 0.35, True)
+        p_last = np.exp(0.35 * np.sum(q[:, :, -1] * k[:, :, -1], -1) - lse[:, :, -1])
+        assert np.max(np.abs(dv[:, :, -1] - p_last[..., None] * g[:, :, -1])) < 1e-13
