@@ -1,0 +1,397 @@
+// Host side of the C ABI declared in include/fa.h: argument validation,
+// TMA tensor-map encoding, kernel launches and the device error word.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/fa.h"
+#include "../../include/fa_selftest.h"
+#include "kernels.h"
+
+namespace fa {
+
+// One error word per device (each device that loads the library has its own
+// copy); kernels get its address as a parameter.
+__device__ unsigned int g_fa_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+unsigned int* g_status_ptr[kMaxDevices] = {};
+std::atomic<unsigned long long> g_limit_ns{2000000000ull};
+thread_local int g_last_launches = 0;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int get_encoder()
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_encode) return FA_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FA_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    return FA_OK;
+}
+
+int get_ctl(WaitCtl* ctl)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_fa_status) != cudaSuccess || !ptr) return FA_ERR_CUDA;
+        g_status_ptr[dev] = static_cast<unsigned int*>(ptr);
+    }
+    ctl->status = g_status_ptr[dev];
+    ctl->limit_ns = g_limit_ns.load();
+    return FA_OK;
+}
+
+// 3-D tiled tensor map over a dense [d2][d1][d0] tensor (d0 innermost).
+int encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* ptr, uint64_t d0, uint64_t d1,
+              uint64_t d2, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw)
+{
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * elem_bytes, d0 * d1 * elem_bytes};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int N, int d, float scale, int causal)
+{
+    if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    const long long elems = static_cast<long long>(B) * H * N * d;
+    if (elems >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(int status)
+{
+    switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    default: return "FA_ERR_UNKNOWN";
+    }
+}
+
+int fa_last_launch_count(void) { return g_last_launches; }
+
+void fa_set_wait_limit_ns(unsigned long long ns) { g_limit_ns.store(ns < 1000000ull ? 1000000ull : ns); }
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, float scale,
+           int causal, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+    if ((st = get_encoder()) != FA_OK) return st;
+    FwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.BH = static_cast<int>(BH);
+    p.N = N;
+    p.n_pairs = (N + 255) / 256;
+    p.scale_log2 = scale * kLog2e;
+    st = cuda_status(launch_fwd_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d)
+{
+    if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+    const size_t rows = static_cast<size_t>(B) * H * (static_cast<size_t>(N + 127) / 128 * 128);
+    return 2 * ((rows * sizeof(float) + 255) & ~size_t(255));
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, float* dq,
+           float* dk, float* dv, void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return FA_ERR_MISALIGNED;
+    if ((st = get_encoder()) != FA_OK) return st;
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    const int n_pad = (N + 127) / 128 * 128;
+    const size_t vec_bytes = (static_cast<size_t>(BH) * n_pad * sizeof(float) + 255) & ~size_t(255);
+    float* delta = static_cast<float*>(workspace);
+    float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + vec_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    BwdPreParams pp;
+    pp.o = static_cast<const __nv_bfloat16*>(o);
+    pp.dO = static_cast<const __nv_bfloat16*>(dO);
+    pp.lse = lse;
+    pp.delta = delta;
+    pp.lse2 = lse2;
+    pp.dq = dq;
+    pp.BH = static_cast<int>(BH);
+    pp.N = N;
+    pp.n_pad = n_pad;
+    pp.d = d;
+
+    BwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint32_t bq = 64;
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, bq,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dO, d, N, BH, 64, bq,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq, d, N, BH, 32, bq,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.dk = dk;
+    p.dv = dv;
+    p.BH = static_cast<int>(BH);
+    p.N = N;
+    p.n_kv_tiles = (N + 127) / 128;
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2e;
+    if ((st = cuda_status(launch_bwd_pre(pp, s))) != FA_OK) return st;
+    g_last_launches = 1;
+    if ((st = cuda_status(launch_bwd_sm100(p, d, causal != 0, s))) != FA_OK) return st;
+    g_last_launches = 2;
+    return FA_OK;
+}
+
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
+               float scale, int causal, int block_k, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (d > 128) return FA_ERR_UNSUPPORTED;
+    if (block_k == 0) block_k = 64;
+    if (block_k < 1 || block_k > 1024) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+    F32Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o_out = o;
+    p.lse_out = lse;
+    p.BH = B * H;
+    p.N = N;
+    p.d = d;
+    p.causal = causal;
+    p.block_k = block_k;
+    p.scale = scale;
+    st = cuda_status(launch_fwd_f32(p, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
+int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* lse, const float* dO,
+               float* dq, float* dk, float* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
+               void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (d > 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return FA_ERR_MISALIGNED;
+    F32Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q;
+    p.k = k;
+    p.v = v;
+    p.o = o;
+    p.lse = lse;
+    p.dO = dO;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.delta = static_cast<float*>(workspace);
+    p.BH = B * H;
+    p.N = N;
+    p.d = d;
+    p.causal = causal;
+    p.scale = scale;
+    st = cuda_status(launch_bwd_f32(p, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 3;
+    return st;
+}
+
+size_t fa_attention_host_arena_bytes(int B, int H, int N, int d)
+{
+    if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+    const size_t E = static_cast<size_t>(B) * H * N * d;
+    const size_t R = static_cast<size_t>(B) * H * N;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    // q k v dO o (bf16), dq dk dv (fp32), lse (fp32), workspace
+    return 5 * up(E * 2) + 3 * up(E * 4) + up(R * 4) + up(fa_bwd_workspace_bytes(B, H, N, d));
+}
+
+int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const void* h_dO, void* h_o, float* h_lse,
+                      float* h_dq, float* h_dk, float* h_dv, void* arena, size_t arena_bytes, int B, int H, int N,
+                      int d, float scale, int causal, void* stream)
+{
+    g_last_launches = 0;
+    if (!h_q || !h_k || !h_v || !h_dO || !arena) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(arena) & 255u) != 0) return FA_ERR_MISALIGNED;
+    if (arena_bytes < fa_attention_host_arena_bytes(B, H, N, d)) return FA_ERR_INVALID_ARG;
+    const size_t E = static_cast<size_t>(B) * H * N * d;
+    const size_t R = static_cast<size_t>(B) * H * N;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    char* a = static_cast<char*>(arena);
+    void* q = a;
+    a += up(E * 2);
+    void* k = a;
+    a += up(E * 2);
+    void* v = a;
+    a += up(E * 2);
+    void* dO = a;
+    a += up(E * 2);
+    void* o = a;
+    a += up(E * 2);
+    float* dq = reinterpret_cast<float*>(a);
+    a += up(E * 4);
+    float* dk = reinterpret_cast<float*>(a);
+    a += up(E * 4);
+    float* dv = reinterpret_cast<float*>(a);
+    a += up(E * 4);
+    float* lse = reinterpret_cast<float*>(a);
+    a += up(R * 4);
+    void* ws = a;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const void* srcs[4] = {h_q, h_k, h_v, h_dO};
+    void* dsts[4] = {q, k, v, dO};
+    for (int i = 0; i < 4; ++i)
+        if (cudaMemcpyAsync(dsts[i], srcs[i], E * 2, cudaMemcpyHostToDevice, s) != cudaSuccess) return FA_ERR_CUDA;
+    if ((st = fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream)) != FA_OK) return st;
+    const int n_fwd = g_last_launches;
+    if ((st = fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, ws, B, H, N, d, scale, causal, stream)) != FA_OK) return st;
+    const int n_bwd = g_last_launches;
+    struct {
+        void* dst;
+        const void* src;
+        size_t bytes;
+    } back[5] = {{h_o, o, E * 2}, {h_lse, lse, R * 4}, {h_dq, dq, E * 4}, {h_dk, dk, E * 4}, {h_dv, dv, E * 4}};
+    for (auto& b : back)
+        if (b.dst && cudaMemcpyAsync(b.dst, b.src, b.bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return FA_ERR_CUDA;
+    g_last_launches = n_fwd + n_bwd;
+    return FA_OK;
+}
+
+int fa_check_device_status(void* stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+    WaitCtl ctl;
+    int st = get_ctl(&ctl);
+    if (st != FA_OK) return st;
+    unsigned int word = 0;
+    if (cudaMemcpy(&word, ctl.status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpy(ctl.status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+        return (word & FA_DEV_TIMEOUT) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+    }
+    return FA_OK;
+}
+
+// ---------------------------------------------------------------- self tests
+
+int fa_selftest_umma(const void* a, const void* b, float* d, int M, int N, int K, int a_mn, int b_mn, int a_tmem,
+                     int b_manual, void* stream)
+{
+    g_last_launches = 0;
+    if (!a || !b || !d) return FA_ERR_INVALID_ARG;
+    if (M != 128 || (N != 64 && N != 128) || (K != 64 && K != 128)) return FA_ERR_UNSUPPORTED;
+    if (a_tmem && a_mn) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(a) || !aligned16(b) || !aligned16(d)) return FA_ERR_MISALIGNED;
+    int st = get_encoder();
+    if (st != FA_OK) return st;
+    UmmaTestParams p;
+    std::memset(&p, 0, sizeof(p));
+    // A storage: K-major [M][K] or MN-major [K][M]; B storage: K-major [N][K] or MN-major [K][N]
+    if ((st = encode_3d(&p.tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, a_mn ? M : K, a_mn ? K : M, 1, 64,
+                        a_mn ? K : M, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, b, b_mn ? N : K, b_mn ? K : N, 1, 64,
+                        b_mn ? K : N, CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    p.a_raw = static_cast<const __nv_bfloat16*>(a);
+    p.b_raw = static_cast<const __nv_bfloat16*>(b);
+    p.d = d;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.a_mn = a_mn;
+    p.b_mn = b_mn;
+    p.a_tmem = a_tmem;
+    p.b_manual = b_manual;
+    st = cuda_status(launch_umma_selftest(p, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
+}  // extern "C"

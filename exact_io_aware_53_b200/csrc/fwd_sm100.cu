@@ -1,0 +1,365 @@
+// Forward attention, bf16 in / fp32 accumulate, sm_100a.
+//
+// One CTA owns 256 query rows of one (batch, head) as two 128-row Q tiles and
+// walks the key/value tiles of 128 keys (the tiling and online softmax of
+// "Tiling and the online softmax", vibeengines.com/paper/flash-attention):
+//
+//   warp 9      TMA producer: Q tiles once, then K_j, V_j through a smem ring
+//   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T (smem x smem -> TMEM),
+//               O_t += P_t V_j (P from TMEM x V from smem -> TMEM)
+//   warps 0-3   softmax for Q tile 0 (thread = query row = TMEM lane)
+//   warps 4-7   softmax for Q tile 1
+//
+// The two softmax warpgroups ping-pong: while one turns its S tile into P, the
+// tensor core runs the other tile's P V and next Q K^T.
+//
+// Softmax per key tile, in base 2 with c = scale * log2(e) (the update rule of
+// "The math, worked with real numbers": m_new = max(m_old, m_block), l_new =
+// l_old e^{m_old-m_new} + sum e^{s-m_new}, O_new = O_old e^{m_old-m_new} + ...):
+//   m_new = max(m, c * rowmax(S));   p = 2^(c s - m);   l = l * alpha + sum p
+// The running max is only moved (and O, l rescaled by alpha = 2^(m - m_new))
+// when it grows by more than RESCALE_LOG2 = 8; otherwise the stale max is kept,
+// which leaves every p <= 2^8 and changes nothing in exact arithmetic because O
+// and l carry the same factor and the result is O / l.
+//
+// TMEM (512 columns x 128 lanes): S_t at columns [128 t, 128 t + 128); P_t (bf16
+// pairs) overwrites the first 64 columns of S_t; O_t at 256 + D t.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace fwdk {
+
+constexpr int BM = 128;  // query rows per Q tile
+constexpr int BN = 128;  // keys per K/V tile
+constexpr int NTHREADS = 320;
+constexpr int MMA_WARP = 8;
+constexpr int LOAD_WARP = 9;
+constexpr float RESCALE_LOG2 = 8.0f;
+constexpr float LN2 = 0.6931471805599453f;
+
+template <int D>
+struct Cfg {
+    static constexpr int NDC = D / 64;              // 128-byte swizzle boxes per row
+    static constexpr int BOX_BYTES = 128 * 128;     // 128 rows x 64 bf16
+    static constexpr int TILE_BYTES = NDC * BOX_BYTES;
+    static constexpr int STAGES = (D == 128) ? 4 : 8;
+    static constexpr int Q_OFF = 0;
+    static constexpr int KV_OFF = 2 * TILE_BYTES;
+    static constexpr int BAR_OFF = KV_OFF + STAGES * TILE_BYTES;
+    static constexpr int NBARS = 1 + 2 * STAGES + 2 + 2 + 2 + 1;
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t O_COL = 256;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p)
+{
+    uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return reinterpret_cast<uint8_t*>((a + 1023) & ~uintptr_t(1023));
+}
+
+// Bounded wait done by every lane of a warp, with a warp-uniform verdict.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c)
+{
+    bool ok = mbar_wait(bar, parity, c);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant__ FwdParams p)
+{
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* sQ = smem + C::Q_OFF;
+    uint8_t* sKV = smem + C::KV_OFF;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = kv_full + C::STAGES;
+    uint64_t* s_full = kv_empty + C::STAGES;  // [2]
+    uint64_t* p_full = s_full + 2;            // [2]
+    uint64_t* o_full = p_full + 2;            // [2]
+    uint64_t* drain = o_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+    const int warp = static_cast<int>(warp_id());
+    const int lane = static_cast<int>(lane_id());
+    const int bh = blockIdx.x;
+    const int pair = CAUSAL ? (p.n_pairs - 1 - static_cast<int>(blockIdx.y)) : static_cast<int>(blockIdx.y);
+    const int q0 = pair * 2 * BM;
+    const int N = p.N;
+    const int n_kv_all = (N + BN - 1) / BN;
+    int n_kv[2];
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int row0 = q0 + t * BM;
+        n_kv[t] = (row0 >= N) ? 0 : (CAUSAL ? min(n_kv_all, row0 / BN + 1) : n_kv_all);
+    }
+    const int n_kv_max = max(n_kv[0], n_kv[1]);
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_full[t], 128);
+            mbar_init(&o_full[t], 1);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == LOAD_WARP && lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == LOAD_WARP) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            uint32_t qbytes = 0;
+            for (int t = 0; t < 2; ++t) qbytes += (n_kv[t] > 0) ? C::TILE_BYTES : 0;
+            mbar_arrive_expect_tx(q_full, qbytes);
+            for (int t = 0; t < 2; ++t)
+                if (n_kv[t] > 0)
+                    for (int c = 0; c < C::NDC; ++c)
+                        tma_load_3d(sQ + t * C::TILE_BYTES + c * C::BOX_BYTES, &p.tm_q, q_full, c * 64,
+                                    q0 + t * BM, bh);
+            int it = 0;
+            bool ok = true;
+            for (int j = 0; j < n_kv_max && ok; ++j) {
+                for (int kind = 0; kind < 2; ++kind) {
+                    const int s = it % C::STAGES;
+                    if (!mbar_wait(&kv_empty[s], ((it / C::STAGES) & 1) ^ 1, p.ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
+                    const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
+                    for (int c = 0; c < C::NDC; ++c)
+                        tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64, j * BN,
+                                    bh);
+                    ++it;
+                }
+            }
+            if (!ok) {
+                // let every copy already issued land before the CTA exits
+                mbar_wait_drain(q_full, 0, p.ctl.limit_ns);
+                for (int i = max(0, it - C::STAGES); i < it; ++i)
+                    mbar_wait_drain(&kv_full[i % C::STAGES], (i / C::STAGES) & 1, p.ctl.limit_ns);
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
+            constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
+            const uint32_t sQa = smem_u32(sQ);
+            const uint32_t sKVa = smem_u32(sKV);
+            auto issue_s = [&](int t, int stage) {
+                const uint32_t qa = sQa + t * C::TILE_BYTES;
+                const uint32_t kb = sKVa + stage * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+                    mma_ss(tmem + 128u * t, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                           idesc_s, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_o = [&](int t, int stage, int j) {
+                const uint32_t vb = sKVa + stage * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    mma_ts(tmem + C::O_COL + D * t, tmem + 128u * t + kk * 8,
+                           sdesc_sw128(vb + kk * 2048, C::BOX_BYTES, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(q_full, 0, p.ctl);
+            int it = 0;
+            if (ok) {
+                const int sK = it % C::STAGES;
+                ok = mbar_wait(&kv_full[sK], (it / C::STAGES) & 1, p.ctl);
+                ++it;
+                if (ok) {
+                    tc_fence_after();
+                    for (int t = 0; t < 2; ++t)
+                        if (n_kv[t] > 0) {
+                            issue_s(t, sK);
+                            mma_commit(&s_full[t]);
+                        }
+                    mma_commit(&kv_empty[sK]);
+                }
+            }
+            for (int j = 0; j < n_kv_max && ok; ++j) {
+                const int sV = it % C::STAGES;
+                if (!(ok = mbar_wait(&kv_full[sV], (it / C::STAGES) & 1, p.ctl))) break;
+                ++it;
+                int sKn = -1;
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (j >= n_kv[t]) continue;
+                    if (!(ok = mbar_wait(&p_full[t], j & 1, p.ctl))) break;
+                    tc_fence_after();
+                    issue_o(t, sV, j);
+                    if (j == n_kv[t] - 1) mma_commit(&o_full[t]);
+                    if (j + 1 < n_kv[t]) {
+                        if (sKn < 0) {
+                            sKn = it % C::STAGES;
+                            if (!(ok = mbar_wait(&kv_full[sKn], (it / C::STAGES) & 1, p.ctl))) break;
+                            ++it;
+                            tc_fence_after();
+                        }
+                        issue_s(t, sKn);
+                        mma_commit(&s_full[t]);
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&kv_empty[sV]);
+                if (sKn >= 0) mma_commit(&kv_empty[sKn]);
+            }
+            // every MMA issued above completes before TMEM is released
+            mma_commit(drain);
+            mbar_wait_drain(drain, 0, p.ctl.limit_ns);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int t = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const int row = q0 + t * BM + r;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + 128u * t;
+        const uint32_t o_addr = tmem + lane_off + C::O_COL + D * t;
+        const float cl2 = p.scale_log2;
+        float m = -INFINITY;
+        float l = 0.f;
+        bool ok = true;
+        const int nk = n_kv[t];
+        for (int j = 0; j < nk; ++j) {
+            if (!(ok = warp_wait(&s_full[t], j & 1, p.ctl))) break;
+            tc_fence_after();
+            float s[BN];
+            tmem_ld32(s_addr + 0, reinterpret_cast<uint32_t*>(s + 0));
+            tmem_ld32(s_addr + 32, reinterpret_cast<uint32_t*>(s + 32));
+            tmem_ld32(s_addr + 64, reinterpret_cast<uint32_t*>(s + 64));
+            tmem_ld32(s_addr + 96, reinterpret_cast<uint32_t*>(s + 96));
+            tmem_wait_ld();
+            if (j == nk - 1) {
+                // last key tile of this Q tile: causal diagonal and/or ragged tail
+                const int limit = min(CAUSAL ? r : BN - 1, N - 1 - j * BN);
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (c > limit) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+            const float m_blk = mx * cl2;
+            float alpha = 1.f;
+            if (j == 0) {
+                m = m_blk;
+            } else if (m_blk > m + RESCALE_LOG2) {
+                alpha = ex2_approx(m - m_blk);
+                m = m_blk;
+            }
+            const float neg_m = -m;
+            float sum = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[BN / 4];
+#pragma unroll
+                for (int c = 0; c < BN / 2; c += 2) {
+                    const float p0 = ex2_approx(fmaf(s[h * (BN / 2) + c], cl2, neg_m));
+                    const float p1 = ex2_approx(fmaf(s[h * (BN / 2) + c + 1], cl2, neg_m));
+                    sum += p0 + p1;
+                    pk[c / 2] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(s_addr + h * (BN / 4), pk);
+            }
+            l = l * alpha + sum;
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                // O_t already holds sum_{j'<j} P V_j' (its MMA precedes this S in
+                // issue order, so S_t's commit covered it); rescale in TMEM.  Done
+                // after P is written so the S registers are dead by now.
+#pragma unroll
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + cc, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(o_addr + cc, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&p_full[t]);
+        }
+        if (ok && nk > 0) {
+            ok = warp_wait(&o_full[t], 0, p.ctl);
+            if (ok) {
+                tc_fence_after();
+                const float inv_l = 1.f / l;
+                __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * N + row) * D;
+#pragma unroll
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + cc, o);
+                    tmem_wait_ld();
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        packed[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                    if (row < N) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + cc);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                    }
+                }
+                if (row < N) p.lse[static_cast<size_t>(bh) * N + row] = (m + __log2f(l)) * LN2;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch(const FwdParams& p, cudaStream_t stream)
+{
+    using C = Cfg<D>;
+    auto kern = fwd_kernel<D, CAUSAL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.BH, p.n_pairs);
+    kern<<<grid, NTHREADS, C::SMEM_BYTES, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace fwdk
+
+cudaError_t launch_fwd_sm100(const FwdParams& p, int d, bool causal, cudaStream_t stream)
+{
+    if (d == 128) return causal ? fwdk::launch<128, true>(p, stream) : fwdk::launch<128, false>(p, stream);
+    return causal ? fwdk::launch<64, true>(p, stream) : fwdk::launch<64, false>(p, stream);
+}
+
+}  // namespace fa

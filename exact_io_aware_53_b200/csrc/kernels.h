@@ -1,0 +1,100 @@
+// Internal interface between the host API (fa_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa_status.h"
+
+namespace fa {
+
+// ---------------------------------------------------------------- bf16 forward
+struct FwdParams {
+    CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle
+    CUtensorMap tm_k;
+    CUtensorMap tm_v;
+    __nv_bfloat16* o;  // [B*H][N][d]
+    float* lse;        // [B*H][N]
+    int BH;
+    int N;
+    int n_pairs;       // ceil(N / 256)
+    float scale_log2;  // scale * log2(e)
+    WaitCtl ctl;
+};
+
+cudaError_t launch_fwd_sm100(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+
+// ---------------------------------------------------------------- bf16 backward
+struct BwdPreParams {
+    const __nv_bfloat16* o;
+    const __nv_bfloat16* dO;
+    const float* lse;
+    float* delta;  // D_i = <dO_i, O_i>            [B*H][n_pad]
+    float* lse2;   // lse_i * log2(e)              [B*H][n_pad]
+    float* dq;     // zeroed                       [B*H][N][d]
+    int BH;
+    int N;
+    int n_pad;     // rows per head in delta / lse2 (N rounded up to 128)
+    int d;
+};
+cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
+
+struct BwdParams {
+    CUtensorMap tm_q;    // {d, N, B*H}, box {64, 64, 1}
+    CUtensorMap tm_do;   // {d, N, B*H}, box {64, 64, 1}
+    CUtensorMap tm_k;    // {d, N, B*H}, box {64, 128, 1}
+    CUtensorMap tm_v;    // {d, N, B*H}, box {64, 128, 1}
+    CUtensorMap tm_dq;   // fp32 {d, N, B*H}, box {32, 64, 1}, reduce-add target
+    const float* lse2;   // [B*H][n_kv_tiles * 128]; +inf past N
+    const float* delta;  // [B*H][n_kv_tiles * 128]; 0 past N
+    float* dk;           // [B*H][N][d]
+    float* dv;           // [B*H][N][d]
+    int BH;
+    int N;
+    int n_kv_tiles;
+    float scale;
+    float scale_log2;
+    WaitCtl ctl;
+};
+cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, cudaStream_t stream);
+
+// ---------------------------------------------------------------- fp32 path
+struct F32Params {
+    const float* q;
+    const float* k;
+    const float* v;
+    const float* o;
+    const float* lse;
+    const float* dO;
+    float* o_out;
+    float* lse_out;
+    float* dq;
+    float* dk;
+    float* dv;
+    float* delta;
+    int BH;
+    int N;
+    int d;
+    int causal;
+    int block_k;
+    float scale;
+};
+cudaError_t launch_fwd_f32(const F32Params& p, cudaStream_t stream);
+cudaError_t launch_bwd_f32(const F32Params& p, cudaStream_t stream);
+
+// ---------------------------------------------------------------- self tests
+struct UmmaTestParams {
+    CUtensorMap tm_a;  // operand A storage (K-major: [M][K], MN-major: [K][M]), box {64, rows, 1}
+    CUtensorMap tm_b;  // operand B storage (K-major: [N][K], MN-major: [K][N])
+    const __nv_bfloat16* a_raw;  // A as [M][K] row-major (for the TMEM-operand variant)
+    const __nv_bfloat16* b_raw;  // B storage (for the manual-swizzle variant)
+    float* d;          // [M][N] fp32 result
+    int M, N, K;
+    int a_mn, b_mn, a_tmem, b_manual;
+    WaitCtl ctl;
+};
+cudaError_t launch_umma_selftest(const UmmaTestParams& p, cudaStream_t stream);
+
+}  // namespace fa

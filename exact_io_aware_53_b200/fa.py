@@ -1,0 +1,204 @@
+"""Python binding of the C ABI in ``include/fa.h`` (argument marshalling only).
+
+Every step of attention runs in the CUDA library ``libfa_sm100.so``; this
+module checks torch tensors, passes their device pointers and the current
+stream, and turns status codes into exceptions.  Importing it fails loudly if
+the library has not been built: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libfa_sm100.so is not built; run `python -m exact_io_aware_53_b200.build` "
+                      "(or __graft_entry__.build()) first")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+P = ctypes.c_void_p
+I = ctypes.c_int
+F = ctypes.c_float
+SZ = ctypes.c_size_t
+
+_SIGS = {
+    "fa_fwd": ([P, P, P, P, P, I, I, I, I, F, I, P], I),
+    "fa_bwd_workspace_bytes": ([I, I, I, I], SZ),
+    "fa_bwd": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
+    "fa_fwd_f32": ([P, P, P, P, P, I, I, I, I, F, I, I, P], I),
+    "fa_bwd_f32": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
+    "fa_attention_host_arena_bytes": ([I, I, I, I], SZ),
+    "fa_attention_host": ([P, P, P, P, P, P, P, P, P, P, SZ, I, I, I, I, F, I, P], I),
+    "fa_check_device_status": ([P], I),
+    "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
+    "fa_status_string": ([I], ctypes.c_char_p),
+    "fa_last_launch_count": ([], I),
+    "fa_selftest_umma": ([P, P, P, I, I, I, I, I, I, I, P], I),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+FA_OK = 0
+FA_ERR_INVALID_ARG = 1
+FA_ERR_UNSUPPORTED = 2
+FA_ERR_MISALIGNED = 3
+FA_ERR_CUDA = 4
+FA_ERR_TIMEOUT = 5
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s" % (what, _lib.fa_status_string(status).decode()))
+
+
+def _check(status: int, what: str):
+    if status != FA_OK:
+        raise FAError(status, what)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def exported_symbols():
+    return list(_SIGS)
+
+
+def status_string(status: int) -> str:
+    return _lib.fa_status_string(status).decode()
+
+
+def last_launch_count() -> int:
+    return int(_lib.fa_last_launch_count())
+
+
+def set_wait_limit_ns(ns: int):
+    _lib.fa_set_wait_limit_ns(int(ns))
+
+
+def check_device_status(stream=None) -> int:
+    return int(_lib.fa_check_device_status(_stream(stream)))
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(int(x) for x in q.shape)
+
+
+def _same(*ts, dtype):
+    ref = ts[0]
+    for t in ts:
+        if t.shape != ref.shape or t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA %s of shape %s" % (dtype, tuple(ref.shape)))
+
+
+# ------------------------------------------------------------------ bf16 path
+
+def fwd_raw(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    return _lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale), int(causal),
+                       _stream(stream))
+
+
+def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):
+    """O, LSE = attention(q, k, v); bf16 [B,H,N,d] in, bf16 O and fp32 LSE [B,H,N] out."""
+    _same(q, k, v, dtype=torch.bfloat16)
+    B, H, N, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(fwd_raw(q, k, v, o, lse, scale, causal, stream), "fa_fwd")
+    return o, lse
+
+
+def bwd_workspace_bytes(B, H, N, d) -> int:
+    return int(_lib.fa_bwd_workspace_bytes(B, H, N, d))
+
+
+def bwd_raw(q, k, v, o, lse, do, dq, dk, dv, ws, scale: float, causal: bool, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    return _lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                       _ptr(ws), B, H, N, d, float(scale), int(causal), _stream(stream))
+
+
+def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, workspace=None, stream=None):
+    """dQ, dK, dV (fp32) of L = sum(O * dO), recomputing the weights from lse."""
+    _same(q, k, v, o, do, dtype=torch.bfloat16)
+    B, H, N, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty_like(dq)
+    dv = torch.empty_like(dq)
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
+    _check(bwd_raw(q, k, v, o, lse, do, dq, dk, dv, workspace, scale, causal, stream), "fa_bwd")
+    return dq, dk, dv
+
+
+# ------------------------------------------------------------------ fp32 path
+
+def fwd_f32(q, k, v, causal: bool = False, scale: float | None = None, block_k: int = 0, stream=None):
+    _same(q, k, v, dtype=torch.float32)
+    B, H, N, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check(_lib.fa_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale), int(causal),
+                           int(block_k), _stream(stream)), "fa_fwd_f32")
+    return o, lse
+
+
+def bwd_f32(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, stream=None):
+    _same(q, k, v, o, do, dtype=torch.float32)
+    B, H, N, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(q)
+    dv = torch.empty_like(q)
+    ws = torch.empty(bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
+    _check(_lib.fa_bwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                           _ptr(ws), B, H, N, d, float(scale), int(causal), _stream(stream)), "fa_bwd_f32")
+    return dq, dk, dv
+
+
+# ------------------------------------------------------------------ host-buffer step
+
+def attention_host_arena_bytes(B, H, N, d) -> int:
+    return int(_lib.fa_attention_host_arena_bytes(B, H, N, d))
+
+
+def attention_host(hq, hk, hv, hdo, arena, outs, causal: bool, scale: float | None = None, stream=None) -> None:
+    """Forward + backward from host (pinned) bf16 tensors; ``outs`` = dict of host
+    tensors o (bf16), lse, dq, dk, dv (fp32), any may be missing.  Enqueues only."""
+    B, H, N, d = _shape(hq)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    g = outs.get
+    _check(_lib.fa_attention_host(_ptr(hq), _ptr(hk), _ptr(hv), _ptr(hdo), _ptr(g("o")), _ptr(g("lse")),
+                                  _ptr(g("dq")), _ptr(g("dk")), _ptr(g("dv")), _ptr(arena),
+                                  arena.numel() * arena.element_size(), B, H, N, d, float(scale), int(causal),
+                                  _stream(stream)), "fa_attention_host")
+
+
+# ------------------------------------------------------------------ diagnostics
+
+def selftest_umma(a, b, M, N, K, a_mn, b_mn, a_tmem=False, b_manual=False, stream=None):
+    d = torch.empty((M, N), dtype=torch.float32, device=a.device)
+    _check(_lib.fa_selftest_umma(_ptr(a), _ptr(b), _ptr(d), M, N, K, int(a_mn), int(b_mn), int(a_tmem),
+                                 int(b_manual), _stream(stream)), "fa_selftest_umma")
+    return d

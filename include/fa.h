@@ -1,0 +1,136 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library libfa_sm100.so.
+ *
+ * The operation is exact scaled-dot-product attention
+ *
+ *     O = softmax(scale * Q K^T [+ causal mask]) V,
+ *
+ * computed tile by tile with the online-softmax update (running max m, running
+ * sum l, accumulator O rescaled by e^{m_old - m_new}, final O / l), so the N x N
+ * score matrix never reaches device memory; see "Tiling and the online softmax"
+ * and "The math, worked with real numbers" (the three update lines) on
+ * vibeengines.com/paper/flash-attention, and "Main concepts to understand" on
+ * chorfi.xyz/research/papers/paper-flashattention.  The backward pass
+ * recomputes the attention weights tile by tile from the saved log-sum-exp
+ * instead of storing them ("What it did not solve", same explainer page; "Study
+ * objectives", the reading guide).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, row-major [B][H][N][d] ("BHND", torch (B,H,N,d)
+ *     contiguous); lse and the workspace vectors are [B][H][N].
+ *   - All pointers are DEVICE pointers owned by the caller unless the name says
+ *     host; the library keeps no pointer after a call returns and allocates no
+ *     device memory.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work; they return before the GPU finishes.
+ *   - Causal masking is square and top-left aligned: query i sees keys j <= i.
+ *   - lse_i = ln sum_j exp(scale * q_i . k_j) over the keys row i sees (natural log).
+ *   - Return value: FA_OK, or an fa_status_t code.  Argument, shape and
+ *     alignment errors are detected before anything is enqueued and leave all
+ *     memory untouched.  A bounded wait that expires inside a kernel is
+ *     reported by fa_check_device_status().
+ */
+#ifndef FA_SM100_H
+#define FA_SM100_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad flag       */
+    FA_ERR_UNSUPPORTED = 2, /* head dim / dtype combination not implemented    */
+    FA_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned                 */
+    FA_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed              */
+    FA_ERR_TIMEOUT = 5      /* a kernel's bounded wait expired (device status)  */
+} fa_status_t;
+
+/*
+ * Forward, bf16.  q, k, v, o: bf16 [B][H][N][d]; lse: fp32 [B][H][N] (output).
+ * d must be 64 or 128; N >= 1; B, H >= 1; B*H*N*d < 2^31.  scale > 0 (the
+ * reading of the pages' standard attention is 1/sqrt(d)).  causal: 0 or 1.
+ * All pointers 16-byte aligned.  q/k/v may alias each other, o and lse must
+ * not overlap any input.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+           float scale, int causal, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: the row terms D_i = <dO_i, O_i> and
+ * the log-sum-exp in base 2, both fp32 [B][H][N] (O(N), never O(N^2)).
+ */
+size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward, bf16 inputs, fp32 gradients.  q, k, v, o, dO: bf16 [B][H][N][d];
+ * lse: fp32 [B][H][N] as written by fa_fwd for the same inputs; dq, dk, dv:
+ * fp32 [B][H][N][d] (outputs; dq is zeroed by the call and accumulated into);
+ * workspace: fa_bwd_workspace_bytes(B,H,N,d) bytes of device memory, 16-byte
+ * aligned, contents irrelevant on entry.  Gradients are of L = sum(O * dO).
+ * Same shape rules as fa_fwd.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+           float* dq, float* dk, float* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
+           void* stream);
+
+/*
+ * Forward, fp32 (all tensors fp32).  1 <= d <= 128.  block_k is the key
+ * block size of the online-softmax walk (1 .. 1024; 0 selects 64): the result
+ * must not depend on it beyond rounding ("Block size never changes the
+ * answer", "Solve it yourself" on the explainer page).
+ */
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int d,
+               float scale, int causal, int block_k, void* stream);
+
+/*
+ * Backward, fp32.  Inputs as fa_fwd_f32 plus o, lse (from it) and dO; outputs
+ * dq, dk, dv fp32 [B][H][N][d].  workspace: fa_bwd_workspace_bytes bytes.
+ */
+int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* lse,
+               const float* dO, float* dq, float* dk, float* dv, void* workspace, int B, int H, int N, int d,
+               float scale, int causal, void* stream);
+
+/*
+ * Bytes of device arena fa_attention_host needs for B,H,N,d (bf16 path).
+ */
+size_t fa_attention_host_arena_bytes(int B, int H, int N, int d);
+
+/*
+ * One forward + backward step from HOST buffers: copies h_q, h_k, h_v, h_dO
+ * (bf16, host memory -- pinned for asynchronous copies) into `arena` (device,
+ * fa_attention_host_arena_bytes bytes, 256-byte aligned), runs fa_fwd and
+ * fa_bwd there, and copies o (bf16), lse, dq, dk, dv (fp32) back to the host
+ * buffers, all on `stream`.  Returns after enqueueing; the host buffers are
+ * valid once the stream is synchronised.  Any output pointer may be NULL to
+ * skip that copy back.
+ */
+int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const void* h_dO, void* h_o,
+                      float* h_lse, float* h_dq, float* h_dk, float* h_dv, void* arena, size_t arena_bytes, int B,
+                      int H, int N, int d, float scale, int causal, void* stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device error word of the
+ * current device: FA_ERR_TIMEOUT if a kernel's bounded wait expired (the
+ * kernel then abandoned its tile and returned), FA_ERR_CUDA if the stream
+ * itself reported an error, else FA_OK.
+ */
+int fa_check_device_status(void* stream);
+
+/* Upper bound, in nanoseconds, on any single wait inside a kernel of this
+ * library (default 2e9).  Values below 1e6 are raised to 1e6.  Process-wide. */
+void fa_set_wait_limit_ns(unsigned long long ns);
+
+/* Human-readable name of a status code (static string). */
+const char* fa_status_string(int status);
+
+/* Number of kernels the most recent fa_* call enqueued on the calling thread. */
+int fa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H */

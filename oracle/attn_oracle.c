@@ -314,3 +314,119 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v, const dou
     }
     return err;
 }
+
+/*
+ * dQ for rows [i0, i1) of ONE head (q, k, v, dO point at that head's [N][d]
+ * blocks; dq receives i1 - i0 rows).  Row i of dQ needs only row i of P and
+ * dP, so sampled rows of workloads too large for the full backward stay cheap.
+ * Same definition as oracle_attn_bwd.
+ */
+int oracle_attn_bwd_dq_rows(const double* q, const double* k, const double* v, const double* dO,
+                            double* dq, long N, long d, long i0, long i1, double scale,
+                            int causal)
+{
+    if (N < 1 || d < 1 || i0 < 0 || i1 > N || i0 > i1) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* prow = (double*)malloc((size_t)N * sizeof(double));
+        double* dprow = (double*)malloc((size_t)N * sizeof(double));
+        if (!prow || !dprow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (long i = i0; i < i1; ++i) {
+            if (!prow || !dprow) continue;
+            const double* qi = q + i * d;
+            const double* doi = dO + i * d;
+            long nk = n_allowed(i, N, causal);
+            double m = -INFINITY;
+            for (long j = 0; j < nk; ++j) {
+                prow[j] = scale * dot(qi, k + j * d, d);
+                if (prow[j] > m) m = prow[j];
+            }
+            double l = 0.0;
+            for (long j = 0; j < nk; ++j) {
+                prow[j] = exp(prow[j] - m);
+                l += prow[j];
+            }
+            for (long j = 0; j < nk; ++j) prow[j] /= l;
+            double D = 0.0;
+            for (long j = 0; j < nk; ++j) {
+                dprow[j] = dot(doi, v + j * d, d);
+                D += prow[j] * dprow[j];
+            }
+            double* dqi = dq + (i - i0) * d;
+            for (long t = 0; t < d; ++t) dqi[t] = 0.0;
+            for (long j = 0; j < nk; ++j) {
+                double ds = prow[j] * (dprow[j] - D);
+                const double* kj = k + j * d;
+                for (long t = 0; t < d; ++t) dqi[t] += ds * kj[t];
+            }
+            for (long t = 0; t < d; ++t) dqi[t] *= scale;
+        }
+        free(prow);
+        free(dprow);
+    }
+    return err;
+}
+
+/*
+ * dK and dV for keys [j0, j1) of ONE head (dk, dv receive j1 - j0 rows).  Every
+ * query row that sees one of these keys is materialised in turn (its P row, dP
+ * row and D_i), and only the columns j0..j1-1 are accumulated.  Cheap for the
+ * last keys of a causal head, which few rows see.  Same definition as
+ * oracle_attn_bwd.
+ */
+int oracle_attn_bwd_kv_rows(const double* q, const double* k, const double* v, const double* dO,
+                            double* dk, double* dv, long N, long d, long j0, long j1,
+                            double scale, int causal)
+{
+    if (N < 1 || d < 1 || j0 < 0 || j1 > N || j0 > j1) return -1;
+    const long nj = j1 - j0;
+    memset(dk, 0, (size_t)(nj * d) * sizeof(double));
+    memset(dv, 0, (size_t)(nj * d) * sizeof(double));
+    double* prow = (double*)malloc((size_t)N * sizeof(double));
+    double* dprow = (double*)malloc((size_t)N * sizeof(double));
+    if (!prow || !dprow) {
+        free(prow);
+        free(dprow);
+        return -1;
+    }
+    for (long i = causal ? j0 : 0; i < N; ++i) {
+        const double* qi = q + i * d;
+        const double* doi = dO + i * d;
+        long nk = n_allowed(i, N, causal);
+        double m = -INFINITY;
+        for (long j = 0; j < nk; ++j) {
+            prow[j] = scale * dot(qi, k + j * d, d);
+            if (prow[j] > m) m = prow[j];
+        }
+        double l = 0.0;
+        for (long j = 0; j < nk; ++j) {
+            prow[j] = exp(prow[j] - m);
+            l += prow[j];
+        }
+        for (long j = 0; j < nk; ++j) prow[j] /= l;
+        double D = 0.0;
+        for (long j = 0; j < nk; ++j) {
+            dprow[j] = dot(doi, v + j * d, d);
+            D += prow[j] * dprow[j];
+        }
+        long jend = j1 < nk ? j1 : nk;
+        for (long j = j0; j < jend; ++j) {
+            double ds = prow[j] * (dprow[j] - D);
+            double* dkj = dk + (j - j0) * d;
+            double* dvj = dv + (j - j0) * d;
+            for (long t = 0; t < d; ++t) {
+                dkj[t] += ds * qi[t];
+                dvj[t] += prow[j] * doi[t];
+            }
+        }
+    }
+    for (long e = 0; e < nj * d; ++e) dk[e] *= scale;
+    free(prow);
+    free(dprow);
+    return 0;
+}

@@ -53,6 +53,10 @@ def _load():
         lib.oracle_attn_fwd_tiled.restype = I
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, D, I]
         lib.oracle_attn_bwd.restype = I
+        lib.oracle_attn_bwd_dq_rows.argtypes = [P, P, P, P, P, L, L, L, L, D, I]
+        lib.oracle_attn_bwd_dq_rows.restype = I
+        lib.oracle_attn_bwd_kv_rows.argtypes = [P, P, P, P, P, P, L, L, L, L, D, I]
+        lib.oracle_attn_bwd_kv_rows.restype = I
         _lib = lib
     return _lib
 
@@ -149,3 +153,28 @@ def attn_bwd(q, k, v, do, scale: float, causal: bool):
     if rc != 0:
         raise RuntimeError("oracle_attn_bwd failed (%d)" % rc)
     return dq, dk, dv
+
+
+def attn_bwd_dq_rows(q, k, v, do, i0: int, i1: int, scale: float, causal: bool):
+    """dQ rows [i0, i1) of ONE head; q, k, v, do are that head's [N, d] arrays."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    N, d = q.shape
+    dq = np.empty((i1 - i0, d))
+    rc = _load().oracle_attn_bwd_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), N, d, i0, i1,
+                                         float(scale), int(bool(causal)))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_bwd_dq_rows failed (%d)" % rc)
+    return dq
+
+
+def attn_bwd_kv_rows(q, k, v, do, j0: int, j1: int, scale: float, causal: bool):
+    """(dK, dV) rows [j0, j1) of ONE head; q, k, v, do are that head's [N, d] arrays."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    N, d = q.shape
+    dk = np.empty((j1 - j0, d))
+    dv = np.empty((j1 - j0, d))
+    rc = _load().oracle_attn_bwd_kv_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dk), _ptr(dv), N, d,
+                                         j0, j1, float(scale), int(bool(causal)))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_bwd_kv_rows failed (%d)" % rc)
+    return dk, dv

@@ -1,0 +1,104 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments before touching the GPU (runs without a GPU)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_io_aware_53_b200 import build
+    build.build()
+    from exact_io_aware_53_b200 import fa
+    return fa
+
+
+def _declared():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?(?:int|void|size_t|char)\s*\*?\s*(fa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert "fa_fwd" in names and "fa_bwd" in names and "fa_selftest_umma" in names
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in names:
+        assert hasattr(so, n), n
+    assert set(names) == set(lib.exported_symbols())
+
+
+def test_status_strings(lib):
+    assert lib.status_string(0) == "FA_OK"
+    assert lib.status_string(5) == "FA_ERR_TIMEOUT"
+    assert lib.status_string(99) == "FA_ERR_UNKNOWN"
+
+
+def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=8, d=64, scale=0.125, causal=0):
+    P = ctypes.c_void_p
+    return lib._lib.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, scale, causal, P(0))
+
+
+def test_fwd_argument_errors_are_returned_before_any_launch(lib):
+    assert _fwd(lib, q=0) == lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, N=0) == lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, B=-1) == lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, causal=2) == lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=0.0) == lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=-1.0) == lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan")) == lib.FA_ERR_INVALID_ARG
+    assert _fwd(lib, d=96) == lib.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, d=256) == lib.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, B=1 << 12, H=1 << 12, N=1 << 12, d=64) == lib.FA_ERR_UNSUPPORTED
+    assert _fwd(lib, k=24) == lib.FA_ERR_MISALIGNED
+    assert _fwd(lib, lse=20) == lib.FA_ERR_MISALIGNED
+
+
+def test_bwd_argument_errors(lib):
+    P = ctypes.c_void_p
+    good = [P(16)] * 10
+    args = lambda ptrs, d=128, N=8: (*ptrs, 1, 1, N, d, 0.1, 1, P(0))
+    assert lib._lib.fa_bwd(*args(good[:9] + [P(0)])) == lib.FA_ERR_INVALID_ARG
+    assert lib._lib.fa_bwd(*args(good, d=32)) == lib.FA_ERR_UNSUPPORTED
+    assert lib._lib.fa_bwd(*args(good[:5] + [P(8)] + good[6:])) == lib.FA_ERR_MISALIGNED
+
+
+def test_f32_argument_errors(lib):
+    P = ctypes.c_void_p
+    f = lib._lib.fa_fwd_f32
+    assert f(P(16), P(16), P(16), P(16), P(16), 1, 1, 8, 129, 0.1, 0, 0, P(0)) == lib.FA_ERR_UNSUPPORTED
+    assert f(P(16), P(16), P(16), P(16), P(16), 1, 1, 8, 64, 0.1, 0, 2000, P(0)) == lib.FA_ERR_INVALID_ARG
+    assert f(P(16), P(16), P(16), P(16), P(16), 1, 1, 8, 64, 0.1, 0, -1, P(0)) == lib.FA_ERR_INVALID_ARG
+    assert f(P(0), P(16), P(16), P(16), P(16), 1, 1, 8, 64, 0.1, 0, 0, P(0)) == lib.FA_ERR_INVALID_ARG
+
+
+def test_workspace_is_linear_in_sequence_length(lib):
+    # two fp32 row vectors per head, padded to 128 rows and 256 bytes: O(N), never O(N^2)
+    for B, H, N, d in [(1, 1, 1, 64), (4, 16, 4096, 128), (1, 16, 16384, 128), (2, 3, 300, 64)]:
+        rows = B * H * (-(-N // 128) * 128)
+        assert lib.bwd_workspace_bytes(B, H, N, d) == 2 * (-(-rows * 4 // 256) * 256)
+    assert lib.bwd_workspace_bytes(0, 1, 1, 64) == 0
+
+
+def test_host_arena_size(lib):
+    B, H, N, d = 2, 3, 300, 64
+    E, R = B * H * N * d, B * H * N
+    up = lambda x: -(-x // 256) * 256
+    want = 5 * up(E * 2) + 3 * up(E * 4) + up(R * 4) + up(lib.bwd_workspace_bytes(B, H, N, d))
+    assert lib.attention_host_arena_bytes(B, H, N, d) == want
+
+
+def test_selftest_argument_errors(lib):
+    P = ctypes.c_void_p
+    f = lib._lib.fa_selftest_umma
+    assert f(P(16), P(16), P(16), 64, 64, 64, 0, 0, 0, 0, P(0)) == lib.FA_ERR_UNSUPPORTED
+    assert f(P(16), P(16), P(16), 128, 64, 64, 1, 0, 1, 0, P(0)) == lib.FA_ERR_UNSUPPORTED
+    assert f(P(0), P(16), P(16), 128, 64, 64, 0, 0, 0, 0, P(0)) == lib.FA_ERR_INVALID_ARG

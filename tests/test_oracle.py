@@ -245,3 +245,22 @@ def test_bwd_invariants(causal):
         o, lse = oracle.attn_fwd(q, k, v, 0.35, True)
         p_last = np.exp(0.35 * np.sum(q[:, :, -1] * k[:, :, -1], -1) - lse[:, :, -1])
         assert np.max(np.abs(dv[:, :, -1] - p_last[..., None] * g[:, :, -1])) < 1e-13
+
+
+def test_bwd_dq_rows_matches_full_backward():
+    shape = (1, 1, 37, 5)
+    q, k, v, g = (_rand(shape, seed=s) for s in (101, 102, 103, 104))
+    for causal in (False, True):
+        dq, _, _ = oracle.attn_bwd(q, k, v, g, 0.45, causal)
+        rows = oracle.attn_bwd_dq_rows(q[0, 0], k[0, 0], v[0, 0], g[0, 0], 5, 29, 0.45, causal)
+        assert np.max(np.abs(rows - dq[0, 0, 5:29])) < 1e-14
+
+
+def test_bwd_kv_rows_matches_full_backward():
+    shape = (1, 1, 41, 6)
+    q, k, v, g = (_rand(shape, seed=s) for s in (111, 112, 113, 114))
+    for causal in (False, True):
+        _, dk, dv = oracle.attn_bwd(q, k, v, g, 0.4, causal)
+        rk, rv = oracle.attn_bwd_kv_rows(q[0, 0], k[0, 0], v[0, 0], g[0, 0], 9, 30, 0.4, causal)
+        assert np.max(np.abs(rk - dk[0, 0, 9:30])) < 1e-14
+        assert np.max(np.abs(rv - dv[0, 0, 9:30])) < 1e-14
