@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Exact attention forward + backward on B200: throughput against the tensor roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl ours|reference]
+
+One step = the whole hot path over one batch of synthetic inputs already
+resident in device memory: fa_fwd (O, LSE), fa_bwd_prep (D, log2 LSE, dQ := 0)
+and fa_bwd_main (dQ, dK, dV).  `value` is whole-job TFLOP/s under the FLOP
+convention 4*B*H*N^2*d forward, 2.5x that backward, halved under the causal
+mask.  Kernels are timed with CUDA events on the launching stream; with N > 1
+ranks each rank runs its own batch (weak scaling, no collective on the data
+path) and the step time is the max over ranks.
+
+--impl reference runs the fp64 CPU oracle on the host cores instead (one
+head of the workload per step) and prints the same JSON line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOPS on 1 B200 and fraction of dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "c4_bf16_4x16x4096x128_causal"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------ ranks
+
+def rank_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def init_dist(world: int, backend: str, device=None):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        kw = {"backend": backend, "timeout": datetime.timedelta(seconds=120)}
+        if device is not None:
+            kw["device_id"] = device
+        dist.init_process_group(**kw)
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Largest value of x over all ranks (a timing collective, not a data-path one)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch of the same shape (weak scaling)."""
+    return base_seed + 7919 * rank
+
+
+# ------------------------------------------------------------------ peaks / clocks
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "of measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "of fallback"
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons with nvidia-smi while running."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str, period_ms: int = 100):
+        self.uuid = uuid
+        self.period_ms = period_ms
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.t:
+            self.t.join(timeout=5)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9 or (self.uuid and parts[0] != self.uuid):
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names[1:], parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(w, heads: int, seed: int):
+    """fp64 oracle forward + backward on `heads` heads of workload w; returns (seconds, flops, threads)."""
+    from exact_io_aware_53_b200.workloads import make_inputs
+    from oracle import oracle
+    x = make_inputs(w, seed=seed, B=1, H=heads)
+    q, k, v, do = (x[n] for n in ("q", "k", "v", "do"))
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, w.scale, w.causal)
+    if w.backward:
+        oracle.attn_bwd(q, k, v, do, w.scale, w.causal)
+    dt = time.perf_counter() - t0
+    per_head = (w.flops_fwd() + (w.flops_bwd() if w.backward else 0.0)) / (w.B * w.H)
+    return dt, per_head * heads, oracle.num_threads()
+
+
+def cpu_baseline(w, seed: int, budget_s: float = 10.0):
+    dt1, fl1, thr = oracle_sample(w, 1, seed)
+    extra = max(0, min(int(budget_s / max(dt1, 1e-3)) - 1, 7))
+    dt, fl = dt1, fl1
+    if extra:
+        dt2, fl2, _ = oracle_sample(w, extra, seed + 1)
+        dt, fl = dt + dt2, fl + fl2
+    heads = 1 + extra
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": thr, "kind": "oracle",
+            "sample": "%d of %d heads (B=1, N=%d, d=%d, causal=%s), fwd%s, fp64, %.1f s" % (
+                heads, w.B * w.H, w.N, w.d, w.causal, "+bwd" if w.backward else "", dt)}
+
+
+def run_reference(args, w):
+    rank, world, _ = rank_env()
+    if rank != 0:
+        return 0
+    for i in range(args.warmup):
+        oracle_sample(w, 1, w.seed + i)
+    times = []
+    flops = 0.0
+    thr = 1
+    for i in range(args.steps):
+        dt, fl, thr = oracle_sample(w, 1, w.seed + 100 + i)
+        times.append(dt)
+        flops = fl
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms / 1e3) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": 1, "H": 1, "N": w.N, "d": w.d, "causal": w.causal,
+                       "sample": "one head per step", "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                             "sample": "one head of %s per step (fwd%s, fp64)" % (
+                                 w.name, "+bwd" if w.backward else "")},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args, w, print_line=True):
+    import torch
+    from exact_io_aware_53_b200 import fa
+    from exact_io_aware_53_b200.workloads import make_inputs
+
+    rank, world, local = rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        init_dist(world, "nccl", torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+
+    x = make_inputs(w, seed=rank_seed(w.seed, rank))
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    B, H, N, d = w.B, w.H, w.N, w.d
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty_like(dq)
+    dv = torch.empty_like(dq)
+    ws = torch.empty(max(1, fa.bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8, device=dev)
+    scale, causal = w.scale, w.causal
+
+    launches = [0]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rc = fa.fwd_raw(q, k, v, o, lse, scale, causal)
+        launches[0] += fa.last_launch_count()
+        if rc:
+            raise fa.FAError(rc, "fa_fwd")
+        if not w.backward:
+            if ev is not None:
+                ev[1].record(stream)
+            return
+        if ev is not None:
+            ev[1].record(stream)
+        rc = fa.bwd_prep_raw(o, lse, do, dq, ws)
+        launches[0] += fa.last_launch_count()
+        if rc:
+            raise fa.FAError(rc, "fa_bwd_prep")
+        if ev is not None:
+            ev[2].record(stream)
+        rc = fa.bwd_main_raw(q, k, v, do, dq, dk, dv, ws, scale, causal)
+        launches[0] += fa.last_launch_count()
+        if rc:
+            raise fa.FAError(rc, "fa_bwd_main")
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after warm-up: %s" % fa.status_string(st))
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    launches[0] = 0
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after timing: %s" % fa.status_string(st))
+    timed_launches = launches[0]
+
+    ms_local = t_start.elapsed_time(t_end) / args.steps
+    ms = max_over_ranks(ms_local, world, dev)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    prep_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) if w.backward else 0.0
+    main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs) if w.backward else 0.0
+    flops_step = w.flops_fwd() + (w.flops_bwd() if w.backward else 0.0)
+    value = world * flops_step / (ms / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    long_region = ms * args.steps > 500.0
+    peak_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    if w.backward:
+        dom_name, dom_ms, dom_flops = "bwd_main", main_ms, w.flops_bwd()
+    else:
+        dom_name, dom_ms, dom_flops = "fwd", fwd_ms, w.flops_fwd()
+    achieved = dom_flops / (dom_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": UNIT,
+                "frac": achieved / peak, "peak_source": "%s %s" % (peak_key, peak_src),
+                "frac_of_burst": achieved / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
+                "algorithmic_flops_per_launch": dom_flops, "ms_per_launch": dom_ms, "traffic": None}
+    fwd_tflops = w.flops_fwd() / (fwd_ms / 1e3) / 1e12
+    kernels = {"fwd": {"ms": fwd_ms, "tflops": fwd_tflops, "frac": fwd_tflops / peak}}
+    if w.backward:
+        bwd_tflops = w.flops_bwd() / ((prep_ms + main_ms) / 1e3) / 1e12
+        kernels["bwd_prep"] = {"ms": prep_ms}
+        kernels["bwd_main"] = {"ms": main_ms, "tflops": achieved, "frac": achieved / peak}
+        kernels["bwd_total"] = {"ms": prep_ms + main_ms, "tflops": bwd_tflops, "frac": bwd_tflops / peak}
+
+    # ---- end to end through the host-buffer entry point
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, fa, x, dev, stream, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, seed=w.seed)
+
+    in_bytes = 4 * B * H * N * d * 2
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                       "backward": w.backward, "global_batch": B * world, "seq_len": N,
+                       "parallelism": "dp%d (independent batches per GPU, no collective)" % world,
+                       "l2": "inputs larger than L2 (q,k,v,dO = %.0f MB per GPU)" % (in_bytes / 1e6)},
+            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": timed_launches, "clocks": clocks}
+    if rank == 0 and print_line:
+        print(json.dumps(line), flush=True)
+    return line
+
+
+def run_e2e(args, w, fa, x, dev, stream, world):
+    import torch
+    B, H, N, d = w.B, w.H, w.N, w.d
+    E, R = B * H * N * d, B * H * N
+    hq, hk, hv, hdo = (x[n].pin_memory() for n in ("q", "k", "v", "do"))
+    outs = {"o": torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory(),
+            "lse": torch.empty((B, H, N), dtype=torch.float32).pin_memory()}
+    if w.backward:
+        for n in ("dq", "dk", "dv"):
+            outs[n] = torch.empty((B, H, N, d), dtype=torch.float32).pin_memory()
+    arena = torch.empty(fa.attention_host_arena_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    if not w.backward:
+        return None
+    steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        fa.attention_host(hq, hk, hv, hdo, arena, outs, w.causal, w.scale)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        fa.attention_host(hq, hk, hv, hdo, arena, outs, w.causal, w.scale)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after e2e: %s" % fa.status_string(st))
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
+    flops = w.flops_fwd() + w.flops_bwd()
+    return {"value": world * flops / (ms / 1e3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": 4 * E * 2, "d2h_bytes_per_step": E * 2 + R * 4 + 3 * E * 4,
+            "steps": steps, "api": "fa_attention_host (pinned host buffers)"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    from exact_io_aware_53_b200.workloads import WORKLOADS
+    if args.workload != "all" and args.workload not in WORKLOADS:
+        ap.error("unknown workload %s (choose from %s)" % (args.workload, ", ".join(WORKLOADS)))
+    names = list(WORKLOADS) if args.workload == "all" else [args.workload]
+    rc = 0
+    try:
+        for name in names:
+            w = WORKLOADS[name]
+            if args.impl == "reference":
+                rc |= run_reference(args, w)
+            elif w.dtype != "bf16":
+                continue  # the fp32 workload is a correctness case, not a bench line
+            else:
+                run_ours(args, w)
+    finally:
+        _, world, _ = rank_env()
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,459 @@
+// Backward attention for head dimension 128, bf16 in / fp32 gradients, sm_100a.
+//
+// Same recomputation as the d = 64 kernel (the attention weights are rebuilt
+// per tile from the saved log-sum-exp, "What it did not solve",
+// vibeengines.com/paper/flash-attention; c = scale * log2 e, lse2 = lse * log2 e):
+//
+//   S^T  = K Q_t^T,  P^T = 2^(c S^T - lse2_t)      dP^T = V dO_t^T
+//   dS^T = P^T o (dP^T - D_t)                        D_t = <dO, O> per query row
+//   dV += P^T dO_t,  dK += dS^T Q_t,  dQ_t^T = K^T dS^T   (dK, dQ times scale)
+//
+// but every tensor-core instruction is 128 x 128 x 16: one CTA owns 128 keys and
+// walks 128-row query tiles (tile t).  A 128 x 64 instruction occupies the
+// tensor pipe about as long as a 128 x 128 one, so the wider query tile nearly
+// doubles the work per instruction.
+//
+// TMEM (512 columns): two 128-column regions R0, R1 and the dV, dK accumulators.
+// Tile t uses X = R[t & 1] for S^T -> P^T (bf16 pairs in its first 64 columns)
+// and then for dQ^T, and Y = R[(t + 1) & 1] for dP^T.  dS^T goes to shared
+// memory only, where it is the K-major A operand of dK and the MN-major B
+// operand of dQ^T; so Y is free once the softmax has read dP^T, and S^T of
+// tile t + 1 is issued there before dK and dQ^T of tile t, overlapping the
+// next softmax with them.  dP^T of tile t + 1 goes to X once the dQ warps have
+// read dQ^T out.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax: thread = key row = TMEM lane
+//   warps 4-7  dQ: thread = head-dim index d; read dQ^T (128 query columns),
+//              scale, stage it as fp32 [64 query][128 d] tiles and TMA
+//              reduce-add them into dQ, two tiles per query block
+//   warp 8     MMA issuer (one thread)
+//   warp 9     TMA producer: K, V once; {Q_t, lse2_t, D_t} in a 2-stage ring, dO_t
+//              in one buffer (its last reader, dV, runs early in a tile and its
+//              next reader, dP^T, late in the previous one)
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace bwd128k {
+
+constexpr int D = 128;
+constexpr int BKV = 128;
+constexpr int BQ = 128;
+constexpr int NTHREADS = 320;
+constexpr int MMA_WARP = 8;
+constexpr int LOAD_WARP = 9;
+constexpr int QSTAGES = 2;
+
+constexpr int BOX = 128 * 128;                    // 128 rows x 128 B (64 bf16)
+constexpr int TILE = 2 * BOX;                      // 128 rows x 128 bf16
+constexpr int K_OFF = 0;
+constexpr int V_OFF = K_OFF + TILE;
+constexpr int Q_OFF = V_OFF + TILE;                // Q_t, 2 stages
+constexpr int DO_OFF = Q_OFF + QSTAGES * TILE;     // dO_t, 1 stage (last read by dV, next needed by dP)
+constexpr int DS_OFF = DO_OFF + TILE;              // dS^T, 2 chunks of 64 query columns
+constexpr int STG_OFF = DS_OFF + TILE;             // dQ staging, fp32 [64 query][128 d]
+constexpr int STG_CHUNK = 64 * 128;                // fp32 [64 query rows][32 d], 128-byte swizzled
+constexpr int VEC_OFF = STG_OFF + 4 * STG_CHUNK;   // [stage][lse2 128 | delta 128]
+constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
+constexpr int NBARS = 16;
+constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// TMEM column of region R[t & 1]
+__device__ __forceinline__ uint32_t rcol(int t) { return 128u * static_cast<uint32_t>(t & 1); }
+constexpr uint32_t DV_COL = 256;
+constexpr uint32_t DK_COL = 384;
+constexpr uint32_t TMEM_COLS = 512;
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c)
+{
+    bool ok = mbar_wait(bar, parity, c);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <bool CAUSAL>
+__global__ void __launch_bounds__(NTHREADS, 1) bwd128_kernel(const __grid_constant__ BwdParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if ((smem_u32(smem) & 1023u) != 0u) {
+        if (threadIdx.x == 0) raise_status(p.ctl, FA_DEV_BAD_TILE);
+        return;
+    }
+    uint8_t* sK = smem + K_OFF;
+    uint8_t* sV = smem + V_OFF;
+    uint8_t* sQ = smem + Q_OFF;
+    uint8_t* sDO = smem + DO_OFF;
+    uint8_t* sDS = smem + DS_OFF;
+    uint8_t* sSTG = smem + STG_OFF;
+    float* sVec = reinterpret_cast<float*>(smem + VEC_OFF);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
+    uint64_t* kv_full = bars + 0;
+    uint64_t* q_full = bars + 1;   // [2]
+    uint64_t* q_empty = bars + 3;  // [2]
+    uint64_t* do_full = bars + 5;
+    uint64_t* do_empty = bars + 6;
+    uint64_t* s_full = bars + 7;
+    uint64_t* dp_full = bars + 8;
+    uint64_t* p_ready = bars + 9;
+    uint64_t* ds_ready = bars + 10;
+    uint64_t* dq_full = bars + 11;
+    uint64_t* dq_empty = bars + 12;
+    uint64_t* dkdv_done = bars + 13;
+    uint64_t* drain = bars + 14;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
+
+    const int warp = static_cast<int>(warp_id());
+    const int lane = static_cast<int>(lane_id());
+    // head-major order: CTAs resident together share a few heads' Q, dO and dQ in L2
+    const int j = blockIdx.x;  // key tile; tile 0 sees the most query tiles under the causal mask
+    const int bh = blockIdx.y;
+    const int N = p.N;
+    const int n_pad = p.n_kv_tiles * BKV;
+    const int n_q = (N + BQ - 1) / BQ;
+    const int i_first = CAUSAL ? j : 0;
+    const int n_it = n_q - i_first;  // >= 1
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < QSTAGES; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+        }
+        mbar_init(do_full, 1);
+        mbar_init(do_empty, 1);
+        mbar_init(s_full, 1);
+        mbar_init(dp_full, 1);
+        mbar_init(p_ready, 128);
+        mbar_init(ds_ready, 128);
+        mbar_init(dq_full, 1);
+        mbar_init(dq_empty, 128);
+        mbar_init(dkdv_done, 1);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == LOAD_WARP && lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_do);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_v);
+        tma_prefetch_desc(&p.tm_dq);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == LOAD_WARP) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(kv_full, 2 * TILE);
+            for (int c = 0; c < 2; ++c) {
+                tma_load_3d(sK + c * BOX, &p.tm_k, kv_full, c * 64, j * BKV, bh);
+                tma_load_3d(sV + c * BOX, &p.tm_v, kv_full, c * 64, j * BKV, bh);
+            }
+            const float* lse2_h = p.lse2 + static_cast<size_t>(bh) * n_pad;
+            const float* delta_h = p.delta + static_cast<size_t>(bh) * n_pad;
+            int t = 0, nq = 0, ndo = 0;  // tiles issued: Q (with its row vectors), dO
+            bool ok = true;
+            for (; t < n_it && ok; ++t) {
+                const int s = t & 1;
+                const int i = i_first + t;
+                if (!(ok = mbar_wait(&q_empty[s], ((t >> 1) & 1) ^ 1, p.ctl))) break;
+                mbar_arrive_expect_tx(&q_full[s], TILE + 2 * BQ * 4);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_3d(sQ + s * TILE + c * BOX, &p.tm_q, &q_full[s], c * 64, i * BQ, bh);
+                bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &q_full[s]);
+                bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &q_full[s]);
+                ++nq;
+                if (!(ok = mbar_wait(do_empty, (t & 1) ^ 1, p.ctl))) break;
+                mbar_arrive_expect_tx(do_full, TILE);
+                for (int c = 0; c < 2; ++c) tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, bh);
+                ++ndo;
+            }
+            if (!ok) {
+                mbar_wait_drain(kv_full, 0, p.ctl.limit_ns);
+                for (int u = max(0, nq - QSTAGES); u < nq; ++u)
+                    mbar_wait_drain(&q_full[u & 1], (u >> 1) & 1, p.ctl.limit_ns);
+                if (ndo > 0) mbar_wait_drain(do_full, (ndo - 1) & 1, p.ctl.limit_ns);
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_kk = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+            constexpr uint32_t idesc_tm = idesc_bf16(128, 128, false, true);   // dV (A in TMEM), dK
+            constexpr uint32_t idesc_mm = idesc_bf16(128, 128, true, true);    // dQ^T
+            const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
+                           aDS = smem_u32(sDS);
+            auto q_base = [&](int t) { return aQ + (t & 1) * TILE; };
+            // (K or V) x (Q or dO)^T, both K-major
+            auto issue_kk = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
+                    mma_ss(tmem + d_col, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
+                           idesc_kk, kk > 0 ? 1u : 0u);
+                }
+            };
+            // dV += P^T (TMEM) x dO (MN-major)
+            auto issue_dv = [&](uint32_t a_col, uint32_t b_base, bool acc0) {
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    mma_ts(tmem + DV_COL, tmem + a_col + kk * 8, sdesc_sw128(b_base + kk * 2048, BOX, 1024), idesc_tm,
+                           (acc0 || kk > 0) ? 1u : 0u);
+            };
+            // dK += dS^T (shared, K-major) x Q (MN-major)
+            auto issue_dk = [&](uint32_t b_base, bool acc0) {
+#pragma unroll
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    mma_ss(tmem + DK_COL, sdesc_sw128(aDS + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024),
+                           sdesc_sw128(b_base + kk * 2048, BOX, 1024), idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
+            };
+            // dQ^T = K^T x dS^T, both MN-major
+            auto issue_dq = [&](uint32_t d_col) {
+#pragma unroll
+                for (int kk = 0; kk < BKV / 16; ++kk)
+                    mma_ss(tmem + d_col, sdesc_sw128(aK + kk * 2048, BOX, 1024),
+                           sdesc_sw128(aDS + kk * 2048, BOX, 1024), idesc_mm, kk > 0 ? 1u : 0u);
+            };
+
+            bool ok = mbar_wait(kv_full, 0, p.ctl) && mbar_wait(&q_full[0], 0, p.ctl);
+            if (ok) {
+                tc_fence_after();
+                issue_kk(rcol(0), aK, q_base(0));
+                mma_commit(s_full);
+                ok = mbar_wait(do_full, 0, p.ctl);
+                if (ok) {
+                    tc_fence_after();
+                    issue_kk(rcol(1), aV, aDO);
+                    mma_commit(dp_full);
+                }
+            }
+            for (int t = 0; t < n_it && ok; ++t) {
+                const uint32_t X = rcol(t), Y = rcol(t + 1);
+                if (!(ok = mbar_wait(p_ready, t & 1, p.ctl))) break;
+                tc_fence_after();
+                issue_dv(X, aDO, t > 0);
+                mma_commit(do_empty);
+                if (!(ok = mbar_wait(ds_ready, t & 1, p.ctl))) break;
+                tc_fence_after();
+                if (t + 1 < n_it) {
+                    // Y held dP^T of tile t, already read by the softmax
+                    if (!(ok = mbar_wait(&q_full[(t + 1) & 1], ((t + 1) >> 1) & 1, p.ctl))) break;
+                    tc_fence_after();
+                    issue_kk(Y, aK, q_base(t + 1));
+                    mma_commit(s_full);
+                }
+                issue_dk(q_base(t), t > 0);
+                mma_commit(&q_empty[t & 1]);
+                issue_dq(X);
+                mma_commit(dq_full);
+                if (t + 1 < n_it) {
+                    if (!(ok = mbar_wait(do_full, (t + 1) & 1, p.ctl))) break;
+                    if (!(ok = mbar_wait(dq_empty, t & 1, p.ctl))) break;
+                    tc_fence_after();
+                    issue_kk(X, aV, aDO);
+                    mma_commit(dp_full);
+                }
+            }
+            if (ok) mma_commit(dkdv_done);
+            mma_commit(drain);
+            mbar_wait_drain(drain, 0, p.ctl.limit_ns);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ softmax (key rows)
+        const int r = warp * 32 + lane;
+        const int key = j * BKV + r;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const float cl2 = p.scale_log2;
+        bool ok = true;
+        for (int t = 0; t < n_it && ok; ++t) {
+            const int s = t & 1;
+            const float* lse2 = sVec + s * 2 * BQ;
+            const float* delta = lse2 + BQ;
+            const uint32_t xa = tmem + lane_off + rcol(t);
+            const uint32_t ya = tmem + lane_off + rcol(t + 1);
+            if (!(ok = warp_wait(s_full, t & 1, p.ctl))) break;
+            if (!(ok = warp_wait(&q_full[s], (t >> 1) & 1, p.ctl))) break;
+            tc_fence_after();
+            // causal: query (t-th tile, column c) sees this key iff key <= query; only
+            // the first (diagonal) tile has such pairs.  Keys past N carry no weight.
+            const bool masked = (CAUSAL && t == 0) || (j * BKV + BKV > N);  // CTA-uniform
+            const int lim = (key >= N) ? BQ : ((CAUSAL && t == 0) ? r : 0);   // zero columns c < lim
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float pv[64];
+                tmem_ld32(xa + h * 64, reinterpret_cast<uint32_t*>(pv));
+                tmem_ld32(xa + h * 64 + 32, reinterpret_cast<uint32_t*>(pv + 32));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4*>(lse2 + h * 64 + c);
+                    pv[c] = ex2_approx(fmaf(pv[c], cl2, -l4.x));
+                    pv[c + 1] = ex2_approx(fmaf(pv[c + 1], cl2, -l4.y));
+                    pv[c + 2] = ex2_approx(fmaf(pv[c + 2], cl2, -l4.z));
+                    pv[c + 3] = ex2_approx(fmaf(pv[c + 3], cl2, -l4.w));
+                }
+                if (masked) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (h * 64 + c < lim) pv[c] = 0.f;
+                }
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) pk[c / 2] = pack_bf16x2(pv[c], pv[c + 1]);
+                tmem_st32(xa + h * 32, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_ready);
+
+            // dP^T of this tile was issued after the dK and dQ^T MMAs of the previous
+            // one, so once it is complete they have read the old dS^T
+            if (!(ok = warp_wait(dp_full, t & 1, p.ctl))) break;
+            tc_fence_after();
+            // dS^T = P^T (dP^T - D), with the bf16 P^T read back from TMEM (it stays in
+            // X until dQ^T is written there, after this tile's dS^T), to shared
+            // memory: row r, query columns in 2 chunks of 64 (128-byte swizzled rows)
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float dp[32];
+                uint32_t pq[16];
+                tmem_ld32(ya + q4 * 32, reinterpret_cast<uint32_t*>(dp));
+                tmem_ld16(xa + q4 * 16, pq);
+                tmem_wait_ld();
+                uint32_t ds[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(delta + q4 * 32 + c);
+                    const float2 pa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pq[c / 2]));
+                    const float2 pb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pq[c / 2 + 1]));
+                    ds[c / 2] = pack_bf16x2(pa.x * (dp[c] - d4.x), pa.y * (dp[c + 1] - d4.y));
+                    ds[c / 2 + 1] = pack_bf16x2(pb.x * (dp[c + 2] - d4.z), pb.y * (dp[c + 3] - d4.w));
+                }
+                uint8_t* chunk = sDS + (q4 >> 1) * BOX;
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc)
+                    *reinterpret_cast<uint4*>(chunk + sw128_offset(r, (q4 & 1) * 4 + pc)) =
+                        make_uint4(ds[4 * pc], ds[4 * pc + 1], ds[4 * pc + 2], ds[4 * pc + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(ds_ready);
+        }
+        // epilogue: dV rows
+        if (ok && warp_wait(dkdv_done, 0, p.ctl)) {
+            tc_fence_after();
+            float* dst = p.dv + (static_cast<size_t>(bh) * N + key) * D;
+#pragma unroll
+            for (int cc = 0; cc < D; cc += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + DV_COL + cc, v);
+                tmem_wait_ld();
+                if (key < N) {
+                    float4* d4 = reinterpret_cast<float4*>(dst + cc);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                            __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ dQ (warps 4-7)
+        const int wq = warp - 4;
+        const int dr = wq * 32 + lane;  // head-dim index = TMEM lane of dQ^T
+        const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+        const bool issuer = (threadIdx.x == 4 * 32);
+        // element (query c, dim dr) of a [64][128] fp32 staging tile: 32-column chunk
+        // dr / 32, row c, 16-byte piece (dr % 32) / 4 swizzled with c % 8
+        uint8_t* stg = sSTG + (dr >> 5) * STG_CHUNK;
+        const uint32_t piece = (dr & 31) >> 2, word = (dr & 3) * 4;
+        bool ok = true;
+        for (int t = 0; t < n_it && ok; ++t) {
+            const int i = i_first + t;
+            if (!(ok = warp_wait(dq_full, t & 1, p.ctl))) break;
+            tc_fence_after();
+            float q[BQ];
+            const uint32_t xa = tmem + lane_off + rcol(t);
+#pragma unroll
+            for (int c = 0; c < BQ; c += 32) tmem_ld32(xa + c, reinterpret_cast<uint32_t*>(q + c));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(dq_empty);
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                // the previous reduce-add must have read the staging tile
+                if (issuer) bulk_wait_group_read0();
+                named_bar_sync(1, 128);
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    *reinterpret_cast<float*>(stg + c * 128 + ((piece ^ (c & 7)) << 4) + word) =
+                        q[half * 64 + c] * p.scale;
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (issuer) {
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch)
+                        tma_reduce_add_3d(&p.tm_dq, sSTG + ch * STG_CHUNK, ch * 32, i * BQ + half * 64, bh);
+                    bulk_commit_group();
+                }
+            }
+        }
+        if (issuer) bulk_wait_group0();
+        // epilogue: dK rows (lanes = key rows)
+        if (ok && warp_wait(dkdv_done, 0, p.ctl)) {
+            tc_fence_after();
+            const int key = j * BKV + wq * 32 + lane;
+            float* dst = p.dk + (static_cast<size_t>(bh) * N + key) * D;
+#pragma unroll
+            for (int cc = 0; cc < D; cc += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_off + DK_COL + cc, v);
+                tmem_wait_ld();
+                if (key < N) {
+                    float4* d4 = reinterpret_cast<float4*>(dst + cc);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        d4[e] = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
+                                            __uint_as_float(v[4 * e + 2]) * p.scale,
+                                            __uint_as_float(v[4 * e + 3]) * p.scale);
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <bool CAUSAL>
+cudaError_t launch(const BwdParams& p, cudaStream_t stream)
+{
+    auto kern = bwd128_kernel<CAUSAL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.n_kv_tiles, p.BH);
+    kern<<<grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace bwd128k
+
+cudaError_t launch_bwd128_sm100(const BwdParams& p, bool causal, cudaStream_t stream)
+{
+    return causal ? bwd128k::launch<true>(p, stream) : bwd128k::launch<false>(p, stream);
+}
+
+}  // namespace fa

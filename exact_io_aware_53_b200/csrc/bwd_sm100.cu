@@ -1,4 +1,5 @@
-// Backward attention, bf16 in / fp32 gradients, sm_100a.
+// Backward attention for head dimension 64, bf16 in / fp32 gradients, sm_100a
+// (head dimension 128 has its own kernel, bwd128_sm100.cu).
 //
 // The attention weights are never stored: each CTA owns one tile of 128 keys
 // (K_j, V_j resident in shared memory) and walks the 64-row query tiles that
@@ -107,8 +108,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
     }
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
-    const int bh = blockIdx.x;
-    const int j = blockIdx.y;  // key tile (heaviest first under the causal mask)
+    // head-major launch order: CTAs resident together share a few heads' Q, dO
+    // and dQ accumulator in L2; key tile 0 (the most query tiles) starts first
+    const int bh = blockIdx.y;
+    const int j = blockIdx.x;
     const int N = p.N;
     const int n_pad = p.n_kv_tiles * BKV;
     const int n_q_all = (N + BQ - 1) / BQ;
@@ -289,7 +292,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             tmem_ld32(sb + 32, reinterpret_cast<uint32_t*>(pv + 32));
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < BQ; ++c) pv[c] = ex2_approx(fmaf(pv[c], cl2, -lse2[c]));
+            for (int c = 0; c < BQ; c += 4) {
+                const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);
+                pv[c] = ex2_approx(fmaf(pv[c], cl2, -l4.x));
+                pv[c + 1] = ex2_approx(fmaf(pv[c + 1], cl2, -l4.y));
+                pv[c + 2] = ex2_approx(fmaf(pv[c + 2], cl2, -l4.z));
+                pv[c + 3] = ex2_approx(fmaf(pv[c + 3], cl2, -l4.w));
+            }
             // causal: query (i*BQ + c) sees this key iff key <= query; keys past N carry no weight
             if (key >= N) {
 #pragma unroll
@@ -316,8 +325,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             tmem_ld32(dpa + 32, reinterpret_cast<uint32_t*>(dp + 32));
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < BQ; c += 2)
-                pk[c / 2] = pack_bf16x2(pv[c] * (dp[c] - delta[c]), pv[c + 1] * (dp[c + 1] - delta[c + 1]));
+            for (int c = 0; c < BQ; c += 4) {
+                const float4 d4 = *reinterpret_cast<const float4*>(delta + c);
+                pk[c / 2] = pack_bf16x2(pv[c] * (dp[c] - d4.x), pv[c + 1] * (dp[c + 1] - d4.y));
+                pk[c / 2 + 1] = pack_bf16x2(pv[c + 2] * (dp[c + 2] - d4.z), pv[c + 3] * (dp[c + 3] - d4.w));
+            }
             tmem_st32(dpa, pk);
             // dS^T row r into the swizzled shared buffer read by the dQ^T MMA
             if (t >= 2 && !(ok = warp_wait(&ds_free[t & 1], ((t >> 1) + 1) & 1, p.ctl))) break;
@@ -426,7 +438,7 @@ cudaError_t launch(const BwdParams& p, cudaStream_t stream)
     auto kern = bwd_kernel<D, CAUSAL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.BH, p.n_kv_tiles);
+    dim3 grid(p.n_kv_tiles, p.BH);
     kern<<<grid, NTHREADS, C::SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
 }
@@ -435,7 +447,7 @@ cudaError_t launch(const BwdParams& p, cudaStream_t stream)
 
 cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, cudaStream_t stream)
 {
-    if (d == 128) return causal ? bwdk::launch<128, true>(p, stream) : bwdk::launch<128, false>(p, stream);
+    if (d == 128) return launch_bwd128_sm100(p, causal, stream);
     return causal ? bwdk::launch<64, true>(p, stream) : bwdk::launch<64, false>(p, stream);
 }
 

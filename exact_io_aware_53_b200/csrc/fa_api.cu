@@ -9,8 +9,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/fa.h"
-#include "../../include/fa_selftest.h"
+#include "fa.h"
+#include "fa_selftest.h"
 #include "kernels.h"
 
 namespace fa {
@@ -152,6 +152,80 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d)
     return 2 * ((rows * sizeof(float) + 255) & ~size_t(255));
 }
 
+int fa_bwd_prep(const void* o, const float* lse, const void* dO, float* dq, void* workspace, int B, int H, int N,
+                int d, void* stream)
+{
+    g_last_launches = 0;
+    if (!o || !lse || !dO || !dq || !workspace) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, 1.f, 0);
+    if (st != FA_OK) return st;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(workspace))
+        return FA_ERR_MISALIGNED;
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    const int n_pad = (N + 127) / 128 * 128;
+    const size_t vec_bytes = (static_cast<size_t>(BH) * n_pad * sizeof(float) + 255) & ~size_t(255);
+    BwdPreParams pp;
+    pp.o = static_cast<const __nv_bfloat16*>(o);
+    pp.dO = static_cast<const __nv_bfloat16*>(dO);
+    pp.lse = lse;
+    pp.delta = static_cast<float*>(workspace);
+    pp.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + vec_bytes);
+    pp.dq = dq;
+    pp.BH = static_cast<int>(BH);
+    pp.N = N;
+    pp.n_pad = n_pad;
+    pp.d = d;
+    st = cuda_status(launch_bwd_pre(pp, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
+int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, float* dq, float* dk, float* dv,
+                const void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv) || !aligned16(workspace))
+        return FA_ERR_MISALIGNED;
+    if ((st = get_encoder()) != FA_OK) return st;
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    const int n_pad = (N + 127) / 128 * 128;
+    const size_t vec_bytes = (static_cast<size_t>(BH) * n_pad * sizeof(float) + 255) & ~size_t(255);
+    BwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint32_t bq = d == 128 ? 128 : 64;  // query rows per backward step
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, bq,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dO, d, N, BH, 64, bq,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq, d, N, BH, 32, 64,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    p.delta = static_cast<const float*>(workspace);
+    p.lse2 = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + vec_bytes);
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.BH = static_cast<int>(BH);
+    p.N = N;
+    p.n_kv_tiles = (N + 127) / 128;
+    p.scale = scale;
+    p.scale_log2 = scale * kLog2e;
+    st = cuda_status(launch_bwd_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, float* dq,
            float* dk, float* dv, void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream)
 {
@@ -164,52 +238,11 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
         return FA_ERR_MISALIGNED;
     if ((st = get_encoder()) != FA_OK) return st;
-    const uint64_t BH = static_cast<uint64_t>(B) * H;
-    const int n_pad = (N + 127) / 128 * 128;
-    const size_t vec_bytes = (static_cast<size_t>(BH) * n_pad * sizeof(float) + 255) & ~size_t(255);
-    float* delta = static_cast<float*>(workspace);
-    float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + vec_bytes);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-    BwdPreParams pp;
-    pp.o = static_cast<const __nv_bfloat16*>(o);
-    pp.dO = static_cast<const __nv_bfloat16*>(dO);
-    pp.lse = lse;
-    pp.delta = delta;
-    pp.lse2 = lse2;
-    pp.dq = dq;
-    pp.BH = static_cast<int>(BH);
-    pp.N = N;
-    pp.n_pad = n_pad;
-    pp.d = d;
-
-    BwdParams p;
-    std::memset(&p, 0, sizeof(p));
-    const uint32_t bq = 64;
-    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, bq,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dO, d, N, BH, 64, bq,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq, d, N, BH, 32, bq,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+    if ((st = fa_bwd_prep(o, lse, dO, dq, workspace, B, H, N, d, stream)) != FA_OK) return st;
+    if ((st = fa_bwd_main(q, k, v, dO, dq, dk, dv, workspace, B, H, N, d, scale, causal, stream)) != FA_OK) {
+        g_last_launches = 1;
         return st;
-    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
-    p.lse2 = lse2;
-    p.delta = delta;
-    p.dk = dk;
-    p.dv = dv;
-    p.BH = static_cast<int>(BH);
-    p.N = N;
-    p.n_kv_tiles = (N + 127) / 128;
-    p.scale = scale;
-    p.scale_log2 = scale * kLog2e;
-    if ((st = cuda_status(launch_bwd_pre(pp, s))) != FA_OK) return st;
-    g_last_launches = 1;
-    if ((st = cuda_status(launch_bwd_sm100(p, d, causal != 0, s))) != FA_OK) return st;
+    }
     g_last_launches = 2;
     return FA_OK;
 }
@@ -390,6 +423,25 @@ int fa_selftest_umma(const void* a, const void* b, float* d, int M, int N, int K
     p.a_tmem = a_tmem;
     p.b_manual = b_manual;
     st = cuda_status(launch_umma_selftest(p, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
+int fa_selftest_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem, int reps, int n_acc, int ctas,
+                          long long* cycles, void* stream)
+{
+    g_last_launches = 0;
+    if (!cycles || reps == 0 || ctas < 1 || n_acc < 1) return FA_ERR_INVALID_ARG;
+    const bool shape_ok = M == 128 && ((K == 128 && !a_mn && !b_mn && !a_tmem && (N == 64 || N == 128 || N == 256)) ||
+                                       (K == 128 && !a_mn && b_mn && a_tmem && (N == 128 || N == 256)) ||
+                                       (K == 64 && !a_mn && b_mn && a_tmem && N == 128) ||
+                                       (K == 128 && a_mn && b_mn && !a_tmem && N == 64));
+    if (!shape_ok || n_acc * N > (a_tmem ? 384 : 512)) return FA_ERR_UNSUPPORTED;
+    WaitCtl ctl;
+    int st = get_ctl(&ctl);
+    if (st != FA_OK) return st;
+    st = cuda_status(launch_umma_rate(M, N, K, a_mn, b_mn, a_tmem, reps, n_acc, ctas, cycles, ctl,
+                                      static_cast<cudaStream_t>(stream)));
     if (st == FA_OK) g_last_launches = 1;
     return st;
 }

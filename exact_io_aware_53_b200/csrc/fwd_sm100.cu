@@ -86,8 +86,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
 
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
-    const int bh = blockIdx.x;
-    const int pair = CAUSAL ? (p.n_pairs - 1 - static_cast<int>(blockIdx.y)) : static_cast<int>(blockIdx.y);
+    // head-major launch order: CTAs resident together share a few heads' K/V in L2;
+    // under the causal mask each head's longest rows start first
+    const int bh = blockIdx.y;
+    const int pair = CAUSAL ? (p.n_pairs - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
     const int q0 = pair * 2 * BM;
     const int N = p.N;
     const int n_kv_all = (N + BN - 1) / BN;
@@ -263,10 +265,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                 for (int c = 0; c < BN; ++c)
                     if (c > limit) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row max as 8 independent chains, then a tree
+            float m8[8];
 #pragma unroll
-            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-            const float m_blk = mx * cl2;
+            for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+            for (int c = 8; c < BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+#pragma unroll
+            for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                for (int e = 0; e < w; ++e) m8[e] = fmaxf(m8[e], m8[e + w]);
+            const float m_blk = m8[0] * cl2;
             float alpha = 1.f;
             if (j == 0) {
                 m = m_blk;
@@ -275,7 +284,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                 m = m_blk;
             }
             const float neg_m = -m;
-            float sum = 0.f;
+            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[BN / 4];
@@ -283,12 +292,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                 for (int c = 0; c < BN / 2; c += 2) {
                     const float p0 = ex2_approx(fmaf(s[h * (BN / 2) + c], cl2, neg_m));
                     const float p1 = ex2_approx(fmaf(s[h * (BN / 2) + c + 1], cl2, neg_m));
-                    sum += p0 + p1;
+                    sum4[(c >> 1) & 3] += p0 + p1;
                     pk[c / 2] = pack_bf16x2(p0, p1);
                 }
                 tmem_st32(s_addr + h * (BN / 4), pk);
             }
-            l = l * alpha + sum;
+            l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 // O_t already holds sum_{j'<j} P V_j' (its MMA precedes this S in
                 // issue order, so S_t's commit covered it); rescale in TMEM.  Done
@@ -349,7 +358,7 @@ cudaError_t launch(const FwdParams& p, cudaStream_t stream)
     auto kern = fwd_kernel<D, CAUSAL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.BH, p.n_pairs);
+    dim3 grid(p.n_pairs, p.BH);
     kern<<<grid, NTHREADS, C::SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
 }

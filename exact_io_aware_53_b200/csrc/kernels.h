@@ -42,13 +42,14 @@ struct BwdPreParams {
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
 
 struct BwdParams {
-    CUtensorMap tm_q;    // {d, N, B*H}, box {64, 64, 1}
-    CUtensorMap tm_do;   // {d, N, B*H}, box {64, 64, 1}
+    CUtensorMap tm_q;    // {d, N, B*H}, box {64, BQ, 1} (BQ = 64 for d = 64, 128 for d = 128)
+    CUtensorMap tm_do;   // {d, N, B*H}, box {64, BQ, 1}
     CUtensorMap tm_k;    // {d, N, B*H}, box {64, 128, 1}
     CUtensorMap tm_v;    // {d, N, B*H}, box {64, 128, 1}
-    CUtensorMap tm_dq;   // fp32 {d, N, B*H}, box {32, 64, 1}, reduce-add target
+    CUtensorMap tm_dq;   // fp32 {d, N, B*H}, box {32, 64, 1}, 128-byte swizzle, reduce-add target
     const float* lse2;   // [B*H][n_kv_tiles * 128]; +inf past N
     const float* delta;  // [B*H][n_kv_tiles * 128]; 0 past N
+    float* dq;           // [B*H][N][d], accumulated into (zeroed by the pre-pass)
     float* dk;           // [B*H][N][d]
     float* dv;           // [B*H][N][d]
     int BH;
@@ -59,6 +60,7 @@ struct BwdParams {
     WaitCtl ctl;
 };
 cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, cudaStream_t stream);
+cudaError_t launch_bwd128_sm100(const BwdParams& p, bool causal, cudaStream_t stream);
 
 // ---------------------------------------------------------------- fp32 path
 struct F32Params {
@@ -96,5 +98,7 @@ struct UmmaTestParams {
     WaitCtl ctl;
 };
 cudaError_t launch_umma_selftest(const UmmaTestParams& p, cudaStream_t stream);
+cudaError_t launch_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem, int reps, int n_acc, int ctas,
+                             long long* cycles, WaitCtl ctl, cudaStream_t stream);
 
 }  // namespace fa

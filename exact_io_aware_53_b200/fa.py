@@ -31,6 +31,8 @@ _SIGS = {
     "fa_fwd": ([P, P, P, P, P, I, I, I, I, F, I, P], I),
     "fa_bwd_workspace_bytes": ([I, I, I, I], SZ),
     "fa_bwd": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
+    "fa_bwd_prep": ([P, P, P, P, P, I, I, I, I, P], I),
+    "fa_bwd_main": ([P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
     "fa_fwd_f32": ([P, P, P, P, P, I, I, I, I, F, I, I, P], I),
     "fa_bwd_f32": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
     "fa_attention_host_arena_bytes": ([I, I, I, I], SZ),
@@ -40,6 +42,7 @@ _SIGS = {
     "fa_status_string": ([I], ctypes.c_char_p),
     "fa_last_launch_count": ([], I),
     "fa_selftest_umma": ([P, P, P, I, I, I, I, I, I, I, P], I),
+    "fa_selftest_umma_rate": ([I, I, I, I, I, I, I, I, I, P, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -137,6 +140,17 @@ def bwd_raw(q, k, v, o, lse, do, dq, dk, dv, ws, scale: float, causal: bool, str
                        _ptr(ws), B, H, N, d, float(scale), int(causal), _stream(stream))
 
 
+def bwd_prep_raw(o, lse, do, dq, ws, stream=None) -> int:
+    B, H, N, d = _shape(o)
+    return _lib.fa_bwd_prep(_ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(ws), B, H, N, d, _stream(stream))
+
+
+def bwd_main_raw(q, k, v, do, dq, dk, dv, ws, scale: float, causal: bool, stream=None) -> int:
+    B, H, N, d = _shape(q)
+    return _lib.fa_bwd_main(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                            B, H, N, d, float(scale), int(causal), _stream(stream))
+
+
 def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, workspace=None, stream=None):
     """dQ, dK, dV (fp32) of L = sum(O * dO), recomputing the weights from lse."""
     _same(q, k, v, o, do, dtype=torch.bfloat16)
@@ -202,3 +216,15 @@ def selftest_umma(a, b, M, N, K, a_mn, b_mn, a_tmem=False, b_manual=False, strea
     _check(_lib.fa_selftest_umma(_ptr(a), _ptr(b), _ptr(d), M, N, K, int(a_mn), int(b_mn), int(a_tmem),
                                  int(b_manual), _stream(stream)), "fa_selftest_umma")
     return d
+
+
+def selftest_umma_rate(N, K, a_mn=0, b_mn=0, a_tmem=0, reps=256, n_acc=1, ctas=1, M=128, converged=True,
+                       stream=None):
+    """(cycles per MMA instruction to completion, cycles per instruction to issue), per CTA."""
+    cyc = torch.zeros(2 * ctas, dtype=torch.int64, device="cuda")
+    r = -int(reps) if converged else int(reps)
+    _check(_lib.fa_selftest_umma_rate(M, N, K, int(a_mn), int(b_mn), int(a_tmem), r, int(n_acc), int(ctas),
+                                      _ptr(cyc), _stream(stream)), "fa_selftest_umma_rate")
+    torch.cuda.synchronize()
+    c = (cyc.double() / (reps * K / 16)).cpu().view(ctas, 2)
+    return c[:, 0], c[:, 1]

@@ -17,7 +17,7 @@
  *
  * Conventions shared by every entry point
  *   - Tensors are dense, row-major [B][H][N][d] ("BHND", torch (B,H,N,d)
- *     contiguous); lse and the workspace vectors are [B][H][N].
+ *     contiguous); lse is [B][H][N].
  *   - All pointers are DEVICE pointers owned by the caller unless the name says
  *     host; the library keeps no pointer after a call returns and allocates no
  *     device memory.
@@ -60,7 +60,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 
 /*
  * Bytes of device workspace fa_bwd needs: the row terms D_i = <dO_i, O_i> and
- * the log-sum-exp in base 2, both fp32 [B][H][N] (O(N), never O(N^2)).
+ * the log-sum-exp in base 2, both fp32 [B][H][N rounded up to 128] (O(N),
+ * never O(N^2)).  Returns 0 for non-positive sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -75,6 +76,19 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
            float* dq, float* dk, float* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
            void* stream);
+
+/*
+ * The two stages of fa_bwd, for callers that time or schedule them apart.
+ * fa_bwd_prep: from o, dO (bf16) and lse, writes the row terms D_i = <dO_i, O_i>
+ * and lse_i * log2(e) into `workspace` and zeroes dq.  fa_bwd_main: the
+ * tensor-core backward proper; it reads that workspace, so it must follow
+ * fa_bwd_prep for the same tensors on the same stream.  Arguments and errors
+ * as fa_bwd.
+ */
+int fa_bwd_prep(const void* o, const float* lse, const void* dO, float* dq, void* workspace, int B, int H, int N,
+                int d, void* stream);
+int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, float* dq, float* dk, float* dv,
+                const void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
  * Forward, fp32 (all tensors fp32).  1 <= d <= 128.  block_k is the key
