@@ -33,6 +33,7 @@ _SIGS = {
     "fa_bwd": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
     "fa_bwd_prep": ([P, P, P, P, P, I, I, I, I, P], I),
     "fa_bwd_main": ([P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
+    "fa_bwd_noalloc": ([P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
     "fa_fwd_f32": ([P, P, P, P, P, I, I, I, I, F, I, I, P], I),
     "fa_bwd_f32": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
     "fa_attention_host_arena_bytes": ([I, I, I, I], SZ),
@@ -163,6 +164,13 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, w
         workspace = torch.empty(bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
     _check(bwd_raw(q, k, v, o, lse, do, dq, dk, dv, workspace, scale, causal, stream), "fa_bwd")
     return dq, dk, dv
+
+
+def bwd_noalloc_raw(q, k, v, o, lse, do, dq, dk, dv, scale: float, causal: bool, stream=None) -> int:
+    """fa_bwd without a workspace argument: the library's built-in scratch area is used."""
+    B, H, N, d = _shape(q)
+    return _lib.fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                               _ptr(dv), B, H, N, d, float(scale), int(causal), _stream(stream))
 
 
 # ------------------------------------------------------------------ fp32 path

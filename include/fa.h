@@ -91,6 +91,34 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, flo
                 const void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
+ * Size of the scratch area built into the library for fa_bwd_noalloc.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * Backward pass that allocates nothing, for callers that cannot call
+ * cudaMalloc: hosts that own all device memory and give a library only its
+ * input and output buffers (plugin and custom-op interfaces), and loops that
+ * must not call cudaMalloc / cudaFree because they can synchronise the device.
+ * The explainer pages have no counterpart to this entry point; it is an
+ * interface convenience only.
+ *
+ * Arguments, results and errors are those of fa_bwd without `workspace`: the
+ * workspace lives in a device array of FA_NOALLOC_SCRATCH_BYTES compiled into
+ * the library (held by every GPU that loads it until the process exits).
+ * Returns FA_ERR_UNSUPPORTED when fa_bwd_workspace_bytes(B,H,N,d) exceeds
+ * FA_NOALLOC_SCRATCH_BYTES (4 MiB: B*H*N up to about 512K rows).
+ * The first call on a device looks the array's device address up (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls on a device share the array and it keeps the last
+ * call's contents (nothing in it needs to start at zero): calls whose work
+ * overlaps on the GPU race on it, so order them on one stream.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   float* dq, float* dk, float* dv, int B, int H, int N, int d, float scale, int causal,
+                   void* stream);
+
+/*
  * Forward, fp32 (all tensors fp32).  1 <= d <= 128.  block_k is the key
  * block size of the online-softmax walk (1 .. 1024; 0 selects 64): the result
  * must not depend on it beyond rounding ("Block size never changes the
