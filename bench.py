@@ -80,6 +80,32 @@ def rank_seed(base_seed: int, rank: int) -> int:
 
 # ------------------------------------------------------------------ peaks / clocks
 
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded in profiles/traffic.txt for this kernel and
+    workload, or None if absent or if the kernel's sources changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    for line in lines:
+        if not line.strip() or line.startswith("#"):
+            continue
+        k, wl, sha, nbytes, files, _ = line.split()[:6]
+        if k != kernel or wl != workload:
+            continue
+        h = hashlib.sha256()
+        try:
+            for f in files.split(","):
+                with open(os.path.join(ROOT, f), "rb") as fh:
+                    h.update(fh.read())
+        except OSError:
+            return None
+        return int(nbytes) if h.hexdigest().startswith(sha) else None
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -309,7 +335,8 @@ def run_ours(args, w, print_line=True):
     roofline = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": UNIT,
                 "frac": achieved / peak, "peak_source": "%s %s" % (peak_key, peak_src),
                 "frac_of_burst": achieved / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
-                "algorithmic_flops_per_launch": dom_flops, "ms_per_launch": dom_ms, "traffic": None}
+                "algorithmic_flops_per_launch": dom_flops, "ms_per_launch": dom_ms,
+                "traffic": measured_traffic(dom_name, w.name), "traffic_unit": "bytes per launch (ncu dram read+write)"}
     fwd_tflops = w.flops_fwd() / (fwd_ms / 1e3) / 1e12
     kernels = {"fwd": {"ms": fwd_ms, "tflops": fwd_tflops, "frac": fwd_tflops / peak}}
     if w.backward:
@@ -379,6 +406,30 @@ def run_e2e(args, w, fa, x, dev, stream, world):
             "steps": steps, "api": "fa_attention_host (pinned host buffers)"}
 
 
+def probe_mma_rate():
+    """Cycles per tcgen05 MMA instruction for the shapes the kernels issue
+    (fa_selftest_umma_rate, one CTA per SM); printed as JSON lines."""
+    from exact_io_aware_53_b200 import fa
+    cases = [  # (N, K, a_mn, b_mn, a_tmem, use)
+        (128, 128, 0, 0, 0, "forward QK^T / backward S^T, dP^T (128x128)"),
+        (64, 128, 0, 0, 0, "backward d=64 S^T, dP^T (128x64)"),
+        (256, 128, 0, 0, 0, "reference: 128x256"),
+        (128, 128, 0, 1, 1, "forward PV / backward dV (A in TMEM)"),
+        (128, 64, 0, 1, 1, "backward d=64 dV, dK (A in TMEM, K=64)"),
+        (64, 128, 1, 1, 0, "backward d=64 dQ^T (both MN-major)"),
+    ]
+    for (N, K, amn, bmn, at, use) in cases:
+        for conv in (False, True):
+            tot, iss = fa.selftest_umma_rate(N, K, amn, bmn, at, reps=2048, n_acc=2 if N <= 128 else 1,
+                                             ctas=148, converged=conv)
+            cyc = float(tot.median())
+            ideal = 2 * 128 * N * 16 / 8192
+            print(json.dumps({"probe": "tcgen05_mma_rate", "shape": "128x%dx16" % N, "K": K, "a_mn": amn,
+                              "b_mn": bmn, "a_tmem": at, "issue": "elected lane of converged warp" if conv
+                              else "one lane of a diverged warp", "clk_per_instr": round(cyc, 1),
+                              "ideal_clk": ideal, "frac_of_ideal": round(ideal / cyc, 3), "use": use}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -388,7 +439,11 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--probe-mma-rate", action="store_true", help="print the tcgen05 issue-rate table and exit")
     args = ap.parse_args(argv)
+    if args.probe_mma_rate:
+        probe_mma_rate()
+        return 0
     from exact_io_aware_53_b200.workloads import WORKLOADS
     if args.workload != "all" and args.workload not in WORKLOADS:
         ap.error("unknown workload %s (choose from %s)" % (args.workload, ", ".join(WORKLOADS)))
