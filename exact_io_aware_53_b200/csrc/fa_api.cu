@@ -427,6 +427,16 @@ int fa_selftest_umma(const void* a, const void* b, float* d, int M, int N, int K
     return st;
 }
 
+int fa_selftest_exp2(const float* x, float* y, int n, int mode, void* stream)
+{
+    g_last_launches = 0;
+    if (!x || !y || n < 1 || (mode != 0 && mode != 1)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return FA_ERR_MISALIGNED;
+    const int st = cuda_status(launch_exp2_selftest(x, y, n, mode, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
 int fa_selftest_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem, int reps, int n_acc, int ctas,
                           long long* cycles, void* stream)
 {

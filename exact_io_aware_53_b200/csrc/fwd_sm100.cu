@@ -5,6 +5,9 @@
 // "Tiling and the online softmax", vibeengines.com/paper/flash-attention):
 //
 //   warp 9      TMA producer: Q tiles once, then K_j, V_j through a smem ring
+//               (stages are handed back by a softmax thread that has seen the
+//               S MMA issued after their last reader complete, so the MMA warp
+//               spends no tcgen05.commit on them)
 //   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T (smem x smem -> TMEM),
 //               O_t += P_t V_j (P from TMEM x V from smem -> TMEM)
 //   warps 0-3   softmax for Q tile 0 (thread = query row = TMEM lane)
@@ -12,6 +15,9 @@
 //
 // The two softmax warpgroups ping-pong: while one turns its S tile into P, the
 // tensor core runs the other tile's P V and next Q K^T.
+//
+// One exponential in four is evaluated by a polynomial on the FMA pipe
+// (ex2_fma) instead of MUFU ex2, which the softmax otherwise saturates.
 //
 // Softmax per key tile, in base 2 with c = scale * log2(e) (the update rule of
 // "The math, worked with real numbers": m_new = max(m_old, m_block), l_new =
@@ -36,6 +42,7 @@ constexpr int NTHREADS = 320;
 constexpr int MMA_WARP = 8;
 constexpr int LOAD_WARP = 9;
 constexpr float RESCALE_LOG2 = 8.0f;
+constexpr int EX2_FMA_EVERY = 4;  // share of a row's exponentials evaluated on the FMA pipe: 1 / this
 constexpr float LN2 = 0.6931471805599453f;
 
 template <int D>
@@ -202,7 +209,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                             issue_s(t, sK);
                             mma_commit(&s_full[t]);
                         }
-                    mma_commit(&kv_empty[sK]);
                 }
             }
             for (int j = 0; j < n_kv_max && ok; ++j) {
@@ -228,8 +234,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                     }
                 }
                 if (!ok) break;
-                mma_commit(&kv_empty[sV]);
-                if (sKn >= 0) mma_commit(&kv_empty[sKn]);
             }
             // every MMA issued above completes before TMEM is released
             mma_commit(drain);
@@ -245,12 +249,21 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
         const uint32_t s_addr = tmem + lane_off + 128u * t;
         const uint32_t o_addr = tmem + lane_off + C::O_COL + D * t;
         const float cl2 = p.scale_log2;
+        // the Q tile with the most key tiles releases the K/V ring stages (it
+        // issues the last S of every key tile); tile 1 unless it lies past N
+        const int releaser = n_kv[1] > 0 ? 1 : 0;
         float m = -INFINITY;
         float l = 0.f;
         bool ok = true;
         const int nk = n_kv[t];
         for (int j = 0; j < nk; ++j) {
             if (!(ok = warp_wait(&s_full[t], j & 1, p.ctl))) break;
+            if (t == releaser && r == 0) {
+                // S_t(j) is complete, so is every MMA issued before it: K_j and
+                // V_{j-1} are consumed; hand their ring stages back to the producer
+                mbar_arrive(&kv_empty[(2 * j) % C::STAGES]);
+                if (j > 0) mbar_arrive(&kv_empty[(2 * j - 1) % C::STAGES]);
+            }
             tc_fence_after();
             float s[BN];
             tmem_ld32(s_addr + 0, reinterpret_cast<uint32_t*>(s + 0));
@@ -265,17 +278,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                 for (int c = 0; c < BN; ++c)
                     if (c > limit) s[c] = -INFINITY;
             }
-            // row max as 8 independent chains, then a tree
+            // row max: 8 independent chains of three-input max, then a tree
             float m8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) m8[e] = s[e];
+            for (int e = 0; e < 8; ++e) m8[e] = fmaxf(s[e], s[e + 8]);
 #pragma unroll
-            for (int c = 8; c < BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], s[c]);
+            for (int c = 16; c < BN; c += 16)
 #pragma unroll
-            for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                for (int e = 0; e < w; ++e) m8[e] = fmaxf(m8[e], m8[e + w]);
-            const float m_blk = m8[0] * cl2;
+                for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
+            const float m_blk = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7])) * cl2;
             float alpha = 1.f;
             if (j == 0) {
                 m = m_blk;
@@ -283,21 +294,25 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                 alpha = ex2_approx(m - m_blk);
                 m = m_blk;
             }
-            const float neg_m = -m;
-            float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+            const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-m, -m);
+            float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[BN / 4];
 #pragma unroll
                 for (int c = 0; c < BN / 2; c += 2) {
-                    const float p0 = ex2_approx(fmaf(s[h * (BN / 2) + c], cl2, neg_m));
-                    const float p1 = ex2_approx(fmaf(s[h * (BN / 2) + c + 1], cl2, neg_m));
-                    sum4[(c >> 1) & 3] += p0 + p1;
+                    // x = c s - m for two scores per instruction; one exponential in
+                    // EX2_FMA_EVERY runs on the FMA pipe, beside MUFU
+                    const float2 x = ffma2(make_float2(s[h * (BN / 2) + c], s[h * (BN / 2) + c + 1]), c2, nm2);
+                    const float p0 = ex2_approx(x.x);
+                    const float p1 = (EX2_FMA_EVERY > 0 && (c + 2) % EX2_FMA_EVERY == 0) ? ex2_fma(x.y) : ex2_approx(x.y);
+                    sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], make_float2(p0, p1));
                     pk[c / 2] = pack_bf16x2(p0, p1);
                 }
                 tmem_st32(s_addr + h * (BN / 4), pk);
             }
-            l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+            const float2 sum_pair = fadd2(sum2[0], sum2[1]);
+            l = l * alpha + (sum_pair.x + sum_pair.y);
             if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 // O_t already holds sum_{j'<j} P V_j' (its MMA precedes this S in
                 // issue order, so S_t's commit covered it); rescale in TMEM.  Done

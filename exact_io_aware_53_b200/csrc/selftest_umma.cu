@@ -270,3 +270,23 @@ cudaError_t launch_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem
 }
 
 }  // namespace fa
+
+namespace fa {
+namespace exp2_test {
+
+// y[i] = 2^x[i] by the FMA-pipe polynomial (mode 0) or ex2.approx (mode 1).
+__global__ void exp2_kernel(const float* x, float* y, int n, int mode)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < n) y[i] = mode == 0 ? ex2_fma(x[i]) : ex2_approx(x[i]);
+}
+
+}  // namespace exp2_test
+
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, int mode, cudaStream_t stream)
+{
+    exp2_test::exp2_kernel<<<(n + 255) / 256, 256, 0, stream>>>(x, y, n, mode);
+    return cudaGetLastError();
+}
+
+}  // namespace fa

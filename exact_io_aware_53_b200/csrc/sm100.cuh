@@ -8,6 +8,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "exp2_poly.h"
 #include "fa_status.h"
 
 namespace fa {
@@ -376,6 +377,64 @@ __device__ __forceinline__ float ex2_approx(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x evaluated on the FMA and integer pipes instead of MUFU, so part of a
+// softmax's exponentials can run beside ex2.approx: n = round(x) by the
+// 1.5 * 2^23 shift, f = x - n in [-1/2, 1/2], p(f) ~ 2^f (minimax, relative
+// error exp2poly::MAX_REL_ERR), then n is added to p's exponent field.
+// x is clamped below at -125 so the exponent stays normal (2^-125 stands for 0);
+// callers keep x <= 64.
+__device__ __forceinline__ float ex2_fma(float x)
+{
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;  // 1.5 * 2^23: rounds x to an integer in the low bits
+    const float n = t - 12582912.0f;
+    const float f = x - n;
+    const float p = fmaf(fmaf(fmaf(exp2poly::C3, f, exp2poly::C2), f, exp2poly::C1), f, exp2poly::C0);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Paired fp32 arithmetic (sm_100 f32x2): one instruction for two lanes of work.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// max of three (sm_100 three-input max.f32)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)

@@ -43,6 +43,7 @@ _SIGS = {
     "fa_status_string": ([I], ctypes.c_char_p),
     "fa_last_launch_count": ([], I),
     "fa_selftest_umma": ([P, P, P, I, I, I, I, I, I, I, P], I),
+    "fa_selftest_exp2": ([P, P, I, I, P], I),
     "fa_selftest_umma_rate": ([I, I, I, I, I, I, I, I, I, P, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -236,3 +237,10 @@ def selftest_umma_rate(N, K, a_mn=0, b_mn=0, a_tmem=0, reps=256, n_acc=1, ctas=1
     torch.cuda.synchronize()
     c = (cyc.double() / (reps * K / 16)).cpu().view(ctas, 2)
     return c[:, 0], c[:, 1]
+
+
+def selftest_exp2(x, mode: int, stream=None):
+    """2^x on the GPU by the FMA-pipe polynomial (mode 0) or ex2.approx (mode 1)."""
+    y = torch.empty_like(x)
+    _check(_lib.fa_selftest_exp2(_ptr(x), _ptr(y), x.numel(), int(mode), _stream(stream)), "fa_selftest_exp2")
+    return y

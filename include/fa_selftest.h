@@ -30,6 +30,14 @@ int fa_selftest_umma(const void* a, const void* b, float* d, int M, int N, int K
                      int b_manual, void* stream);
 
 /*
+ * y[i] = 2^x[i] for n device floats, by the kernels' FMA-pipe polynomial
+ * (mode 0: round-to-nearest range reduction, degree-3 minimax polynomial for
+ * 2^f on [-1/2, 1/2], exponent insertion; inputs below -125 give 2^-125) or
+ * by ex2.approx (mode 1).  Pointers 16-byte aligned.
+ */
+int fa_selftest_exp2(const float* x, float* y, int n, int mode, void* stream);
+
+/*
  * Tensor-core issue-rate probe: `ctas` CTAs (one per SM when ctas <= SM count)
  * each stage dummy operands once and issue `reps` back-to-back copies of the
  * K/16-instruction 128 x N x K MMA sequence (same operand kinds as

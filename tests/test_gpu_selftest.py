@@ -39,3 +39,26 @@ def test_umma_tmem_a_operand(fa_lib, N, K, b_mn):
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 1), (1, 1), (0, 0)])
 def test_umma_software_swizzled_b(fa_lib, N, K, a_mn, b_mn):
     _case(fa_lib, N, K, a_mn, b_mn, 0, 1, seed=3 + N + K + a_mn + b_mn)
+
+
+def test_fma_pipe_exp2_within_its_fitted_bound(fa_lib):
+    """The polynomial exp2 the kernels use beside ex2.approx: relative error
+    against float64 2^x within the Remez fit's bound (exp2_poly.h) plus float32
+    evaluation rounding, over the range the kernels feed it."""
+    import re
+    hdr = open("exact_io_aware_53_b200/csrc/exp2_poly.h").read()
+    bound = float(re.search(r"MAX_REL_ERR = ([0-9.e+-]+)f", hdr).group(1))
+    g = torch.Generator().manual_seed(3)
+    x = torch.cat([torch.linspace(-124.0, 64.0, 1 << 20), torch.rand(1 << 20, generator=g) * 20 - 16,
+                   torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.999, -124.5])])
+    x = x.contiguous().cuda()
+    y = fa_lib.selftest_exp2(x, 0)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref) / ref).abs().max().item()
+    assert rel <= bound + 8 * 2.0 ** -24, rel
+    # below the clamp the result stands for zero
+    lo = fa_lib.selftest_exp2(torch.tensor([-200.0, float("-inf"), -126.0, 0, 0, 0, 0, 0]).cuda(), 0)
+    assert float(lo[:3].max()) <= 2.0 ** -124
+    # the hardware approximation it runs beside, for comparison
+    y1 = fa_lib.selftest_exp2(x, 1)
+    assert ((y1.double() - ref) / ref).abs().max().item() < 2.0 ** -20
