@@ -44,6 +44,7 @@ constexpr int NTHREADS = 320;
 constexpr int MMA_WARP = 8;
 constexpr int LOAD_WARP = 9;
 constexpr int QSTAGES = 2;
+constexpr bool EX2_FMA_QUARTER = false;  // one exponential in four on the FMA pipe (off: no gain measured here)
 
 constexpr int BOX = 128 * 128;                    // 128 rows x 128 B (64 bf16)
 constexpr int TILE = 2 * BOX;                      // 128 rows x 128 bf16
@@ -293,13 +294,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd128_kernel(const __grid_consta
                 tmem_ld32(xa + h * 64, reinterpret_cast<uint32_t*>(pv));
                 tmem_ld32(xa + h * 64 + 32, reinterpret_cast<uint32_t*>(pv + 32));
                 tmem_wait_ld();
+                const float2 c2 = make_float2(cl2, cl2);
 #pragma unroll
                 for (int c = 0; c < 64; c += 4) {
+                    // x = c s - lse2 two at a time; one exponential in four on the FMA pipe
                     const float4 l4 = *reinterpret_cast<const float4*>(lse2 + h * 64 + c);
-                    pv[c] = ex2_approx(fmaf(pv[c], cl2, -l4.x));
-                    pv[c + 1] = ex2_approx(fmaf(pv[c + 1], cl2, -l4.y));
-                    pv[c + 2] = ex2_approx(fmaf(pv[c + 2], cl2, -l4.z));
-                    pv[c + 3] = ex2_approx(fmaf(pv[c + 3], cl2, -l4.w));
+                    const float2 xa = ffma2(make_float2(pv[c], pv[c + 1]), c2, make_float2(-l4.x, -l4.y));
+                    const float2 xb = ffma2(make_float2(pv[c + 2], pv[c + 3]), c2, make_float2(-l4.z, -l4.w));
+                    pv[c] = ex2_approx(xa.x);
+                    pv[c + 1] = ex2_approx(xa.y);
+                    pv[c + 2] = ex2_approx(xb.x);
+                    pv[c + 3] = EX2_FMA_QUARTER ? ex2_fma(xb.y) : ex2_approx(xb.y);
                 }
                 if (masked) {
 #pragma unroll
@@ -335,8 +340,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd128_kernel(const __grid_consta
                     const float4 d4 = *reinterpret_cast<const float4*>(delta + q4 * 32 + c);
                     const float2 pa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pq[c / 2]));
                     const float2 pb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pq[c / 2 + 1]));
-                    ds[c / 2] = pack_bf16x2(pa.x * (dp[c] - d4.x), pa.y * (dp[c + 1] - d4.y));
-                    ds[c / 2 + 1] = pack_bf16x2(pb.x * (dp[c + 2] - d4.z), pb.y * (dp[c + 3] - d4.w));
+                    const float2 ga = fmul2(pa, fadd2(make_float2(dp[c], dp[c + 1]), make_float2(-d4.x, -d4.y)));
+                    const float2 gb = fmul2(pb, fadd2(make_float2(dp[c + 2], dp[c + 3]), make_float2(-d4.z, -d4.w)));
+                    ds[c / 2] = pack_bf16x2(ga.x, ga.y);
+                    ds[c / 2 + 1] = pack_bf16x2(gb.x, gb.y);
                 }
                 uint8_t* chunk = sDS + (q4 >> 1) * BOX;
 #pragma unroll

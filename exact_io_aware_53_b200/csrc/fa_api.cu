@@ -427,6 +427,19 @@ int fa_selftest_umma(const void* a, const void* b, float* d, int M, int N, int K
     return st;
 }
 
+int fa_selftest_wait_timeout(unsigned long long limit_ns, unsigned int* gave_up, void* stream)
+{
+    g_last_launches = 0;
+    if (!gave_up || limit_ns < 1000000ull || limit_ns > 2000000000ull) return FA_ERR_INVALID_ARG;
+    WaitCtl ctl;
+    int st = get_ctl(&ctl);
+    if (st != FA_OK) return st;
+    ctl.limit_ns = limit_ns;
+    st = cuda_status(launch_wait_timeout_selftest(ctl, gave_up, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
 int fa_selftest_exp2(const float* x, float* y, int n, int mode, void* stream)
 {
     g_last_launches = 0;

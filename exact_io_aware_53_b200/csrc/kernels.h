@@ -98,6 +98,7 @@ struct UmmaTestParams {
     WaitCtl ctl;
 };
 cudaError_t launch_umma_selftest(const UmmaTestParams& p, cudaStream_t stream);
+cudaError_t launch_wait_timeout_selftest(WaitCtl ctl, unsigned int* gave_up, cudaStream_t stream);
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, int mode, cudaStream_t stream);
 cudaError_t launch_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem, int reps, int n_acc, int ctas,
                              long long* cycles, WaitCtl ctl, cudaStream_t stream);

@@ -290,3 +290,31 @@ cudaError_t launch_exp2_selftest(const float* x, float* y, int n, int mode, cuda
 }
 
 }  // namespace fa
+
+namespace fa {
+namespace wait_test {
+
+// One warp waits, with the kernels' bounded wait, for an mbarrier phase that
+// nothing completes: every lane gives up after ctl.limit_ns, the device error
+// word gets FA_DEV_TIMEOUT, and the kernel returns normally.
+__global__ void wait_timeout_kernel(WaitCtl ctl, unsigned int* gave_up)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    const bool ok = mbar_wait(&bar, 0, ctl);
+    if (!ok) atomicAdd(gave_up, 1u);
+}
+
+}  // namespace wait_test
+
+cudaError_t launch_wait_timeout_selftest(WaitCtl ctl, unsigned int* gave_up, cudaStream_t stream)
+{
+    wait_test::wait_timeout_kernel<<<1, 32, 0, stream>>>(ctl, gave_up);
+    return cudaGetLastError();
+}
+
+}  // namespace fa

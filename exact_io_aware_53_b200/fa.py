@@ -44,6 +44,7 @@ _SIGS = {
     "fa_last_launch_count": ([], I),
     "fa_selftest_umma": ([P, P, P, I, I, I, I, I, I, I, P], I),
     "fa_selftest_exp2": ([P, P, I, I, P], I),
+    "fa_selftest_wait_timeout": ([ctypes.c_ulonglong, P, P], I),
     "fa_selftest_umma_rate": ([I, I, I, I, I, I, I, I, I, P, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -244,3 +245,11 @@ def selftest_exp2(x, mode: int, stream=None):
     y = torch.empty_like(x)
     _check(_lib.fa_selftest_exp2(_ptr(x), _ptr(y), x.numel(), int(mode), _stream(stream)), "fa_selftest_exp2")
     return y
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    """Runs the bounded-wait failure check; returns how many lanes gave up."""
+    gave_up = torch.zeros(1, dtype=torch.int32, device="cuda")
+    _check(_lib.fa_selftest_wait_timeout(int(limit_ns), _ptr(gave_up), _stream(stream)), "fa_selftest_wait_timeout")
+    torch.cuda.synchronize()
+    return int(gave_up.item())

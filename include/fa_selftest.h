@@ -30,6 +30,16 @@ int fa_selftest_umma(const void* a, const void* b, float* d, int M, int N, int K
                      int b_manual, void* stream);
 
 /*
+ * Failure-path check of the kernels' bounded waits: one warp waits for an
+ * mbarrier phase that nothing completes.  Each lane gives up after limit_ns
+ * (1e6 .. 2e9), adds 1 to *gave_up (device counter) and the kernel returns;
+ * the device error word then holds the timeout, so the next
+ * fa_check_device_status() returns FA_ERR_TIMEOUT (and clears it).  No fault,
+ * trap or hang is involved.
+ */
+int fa_selftest_wait_timeout(unsigned long long limit_ns, unsigned int* gave_up, void* stream);
+
+/*
  * y[i] = 2^x[i] for n device floats, by the kernels' FMA-pipe polynomial
  * (mode 0: round-to-nearest range reduction, degree-3 minimax polynomial for
  * 2^f on [-1/2, 1/2], exponent insertion; inputs below -125 give 2^-125) or
