@@ -57,7 +57,7 @@ constexpr int STG_OFF = DS_OFF + TILE;             // dQ staging, fp32 [64 query
 constexpr int STG_CHUNK = 64 * 128;                // fp32 [64 query rows][32 d], 128-byte swizzled
 constexpr int VEC_OFF = STG_OFF + 4 * STG_CHUNK;   // [stage][lse2 128 | delta 128]
 constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
-constexpr int NBARS = 16;
+constexpr int NBARS = 17;
 constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd128_kernel(const __grid_consta
     uint64_t* dq_empty = bars + 12;
     uint64_t* dkdv_done = bars + 13;
     uint64_t* drain = bars + 14;
+    uint64_t* dqw_bar = bars + 15;  // the 4 dQ warps (128 threads)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NBARS);
 
     const int warp = static_cast<int>(warp_id());
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd128_kernel(const __grid_consta
         mbar_init(dq_empty, 128);
         mbar_init(dkdv_done, 1);
         mbar_init(drain, 1);
+        mbar_init(dqw_bar, 128);
         fence_mbar_init();
     }
     if (warp == MMA_WARP) {
@@ -379,6 +381,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd128_kernel(const __grid_consta
         const int dr = wq * 32 + lane;  // head-dim index = TMEM lane of dQ^T
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
         const bool issuer = (threadIdx.x == 4 * 32);
+        // thread barrier on an mbarrier with the bounded wait (never bar.sync), so a
+        // warp that gives up on a wait cannot strand the others at a barrier
+        int bar_uses = 0;
+        auto sync_dq = [&]() -> bool {
+            mbar_arrive(dqw_bar);
+            return warp_wait(dqw_bar, (bar_uses++) & 1, p.ctl);
+        };
         // element (query c, dim dr) of a [64][128] fp32 staging tile: 32-column chunk
         // dr / 32, row c, 16-byte piece (dr % 32) / 4 swizzled with c % 8
         uint8_t* stg = sSTG + (dr >> 5) * STG_CHUNK;
@@ -399,13 +408,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd128_kernel(const __grid_consta
             for (int half = 0; half < 2; ++half) {
                 // the previous reduce-add must have read the staging tile
                 if (issuer) bulk_wait_group_read0();
-                named_bar_sync(1, 128);
+                if (!(ok = sync_dq())) break;
 #pragma unroll
                 for (int c = 0; c < 64; ++c)
                     *reinterpret_cast<float*>(stg + c * 128 + ((piece ^ (c & 7)) << 4) + word) =
                         q[half * 64 + c] * p.scale;
                 fence_proxy_async_smem();
-                named_bar_sync(1, 128);
+                if (!(ok = sync_dq())) break;
                 if (issuer) {
 #pragma unroll
                     for (int ch = 0; ch < D / 32; ++ch)

@@ -57,7 +57,7 @@ struct Cfg {
     static constexpr int DQ_CHUNK = BQ * 128;
     static constexpr int VEC_OFF = DQ_OFF + (D / 32) * DQ_CHUNK;    // [QSTAGES][lse2 64 | delta 64]
     static constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
-    static constexpr int NBARS = 18;
+    static constexpr int NBARS = 19;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t DV_COL = 0;
@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
     uint64_t* dq_empty = bars + 15;
     uint64_t* dkdv_done = bars + 16;
     uint64_t* drain = bars + 17;
+    uint64_t* dqw_bar = bars + 18;  // the 4 dQ warps (128 threads)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
 
     // the 128-byte-swizzled tiles need a 1024-byte aligned base; the layout
@@ -135,6 +136,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
         mbar_init(dq_empty, 128);
         mbar_init(dkdv_done, 1);
         mbar_init(drain, 1);
+        mbar_init(dqw_bar, 128);
         fence_mbar_init();
     }
     if (D == 64) {
@@ -369,6 +371,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
         const bool has_rows = (wq * 32) < D;  // warp-uniform
         const bool issuer = (threadIdx.x == 4 * 32);
         bool ok = true;
+        // thread barrier on an mbarrier with the bounded wait (never bar.sync), so a
+        // warp that gives up on a wait cannot strand the others at a barrier
+        int bar_uses = 0;
+        auto sync_dq = [&]() -> bool {
+            mbar_arrive(dqw_bar);
+            return warp_wait(dqw_bar, (bar_uses++) & 1, p.ctl);
+        };
         for (int t = 0; t < n_it && ok; ++t) {
             const int i = i_first + t;
             if (!(ok = warp_wait(dq_full, t & 1, p.ctl))) break;
@@ -383,7 +392,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             mbar_arrive(dq_empty);
             // staging is free once the previous reduce-add has read it
             if (issuer) bulk_wait_group_read0();
-            named_bar_sync(1, 128);
+            if (!(ok = sync_dq())) break;
             if (has_rows) {
                 // element (query c, dim dr) of a [BQ][D] fp32 tile in 32-column swizzled chunks
                 uint8_t* chunk = sDQ + (dr >> 5) * C::DQ_CHUNK;
@@ -393,7 +402,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
                     *reinterpret_cast<float*>(chunk + c * 128 + ((piece ^ (c & 7)) << 4) + word) = q[c] * p.scale;
             }
             fence_proxy_async_smem();
-            named_bar_sync(1, 128);
+            if (!(ok = sync_dq())) break;
             if (issuer) {
                 for (int ch = 0; ch < D / 32; ++ch)
                     tma_reduce_add_3d(&p.tm_dq, sDQ + ch * C::DQ_CHUNK, ch * 32, i * BQ, bh);
