@@ -107,9 +107,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd128_kernel(const __grid_consta
 
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
-    // head-major order: CTAs resident together share a few heads' Q, dO and dQ in L2
-    const int j = blockIdx.x;  // key tile; tile 0 sees the most query tiles under the causal mask
-    const int bh = blockIdx.y;
+    // grouped longest-first order over (key tile, head): key tile 0 sees the
+    // most query tiles under the causal mask; a group's Q, dO and dQ share L2
+    int bh, j;
+    grouped_order(static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x), p.BH, p.n_kv_tiles, p.group_heads, bh, j);
     const int N = p.N;
     const int n_pad = p.n_kv_tiles * BKV;
     const int n_q = (N + BQ - 1) / BQ;

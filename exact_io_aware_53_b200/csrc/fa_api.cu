@@ -4,7 +4,12 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <functional>
+#include <map>
 #include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -60,6 +65,28 @@ int get_ctl(WaitCtl* ctl)
     return FA_OK;
 }
 
+// Finishing time of the last CTA when every SM that frees up takes the next
+// CTA in linear order (one resident CTA per SM), for grouped_order's layout.
+double grouped_makespan(int BH, int n_levels, const double* work, int G, int n_sm, double fixed)
+{
+    std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+    for (int i = 0; i < n_sm; ++i) free_at.push(0.0);
+    double last = 0.0;
+    for (int g0 = 0; g0 < BH; g0 += G) {
+        const int gh = std::min(G, BH - g0);
+        for (int v = 0; v < n_levels; ++v)
+            for (int h = 0; h < gh; ++h) {
+                const double t = free_at.top() + work[v] + fixed;
+                free_at.pop();
+                free_at.push(t);
+                last = std::max(last, t);
+            }
+    }
+    return last;
+}
+
+std::map<std::tuple<int, int, int, size_t, std::vector<double>>, int> g_group_cache;
+
 // 3-D tiled tensor map over a dense [d2][d1][d0] tensor (d0 innermost).
 int encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void* ptr, uint64_t d0, uint64_t d1,
               uint64_t d2, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw)
@@ -90,6 +117,41 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; 
 constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace
+
+// Group size for grouped_order: the one with the shortest modelled makespan
+// (a CTA costs its work plus a fixed prologue/epilogue share of two units)
+// among the sizes whose heads' shared data fits in half of L2; the smaller
+// size wins ties within half a percent.  Memoised per shape and device.
+int choose_group_heads(int BH, int n_levels, const double* work, size_t bytes_per_head)
+{
+    if (BH <= 1 || n_levels <= 1) return 1;
+    int dev = 0, n_sm = 0, l2 = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || n_sm < 1)
+        return 1;
+    auto key = std::make_tuple(n_sm, BH, l2, bytes_per_head, std::vector<double>(work, work + n_levels));
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        auto it = g_group_cache.find(key);
+        if (it != g_group_cache.end()) return it->second;
+    }
+    const size_t budget = static_cast<size_t>(l2) / 2;
+    const int g_max = std::max(1, static_cast<int>(std::min<size_t>(BH, budget / std::max<size_t>(bytes_per_head, 1))));
+    int best_g = 1;
+    double best = grouped_makespan(BH, n_levels, work, 1, n_sm, 2.0);
+    for (int G = 2; G <= g_max; G = (G < 16) ? G + 1 : G + G / 4) {
+        const double t = grouped_makespan(BH, n_levels, work, G, n_sm, 2.0);
+        if (t < best * 0.995) {
+            best = t;
+            best_g = G;
+        }
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_group_cache[key] = best_g;
+    return best_g;
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -139,6 +201,17 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.BH = static_cast<int>(BH);
     p.N = N;
     p.n_pairs = (N + 255) / 256;
+    p.group_heads = 1;
+    if (causal) {
+        // a pair's CTA runs the key tiles of both its Q tiles (levels = pairs, longest first)
+        const int n_t = (N + 127) / 128;
+        std::vector<double> work(p.n_pairs);
+        for (int v = 0; v < p.n_pairs; ++v) {
+            const int t0 = 2 * (p.n_pairs - 1 - v);
+            work[v] = (t0 < n_t ? t0 + 1 : 0) + (t0 + 1 < n_t ? t0 + 2 : 0);
+        }
+        p.group_heads = choose_group_heads(p.BH, p.n_pairs, work.data(), static_cast<size_t>(N) * d * 2 * 2);
+    }
     p.scale_log2 = scale * kLog2e;
     st = cuda_status(launch_fwd_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
     if (st == FA_OK) g_last_launches = 1;
@@ -219,6 +292,16 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, flo
     p.BH = static_cast<int>(BH);
     p.N = N;
     p.n_kv_tiles = (N + 127) / 128;
+    p.group_heads = 1;
+    if (causal) {
+        // key tile j runs the query tiles from its diagonal on (levels = key tiles)
+        const int n_q = (N + static_cast<int>(bq) - 1) / static_cast<int>(bq);
+        const int per_kv = 128 / static_cast<int>(bq);
+        std::vector<double> work(p.n_kv_tiles);
+        for (int j = 0; j < p.n_kv_tiles; ++j) work[j] = static_cast<double>(n_q - j * per_kv) / per_kv;
+        // Q, dO (bf16) and the fp32 dQ accumulator of a head
+        p.group_heads = choose_group_heads(p.BH, p.n_kv_tiles, work.data(), static_cast<size_t>(N) * d * 8);
+    }
     p.scale = scale;
     p.scale_log2 = scale * kLog2e;
     st = cuda_status(launch_bwd_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));

@@ -93,10 +93,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
 
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
-    // head-major launch order: CTAs resident together share a few heads' K/V in L2;
-    // under the causal mask each head's longest rows start first
-    const int bh = blockIdx.y;
-    const int pair = CAUSAL ? (p.n_pairs - 1 - static_cast<int>(blockIdx.x)) : static_cast<int>(blockIdx.x);
+    // grouped longest-first order: under the causal mask the pairs with the
+    // most key tiles (level 0 = the last pair) of a group of heads start first
+    int bh, level;
+    grouped_order(static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x), p.BH, p.n_pairs, p.group_heads, bh, level);
+    const int pair = CAUSAL ? (p.n_pairs - 1 - level) : level;
     const int q0 = pair * 2 * BM;
     const int N = p.N;
     const int n_kv_all = (N + BN - 1) / BN;

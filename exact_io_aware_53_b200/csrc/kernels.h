@@ -20,11 +20,17 @@ struct FwdParams {
     int BH;
     int N;
     int n_pairs;       // ceil(N / 256)
+    int group_heads;   // dispatch grouping of the (pair, head) grid, >= 1 (grouped_order)
     float scale_log2;  // scale * log2(e)
     WaitCtl ctl;
 };
 
 cudaError_t launch_fwd_sm100(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+
+// Heads per dispatch group for a causal grid: work[v] is the relative cost of
+// a CTA at level v (levels in dispatch order), bytes_per_head the data a head's
+// CTAs share through L2.  Host code (fa_api.cu).
+int choose_group_heads(int BH, int n_levels, const double* work, size_t bytes_per_head);
 
 // ---------------------------------------------------------------- bf16 backward
 struct BwdPreParams {
@@ -55,6 +61,7 @@ struct BwdParams {
     int BH;
     int N;
     int n_kv_tiles;
+    int group_heads;  // dispatch grouping of the (key tile, head) grid, >= 1 (grouped_order)
     float scale;
     float scale_log2;
     WaitCtl ctl;

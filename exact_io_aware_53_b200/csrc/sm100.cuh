@@ -30,6 +30,24 @@ __device__ __forceinline__ uint64_t global_timer_ns()
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ uint32_t warp_id() { return threadIdx.x >> 5; }
 
+// Dispatch order of a (level, head) grid whose CTA work shrinks with the
+// level.  The block dispatcher hands out CTAs in linear-index order; here heads
+// are taken in groups of `group_heads` and, inside a group, every head's
+// level-0 CTA comes first, then every head's level 1, and so on.  The longest
+// CTAs therefore start early instead of at the end of the grid, and CTAs
+// resident together touch the per-head data of one group only, which stays in
+// L2.  group_heads = 1 is plain head-major order.
+__device__ __forceinline__ void grouped_order(int lin, int BH, int n_levels, int group_heads, int& bh, int& level)
+{
+    const int G = max(group_heads, 1);
+    const int per_group = G * n_levels;
+    const int g = lin / per_group;
+    const int rem = lin - g * per_group;
+    const int gh = min(G, BH - g * G);
+    level = rem / gh;
+    bh = g * G + (rem - level * gh);
+}
+
 // Named barrier over `nthreads` threads (a multiple of 32) with id 1..15.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads)
 {
