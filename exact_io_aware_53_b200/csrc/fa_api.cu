@@ -53,11 +53,14 @@ int get_encoder()
 int get_ctl(WaitCtl* ctl)
 {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    int st = cuda_status(cudaGetDevice(&dev));
+    if (st != FA_OK) return st;
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_status_ptr[dev]) {
         void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_fa_status) != cudaSuccess || !ptr) return FA_ERR_CUDA;
+        if ((st = cuda_status(cudaGetSymbolAddress(&ptr, g_fa_status))) != FA_OK) return st;
+        if (!ptr) return FA_ERR_CUDA;
         g_status_ptr[dev] = static_cast<unsigned int*>(ptr);
     }
     ctl->status = g_status_ptr[dev];
@@ -112,11 +115,18 @@ int check_shape(int B, int H, int N, int d, float scale, int causal)
     return FA_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+thread_local int g_last_cuda_error = 0;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace
+
+int cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return FA_OK;
+    g_last_cuda_error = static_cast<int>(e);
+    return FA_ERR_CUDA;
+}
 
 // Group size for grouped_order: the one with the shortest modelled makespan
 // (a CTA costs its work plus a fixed prologue/epilogue share of two units)
@@ -172,6 +182,10 @@ const char* fa_status_string(int status)
 }
 
 int fa_last_launch_count(void) { return g_last_launches; }
+
+int fa_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* fa_cuda_error_string(int code) { return cudaGetErrorString(static_cast<cudaError_t>(code)); }
 
 void fa_set_wait_limit_ns(unsigned long long ns) { g_limit_ns.store(ns < 1000000ull ? 1000000ull : ns); }
 
@@ -441,7 +455,7 @@ int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const v
     const void* srcs[4] = {h_q, h_k, h_v, h_dO};
     void* dsts[4] = {q, k, v, dO};
     for (int i = 0; i < 4; ++i)
-        if (cudaMemcpyAsync(dsts[i], srcs[i], E * 2, cudaMemcpyHostToDevice, s) != cudaSuccess) return FA_ERR_CUDA;
+        if ((st = cuda_status(cudaMemcpyAsync(dsts[i], srcs[i], E * 2, cudaMemcpyHostToDevice, s))) != FA_OK) return st;
     if ((st = fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream)) != FA_OK) return st;
     const int n_fwd = g_last_launches;
     if ((st = fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, ws, B, H, N, d, scale, causal, stream)) != FA_OK) return st;
@@ -452,23 +466,23 @@ int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const v
         size_t bytes;
     } back[5] = {{h_o, o, E * 2}, {h_lse, lse, R * 4}, {h_dq, dq, E * 4}, {h_dk, dk, E * 4}, {h_dv, dv, E * 4}};
     for (auto& b : back)
-        if (b.dst && cudaMemcpyAsync(b.dst, b.src, b.bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-            return FA_ERR_CUDA;
+        if (b.dst && (st = cuda_status(cudaMemcpyAsync(b.dst, b.src, b.bytes, cudaMemcpyDeviceToHost, s))) != FA_OK)
+            return st;
     g_last_launches = n_fwd + n_bwd;
     return FA_OK;
 }
 
 int fa_check_device_status(void* stream)
 {
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
-    WaitCtl ctl;
-    int st = get_ctl(&ctl);
+    int st = cuda_status(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
     if (st != FA_OK) return st;
+    WaitCtl ctl;
+    if ((st = get_ctl(&ctl)) != FA_OK) return st;
     unsigned int word = 0;
-    if (cudaMemcpy(&word, ctl.status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+    if ((st = cuda_status(cudaMemcpy(&word, ctl.status, sizeof(word), cudaMemcpyDeviceToHost))) != FA_OK) return st;
     if (word != 0) {
         const unsigned int zero = 0;
-        if (cudaMemcpy(ctl.status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return FA_ERR_CUDA;
+        if ((st = cuda_status(cudaMemcpy(ctl.status, &zero, sizeof(zero), cudaMemcpyHostToDevice))) != FA_OK) return st;
         return (word & FA_DEV_TIMEOUT) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
     }
     return FA_OK;

@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 
 #include "fa.h"
+#include "kernels.h"
 
 namespace {
 
@@ -36,11 +37,14 @@ void* g_scratch_ptr[kMaxDevices] = {};
 int scratch_for_current_device(void** out)
 {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    int st = fa::cuda_status(cudaGetDevice(&dev));
+    if (st != FA_OK) return st;
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_scratch_ptr[dev]) {
         void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
+        if ((st = fa::cuda_status(cudaGetSymbolAddress(&ptr, g_noalloc_scratch))) != FA_OK) return st;
+        if (ptr == nullptr) return FA_ERR_CUDA;
         g_scratch_ptr[dev] = ptr;
     }
     *out = g_scratch_ptr[dev];

@@ -10,6 +10,10 @@
 
 namespace fa {
 
+// FA_OK for cudaSuccess; otherwise records e as the calling thread's last CUDA
+// error (fa_last_cuda_error) and returns FA_ERR_CUDA.  Host code (fa_api.cu).
+int cuda_status(cudaError_t e);
+
 // ---------------------------------------------------------------- bf16 forward
 struct FwdParams {
     CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle

@@ -42,6 +42,8 @@ _SIGS = {
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
     "fa_status_string": ([I], ctypes.c_char_p),
     "fa_last_launch_count": ([], I),
+    "fa_last_cuda_error": ([], I),
+    "fa_cuda_error_string": ([I], ctypes.c_char_p),
     "fa_selftest_umma": ([P, P, P, I, I, I, I, I, I, I, P], I),
     "fa_selftest_exp2": ([P, P, I, I, P], I),
     "fa_selftest_wait_timeout": ([ctypes.c_ulonglong, P, P], I),
@@ -63,7 +65,11 @@ FA_ERR_TIMEOUT = 5
 class FAError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__("%s: %s" % (what, _lib.fa_status_string(status).decode()))
+        msg = "%s: %s" % (what, _lib.fa_status_string(status).decode())
+        if status == FA_ERR_CUDA:
+            code = int(_lib.fa_last_cuda_error())
+            msg += " (CUDA error %d: %s)" % (code, _lib.fa_cuda_error_string(code).decode())
+        super().__init__(msg)
 
 
 def _check(status: int, what: str):

@@ -171,6 +171,13 @@ const char* fa_status_string(int status);
 /* Number of kernels the most recent fa_* call enqueued on the calling thread. */
 int fa_last_launch_count(void);
 
+/* The CUDA runtime error code (a cudaError_t value) behind the most recent
+ * FA_ERR_CUDA returned on the calling thread, 0 if none has been returned, and
+ * its description (static string; "no error" for 0).  Diagnostics only: no
+ * state of the library depends on them. */
+int fa_last_cuda_error(void);
+const char* fa_cuda_error_string(int code);
+
 #ifdef __cplusplus
 }
 #endif

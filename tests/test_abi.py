@@ -42,6 +42,14 @@ def test_status_strings(lib):
     assert lib.status_string(99) == "FA_ERR_UNKNOWN"
 
 
+def test_cuda_error_diagnostics(lib):
+    # argument errors record no CUDA error; the description table needs no GPU
+    assert _fwd(lib, q=0) == lib.FA_ERR_INVALID_ARG
+    assert lib._lib.fa_last_cuda_error() == 0
+    assert lib._lib.fa_cuda_error_string(0).decode() == "no error"
+    assert "resources" in lib._lib.fa_cuda_error_string(701).decode()
+
+
 def _fwd(lib, q=16, k=16, v=16, o=16, lse=16, B=1, H=1, N=8, d=64, scale=0.125, causal=0):
     P = ctypes.c_void_p
     return lib._lib.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, H, N, d, scale, causal, P(0))
