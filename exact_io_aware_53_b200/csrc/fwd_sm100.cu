@@ -23,10 +23,12 @@
 // "The math, worked with real numbers": m_new = max(m_old, m_block), l_new =
 // l_old e^{m_old-m_new} + sum e^{s-m_new}, O_new = O_old e^{m_old-m_new} + ...):
 //   m_new = max(m, c * rowmax(S));   p = 2^(c s - m);   l = l * alpha + sum p
-// The running max is only moved (and O, l rescaled by alpha = 2^(m - m_new))
-// when it grows by more than RESCALE_LOG2 = 8; otherwise the stale max is kept,
-// which leaves every p <= 2^8 and changes nothing in exact arithmetic because O
-// and l carry the same factor and the result is O / l.
+// The row max is taken for the first key tile only.  Later tiles are
+// exponentiated against the running max as it stands, and the max is moved
+// (O, l rescaled by alpha = 2^(m - m_new)) only when the tile's row sum exceeds
+// SUM_LIMIT, i.e. some score lies more than 16 (base 2) above m.  Any reference
+// m gives the same O / l in exact arithmetic (O and l carry the same factor);
+// the check keeps every p <= SUM_LIMIT.
 //
 // TMEM (512 columns x 128 lanes): S_t at columns [128 t, 128 t + 128); P_t (bf16
 // pairs) overwrites the first 64 columns of S_t; O_t at 256 + D t.
@@ -41,7 +43,8 @@ constexpr int BN = 128;  // keys per K/V tile
 constexpr int NTHREADS = 320;
 constexpr int MMA_WARP = 8;
 constexpr int LOAD_WARP = 9;
-constexpr float RESCALE_LOG2 = 8.0f;
+// A key tile whose row sum of 2^(c s - m) exceeds this moves the running max.
+constexpr float SUM_LIMIT = 65536.0f;
 constexpr int EX2_FMA_EVERY = 4;  // share of a row's exponentials evaluated on the FMA pipe: 1 / this
 constexpr float LN2 = 0.6931471805599453f;
 
@@ -267,57 +270,71 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
             }
             tc_fence_after();
             float s[BN];
-            tmem_ld32(s_addr + 0, reinterpret_cast<uint32_t*>(s + 0));
-            tmem_ld32(s_addr + 32, reinterpret_cast<uint32_t*>(s + 32));
-            tmem_ld32(s_addr + 64, reinterpret_cast<uint32_t*>(s + 64));
-            tmem_ld32(s_addr + 96, reinterpret_cast<uint32_t*>(s + 96));
-            tmem_wait_ld();
-            if (j == nk - 1) {
-                // last key tile of this Q tile: causal diagonal and/or ragged tail
-                const int limit = min(CAUSAL ? r : BN - 1, N - 1 - j * BN);
+            auto load_s = [&]() {
+                tmem_ld32(s_addr + 0, reinterpret_cast<uint32_t*>(s + 0));
+                tmem_ld32(s_addr + 32, reinterpret_cast<uint32_t*>(s + 32));
+                tmem_ld32(s_addr + 64, reinterpret_cast<uint32_t*>(s + 64));
+                tmem_ld32(s_addr + 96, reinterpret_cast<uint32_t*>(s + 96));
+                tmem_wait_ld();
+                if (j == nk - 1) {
+                    // last key tile of this Q tile: causal diagonal and/or ragged tail
+                    const int limit = min(CAUSAL ? r : BN - 1, N - 1 - j * BN);
 #pragma unroll
-                for (int c = 0; c < BN; ++c)
-                    if (c > limit) s[c] = -INFINITY;
-            }
-            // row max: 8 independent chains of three-input max, then a tree
-            float m8[8];
+                    for (int c = 0; c < BN; ++c)
+                        if (c > limit) s[c] = -INFINITY;
+                }
+            };
+            auto row_max = [&]() {
+                // 8 independent chains of three-input max, then a tree
+                float m8[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) m8[e] = fmaxf(s[e], s[e + 8]);
+                for (int e = 0; e < 8; ++e) m8[e] = fmaxf(s[e], s[e + 8]);
 #pragma unroll
-            for (int c = 16; c < BN; c += 16)
+                for (int c = 16; c < BN; c += 16)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
-            const float m_blk = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7])) * cl2;
+                    for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
+                return fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7])) * cl2;
+            };
+            load_s();
+            // The exponentials use the running max m as it stands: the row max of
+            // this tile is only taken (and m moved, O and l rescaled) when the
+            // tile's sum shows a score more than log2(SUM_LIMIT) above m.  Any
+            // reference m gives the same O / l and LSE in exact arithmetic; the
+            // check bounds every p by SUM_LIMIT.  P stays in registers until then,
+            // so S is still intact in TMEM for the second pass.
+            if (j == 0) m = row_max();
             float alpha = 1.f;
-            if (j == 0) {
-                m = m_blk;
-            } else if (m_blk > m + RESCALE_LOG2) {
-                alpha = ex2_approx(m - m_blk);
-                m = m_blk;
-            }
-            const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-m, -m);
-            float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            bool redo = false;
+            uint32_t pk[BN / 2];
+            float tsum;
+            for (;;) {
+                const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-m, -m);
+                float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[BN / 4];
-#pragma unroll
-                for (int c = 0; c < BN / 2; c += 2) {
+                for (int c = 0; c < BN; c += 2) {
                     // x = c s - m for two scores per instruction; one exponential in
                     // EX2_FMA_EVERY runs on the FMA pipe, beside MUFU
-                    const float2 x = ffma2(make_float2(s[h * (BN / 2) + c], s[h * (BN / 2) + c + 1]), c2, nm2);
+                    const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2, nm2);
                     const float p0 = ex2_approx(x.x);
                     const float p1 = (EX2_FMA_EVERY > 0 && (c + 2) % EX2_FMA_EVERY == 0) ? ex2_fma(x.y) : ex2_approx(x.y);
                     sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], make_float2(p0, p1));
                     pk[c / 2] = pack_bf16x2(p0, p1);
                 }
-                tmem_st32(s_addr + h * (BN / 4), pk);
+                const float2 sum_pair = fadd2(sum2[0], sum2[1]);
+                tsum = sum_pair.x + sum_pair.y;
+                if (redo || j == 0 || !__any_sync(0xffffffffu, !(tsum <= SUM_LIMIT))) break;
+                // a score far above m in some row of this warp: take the true row
+                // maxima (the whole warp, so TMEM access stays warp-wide)
+                redo = true;
+                load_s();
+                const float m_new = fmaxf(m, row_max());
+                alpha = ex2_approx(m - m_new);
+                m = m_new;
             }
-            const float2 sum_pair = fadd2(sum2[0], sum2[1]);
-            l = l * alpha + (sum_pair.x + sum_pair.y);
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                // O_t already holds sum_{j'<j} P V_j' (its MMA precedes this S in
-                // issue order, so S_t's commit covered it); rescale in TMEM.  Done
-                // after P is written so the S registers are dead by now.
+            l = l * alpha + tsum;
+            if (redo) {
+                // O_t holds sum_{j'<j} P V_j' (its MMA precedes this S in issue
+                // order, so S_t's commit covered it): rescale it in TMEM
 #pragma unroll
                 for (int cc = 0; cc < D; cc += 32) {
                     uint32_t o[32];
@@ -328,6 +345,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                     tmem_st32(o_addr + cc, o);
                 }
             }
+            tmem_st32(s_addr, pk);
+            tmem_st32(s_addr + BN / 4, pk + BN / 4);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[t]);

@@ -71,6 +71,35 @@ def test_sharp_softmax_rescaling_fwd(fa_lib, d):
     assert max_abs(out["lse"], rlse) <= LSE_TOL
 
 
+@pytest.mark.parametrize("d,causal", [(128, False), (128, True), (64, True)])
+def test_late_dominant_key_moves_the_running_max(fa_lib, d, causal):
+    """Key 400 (fourth key tile) scores 2 sqrt(d) for every query, 16 to 23
+    natural units (23 to 33 in base 2) above every other key.  The first key
+    tile's max is then far too low for the rows that see key 400, so the
+    forward has to move its running max and rescale O and l in the middle of
+    the row; under the causal mask rows 384..399 share a warp with rows that
+    do and must come out unchanged."""
+    N = 600
+    g = torch.Generator().manual_seed(5 + d)
+    u = torch.randn(d, generator=g)
+    u = u / u.norm() * math.sqrt(d)
+    q = (u + 0.05 * torch.randn(1, 1, N, d, generator=g)).to(torch.bfloat16)
+    k = 0.1 * torch.randn(1, 1, N, d, generator=g)
+    k[0, 0, 400] = 2 * u
+    k = k.to(torch.bfloat16)
+    v = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    do = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    x = {"q": q, "k": k, "v": v, "do": do}
+    scale = 1 / math.sqrt(d)
+    out = gpu_fwd_bwd(fa_lib, to_cuda(x), scale, causal, backward=False)
+    ro, rlse = oracle.attn_fwd(q, k, v, scale, causal)
+    assert max_abs(out["o"], ro) <= BF16_TOL
+    assert max_abs(out["lse"], rlse) <= LSE_TOL
+    # the rows that see key 400 are (almost) exactly its value row
+    seen = slice(400, N) if causal else slice(0, N)
+    assert max_abs(out["o"][0, 0, seen], v[0, 0, 400].float().expand(N - (400 if causal else 0), d)) <= BF16_TOL
+
+
 def _d_rounding_bounds(x, scale, causal):
     """First-order effect on dQ and dK of forming D_i = <dO_i, O_i> from the bf16
     O the backward is given (the oracle uses D_i = sum_j P_ij dP_ij exactly).
