@@ -216,10 +216,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                 }
             }
             for (int j = 0; j < n_kv_max && ok; ++j) {
+                // V_j and K_{j+1} are waited for first, while the tensor pipe
+                // still works through the previous key tile's MMAs; the waits
+                // between the MMA bursts below are then only on the softmax
                 const int sV = it % C::STAGES;
                 if (!(ok = mbar_wait(&kv_full[sV], (it / C::STAGES) & 1, p.ctl))) break;
                 ++it;
                 int sKn = -1;
+                if (j + 1 < n_kv_max) {
+                    sKn = it % C::STAGES;
+                    if (!(ok = mbar_wait(&kv_full[sKn], (it / C::STAGES) & 1, p.ctl))) break;
+                    ++it;
+                }
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (j >= n_kv[t]) continue;
                     if (!(ok = mbar_wait(&p_full[t], j & 1, p.ctl))) break;
@@ -227,12 +235,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
                     issue_o(t, sV, j);
                     if (j == n_kv[t] - 1) mma_commit(&o_full[t]);
                     if (j + 1 < n_kv[t]) {
-                        if (sKn < 0) {
-                            sKn = it % C::STAGES;
-                            if (!(ok = mbar_wait(&kv_full[sKn], (it / C::STAGES) & 1, p.ctl))) break;
-                            ++it;
-                            tc_fence_after();
-                        }
                         issue_s(t, sKn);
                         mma_commit(&s_full[t]);
                     }
