@@ -194,7 +194,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
         __syncwarp();
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop in step and elect.sync picks the lane
+        // that issues each tcgen05 instruction (from one lane of a diverged warp
+        // the same MMAs measured ~92 cycles each instead of ~65, B200).
+        {
             constexpr uint32_t idesc_st = idesc_bf16(BKV, BQ, false, false);
             constexpr uint32_t idesc_dkv = idesc_bf16(BKV, D, false, true);
             constexpr uint32_t idesc_dq = idesc_bf16(128, BQ, true, true);
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t ka = (kk >> 2) * C::KBOX + (kk & 3) * 32;
                     const uint32_t kb = (kk >> 2) * C::QBOX + (kk & 3) * 32;
-                    mma_ss(tmem + d_col, sdesc_sw128(a_base + ka, 16, 1024), sdesc_sw128(b_base + kb, 16, 1024),
+                    mma_ss_elect(tmem + d_col, sdesc_sw128(a_base + ka, 16, 1024), sdesc_sw128(b_base + kb, 16, 1024),
                            idesc_st, kk > 0 ? 1u : 0u);
                 }
             };
@@ -213,63 +216,63 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             auto issue_dkv = [&](uint32_t d_col, uint32_t a_col, uint32_t b_base, bool acc0) {
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    mma_ts(tmem + d_col, tmem + a_col + kk * 8, sdesc_sw128(b_base + kk * 2048, C::QBOX, 1024),
+                    mma_ts_elect(tmem + d_col, tmem + a_col + kk * 8, sdesc_sw128(b_base + kk * 2048, C::QBOX, 1024),
                            idesc_dkv, (acc0 || kk > 0) ? 1u : 0u);
             };
             // dQ^T = K^T (MN-major) x dS^T (MN-major, software-swizzled)
             auto issue_dq = [&](uint32_t ds_base) {
 #pragma unroll
                 for (int kk = 0; kk < BKV / 16; ++kk)
-                    mma_ss(tmem + C::DQ_COL, sdesc_sw128(aK + kk * 2048, C::KBOX, 1024),
+                    mma_ss_elect(tmem + C::DQ_COL, sdesc_sw128(aK + kk * 2048, C::KBOX, 1024),
                            sdesc_sw128(ds_base + kk * 2048, C::KBOX, 1024), idesc_dq, kk > 0 ? 1u : 0u);
             };
             auto q_base = [&](int t) { return aQS + (t % QSTAGES) * C::QSTAGE_BYTES; };
             auto do_base = [&](int t) { return aQS + (t % QSTAGES) * C::QSTAGE_BYTES + C::NDC * C::QBOX; };
 
-            bool ok = mbar_wait(kv_full, 0, p.ctl);
-            if (ok) ok = mbar_wait(&qdo_full[0], 0, p.ctl);
+            bool ok = warp_wait(kv_full, 0, p.ctl);
+            if (ok) ok = warp_wait(&qdo_full[0], 0, p.ctl);
             if (ok) {
                 tc_fence_after();
                 issue_sT(C::S_COL, aK, q_base(0));
-                mma_commit(&s_full[0]);
+                mma_commit_elect(&s_full[0]);
                 issue_sT(C::DP_COL, aV, do_base(0));
-                mma_commit(dp_full);
+                mma_commit_elect(dp_full);
                 if (n_it > 1) {
-                    ok = mbar_wait(&qdo_full[1], 0, p.ctl);
+                    ok = warp_wait(&qdo_full[1], 0, p.ctl);
                     if (ok) {
                         tc_fence_after();
                         issue_sT(C::S_COL + 64, aK, q_base(1));
-                        mma_commit(&s_full[1]);
+                        mma_commit_elect(&s_full[1]);
                     }
                 }
             }
             for (int t = 0; t < n_it && ok; ++t) {
                 const uint32_t sb = C::S_COL + 64 * (t & 1);
-                if (!(ok = mbar_wait(p_ready, t & 1, p.ctl))) break;
+                if (!(ok = warp_wait(p_ready, t & 1, p.ctl))) break;
                 tc_fence_after();
                 issue_dkv(C::DV_COL, sb, do_base(t), t > 0);
-                if (!(ok = mbar_wait(ds_ready, t & 1, p.ctl))) break;
+                if (!(ok = warp_wait(ds_ready, t & 1, p.ctl))) break;
                 tc_fence_after();
                 issue_dkv(C::DK_COL, C::DP_COL, q_base(t), t > 0);
-                mma_commit(&qdo_empty[t % QSTAGES]);
+                mma_commit_elect(&qdo_empty[t % QSTAGES]);
                 if (t + 1 < n_it) {
                     issue_sT(C::DP_COL, aV, do_base(t + 1));
-                    mma_commit(dp_full);
+                    mma_commit_elect(dp_full);
                 }
-                if (t > 0 && !(ok = mbar_wait(dq_empty, (t - 1) & 1, p.ctl))) break;
+                if (t > 0 && !(ok = warp_wait(dq_empty, (t - 1) & 1, p.ctl))) break;
                 tc_fence_after();
                 issue_dq(aDS + (t & 1) * C::DS_BYTES);
-                mma_commit(dq_full);
-                mma_commit(&ds_free[t & 1]);
+                mma_commit_elect(dq_full);
+                mma_commit_elect(&ds_free[t & 1]);
                 if (t + 2 < n_it) {
-                    if (!(ok = mbar_wait(&qdo_full[(t + 2) % QSTAGES], ((t + 2) / QSTAGES) & 1, p.ctl))) break;
+                    if (!(ok = warp_wait(&qdo_full[(t + 2) % QSTAGES], ((t + 2) / QSTAGES) & 1, p.ctl))) break;
                     tc_fence_after();
                     issue_sT(sb, aK, q_base(t + 2));
-                    mma_commit(&s_full[t & 1]);
+                    mma_commit_elect(&s_full[t & 1]);
                 }
             }
-            if (ok) mma_commit(dkdv_done);
-            mma_commit(drain);
+            if (ok) mma_commit_elect(dkdv_done);
+            mma_commit_elect(drain);
             mbar_wait_drain(drain, 0, p.ctl.limit_ns);
         }
         __syncwarp();
