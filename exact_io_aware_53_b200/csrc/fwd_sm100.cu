@@ -4,17 +4,21 @@
 // walks the key/value tiles of 128 keys (the tiling and online softmax of
 // "Tiling and the online softmax", vibeengines.com/paper/flash-attention):
 //
-//   warp 9      TMA producer: Q tiles once, then K_j, V_j through a smem ring
+//   warp 17     TMA producer: Q tiles once, then K_j, V_j through a smem ring
 //               (stages are handed back by a softmax thread that has seen the
 //               S MMA issued after their last reader complete, so the MMA warp
 //               spends no tcgen05.commit on them)
-//   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T (smem x smem -> TMEM),
+//   warp 16     MMA issuer: S_t = Q_t K_j^T (smem x smem -> TMEM),
 //               O_t += P_t V_j (P from TMEM x V from smem -> TMEM)
-//   warps 0-3   softmax for Q tile 0 (thread = query row = TMEM lane)
-//   warps 4-7   softmax for Q tile 1
+//   warps 0-7   softmax for Q tile 0, warps 8-15 for Q tile 1
 //
-// The two softmax warpgroups ping-pong: while one turns its S tile into P, the
-// tensor core runs the other tile's P V and next Q K^T.
+// Each Q tile has two softmax warps per SM sub-partition.  Warp w reaches the
+// TMEM lanes of quadrant w % 4 only, so the two warps of a quadrant take 16
+// lanes (rows) each through the 16-lane tcgen05.ld/st shapes, in which a row
+// is spread over four threads: the row max and sum need two shuffles, and the
+// two warps interleave their MUFU and FMA-pipe work, which a single warp does
+// not overlap.  The two Q tiles ping-pong: while one turns its S tile into P,
+// the tensor core runs the other tile's P V and next Q K^T.
 //
 // One exponential in four is evaluated by a polynomial on the FMA pipe
 // (ex2_fma) instead of MUFU ex2, which the softmax otherwise saturates.
@@ -40,12 +44,14 @@ namespace fwdk {
 
 constexpr int BM = 128;  // query rows per Q tile
 constexpr int BN = 128;  // keys per K/V tile
-constexpr int NTHREADS = 320;
-constexpr int MMA_WARP = 8;
-constexpr int LOAD_WARP = 9;
+constexpr int NTHREADS = 576;
+constexpr int MMA_WARP = 16;
+constexpr int LOAD_WARP = 17;
+// 18 warps leave five on two SM sub-partitions, whose 16K registers then allow
+// 102 per thread: the kernel is built for 96 (a softmax thread holds 64 scores)
+constexpr int MAX_REGS = 96;
 // A key tile whose row sum of 2^(c s - m) exceeds this moves the running max.
 constexpr float SUM_LIMIT = 65536.0f;
-constexpr int EX2_FMA_EVERY = 4;  // share of a row's exponentials evaluated on the FMA pipe: 1 / this
 constexpr float LN2 = 0.6931471805599453f;
 
 template <int D>
@@ -77,7 +83,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant__ FwdParams p)
+__global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdParams p)
 {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -120,7 +126,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&s_full[t], 1);
-            mbar_init(&p_full[t], 128);
+            mbar_init(&p_full[t], 256);
             mbar_init(&o_full[t], 1);
         }
         mbar_init(drain, 1);
@@ -252,107 +258,137 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
-        const int t = warp >> 2;
-        const int r = (warp & 3) * 32 + lane;
-        const int row = q0 + t * BM + r;
-        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t s_addr = tmem + lane_off + 128u * t;
-        const uint32_t o_addr = tmem + lane_off + C::O_COL + D * t;
+        // warp (quad, sub) of tile t owns TMEM lanes base .. base + 15; thread
+        // i holds rows rr0 = base + i/4 and rr0 + 8, columns 8n + cg + {0, 1}
+        // of each 8-column group n, in s[4n .. 4n + 3] (16x256b layout)
+        const int t = warp >> 3;
+        const int quad = warp & 3;
+        const int sub = (warp >> 2) & 1;
+        const int base = 32 * quad + 16 * sub;
+        const int rr0 = base + (lane >> 2);
+        const int cg = 2 * (lane & 3);
+        const uint32_t s_addr = tmem + (static_cast<uint32_t>(base) << 16) + 128u * t;
+        const uint32_t o_addr = s_addr + (C::O_COL + (D - 128) * t);
         const float cl2 = p.scale_log2;
         // the Q tile with the most key tiles releases the K/V ring stages (it
-        // issues the last S of every key tile); tile 1 unless it lies past N
-        const int releaser = n_kv[1] > 0 ? 1 : 0;
-        float m = -INFINITY;
-        float l = 0.f;
+        // issues the last S of every key tile): tile 1 unless it lies past N
+        const bool releases = (t == (n_kv[1] > 0 ? 1 : 0)) && warp == 8 * t && lane == 0;
+        float m0 = -INFINITY, m1 = -INFINITY;  // running max (base 2) of rows rr0, rr0 + 8
+        float l0 = 0.f, l1 = 0.f;              // this thread's share of their running sums
         bool ok = true;
         const int nk = n_kv[t];
         for (int j = 0; j < nk; ++j) {
             if (!(ok = warp_wait(&s_full[t], j & 1, p.ctl))) break;
-            if (t == releaser && r == 0) {
+            if (releases) {
                 // S_t(j) is complete, so is every MMA issued before it: K_j and
                 // V_{j-1} are consumed; hand their ring stages back to the producer
                 mbar_arrive(&kv_empty[(2 * j) % C::STAGES]);
                 if (j > 0) mbar_arrive(&kv_empty[(2 * j - 1) % C::STAGES]);
             }
             tc_fence_after();
-            float s[BN];
+            float s[64];
             auto load_s = [&]() {
-                tmem_ld32(s_addr + 0, reinterpret_cast<uint32_t*>(s + 0));
-                tmem_ld32(s_addr + 32, reinterpret_cast<uint32_t*>(s + 32));
-                tmem_ld32(s_addr + 64, reinterpret_cast<uint32_t*>(s + 64));
-                tmem_ld32(s_addr + 96, reinterpret_cast<uint32_t*>(s + 96));
+                tmem_ld_16x256b_x8(s_addr, reinterpret_cast<uint32_t*>(s));
+                tmem_ld_16x256b_x8(s_addr + 64, reinterpret_cast<uint32_t*>(s + 32));
                 tmem_wait_ld();
                 if (j == nk - 1) {
                     // last key tile of this Q tile: causal diagonal and/or ragged tail
-                    const int limit = min(CAUSAL ? r : BN - 1, N - 1 - j * BN);
+                    const int tail = N - 1 - j * BN;
+                    const int lim0 = min(CAUSAL ? rr0 : BN - 1, tail);
+                    const int lim1 = min(CAUSAL ? rr0 + 8 : BN - 1, tail);
 #pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        if (c > limit) s[c] = -INFINITY;
+                    for (int n = 0; n < 16; ++n)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int c = 8 * n + cg + e;
+                            if (c > lim0) s[4 * n + e] = -INFINITY;
+                            if (c > lim1) s[4 * n + 2 + e] = -INFINITY;
+                        }
                 }
             };
-            auto row_max = [&]() {
-                // 8 independent chains of three-input max, then a tree
-                float m8[8];
+            // row maxima (base 2) of rows rr0, rr0 + 8: two chains of three-input
+            // max per row, then the row's four threads (lanes 4(i/4) .. + 3)
+            auto row_max = [&](float& mx0, float& mx1) {
+                float x0 = fmaxf(s[0], s[1]), y0 = fmaxf(s[4], s[5]);
+                float x1 = fmaxf(s[2], s[3]), y1 = fmaxf(s[6], s[7]);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) m8[e] = fmaxf(s[e], s[e + 8]);
-#pragma unroll
-                for (int c = 16; c < BN; c += 16)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
-                return fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(fmax3(m8[3], m8[4], m8[5]), m8[6], m8[7])) * cl2;
+                for (int n = 2; n < 16; n += 2) {
+                    x0 = fmax3(x0, s[4 * n], s[4 * n + 1]);
+                    y0 = fmax3(y0, s[4 * n + 4], s[4 * n + 5]);
+                    x1 = fmax3(x1, s[4 * n + 2], s[4 * n + 3]);
+                    y1 = fmax3(y1, s[4 * n + 6], s[4 * n + 7]);
+                }
+                mx0 = fmaxf(x0, y0);
+                mx1 = fmaxf(x1, y1);
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2)) * cl2;
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2)) * cl2;
             };
             load_s();
-            // The exponentials use the running max m as it stands: the row max of
-            // this tile is only taken (and m moved, O and l rescaled) when the
-            // tile's sum shows a score more than log2(SUM_LIMIT) above m.  Any
-            // reference m gives the same O / l and LSE in exact arithmetic; the
-            // check bounds every p by SUM_LIMIT.  P stays in registers until then,
-            // so S is still intact in TMEM for the second pass.
-            if (j == 0) m = row_max();
-            float alpha = 1.f;
+            // The exponentials use the running max as it stands: the row max of
+            // this tile is only taken (and m moved, O and l rescaled) when a
+            // thread's share of a row sum shows a score more than log2(SUM_LIMIT)
+            // above m.  Any reference m gives the same O / l and LSE in exact
+            // arithmetic, and each p is bounded by the share it is part of.  P
+            // stays in registers until then, so S is still intact in TMEM.
+            if (j == 0) row_max(m0, m1);
+            float al0 = 1.f, al1 = 1.f;
             bool redo = false;
-            uint32_t pk[BN / 2];
-            float tsum;
+            uint32_t pk[32];
+            float ts0, ts1;
             for (;;) {
-                const float2 c2 = make_float2(cl2, cl2), nm2 = make_float2(-m, -m);
-                float2 sum2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                const float2 c2 = make_float2(cl2, cl2), n0 = make_float2(-m0, -m0), n1 = make_float2(-m1, -m1);
+                float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int c = 0; c < BN; c += 2) {
-                    // x = c s - m for two scores per instruction; one exponential in
-                    // EX2_FMA_EVERY runs on the FMA pipe, beside MUFU
-                    const float2 x = ffma2(make_float2(s[c], s[c + 1]), c2, nm2);
-                    const float p0 = ex2_approx(x.x);
-                    const float p1 = (EX2_FMA_EVERY > 0 && (c + 2) % EX2_FMA_EVERY == 0) ? ex2_fma(x.y) : ex2_approx(x.y);
-                    sum2[(c >> 1) & 1] = fadd2(sum2[(c >> 1) & 1], make_float2(p0, p1));
-                    pk[c / 2] = pack_bf16x2(p0, p1);
+                for (int n = 0; n < 16; ++n) {
+                    // one exponential in four on the FMA pipe, beside MUFU
+                    const float2 xa = ffma2(make_float2(s[4 * n], s[4 * n + 1]), c2, n0);
+                    const float2 xb = ffma2(make_float2(s[4 * n + 2], s[4 * n + 3]), c2, n1);
+                    const float2 pa = make_float2(ex2_approx(xa.x), ex2_approx(xa.y));
+                    const float2 pb = make_float2(ex2_approx(xb.x), ex2_fma(xb.y));
+                    sum0 = fadd2(sum0, pa);
+                    sum1 = fadd2(sum1, pb);
+                    // packed pairs in the 16x128b layout: column 4n + i%4
+                    pk[2 * n] = pack_bf16x2(pa.x, pa.y);
+                    pk[2 * n + 1] = pack_bf16x2(pb.x, pb.y);
                 }
-                const float2 sum_pair = fadd2(sum2[0], sum2[1]);
-                tsum = sum_pair.x + sum_pair.y;
-                if (redo || j == 0 || !__any_sync(0xffffffffu, !(tsum <= SUM_LIMIT))) break;
+                ts0 = sum0.x + sum0.y;
+                ts1 = sum1.x + sum1.y;
+                if (redo || j == 0 || !__any_sync(0xffffffffu, !(ts0 <= SUM_LIMIT && ts1 <= SUM_LIMIT))) break;
                 // a score far above m in some row of this warp: take the true row
                 // maxima (the whole warp, so TMEM access stays warp-wide)
                 redo = true;
                 load_s();
-                const float m_new = fmaxf(m, row_max());
-                alpha = ex2_approx(m - m_new);
-                m = m_new;
+                float mx0, mx1;
+                row_max(mx0, mx1);
+                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                al0 = ex2_approx(m0 - mn0);
+                al1 = ex2_approx(m1 - mn1);
+                m0 = mn0;
+                m1 = mn1;
             }
-            l = l * alpha + tsum;
+            l0 = l0 * al0 + ts0;
+            l1 = l1 * al1 + ts1;
             if (redo) {
                 // O_t holds sum_{j'<j} P V_j' (its MMA precedes this S in issue
                 // order, so S_t's commit covered it): rescale it in TMEM
 #pragma unroll
                 for (int cc = 0; cc < D; cc += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(o_addr + cc, o);
+                    uint32_t o[16];
+                    tmem_ld_16x256b_x4(o_addr + cc, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                    tmem_st32(o_addr + cc, o);
+                    for (int n = 0; n < 4; ++n) {
+                        o[4 * n] = __float_as_uint(__uint_as_float(o[4 * n]) * al0);
+                        o[4 * n + 1] = __float_as_uint(__uint_as_float(o[4 * n + 1]) * al0);
+                        o[4 * n + 2] = __float_as_uint(__uint_as_float(o[4 * n + 2]) * al1);
+                        o[4 * n + 3] = __float_as_uint(__uint_as_float(o[4 * n + 3]) * al1);
+                    }
+                    tmem_st_16x256b_x4(o_addr + cc, o);
                 }
             }
-            tmem_st32(s_addr, pk);
-            tmem_st32(s_addr + BN / 4, pk + BN / 4);
+            tmem_st_16x128b_x16(s_addr, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&p_full[t]);
@@ -361,25 +397,35 @@ __global__ void __launch_bounds__(NTHREADS, 1) fwd_kernel(const __grid_constant_
             ok = warp_wait(&o_full[t], 0, p.ctl);
             if (ok) {
                 tc_fence_after();
-                const float inv_l = 1.f / l;
-                __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * N + row) * D;
+                // each row's sum is split over its four threads
+                l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+                l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+                const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+                const int row0 = q0 + t * BM + rr0, row1 = row0 + 8;
+                __nv_bfloat16* orow0 = p.o + (static_cast<size_t>(bh) * N + row0) * D;
+                __nv_bfloat16* orow1 = orow0 + 8 * D;
 #pragma unroll
                 for (int cc = 0; cc < D; cc += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(o_addr + cc, o);
+                    uint32_t o[16];
+                    tmem_ld_16x256b_x4(o_addr + cc, o);
                     tmem_wait_ld();
-                    uint32_t packed[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        packed[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-                    if (row < N) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + cc);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+                    for (int n = 0; n < 4; ++n) {
+                        const int col = cc + 8 * n + cg;
+                        if (row0 < N)
+                            *reinterpret_cast<uint32_t*>(orow0 + col) =
+                                pack_bf16x2(__uint_as_float(o[4 * n]) * inv0, __uint_as_float(o[4 * n + 1]) * inv0);
+                        if (row1 < N)
+                            *reinterpret_cast<uint32_t*>(orow1 + col) = pack_bf16x2(
+                                __uint_as_float(o[4 * n + 2]) * inv1, __uint_as_float(o[4 * n + 3]) * inv1);
                     }
                 }
-                if (row < N) p.lse[static_cast<size_t>(bh) * N + row] = (m + __log2f(l)) * LN2;
+                if ((lane & 3) == 0) {
+                    if (row0 < N) p.lse[static_cast<size_t>(bh) * N + row0] = (m0 + __log2f(l0)) * LN2;
+                    if (row1 < N) p.lse[static_cast<size_t>(bh) * N + row1] = (m1 + __log2f(l1)) * LN2;
+                }
             }
         }
     }
