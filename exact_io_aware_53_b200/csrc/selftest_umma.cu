@@ -157,9 +157,8 @@ namespace umma_rate {
 // issue pattern the attention kernels use.  Issued either by one lane of a
 // diverged warp or by a converged warp with an elected lane per instruction.
 // cycles[2 cta] = first issue -> completion, cycles[2 cta + 1] = first -> last issue.
-template <int N, int K, bool AMN, bool BMN, bool ATMEM>
-__global__ void __launch_bounds__(128, 1) umma_rate_kernel(int reps, int n_acc, int converged, long long* cycles,
-                                                            WaitCtl ctl)
+template <int N, int K, bool AMN, bool BMN, bool ATMEM, bool CONV>
+__global__ void __launch_bounds__(128, 1) umma_rate_kernel(int reps, int n_acc, long long* cycles, WaitCtl ctl)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -185,32 +184,35 @@ __global__ void __launch_bounds__(128, 1) umma_rate_kernel(int reps, int n_acc, 
     const uint32_t tmem = *tmem_slot;
     constexpr uint32_t idesc = idesc_bf16(128, N, AMN, BMN);
     const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
-    auto issue = [&](uint32_t d, bool elect) {
+    // CONV: the whole warp runs the loop and elect.sync picks the issuing lane;
+    // otherwise lane 0 alone.  A compile-time choice: a run-time branch around
+    // every MMA would itself slow the issue stream.
+    auto issue = [&](uint32_t d) {
 #pragma unroll
         for (int kk = 0; kk < K / 16; ++kk) {
             const uint32_t acc = kk > 0 ? 1u : 0u;
             const uint64_t bdesc = BMN ? sdesc_sw128(b0 + kk * 2048, K * 128, 1024)
                                        : sdesc_sw128(b0 + (kk >> 2) * N * 128 + (kk & 3) * 32, 16, 1024);
             if constexpr (ATMEM) {
-                if (elect) mma_ts_elect(d, tmem + 384 + kk * 8, bdesc, idesc, acc);
+                if constexpr (CONV) mma_ts_elect(d, tmem + 384 + kk * 8, bdesc, idesc, acc);
                 else mma_ts(d, tmem + 384 + kk * 8, bdesc, idesc, acc);
             } else {
                 const uint64_t adesc = AMN ? sdesc_sw128(a0 + kk * 2048, K * 128, 1024)
                                            : sdesc_sw128(a0 + (kk >> 2) * 128 * 128 + (kk & 3) * 32, 16, 1024);
-                if (elect) mma_ss_elect(d, adesc, bdesc, idesc, acc);
+                if constexpr (CONV) mma_ss_elect(d, adesc, bdesc, idesc, acc);
                 else mma_ss(d, adesc, bdesc, idesc, acc);
             }
         }
     };
-    if (converged ? (warp == 0) : (threadIdx.x == 0)) {
+    if (CONV ? (warp == 0) : (threadIdx.x == 0)) {
         const long long t0 = clock64();
         int a = 0;
         for (int r = 0; r < reps; ++r) {
-            issue(tmem + static_cast<uint32_t>(a * N), converged != 0);
+            issue(tmem + static_cast<uint32_t>(a * N));
             a = (a + 1 == n_acc) ? 0 : a + 1;
         }
         const long long t1 = clock64();
-        if (converged)
+        if constexpr (CONV)
             mma_commit_elect(bar);
         else
             mma_commit(bar);
@@ -230,16 +232,23 @@ __global__ void __launch_bounds__(128, 1) umma_rate_kernel(int reps, int n_acc, 
     }
 }
 
+template <int N, int K, bool AMN, bool BMN, bool ATMEM, bool CONV>
+cudaError_t launch_rate_as(int reps, int n_acc, int ctas, long long* cycles, WaitCtl ctl, cudaStream_t stream)
+{
+    const int smem = 96 * 1024 + 64 + 1024;
+    auto kern = umma_rate_kernel<N, K, AMN, BMN, ATMEM, CONV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, 128, smem, stream>>>(reps, n_acc, cycles, ctl);
+    return cudaGetLastError();
+}
+
 template <int N, int K, bool AMN, bool BMN, bool ATMEM>
 cudaError_t launch_rate(int reps, int n_acc, int converged, int ctas, long long* cycles, WaitCtl ctl,
                         cudaStream_t stream)
 {
-    const int smem = 96 * 1024 + 64 + 1024;
-    auto kern = umma_rate_kernel<N, K, AMN, BMN, ATMEM>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    kern<<<ctas, 128, smem, stream>>>(reps, n_acc, converged, cycles, ctl);
-    return cudaGetLastError();
+    return converged ? launch_rate_as<N, K, AMN, BMN, ATMEM, true>(reps, n_acc, ctas, cycles, ctl, stream)
+                     : launch_rate_as<N, K, AMN, BMN, ATMEM, false>(reps, n_acc, ctas, cycles, ctl, stream);
 }
 
 }  // namespace umma_rate
