@@ -215,6 +215,18 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.BH = static_cast<int>(BH);
     p.N = N;
     p.n_pairs = (N + 255) / 256;
+    {
+        // persistent grid: one CTA per SM, no more than there are work items;
+        // each launch takes the next work-queue slot in turn (a slot is reused
+        // only after 63 other forward launches)
+        int dev = 0, n_sm = 0;
+        if ((st = cuda_status(cudaGetDevice(&dev))) != FA_OK) return st;
+        if ((st = cuda_status(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev))) != FA_OK) return st;
+        const long long items = static_cast<long long>(BH) * p.n_pairs;
+        p.n_ctas = static_cast<int>(std::max<long long>(1, std::min<long long>(n_sm, items)));
+        static std::atomic<unsigned int> launches{0};
+        p.queue_slot = static_cast<int>(launches.fetch_add(1) % 64u);
+    }
     p.group_heads = 1;
     if (causal) {
         // a pair's CTA runs the key tiles of both its Q tiles (levels = pairs, longest first)

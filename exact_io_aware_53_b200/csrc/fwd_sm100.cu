@@ -1,10 +1,16 @@
 // Forward attention, bf16 in / fp32 accumulate, sm_100a.
 //
-// One CTA owns 256 query rows of one (batch, head) as two 128-row Q tiles and
-// walks the key/value tiles of 128 keys (the tiling and online softmax of
-// "Tiling and the online softmax", vibeengines.com/paper/flash-attention):
+// A work item is 256 query rows of one (batch, head), as two 128-row Q tiles,
+// walking the key/value tiles of 128 keys (the tiling and online softmax of
+// "Tiling and the online softmax", vibeengines.com/paper/flash-attention).
+// The kernel is persistent: one CTA per SM takes items from a queue in the
+// grouped longest-first order until none are left, and one item's Q load and
+// first S overlap the previous item's last softmax and epilogue.
 //
-//   warp 17     TMA producer: Q tiles once, then K_j, V_j through a smem ring
+//   warp 17     TMA producer: takes the next item from the queue and hands it
+//               to the other warps through a two-slot ring; Q tiles once per
+//               item (after the previous item's last S MMA), then K_j, V_j
+//               through a smem ring
 //               (stages are handed back by a softmax thread that has seen the
 //               S MMA issued after their last reader complete, so the MMA warp
 //               spends no tcgen05.commit on them)
@@ -54,6 +60,13 @@ constexpr int MAX_REGS = 96;
 constexpr float SUM_LIMIT = 65536.0f;
 constexpr float LN2 = 0.6931471805599453f;
 
+// Work queues: slot k holds {next item, CTAs finished} for one launch in
+// flight.  The host gives each launch the next slot in turn; a launch's last
+// CTA returns its slot to {0, 0} (device memory starts zeroed), so launches
+// allocate nothing.
+constexpr int QUEUE_SLOTS = 64;
+__device__ unsigned int g_queue[QUEUE_SLOTS][2];
+
 template <int D>
 struct Cfg {
     static constexpr int NDC = D / 64;              // 128-byte swizzle boxes per row
@@ -63,8 +76,10 @@ struct Cfg {
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = 2 * TILE_BYTES;
     static constexpr int BAR_OFF = KV_OFF + STAGES * TILE_BYTES;
-    static constexpr int NBARS = 1 + 2 * STAGES + 2 + 2 + 2 + 1;
-    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
+    // q_full, q_empty, kv_full/empty[S], s_full, p_full, o_full, o_free [2],
+    // item_full, item_empty [2], drain
+    static constexpr int NBARS = 2 + 2 * STAGES + 4 * 2 + 2 * 2 + 1;
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;  // + TMEM slot and item ring
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t O_COL = 256;
 };
@@ -82,6 +97,35 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
     return __all_sync(0xffffffffu, ok);
 }
 
+// A work item: (batch * head, pair of Q tiles) by grouped_order, with the
+// number of key tiles each Q tile sees.
+struct Item {
+    int bh;
+    int q0;       // first query row
+    int n_kv[2];  // key tiles of Q tiles 0, 1 (0: the tile lies past N)
+    int n_kv_max;
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ Item decode_item(const FwdParams& p, int item)
+{
+    Item w;
+    int level;
+    grouped_order(item, p.BH, p.n_pairs, p.group_heads, w.bh, level);
+    // under the causal mask the pairs with the most key tiles (level 0 = the
+    // last pair) of a group of heads come first
+    const int pair = CAUSAL ? (p.n_pairs - 1 - level) : level;
+    w.q0 = pair * 2 * BM;
+    const int n_kv_all = (p.N + BN - 1) / BN;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int row0 = w.q0 + t * BM;
+        w.n_kv[t] = (row0 >= p.N) ? 0 : (CAUSAL ? min(n_kv_all, row0 / BN + 1) : n_kv_all);
+    }
+    w.n_kv_max = max(w.n_kv[0], w.n_kv[1]);
+    return w;
+}
+
 template <int D, bool CAUSAL>
 __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdParams p)
 {
@@ -92,34 +136,28 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     uint8_t* sKV = smem + C::KV_OFF;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
     uint64_t* q_full = bars;
-    uint64_t* kv_full = bars + 1;
+    uint64_t* q_empty = bars + 1;
+    uint64_t* kv_full = bars + 2;
     uint64_t* kv_empty = kv_full + C::STAGES;
     uint64_t* s_full = kv_empty + C::STAGES;  // [2]
     uint64_t* p_full = s_full + 2;            // [2]
     uint64_t* o_full = p_full + 2;            // [2]
-    uint64_t* drain = o_full + 2;
+    uint64_t* o_free = o_full + 2;            // [2] the epilogue has read O_t
+    uint64_t* item_full = o_free + 2;         // [2]
+    uint64_t* item_empty = item_full + 2;     // [2]
+    uint64_t* drain = item_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    int* item_buf = reinterpret_cast<int*>(tmem_slot + 1);  // [2]
 
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
-    // grouped longest-first order: under the causal mask the pairs with the
-    // most key tiles (level 0 = the last pair) of a group of heads start first
-    int bh, level;
-    grouped_order(static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x), p.BH, p.n_pairs, p.group_heads, bh, level);
-    const int pair = CAUSAL ? (p.n_pairs - 1 - level) : level;
-    const int q0 = pair * 2 * BM;
     const int N = p.N;
-    const int n_kv_all = (N + BN - 1) / BN;
-    int n_kv[2];
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        const int row0 = q0 + t * BM;
-        n_kv[t] = (row0 >= N) ? 0 : (CAUSAL ? min(n_kv_all, row0 / BN + 1) : n_kv_all);
-    }
-    const int n_kv_max = max(n_kv[0], n_kv[1]);
+    const int total = p.BH * p.n_pairs;
+    unsigned int* queue = g_queue[p.queue_slot];
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
@@ -128,6 +166,9 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
             mbar_init(&s_full[t], 1);
             mbar_init(&p_full[t], 256);
             mbar_init(&o_full[t], 1);
+            mbar_init(&o_free[t], 256);
+            mbar_init(&item_full[t], 1);
+            mbar_init(&item_empty[t], 1 + 16);  // the MMA warp and the 16 softmax warps
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -149,34 +190,47 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     if (warp == LOAD_WARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            uint32_t qbytes = 0;
-            for (int t = 0; t < 2; ++t) qbytes += (n_kv[t] > 0) ? C::TILE_BYTES : 0;
-            mbar_arrive_expect_tx(q_full, qbytes);
-            for (int t = 0; t < 2; ++t)
-                if (n_kv[t] > 0)
-                    for (int c = 0; c < C::NDC; ++c)
-                        tma_load_3d(sQ + t * C::TILE_BYTES + c * C::BOX_BYTES, &p.tm_q, q_full, c * 64,
-                                    q0 + t * BM, bh);
-            int it = 0;
+            int it = 0, nq = 0;  // K/V ring slots and Q tiles issued so far
             bool ok = true;
-            for (int j = 0; j < n_kv_max && ok; ++j) {
-                for (int kind = 0; kind < 2; ++kind) {
-                    const int s = it % C::STAGES;
-                    if (!mbar_wait(&kv_empty[s], ((it / C::STAGES) & 1) ^ 1, p.ctl)) {
-                        ok = false;
-                        break;
+            for (int n = 0; ok; ++n) {
+                const int slot = n & 1;
+                const int raw = static_cast<int>(atomicAdd(&queue[0], 1u));
+                const int item = raw < total ? raw : -1;
+                if (!(ok = mbar_wait(&item_empty[slot], ((n >> 1) & 1) ^ 1, p.ctl))) break;
+                item_buf[slot] = item;
+                mbar_arrive(&item_full[slot]);  // release: the waiters see item_buf
+                if (item < 0) break;
+                const Item w = decode_item<CAUSAL>(p, item);
+                // the previous item's last S MMA has read the Q tiles
+                if (!(ok = mbar_wait(q_empty, (n & 1) ^ 1, p.ctl))) break;
+                uint32_t qbytes = 0;
+                for (int t = 0; t < 2; ++t) qbytes += (w.n_kv[t] > 0) ? C::TILE_BYTES : 0;
+                mbar_arrive_expect_tx(q_full, qbytes);
+                for (int t = 0; t < 2; ++t)
+                    if (w.n_kv[t] > 0)
+                        for (int c = 0; c < C::NDC; ++c)
+                            tma_load_3d(sQ + t * C::TILE_BYTES + c * C::BOX_BYTES, &p.tm_q, q_full, c * 64,
+                                        w.q0 + t * BM, w.bh);
+                ++nq;
+                for (int j = 0; j < w.n_kv_max && ok; ++j) {
+                    for (int kind = 0; kind < 2; ++kind) {
+                        const int s = it % C::STAGES;
+                        if (!mbar_wait(&kv_empty[s], ((it / C::STAGES) & 1) ^ 1, p.ctl)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
+                        const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
+                        for (int c = 0; c < C::NDC; ++c)
+                            tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64,
+                                        j * BN, w.bh);
+                        ++it;
                     }
-                    mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
-                    const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
-                    for (int c = 0; c < C::NDC; ++c)
-                        tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64, j * BN,
-                                    bh);
-                    ++it;
                 }
             }
             if (!ok) {
                 // let every copy already issued land before the CTA exits
-                mbar_wait_drain(q_full, 0, p.ctl.limit_ns);
+                if (nq > 0) mbar_wait_drain(q_full, (nq - 1) & 1, p.ctl.limit_ns);
                 for (int i = max(0, it - C::STAGES); i < it; ++i)
                     mbar_wait_drain(&kv_full[i % C::STAGES], (i / C::STAGES) & 1, p.ctl.limit_ns);
             }
@@ -210,46 +264,61 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                     mma_ts_elect(tmem + C::O_COL + D * t, tmem + 128u * t + kk * 8,
                            sdesc_sw128(vb + kk * 2048, C::BOX_BYTES, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
             };
-            bool ok = warp_wait(q_full, 0, p.ctl);
-            int it = 0;
-            if (ok) {
+            int it = 0;                 // K/V ring slots consumed
+            int pc[2] = {0, 0};         // key tiles of Q tile t done (s_full / p_full phases)
+            int nact[2] = {0, 0};       // items in which Q tile t was present (o_full / o_free phases)
+            bool ok = true;
+            for (int n = 0; ok; ++n) {
+                const int slot = n & 1;
+                if (!(ok = warp_wait(&item_full[slot], (n >> 1) & 1, p.ctl))) break;
+                const int item = *reinterpret_cast<volatile int*>(&item_buf[slot]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&item_empty[slot]);
+                if (item < 0) break;
+                const Item w = decode_item<CAUSAL>(p, item);
+                if (!(ok = warp_wait(q_full, n & 1, p.ctl))) break;
                 const int sK = it % C::STAGES;
-                ok = warp_wait(&kv_full[sK], (it / C::STAGES) & 1, p.ctl);
+                if (!(ok = warp_wait(&kv_full[sK], (it / C::STAGES) & 1, p.ctl))) break;
                 ++it;
-                if (ok) {
-                    tc_fence_after();
-                    for (int t = 0; t < 2; ++t)
-                        if (n_kv[t] > 0) {
-                            issue_s(t, sK);
-                            mma_commit_elect(&s_full[t]);
-                        }
-                }
-            }
-            for (int j = 0; j < n_kv_max && ok; ++j) {
-                // V_j and K_{j+1} are waited for first, while the tensor pipe
-                // still works through the previous key tile's MMAs; the waits
-                // between the MMA bursts below are then only on the softmax
-                const int sV = it % C::STAGES;
-                if (!(ok = warp_wait(&kv_full[sV], (it / C::STAGES) & 1, p.ctl))) break;
-                ++it;
-                int sKn = -1;
-                if (j + 1 < n_kv_max) {
-                    sKn = it % C::STAGES;
-                    if (!(ok = warp_wait(&kv_full[sKn], (it / C::STAGES) & 1, p.ctl))) break;
-                    ++it;
-                }
-                for (int t = 0; t < 2 && ok; ++t) {
-                    if (j >= n_kv[t]) continue;
-                    if (!(ok = warp_wait(&p_full[t], j & 1, p.ctl))) break;
-                    tc_fence_after();
-                    issue_o(t, sV, j);
-                    if (j == n_kv[t] - 1) mma_commit_elect(&o_full[t]);
-                    if (j + 1 < n_kv[t]) {
-                        issue_s(t, sKn);
+                tc_fence_after();
+                for (int t = 0; t < 2; ++t)
+                    if (w.n_kv[t] > 0) {
+                        issue_s(t, sK);
                         mma_commit_elect(&s_full[t]);
                     }
+                if (w.n_kv_max == 1) mma_commit_elect(q_empty);  // that was the item's last S
+                for (int j = 0; j < w.n_kv_max && ok; ++j) {
+                    // V_j and K_{j+1} are waited for first, while the tensor pipe
+                    // still works through the previous key tile's MMAs; the waits
+                    // between the MMA bursts below are then only on the softmax
+                    const int sV = it % C::STAGES;
+                    if (!(ok = warp_wait(&kv_full[sV], (it / C::STAGES) & 1, p.ctl))) break;
+                    ++it;
+                    int sKn = -1;
+                    if (j + 1 < w.n_kv_max) {
+                        sKn = it % C::STAGES;
+                        if (!(ok = warp_wait(&kv_full[sKn], (it / C::STAGES) & 1, p.ctl))) break;
+                        ++it;
+                    }
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (j >= w.n_kv[t]) continue;
+                        if (!(ok = warp_wait(&p_full[t], pc[t] & 1, p.ctl))) break;
+                        // the first P V of an item overwrites O_t: the previous
+                        // item's epilogue must have read it
+                        if (j == 0 && nact[t] > 0 && !(ok = warp_wait(&o_free[t], (nact[t] - 1) & 1, p.ctl))) break;
+                        tc_fence_after();
+                        issue_o(t, sV, j);
+                        ++pc[t];
+                        if (j == w.n_kv[t] - 1) mma_commit_elect(&o_full[t]);
+                        if (j + 1 < w.n_kv[t]) {
+                            issue_s(t, sKn);
+                            mma_commit_elect(&s_full[t]);
+                        }
+                    }
+                    if (j + 2 == w.n_kv_max) mma_commit_elect(q_empty);  // S(j + 1) was the item's last S
+                    if (!ok) break;
                 }
-                if (!ok) break;
+                for (int t = 0; t < 2; ++t) nact[t] += (w.n_kv[t] > 0) ? 1 : 0;
             }
             // every MMA issued above completes before TMEM is released
             mma_commit_elect(drain);
@@ -270,163 +339,183 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
         const uint32_t s_addr = tmem + (static_cast<uint32_t>(base) << 16) + 128u * t;
         const uint32_t o_addr = s_addr + (C::O_COL + (D - 128) * t);
         const float cl2 = p.scale_log2;
-        // the Q tile with the most key tiles releases the K/V ring stages (it
-        // issues the last S of every key tile): tile 1 unless it lies past N
-        const bool releases = (t == (n_kv[1] > 0 ? 1 : 0)) && warp == 8 * t && lane == 0;
-        float m0 = -INFINITY, m1 = -INFINITY;  // running max (base 2) of rows rr0, rr0 + 8
-        float l0 = 0.f, l1 = 0.f;              // this thread's share of their running sums
+        int pc = 0;       // key tiles of this Q tile done over all items (s_full / p_full phases)
+        int oc = 0;       // items in which this Q tile was present (o_full phases)
+        int ring0 = 0;    // K/V ring slots used by earlier items
         bool ok = true;
-        const int nk = n_kv[t];
-        for (int j = 0; j < nk; ++j) {
-            if (!(ok = warp_wait(&s_full[t], j & 1, p.ctl))) break;
-            if (releases) {
-                // S_t(j) is complete, so is every MMA issued before it: K_j and
-                // V_{j-1} are consumed; hand their ring stages back to the producer
-                mbar_arrive(&kv_empty[(2 * j) % C::STAGES]);
-                if (j > 0) mbar_arrive(&kv_empty[(2 * j - 1) % C::STAGES]);
-            }
-            tc_fence_after();
-            float s[64];
-            auto load_s = [&]() {
-                tmem_ld_16x256b_x8(s_addr, reinterpret_cast<uint32_t*>(s));
-                tmem_ld_16x256b_x8(s_addr + 64, reinterpret_cast<uint32_t*>(s + 32));
-                tmem_wait_ld();
-                if (j == nk - 1) {
-                    // last key tile of this Q tile: causal diagonal and/or ragged tail
-                    const int tail = N - 1 - j * BN;
-                    const int lim0 = min(CAUSAL ? rr0 : BN - 1, tail);
-                    const int lim1 = min(CAUSAL ? rr0 + 8 : BN - 1, tail);
-#pragma unroll
-                    for (int n = 0; n < 16; ++n)
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int c = 8 * n + cg + e;
-                            if (c > lim0) s[4 * n + e] = -INFINITY;
-                            if (c > lim1) s[4 * n + 2 + e] = -INFINITY;
-                        }
+        for (int n = 0; ok; ++n) {
+            const int slot = n & 1;
+            if (!(ok = warp_wait(&item_full[slot], (n >> 1) & 1, p.ctl))) break;
+            const int item = *reinterpret_cast<volatile int*>(&item_buf[slot]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[slot]);
+            if (item < 0) break;
+            const Item w = decode_item<CAUSAL>(p, item);
+            // the Q tile with the most key tiles releases the K/V ring stages (it
+            // issues the last S of every key tile): tile 1 unless it lies past N
+            const bool releases = (t == (w.n_kv[1] > 0 ? 1 : 0)) && warp == 8 * t && lane == 0;
+            float m0 = -INFINITY, m1 = -INFINITY;  // running max (base 2) of rows rr0, rr0 + 8
+            float l0 = 0.f, l1 = 0.f;              // this thread's share of their running sums
+            const int nk = w.n_kv[t];
+            for (int j = 0; j < nk; ++j) {
+                if (!(ok = warp_wait(&s_full[t], pc & 1, p.ctl))) break;
+                if (releases) {
+                    // S_t(j) is complete, so is every MMA issued before it: K_j and
+                    // V_{j-1} (at j = 0 the previous item's last V) are consumed;
+                    // hand their ring stages back to the producer
+                    const int k_slot = ring0 + 2 * j;
+                    mbar_arrive(&kv_empty[k_slot % C::STAGES]);
+                    if (k_slot > 0) mbar_arrive(&kv_empty[(k_slot - 1) % C::STAGES]);
                 }
-            };
-            // row maxima (base 2) of rows rr0, rr0 + 8: two chains of three-input
-            // max per row, then the row's four threads (lanes 4(i/4) .. + 3)
-            auto row_max = [&](float& mx0, float& mx1) {
-                float x0 = fmaxf(s[0], s[1]), y0 = fmaxf(s[4], s[5]);
-                float x1 = fmaxf(s[2], s[3]), y1 = fmaxf(s[6], s[7]);
-#pragma unroll
-                for (int n = 2; n < 16; n += 2) {
-                    x0 = fmax3(x0, s[4 * n], s[4 * n + 1]);
-                    y0 = fmax3(y0, s[4 * n + 4], s[4 * n + 5]);
-                    x1 = fmax3(x1, s[4 * n + 2], s[4 * n + 3]);
-                    y1 = fmax3(y1, s[4 * n + 6], s[4 * n + 7]);
-                }
-                mx0 = fmaxf(x0, y0);
-                mx1 = fmaxf(x1, y1);
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2)) * cl2;
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2)) * cl2;
-            };
-            load_s();
-            // The exponentials use the running max as it stands: the row max of
-            // this tile is only taken (and m moved, O and l rescaled) when a
-            // thread's share of a row sum shows a score more than log2(SUM_LIMIT)
-            // above m.  Any reference m gives the same O / l and LSE in exact
-            // arithmetic, and each p is bounded by the share it is part of.  P
-            // stays in registers until then, so S is still intact in TMEM.
-            if (j == 0) row_max(m0, m1);
-            float al0 = 1.f, al1 = 1.f;
-            bool redo = false;
-            uint32_t pk[32];
-            float ts0, ts1;
-            for (;;) {
-                const float2 c2 = make_float2(cl2, cl2), n0 = make_float2(-m0, -m0), n1 = make_float2(-m1, -m1);
-                float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int n = 0; n < 16; ++n) {
-                    // one exponential in four on the FMA pipe, beside MUFU
-                    const float2 xa = ffma2(make_float2(s[4 * n], s[4 * n + 1]), c2, n0);
-                    const float2 xb = ffma2(make_float2(s[4 * n + 2], s[4 * n + 3]), c2, n1);
-                    const float2 pa = make_float2(ex2_approx(xa.x), ex2_approx(xa.y));
-                    const float2 pb = make_float2(ex2_approx(xb.x), ex2_fma(xb.y));
-                    sum0 = fadd2(sum0, pa);
-                    sum1 = fadd2(sum1, pb);
-                    // packed pairs in the 16x128b layout: column 4n + i%4
-                    pk[2 * n] = pack_bf16x2(pa.x, pa.y);
-                    pk[2 * n + 1] = pack_bf16x2(pb.x, pb.y);
-                }
-                ts0 = sum0.x + sum0.y;
-                ts1 = sum1.x + sum1.y;
-                if (redo || j == 0 || !__any_sync(0xffffffffu, !(ts0 <= SUM_LIMIT && ts1 <= SUM_LIMIT))) break;
-                // a score far above m in some row of this warp: take the true row
-                // maxima (the whole warp, so TMEM access stays warp-wide)
-                redo = true;
-                load_s();
-                float mx0, mx1;
-                row_max(mx0, mx1);
-                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                al0 = ex2_approx(m0 - mn0);
-                al1 = ex2_approx(m1 - mn1);
-                m0 = mn0;
-                m1 = mn1;
-            }
-            l0 = l0 * al0 + ts0;
-            l1 = l1 * al1 + ts1;
-            if (redo) {
-                // O_t holds sum_{j'<j} P V_j' (its MMA precedes this S in issue
-                // order, so S_t's commit covered it): rescale it in TMEM
-#pragma unroll
-                for (int cc = 0; cc < D; cc += 32) {
-                    uint32_t o[16];
-                    tmem_ld_16x256b_x4(o_addr + cc, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        o[4 * n] = __float_as_uint(__uint_as_float(o[4 * n]) * al0);
-                        o[4 * n + 1] = __float_as_uint(__uint_as_float(o[4 * n + 1]) * al0);
-                        o[4 * n + 2] = __float_as_uint(__uint_as_float(o[4 * n + 2]) * al1);
-                        o[4 * n + 3] = __float_as_uint(__uint_as_float(o[4 * n + 3]) * al1);
-                    }
-                    tmem_st_16x256b_x4(o_addr + cc, o);
-                }
-            }
-            tmem_st_16x128b_x16(s_addr, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&p_full[t]);
-        }
-        if (ok && nk > 0) {
-            ok = warp_wait(&o_full[t], 0, p.ctl);
-            if (ok) {
                 tc_fence_after();
-                // each row's sum is split over its four threads
-                l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-                l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-                l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-                l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-                const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-                const int row0 = q0 + t * BM + rr0, row1 = row0 + 8;
-                __nv_bfloat16* orow0 = p.o + (static_cast<size_t>(bh) * N + row0) * D;
-                __nv_bfloat16* orow1 = orow0 + 8 * D;
-#pragma unroll
-                for (int cc = 0; cc < D; cc += 32) {
-                    uint32_t o[16];
-                    tmem_ld_16x256b_x4(o_addr + cc, o);
+                float s[64];
+                auto load_s = [&]() {
+                    tmem_ld_16x256b_x8(s_addr, reinterpret_cast<uint32_t*>(s));
+                    tmem_ld_16x256b_x8(s_addr + 64, reinterpret_cast<uint32_t*>(s + 32));
                     tmem_wait_ld();
-#pragma unroll
-                    for (int n = 0; n < 4; ++n) {
-                        const int col = cc + 8 * n + cg;
-                        if (row0 < N)
-                            *reinterpret_cast<uint32_t*>(orow0 + col) =
-                                pack_bf16x2(__uint_as_float(o[4 * n]) * inv0, __uint_as_float(o[4 * n + 1]) * inv0);
-                        if (row1 < N)
-                            *reinterpret_cast<uint32_t*>(orow1 + col) = pack_bf16x2(
-                                __uint_as_float(o[4 * n + 2]) * inv1, __uint_as_float(o[4 * n + 3]) * inv1);
+                    if (j == nk - 1) {
+                        // last key tile of this Q tile: causal diagonal and/or ragged tail
+                        const int tail = N - 1 - j * BN;
+                        const int lim0 = min(CAUSAL ? rr0 : BN - 1, tail);
+                        const int lim1 = min(CAUSAL ? rr0 + 8 : BN - 1, tail);
+    #pragma unroll
+                        for (int n = 0; n < 16; ++n)
+    #pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int c = 8 * n + cg + e;
+                                if (c > lim0) s[4 * n + e] = -INFINITY;
+                                if (c > lim1) s[4 * n + 2 + e] = -INFINITY;
+                            }
+                    }
+                };
+                // row maxima (base 2) of rows rr0, rr0 + 8: two chains of three-input
+                // max per row, then the row's four threads (lanes 4(i/4) .. + 3)
+                auto row_max = [&](float& mx0, float& mx1) {
+                    float x0 = fmaxf(s[0], s[1]), y0 = fmaxf(s[4], s[5]);
+                    float x1 = fmaxf(s[2], s[3]), y1 = fmaxf(s[6], s[7]);
+    #pragma unroll
+                    for (int n = 2; n < 16; n += 2) {
+                        x0 = fmax3(x0, s[4 * n], s[4 * n + 1]);
+                        y0 = fmax3(y0, s[4 * n + 4], s[4 * n + 5]);
+                        x1 = fmax3(x1, s[4 * n + 2], s[4 * n + 3]);
+                        y1 = fmax3(y1, s[4 * n + 6], s[4 * n + 7]);
+                    }
+                    mx0 = fmaxf(x0, y0);
+                    mx1 = fmaxf(x1, y1);
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2)) * cl2;
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2)) * cl2;
+                };
+                load_s();
+                // The exponentials use the running max as it stands: the row max of
+                // this tile is only taken (and m moved, O and l rescaled) when a
+                // thread's share of a row sum shows a score more than log2(SUM_LIMIT)
+                // above m.  Any reference m gives the same O / l and LSE in exact
+                // arithmetic, and each p is bounded by the share it is part of.  P
+                // stays in registers until then, so S is still intact in TMEM.
+                if (j == 0) row_max(m0, m1);
+                float al0 = 1.f, al1 = 1.f;
+                bool redo = false;
+                uint32_t pk[32];
+                float ts0, ts1;
+                for (;;) {
+                    const float2 c2 = make_float2(cl2, cl2), n0 = make_float2(-m0, -m0), n1 = make_float2(-m1, -m1);
+                    float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
+    #pragma unroll
+                    for (int n = 0; n < 16; ++n) {
+                        // one exponential in four on the FMA pipe, beside MUFU
+                        const float2 xa = ffma2(make_float2(s[4 * n], s[4 * n + 1]), c2, n0);
+                        const float2 xb = ffma2(make_float2(s[4 * n + 2], s[4 * n + 3]), c2, n1);
+                        const float2 pa = make_float2(ex2_approx(xa.x), ex2_approx(xa.y));
+                        const float2 pb = make_float2(ex2_approx(xb.x), ex2_fma(xb.y));
+                        sum0 = fadd2(sum0, pa);
+                        sum1 = fadd2(sum1, pb);
+                        // packed pairs in the 16x128b layout: column 4n + i%4
+                        pk[2 * n] = pack_bf16x2(pa.x, pa.y);
+                        pk[2 * n + 1] = pack_bf16x2(pb.x, pb.y);
+                    }
+                    ts0 = sum0.x + sum0.y;
+                    ts1 = sum1.x + sum1.y;
+                    if (redo || j == 0 || !__any_sync(0xffffffffu, !(ts0 <= SUM_LIMIT && ts1 <= SUM_LIMIT))) break;
+                    // a score far above m in some row of this warp: take the true row
+                    // maxima (the whole warp, so TMEM access stays warp-wide)
+                    redo = true;
+                    load_s();
+                    float mx0, mx1;
+                    row_max(mx0, mx1);
+                    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                    al0 = ex2_approx(m0 - mn0);
+                    al1 = ex2_approx(m1 - mn1);
+                    m0 = mn0;
+                    m1 = mn1;
+                }
+                l0 = l0 * al0 + ts0;
+                l1 = l1 * al1 + ts1;
+                if (redo) {
+                    // O_t holds sum_{j'<j} P V_j' (its MMA precedes this S in issue
+                    // order, so S_t's commit covered it): rescale it in TMEM
+    #pragma unroll
+                    for (int cc = 0; cc < D; cc += 32) {
+                        uint32_t o[16];
+                        tmem_ld_16x256b_x4(o_addr + cc, o);
+                        tmem_wait_ld();
+    #pragma unroll
+                        for (int n = 0; n < 4; ++n) {
+                            o[4 * n] = __float_as_uint(__uint_as_float(o[4 * n]) * al0);
+                            o[4 * n + 1] = __float_as_uint(__uint_as_float(o[4 * n + 1]) * al0);
+                            o[4 * n + 2] = __float_as_uint(__uint_as_float(o[4 * n + 2]) * al1);
+                            o[4 * n + 3] = __float_as_uint(__uint_as_float(o[4 * n + 3]) * al1);
+                        }
+                        tmem_st_16x256b_x4(o_addr + cc, o);
                     }
                 }
-                if ((lane & 3) == 0) {
-                    if (row0 < N) p.lse[static_cast<size_t>(bh) * N + row0] = (m0 + __log2f(l0)) * LN2;
-                    if (row1 < N) p.lse[static_cast<size_t>(bh) * N + row1] = (m1 + __log2f(l1)) * LN2;
+                tmem_st_16x128b_x16(s_addr, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&p_full[t]);
+                ++pc;
+            }
+            if (ok && nk > 0) {
+                ok = warp_wait(&o_full[t], oc & 1, p.ctl);
+                ++oc;
+                if (ok) {
+                    tc_fence_after();
+                    // each row's sum is split over its four threads
+                    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+                    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+                    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+                    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+                    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+                    const int row0 = w.q0 + t * BM + rr0, row1 = row0 + 8;
+                    __nv_bfloat16* orow0 = p.o + (static_cast<size_t>(w.bh) * N + row0) * D;
+                    __nv_bfloat16* orow1 = orow0 + 8 * D;
+    #pragma unroll
+                    for (int cc = 0; cc < D; cc += 32) {
+                        uint32_t o[16];
+                        tmem_ld_16x256b_x4(o_addr + cc, o);
+                        tmem_wait_ld();
+    #pragma unroll
+                        for (int n = 0; n < 4; ++n) {
+                            const int col = cc + 8 * n + cg;
+                            if (row0 < N)
+                                *reinterpret_cast<uint32_t*>(orow0 + col) =
+                                    pack_bf16x2(__uint_as_float(o[4 * n]) * inv0, __uint_as_float(o[4 * n + 1]) * inv0);
+                            if (row1 < N)
+                                *reinterpret_cast<uint32_t*>(orow1 + col) = pack_bf16x2(
+                                    __uint_as_float(o[4 * n + 2]) * inv1, __uint_as_float(o[4 * n + 3]) * inv1);
+                        }
+                    }
+                    if ((lane & 3) == 0) {
+                        if (row0 < N) p.lse[static_cast<size_t>(w.bh) * N + row0] = (m0 + __log2f(l0)) * LN2;
+                        if (row1 < N) p.lse[static_cast<size_t>(w.bh) * N + row1] = (m1 + __log2f(l1)) * LN2;
+                    }
+                    // O_t has been read: the next item's first P V may overwrite it
+                    tc_fence_before();
+                    mbar_arrive(&o_free[t]);
                 }
             }
+            ring0 += 2 * w.n_kv_max;
         }
     }
 
@@ -435,6 +524,12 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     if (warp == MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+    // every CTA has taken its last item by now; the last one to get here
+    // returns the queue slot to {0, 0} for a later launch
+    if (threadIdx.x == 0 && atomicAdd(&queue[1], 1u) == gridDim.x - 1) {
+        atomicExch(&queue[0], 0u);
+        atomicExch(&queue[1], 0u);
     }
 }
 
@@ -445,8 +540,7 @@ cudaError_t launch(const FwdParams& p, cudaStream_t stream)
     auto kern = fwd_kernel<D, CAUSAL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_pairs, p.BH);
-    kern<<<grid, NTHREADS, C::SMEM_BYTES, stream>>>(p);
+    kern<<<p.n_ctas, NTHREADS, C::SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
 }
 

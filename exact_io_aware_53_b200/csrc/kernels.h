@@ -24,7 +24,9 @@ struct FwdParams {
     int BH;
     int N;
     int n_pairs;       // ceil(N / 256)
-    int group_heads;   // dispatch grouping of the (pair, head) grid, >= 1 (grouped_order)
+    int group_heads;   // grouping of the (pair, head) work items, >= 1 (grouped_order)
+    int n_ctas;        // persistent CTAs, <= min(SMs, B*H*n_pairs)
+    int queue_slot;    // work queue slot of this launch, < 64
     float scale_log2;  // scale * log2(e)
     WaitCtl ctl;
 };
