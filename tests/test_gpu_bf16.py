@@ -100,6 +100,28 @@ def test_late_dominant_key_moves_the_running_max(fa_lib, d, causal):
     assert max_abs(out["o"][0, 0, seen], v[0, 0, 400].float().expand(N - (400 if causal else 0), d)) <= BF16_TOL
 
 
+@pytest.mark.parametrize("d,causal", [(128, True), (64, False)])
+def test_forward_work_queue_survives_many_launches(fa_lib, d, causal):
+    """The persistent forward takes its work items from one of 64 queue slots
+    per launch, and the launch's last CTA returns the slot to zero.  150
+    launches in a row wrap the slots more than twice; every output must match
+    the first bit for bit (the forward's arithmetic has no atomics), and the
+    first must match the oracle."""
+    x = _inputs((2, 3, 700, d), seed=321 + d)
+    scale = 1 / math.sqrt(d)
+    xc = to_cuda(x)
+    o0, lse0 = fa_lib.fwd(xc["q"], xc["k"], xc["v"], causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    ro, rlse = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, causal)
+    assert max_abs(o0, ro) <= BF16_TOL
+    assert max_abs(lse0, rlse) <= LSE_TOL
+    outs = [fa_lib.fwd(xc["q"], xc["k"], xc["v"], causal=causal, scale=scale) for _ in range(149)]
+    torch.cuda.synchronize()
+    assert fa_lib.check_device_status() == 0
+    for o, lse in outs:
+        assert torch.equal(o, o0) and torch.equal(lse, lse0)
+
+
 def _d_rounding_bounds(x, scale, causal):
     """First-order effect on dQ and dK of forming D_i = <dO_i, O_i> from the bf16
     O the backward is given (the oracle uses D_i = sum_j P_ij dP_ij exactly).
