@@ -54,6 +54,11 @@ typedef enum {
  * reading of the pages' standard attention is 1/sqrt(d)).  causal: 0 or 1.
  * All pointers 16-byte aligned.  q/k/v may alias each other, o and lse must
  * not overlap any input.
+ * The kernel is persistent: one CTA per SM takes work items from a queue in
+ * the library's device memory (64 slots, one per launch in turn, returned to
+ * zero by each launch's last CTA).  Launches may run concurrently on several
+ * streams as long as fewer than 64 forward launches are in flight on a device
+ * at once.
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, void* stream);
