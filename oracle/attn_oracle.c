@@ -110,11 +110,9 @@ static double dot(const double* a, const double* b, long d)
  * One query row of one head: materialise the score row into srow (length N),
  * turn it into P in place, write O_i and LSE_i.
  */
-static void fwd_row(const double* qi, const double* k, const double* v, double* oi,
-                    double* lse_i, long i, long N, long d, double scale, int causal,
-                    double* srow)
+static void fwd_row_nk(const double* qi, const double* k, const double* v, double* oi,
+                       double* lse_i, long nk, long d, double scale, double* srow)
 {
-    long nk = n_allowed(i, N, causal);
     double m = -INFINITY;
     for (long j = 0; j < nk; ++j) {
         srow[j] = scale * dot(qi, k + j * d, d);
@@ -132,6 +130,14 @@ static void fwd_row(const double* qi, const double* k, const double* v, double* 
         for (long t = 0; t < d; ++t) oi[t] += p * vj[t];
     }
     *lse_i = m + log(l);
+}
+
+/* One query row i of a square [N x N] problem. */
+static void fwd_row(const double* qi, const double* k, const double* v, double* oi,
+                    double* lse_i, long i, long N, long d, double scale, int causal,
+                    double* srow)
+{
+    fwd_row_nk(qi, k, v, oi, lse_i, n_allowed(i, N, causal), d, scale, srow);
 }
 
 /* Forward over all heads and rows.  Returns 0, or -1 on bad sizes / no memory. */
@@ -154,6 +160,40 @@ int oracle_attn_fwd(const double* q, const double* k, const double* v, double* o
                 const long base = h * N * d;
                 fwd_row(q + base + i * d, k + base, v + base, o + base + i * d,
                         lse + h * N + i, i, N, d, scale, causal, srow);
+            }
+        free(srow);
+    }
+    return err;
+}
+
+/*
+ * Forward with Nq queries against Nk keys (q: [BH][Nq][d]; k, v: [BH][Nk][d];
+ * o: [BH][Nq][d]; lse: [BH][Nq]), the shape of decoding against a key/value
+ * cache.  Causal reading (the pages fix no convention for Nq != Nk): the
+ * queries are the last Nq positions of the sequence, so query i sees keys
+ * j <= Nk - Nq + i; this needs Nk >= Nq and gives the square mask when Nq = Nk.
+ * Returns 0, or -1 on bad sizes / no memory.
+ */
+int oracle_attn_fwd_rect(const double* q, const double* k, const double* v, double* o,
+                         double* lse, long BH, long Nq, long Nk, long d, double scale,
+                         int causal)
+{
+    if (BH < 0 || Nq < 0 || Nk < 1 || d < 1 || (causal && Nk < Nq)) return -1;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* srow = (double*)malloc((size_t)Nk * sizeof(double));
+        if (!srow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 16) collapse(2)
+        for (long h = 0; h < BH; ++h)
+            for (long i = 0; i < Nq; ++i) {
+                if (!srow) continue;
+                const long nk = causal ? Nk - Nq + i + 1 : Nk;
+                fwd_row_nk(q + (h * Nq + i) * d, k + h * Nk * d, v + h * Nk * d, o + (h * Nq + i) * d,
+                           lse + h * Nq + i, nk, d, scale, srow);
             }
         free(srow);
     }

@@ -49,6 +49,8 @@ def _load():
         lib.oracle_attn_fwd.restype = I
         lib.oracle_attn_fwd_rows.argtypes = [P, P, P, P, P, L, L, L, L, D, I]
         lib.oracle_attn_fwd_rows.restype = I
+        lib.oracle_attn_fwd_rect.argtypes = [P, P, P, P, P, L, L, L, L, D, I]
+        lib.oracle_attn_fwd_rect.restype = I
         lib.oracle_attn_fwd_tiled.argtypes = [P, P, P, P, P, L, L, L, D, I, L]
         lib.oracle_attn_fwd_tiled.restype = I
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, D, I]
@@ -110,6 +112,22 @@ def attn_fwd(q, k, v, scale: float, causal: bool):
                                  B * H, N, d, float(scale), int(bool(causal)))
     if rc != 0:
         raise RuntimeError("oracle_attn_fwd failed (%d)" % rc)
+    return o, lse
+
+
+def attn_fwd_rect(q, k, v, scale: float, causal: bool):
+    """Nq queries against Nk keys: q [B,H,Nq,d], k and v [B,H,Nk,d].  Causal:
+    query i sees keys j <= Nk - Nq + i (needs Nk >= Nq).  Returns (O, LSE)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    assert k.shape == (B, H, Nk, d) and v.shape == k.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, H, Nq))
+    rc = _load().oracle_attn_fwd_rect(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                      B * H, Nq, Nk, d, float(scale), int(bool(causal)))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd_rect failed (%d)" % rc)
     return o, lse
 
 

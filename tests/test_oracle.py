@@ -264,3 +264,73 @@ def test_bwd_kv_rows_matches_full_backward():
         rk, rv = oracle.attn_bwd_kv_rows(q[0, 0], k[0, 0], v[0, 0], g[0, 0], 9, 30, 0.4, causal)
         assert np.max(np.abs(rk - dk[0, 0, 9:30])) < 1e-14
         assert np.max(np.abs(rv - dv[0, 0, 9:30])) < 1e-14
+
+
+# ---------------------------------------------------------------- Nq queries against Nk keys
+# (the decode / split-KV shape).  Causal reading: the queries are the last Nq
+# positions, so query i sees keys j <= Nk - Nq + i.
+
+def _torch_attention_rect(q, k, v, scale, causal):
+    """Library brute force: torch fp64 softmax(Q K^T scale + mask) V with the
+    mask built by torch.tril on a rectangular matrix."""
+    q, k, v = (torch.as_tensor(np.asarray(t, dtype=np.float64)) for t in (q, k, v))
+    s = torch.matmul(q, k.transpose(-1, -2)) * scale
+    Nq, Nk = s.shape[-2], s.shape[-1]
+    if causal:
+        keep = torch.tril(torch.ones(Nq, Nk, dtype=torch.bool), diagonal=Nk - Nq)
+        s = s.masked_fill(~keep, float("-inf"))
+    return torch.matmul(torch.softmax(s, dim=-1), v).numpy(), torch.logsumexp(s, dim=-1).numpy()
+
+
+@pytest.mark.parametrize("Nq,Nk", [(1, 1), (1, 9), (3, 11), (7, 7), (5, 130)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rect_fwd_matches_library_bruteforce(Nq, Nk, causal):
+    q = _rand((2, 2, Nq, 6), seed=Nq * 31 + Nk)
+    k = _rand((2, 2, Nk, 6), seed=Nq * 37 + Nk)
+    v = _rand((2, 2, Nk, 6), seed=Nq * 41 + Nk)
+    o, lse = oracle.attn_fwd_rect(q, k, v, 0.4, causal)
+    ro, rlse = _torch_attention_rect(q, k, v, 0.4, causal)
+    assert np.max(np.abs(o - ro)) < 1e-12
+    assert np.max(np.abs(lse - rlse)) < 1e-12
+
+
+def test_rect_single_query_sees_every_key_even_causal():
+    """With one query the causal mask allows all Nk keys (j <= Nk - 1)."""
+    q, k, v = _rand((1, 3, 1, 8), 1), _rand((1, 3, 50, 8), 2), _rand((1, 3, 50, 8), 3)
+    o_c, lse_c = oracle.attn_fwd_rect(q, k, v, 0.3, True)
+    o_n, lse_n = oracle.attn_fwd_rect(q, k, v, 0.3, False)
+    assert np.array_equal(o_c, o_n) and np.array_equal(lse_c, lse_n)
+
+
+def test_rect_zero_queries_give_prefix_means():
+    """Q = 0: uniform weights over the allowed keys, so causal row i is the mean
+    of v[0 .. Nk - Nq + i] and LSE = ln(Nk - Nq + i + 1)."""
+    Nq, Nk = 4, 10
+    q = np.zeros((1, 1, Nq, 5))
+    k, v = _rand((1, 1, Nk, 5), 7), _rand((1, 1, Nk, 5), 8)
+    o, lse = oracle.attn_fwd_rect(q, k, v, 1.0, True)
+    for i in range(Nq):
+        n = Nk - Nq + i + 1
+        assert np.allclose(o[0, 0, i], v[0, 0, :n].mean(axis=0), atol=1e-14)
+        assert abs(lse[0, 0, i] - math.log(n)) < 1e-14
+
+
+def test_rect_with_nq_equal_nk_is_the_square_problem():
+    """Nq = Nk reduces the bottom-right mask to the square top-left one."""
+    q, k, v = _rand((2, 2, 9, 4), 11), _rand((2, 2, 9, 4), 12), _rand((2, 2, 9, 4), 13)
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd_rect(q, k, v, 0.5, causal)
+        ro, rlse = _torch_attention(q, k, v, 0.5, causal)
+        assert np.max(np.abs(o - ro)) < 1e-12 and np.max(np.abs(lse - rlse)) < 1e-12
+
+
+def test_rect_key_splits_combine_by_the_rescale_rule():
+    """Attention over disjoint key ranges, each with its own (O_s, LSE_s),
+    recombines exactly: LSE = ln sum_s e^{LSE_s}, O = sum_s e^{LSE_s - LSE} O_s
+    (the online-softmax update applied to whole blocks)."""
+    q, k, v = _rand((1, 2, 3, 6), 21), _rand((1, 2, 40, 6), 22), _rand((1, 2, 40, 6), 23)
+    o, lse = oracle.attn_fwd_rect(q, k, v, 0.7, False)
+    parts = [oracle.attn_fwd_rect(q, k[:, :, a:b], v[:, :, a:b], 0.7, False) for a, b in ((0, 13), (13, 14), (14, 40))]
+    L = np.log(sum(np.exp(p[1]) for p in parts))
+    O = sum(np.exp(p[1] - L)[..., None] * p[0] for p in parts)
+    assert np.max(np.abs(L - lse)) < 1e-12 and np.max(np.abs(O - o)) < 1e-12
