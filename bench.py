@@ -406,6 +406,173 @@ def run_e2e(args, w, fa, x, dev, stream, world):
             "steps": steps, "api": "fa_attention_host (pinned host buffers)"}
 
 
+# ------------------------------------------------------------------ decode (split-KV)
+
+DECODE_METRIC = "split-KV decode forward: HBM GB/s (q, k, v read + o, lse written) on 1 B200"
+DECODE_UNIT = "GB/s"
+
+
+def decode_oracle_sample(w, heads: int, seed: int):
+    """fp64 oracle rectangular forward on `heads` heads of decode workload w;
+    returns (seconds, algorithmic bytes of those heads, threads)."""
+    from exact_io_aware_53_b200.workloads import make_decode_inputs
+    from oracle import oracle
+    x = make_decode_inputs(w, seed=seed, B=1, H=heads)
+    t0 = time.perf_counter()
+    oracle.attn_fwd_rect(x["q"], x["k"], x["v"], w.scale, w.causal)
+    dt = time.perf_counter() - t0
+    return dt, w.bytes_min() / (w.B * w.H) * heads, oracle.num_threads()
+
+
+def decode_cpu_baseline(w, seed: int, budget_s: float = 10.0):
+    dt1, b1, thr = decode_oracle_sample(w, 1, seed)
+    heads = max(1, min(int(budget_s / max(dt1, 1e-3)), w.B * w.H))
+    dt, by, _ = decode_oracle_sample(w, heads, seed + 1)
+    return {"value": by / dt / 1e9, "unit": DECODE_UNIT, "cores": thr, "kind": "oracle",
+            "sample": "%d of %d heads (Nq=%d, Nk=%d, d=%d, causal=%s), fp64, %.2f s" % (
+                heads, w.B * w.H, w.Nq, w.Nk, w.d, w.causal, dt)}
+
+
+def run_reference_decode(args, w):
+    rank, world, _ = rank_env()
+    if rank != 0:
+        return 0
+    heads = min(8, w.B * w.H)
+    for i in range(args.warmup):
+        decode_oracle_sample(w, heads, w.seed + i)
+    times, by, thr = [], 0.0, 1
+    for i in range(args.steps):
+        dt, by, thr = decode_oracle_sample(w, heads, w.seed + 100 + i)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = by / (ms / 1e3) / 1e9
+    line = {"impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": 1, "H": heads, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                       "causal": w.causal, "sample": "%d heads per step" % heads, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": DECODE_UNIT, "cores": thr, "kind": "oracle",
+                             "sample": "%d heads of %s per step (fp64)" % (heads, w.name)},
+            "e2e": {"value": value, "unit": DECODE_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_decode(args, w):
+    """One step = fa_fwd_splitkv over the whole batch (range kernel + merge
+    kernel) with q and the key/value cache resident in device memory."""
+    import torch
+    from exact_io_aware_53_b200 import fa
+    from exact_io_aware_53_b200.workloads import make_decode_inputs
+
+    rank, world, local = rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        init_dist(world, "nccl", torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    x = make_decode_inputs(w, seed=rank_seed(w.seed, rank))
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    B, H, Nq, Nk, d = w.B, w.H, w.Nq, w.Nk, w.d
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    n_split = args.n_split
+    ws = torch.empty(max(16, fa.splitkv_workspace_bytes(B, H, Nq, Nk, d, n_split)), dtype=torch.uint8, device=dev)
+    launches = [0]
+
+    def step():
+        rc = fa.fwd_splitkv_raw(q, k, v, o, lse, ws, w.scale, w.causal, n_split)
+        launches[0] += fa.last_launch_count()
+        if rc:
+            raise fa.FAError(rc, "fa_fwd_splitkv")
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after warm-up: %s" % fa.status_string(st))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    launches[0] = 0
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after timing: %s" % fa.status_string(st))
+    ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ms = max_over_ranks(ms_local, world, dev)
+    by = w.bytes_min()
+    value = world * by / (ms / 1e3) / 1e9
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = by / (ms_local / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "fa_fwd_splitkv (range + merge kernels)", "achieved": achieved,
+                "peak": peak, "unit": DECODE_UNIT, "frac": achieved / peak, "peak_source": "hbm_gbs %s" % peak_src,
+                "algorithmic_bytes_per_launch": by, "ms_per_launch": ms_local,
+                "traffic": measured_traffic("decode", w.name),
+                "traffic_unit": "bytes per launch (ncu dram read+write)"}
+
+    # end to end: the query comes from pinned host memory and O, LSE go back
+    # each step; the key/value cache stays resident (it is the decoder's state)
+    e2e = None
+    if not args.no_e2e:
+        hq = x["q"].pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        steps = max(3, min(args.steps, 50))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
+        e2e = {"value": world * by / (ems / 1e3) / 1e9, "unit": DECODE_UNIT, "ms_per_step": ems,
+               "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size(),
+               "steps": steps, "api": "fa.fwd_splitkv_raw with q from and o, lse to pinned host memory; "
+                                      "key/value cache resident on the device"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = decode_cpu_baseline(w, seed=w.seed)
+    ranges = (Nk + 127) // 128 if n_split > (Nk + 127) // 128 else n_split
+    line = {"metric": DECODE_METRIC, "value": value, "unit": DECODE_UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "Nq": Nq, "Nk": Nk, "d": d, "causal": w.causal,
+                       "n_split": ranges if n_split else "library choice",
+                       "parallelism": "dp%d (independent batches per GPU, no collective)" % world,
+                       "l2": "inputs larger than L2 (k, v = %.0f MB per GPU)" % (B * H * Nk * d * 4 / 1e6)},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches[0], "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return line
+
+
 def probe_mma_rate():
     """Cycles per tcgen05 MMA instruction for the shapes the kernels issue
     (fa_selftest_umma_rate, one CTA per SM); printed as JSON lines."""
@@ -437,6 +604,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--n-split", type=int, default=0, help="key ranges for the decode workloads (0: library choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe-mma-rate", action="store_true", help="print the tcgen05 issue-rate table and exit")
@@ -444,13 +612,21 @@ def main(argv=None):
     if args.probe_mma_rate:
         probe_mma_rate()
         return 0
-    from exact_io_aware_53_b200.workloads import WORKLOADS
-    if args.workload != "all" and args.workload not in WORKLOADS:
-        ap.error("unknown workload %s (choose from %s)" % (args.workload, ", ".join(WORKLOADS)))
-    names = list(WORKLOADS) if args.workload == "all" else [args.workload]
+    from exact_io_aware_53_b200.workloads import DECODE_WORKLOADS, WORKLOADS
+    known = list(WORKLOADS) + list(DECODE_WORKLOADS)
+    if args.workload != "all" and args.workload not in known:
+        ap.error("unknown workload %s (choose from %s)" % (args.workload, ", ".join(known)))
+    names = known if args.workload == "all" else [args.workload]
     rc = 0
     try:
         for name in names:
+            if name in DECODE_WORKLOADS:
+                w = DECODE_WORKLOADS[name]
+                if args.impl == "reference":
+                    rc |= run_reference_decode(args, w)
+                else:
+                    run_decode(args, w)
+                continue
             w = WORKLOADS[name]
             if args.impl == "reference":
                 rc |= run_reference(args, w)

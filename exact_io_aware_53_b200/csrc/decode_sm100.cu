@@ -1,0 +1,372 @@
+// Split-KV forward for a few queries against a long key/value sequence (the
+// shape of decoding against a key/value cache), bf16 in / fp32 accumulate.
+//
+// Nq queries (one 128-row Q tile per CTA; TMA zero-fills rows past Nq) meet Nk
+// keys split into n_split ranges of whole 128-key tiles.  Each CTA runs the
+// forward's tile loop (S = Q K_j^T, online softmax, O += P V; "Tiling and the
+// online softmax", vibeengines.com/paper/flash-attention) over its range and
+// writes that range's normalised O_s (fp32) and LSE_s (natural log, -inf when
+// no key of the range is allowed).  A second kernel merges the ranges by the
+// same update rule applied to whole blocks ("The math, worked with real
+// numbers": a block with log-sum-exp L_s joins with weight e^{L_s - L}):
+//   L = ln sum_s e^{L_s},   O = sum_s e^{L_s - L} O_s.
+//
+// Causal reading for Nq != Nk: the queries are the last Nq positions, so query
+// i sees keys j <= Nk - Nq + i.
+//
+// The work is bound by reading K and V.  A CTA keeps one Q tile, so S and P
+// share TMEM without a second tile to ping-pong with; instead two CTAs share
+// an SM (96 KB shared memory, 256 TMEM columns each) and one's softmax runs
+// while the other's loads and MMAs do.
+//
+//   warp 5      TMA producer: Q tile, then K_j, V_j through a smem ring
+//   warp 4      MMA issuer (converged warp, elected lane)
+//   warps 0-3   softmax: thread = query row = TMEM lane
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace fa {
+namespace deck {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int NTHREADS = 192;
+constexpr int MMA_WARP = 4;
+constexpr int LOAD_WARP = 5;
+constexpr float RESCALE_LOG2 = 8.0f;  // move the running max only when it grows by more
+constexpr float LN2 = 0.6931471805599453f;
+
+template <int D>
+struct Cfg {
+    static constexpr int NDC = D / 64;
+    static constexpr int BOX_BYTES = 128 * 128;  // 128 rows x 64 bf16
+    static constexpr int TILE_BYTES = NDC * BOX_BYTES;
+    static constexpr int STAGES = (D == 128) ? 2 : 4;
+    static constexpr int Q_OFF = 0;
+    static constexpr int KV_OFF = TILE_BYTES;
+    static constexpr int BAR_OFF = KV_OFF + STAGES * TILE_BYTES;
+    static constexpr int NBARS = 1 + 2 * STAGES + 3 + 1;  // q, kv full/empty, s, p, o, drain
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
+    static constexpr uint32_t TMEM_COLS = 256;
+    static constexpr uint32_t O_COL = 128;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p)
+{
+    uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return reinterpret_cast<uint8_t*>((a + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c)
+{
+    bool ok = mbar_wait(bar, parity, c);
+    return __all_sync(0xffffffffu, ok);
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __grid_constant__ DecodeParams p)
+{
+    using C = Cfg<D>;
+    const int split = blockIdx.x, qt = blockIdx.y, bh = blockIdx.z;
+    const int Nq = p.Nq, Nk = p.Nk;
+    const int n_kv = (Nk + BN - 1) / BN;
+    // key tiles of this split, clipped to those the tile's last query row sees
+    const int j0 = split * p.tiles_per_split;
+    int j1 = min(n_kv, j0 + p.tiles_per_split);
+    const int row_last = min(Nq, (qt + 1) * BM) - 1;
+    if (CAUSAL) j1 = min(j1, (Nk - Nq + row_last) / BN + 1);
+    const size_t part_row0 = (static_cast<size_t>(split) * p.BH + bh) * Nq;
+    if (j0 >= j1) {
+        // no key of this range reaches this Q tile
+        for (int r = threadIdx.x; r < BM; r += NTHREADS) {
+            const int row = qt * BM + r;
+            if (row >= Nq) continue;
+            p.lse_part[part_row0 + row] = -INFINITY;
+            float4* op = reinterpret_cast<float4*>(p.o_part + (part_row0 + row) * D);
+            for (int c = 0; c < D / 4; ++c) op[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        return;
+    }
+    const int nj = j1 - j0;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* sQ = smem + C::Q_OFF;
+    uint8_t* sKV = smem + C::KV_OFF;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;
+    uint64_t* kv_empty = kv_full + C::STAGES;
+    uint64_t* s_full = kv_empty + C::STAGES;
+    uint64_t* p_full = s_full + 1;
+    uint64_t* o_full = p_full + 1;
+    uint64_t* drain = o_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    const int warp = static_cast<int>(warp_id());
+    const int lane = static_cast<int>(lane_id());
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(o_full, 1);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == LOAD_WARP && lane == 0) {
+        tma_prefetch_desc(&p.tm_q);
+        tma_prefetch_desc(&p.tm_k);
+        tma_prefetch_desc(&p.tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == LOAD_WARP) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+            for (int c = 0; c < C::NDC; ++c)
+                tma_load_3d(sQ + c * C::BOX_BYTES, &p.tm_q, q_full, c * 64, qt * BM, bh);
+            int it = 0;
+            bool ok = true;
+            for (int jj = 0; jj < nj && ok; ++jj) {
+                for (int kind = 0; kind < 2; ++kind) {
+                    const int s = it % C::STAGES;
+                    if (!mbar_wait(&kv_empty[s], ((it / C::STAGES) & 1) ^ 1, p.ctl)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
+                    const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
+                    for (int c = 0; c < C::NDC; ++c)
+                        tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64,
+                                    (j0 + jj) * BN, bh);
+                    ++it;
+                }
+            }
+            if (!ok) {
+                mbar_wait_drain(q_full, 0, p.ctl.limit_ns);
+                for (int i = max(0, it - C::STAGES); i < it; ++i)
+                    mbar_wait_drain(&kv_full[i % C::STAGES], (i / C::STAGES) & 1, p.ctl.limit_ns);
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA_WARP) {
+        // ------------------------------------------------------------ MMA issuer
+        // S and P share TMEM columns 0..127, so S of the next key tile is
+        // issued after the P V that reads this one's P
+        constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
+        constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
+        const uint32_t qa = smem_u32(sQ), kva = smem_u32(sKV);
+        auto issue_s = [&](int stage) {
+            const uint32_t kb = kva + stage * C::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+                mma_ss_elect(tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_s,
+                             kk > 0 ? 1u : 0u);
+            }
+        };
+        auto issue_o = [&](int stage, int jj) {
+            const uint32_t vb = kva + stage * C::TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+                mma_ts_elect(tmem + C::O_COL, tmem + kk * 8, sdesc_sw128(vb + kk * 2048, C::BOX_BYTES, 1024),
+                             idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+        };
+        int it = 0;
+        bool ok = warp_wait(q_full, 0, p.ctl);
+        if (ok && (ok = warp_wait(&kv_full[0], 0, p.ctl))) {
+            ++it;
+            tc_fence_after();
+            issue_s(0);
+            mma_commit_elect(s_full);
+        }
+        for (int jj = 0; jj < nj && ok; ++jj) {
+            const int sV = it % C::STAGES;
+            if (!(ok = warp_wait(&kv_full[sV], (it / C::STAGES) & 1, p.ctl))) break;
+            ++it;
+            if (!(ok = warp_wait(p_full, jj & 1, p.ctl))) break;
+            tc_fence_after();
+            issue_o(sV, jj);
+            if (jj + 1 < nj) {
+                const int sK = it % C::STAGES;
+                if (!(ok = warp_wait(&kv_full[sK], (it / C::STAGES) & 1, p.ctl))) break;
+                ++it;
+                tc_fence_after();
+                issue_s(sK);
+                mma_commit_elect(s_full);
+            } else {
+                mma_commit_elect(o_full);
+            }
+        }
+        mma_commit_elect(drain);
+        mbar_wait_drain(drain, 0, p.ctl.limit_ns);
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int r = warp * 32 + lane;
+        const int row = qt * BM + r;
+        // largest key index this row may see (rows past Nq are zero-filled padding)
+        const int key_max = CAUSAL ? min(Nk - 1, Nk - Nq + row) : Nk - 1;
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off;
+        const uint32_t o_addr = tmem + lane_off + C::O_COL;
+        const float cl2 = p.scale_log2;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int jj = 0; jj < nj; ++jj) {
+            if (!(ok = warp_wait(s_full, jj & 1, p.ctl))) break;
+            if (r == 0) {
+                // S(jj) is complete, so is every MMA issued before it: K_jj and
+                // V_{jj-1} are consumed; hand their ring stages back
+                mbar_arrive(&kv_empty[(2 * jj) % C::STAGES]);
+                if (jj > 0) mbar_arrive(&kv_empty[(2 * jj - 1) % C::STAGES]);
+            }
+            tc_fence_after();
+            float s[BN];
+#pragma unroll
+            for (int c = 0; c < BN; c += 32) tmem_ld32(s_addr + c, reinterpret_cast<uint32_t*>(s + c));
+            tmem_wait_ld();
+            const int limit = key_max - (j0 + jj) * BN;  // columns c <= limit are allowed
+            if (limit < BN - 1) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (c > limit) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+            const float m_blk = mx * cl2;
+            float alpha = 1.f;
+            if (m_blk > m + RESCALE_LOG2) {
+                // also the first tile with an allowed key (m = -inf gives alpha = 0)
+                alpha = ex2_approx(m - m_blk);
+                m = m_blk;
+            }
+            // while no key has been allowed m is -inf and every p is 0
+            const float m_use = (m == -INFINITY) ? 0.f : m;
+            uint32_t pk[BN / 2];
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < BN; c += 2) {
+                const float p0 = ex2_approx(fmaf(s[c], cl2, -m_use));
+                const float p1 = ex2_approx(fmaf(s[c + 1], cl2, -m_use));
+                sum += p0 + p1;
+                pk[c / 2] = pack_bf16x2(p0, p1);
+            }
+            l = l * alpha + sum;
+            if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                // O holds the earlier tiles' P V (their MMA precedes this S)
+#pragma unroll
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + cc, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(o_addr + cc, o);
+                }
+            }
+            tmem_st32(s_addr, pk);
+            tmem_st32(s_addr + BN / 4, pk + BN / 4);
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        if (ok && warp_wait(o_full, 0, p.ctl)) {
+            tc_fence_after();
+            const bool any = l > 0.f;
+            const float inv_l = any ? 1.f / l : 0.f;
+            float* op = p.o_part + (part_row0 + row) * D;
+#pragma unroll
+            for (int cc = 0; cc < D; cc += 32) {
+                uint32_t o[32];
+                tmem_ld32(o_addr + cc, o);
+                tmem_wait_ld();
+                if (row < Nq) {
+                    float4* d4 = reinterpret_cast<float4*>(op + cc);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        d4[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
+                                            __uint_as_float(o[4 * e + 2]) * inv_l,
+                                            __uint_as_float(o[4 * e + 3]) * inv_l);
+                }
+            }
+            if (row < Nq) p.lse_part[part_row0 + row] = any ? (m + __log2f(l)) * LN2 : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// One warp per query row: L = ln sum_s e^{L_s}, O = sum_s e^{L_s - L} O_s.
+template <int D>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p)
+{
+    constexpr int PER = D / 32;  // columns per lane
+    const int lane = static_cast<int>(threadIdx.x & 31);
+    const long long rid = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+    if (rid >= static_cast<long long>(p.BH) * p.Nq) return;
+    const size_t stride = static_cast<size_t>(p.BH) * p.Nq;  // between splits
+    float M = -INFINITY;
+    for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, p.lse_part[s * stride + rid]);
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    float W = 0.f;
+    for (int s = 0; s < p.n_split; ++s) {
+        const float L = p.lse_part[s * stride + rid];
+        if (L == -INFINITY) continue;
+        const float w = __expf(L - M);
+        W += w;
+        const float* op = p.o_part + (s * stride + rid) * D + lane * PER;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, op[e], acc[e]);
+    }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    __nv_bfloat16* out = p.o + rid * D + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; e += 2) *reinterpret_cast<uint32_t*>(out + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+    if (lane == 0) p.lse[rid] = W > 0.f ? M + __logf(W) : -INFINITY;
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch(const DecodeParams& p, cudaStream_t stream)
+{
+    using C = Cfg<D>;
+    auto kern = decode_partial_kernel<D, CAUSAL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.n_split, (p.Nq + BM - 1) / BM, p.BH);
+    kern<<<grid, NTHREADS, C::SMEM_BYTES, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const long long rows = static_cast<long long>(p.BH) * p.Nq;
+    decode_combine_kernel<D><<<static_cast<unsigned int>((rows + 3) / 4), 128, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace deck
+
+cudaError_t launch_decode_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream)
+{
+    if (d == 128) return causal ? deck::launch<128, true>(p, stream) : deck::launch<128, false>(p, stream);
+    return causal ? deck::launch<64, true>(p, stream) : deck::launch<64, false>(p, stream);
+}
+
+}  // namespace fa

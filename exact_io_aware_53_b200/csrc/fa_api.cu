@@ -244,6 +244,85 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     return st;
 }
 
+// ---------------------------------------------------------------- split-KV forward
+
+namespace {
+
+// Key ranges for the split-KV forward: the caller's count (capped at the number
+// of 128-key tiles), or about two CTAs per SM; 0 on bad sizes or device errors.
+int splitkv_ranges(int B, int H, int Nq, int Nk, int n_split)
+{
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || n_split < 0) return 0;
+    const int n_kv = (Nk + 127) / 128;
+    if (n_split > 0) return std::min(n_split, n_kv);
+    int dev = 0, n_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm < 1)
+        return 0;
+    const long long base = static_cast<long long>(B) * H * ((Nq + 127) / 128);
+    const long long want = (2ll * n_sm + base - 1) / base;
+    return static_cast<int>(std::max(1ll, std::min<long long>(want, n_kv)));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_split)
+{
+    const int s = splitkv_ranges(B, H, Nq, Nk, n_split);
+    if (s == 0 || d < 1) return 0;
+    const size_t rows = static_cast<size_t>(s) * B * H * Nq;
+    return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B, int H,
+                   int Nq, int Nk, int d, float scale, int causal, int n_split, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, std::max(Nq, Nk), d, scale, causal);
+    if (st != FA_OK) return st;
+    if (Nq < 1 || Nk < 1 || n_split < 0) return FA_ERR_INVALID_ARG;
+    if (causal && Nk < Nq) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    // grid (ranges, query tiles, heads): y and z are limited to 65535
+    if (static_cast<long long>(B) * H > 65535 || (Nq + 127) / 128 > 65535) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(workspace))
+        return FA_ERR_MISALIGNED;
+    const int s_req = splitkv_ranges(B, H, Nq, Nk, n_split);
+    if (s_req == 0) return FA_ERR_CUDA;
+    if ((st = get_encoder()) != FA_OK) return st;
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, Nq, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, Nk, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, Nk, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    // whole 128-key tiles per range; the last ranges may come out empty and
+    // are dropped (fewer ranges than the workspace was sized for)
+    const int n_kv = (Nk + 127) / 128;
+    p.tiles_per_split = (n_kv + s_req - 1) / s_req;
+    p.n_split = (n_kv + p.tiles_per_split - 1) / p.tiles_per_split;
+    const size_t rows = static_cast<size_t>(p.n_split) * BH * Nq;
+    p.o_part = static_cast<float*>(workspace);
+    p.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * d * sizeof(float)));
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.BH = static_cast<int>(BH);
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.scale_log2 = scale * kLog2e;
+    st = cuda_status(launch_decode_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 2;
+    return st;
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d)
 {
     if (B < 1 || H < 1 || N < 1 || d < 1) return 0;

@@ -38,6 +38,26 @@ cudaError_t launch_fwd_sm100(const FwdParams& p, int d, bool causal, cudaStream_
 // CTAs share through L2.  Host code (fa_api.cu).
 int choose_group_heads(int BH, int n_levels, const double* work, size_t bytes_per_head);
 
+// ---------------------------------------------------------------- split-KV forward (decode shape)
+struct DecodeParams {
+    CUtensorMap tm_q;   // {d, Nq, B*H}, box {64, 128, 1}, 128-byte swizzle
+    CUtensorMap tm_k;   // {d, Nk, B*H}
+    CUtensorMap tm_v;
+    float* o_part;      // [n_split][B*H][Nq][d] normalised partial outputs
+    float* lse_part;    // [n_split][B*H][Nq] natural log; -inf: no key of that range
+    __nv_bfloat16* o;   // [B*H][Nq][d]
+    float* lse;         // [B*H][Nq]
+    int BH;
+    int Nq;
+    int Nk;
+    int n_split;
+    int tiles_per_split;  // 128-key tiles per range
+    float scale_log2;
+    WaitCtl ctl;
+};
+// Partial kernel over (range, Q tile, head) plus the combine kernel.
+cudaError_t launch_decode_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream);
+
 // ---------------------------------------------------------------- bf16 backward
 struct BwdPreParams {
     const __nv_bfloat16* o;

@@ -40,6 +40,8 @@ _SIGS = {
     "fa_attention_host": ([P, P, P, P, P, P, P, P, P, P, SZ, I, I, I, I, F, I, P], I),
     "fa_check_device_status": ([P], I),
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
+    "fa_fwd_splitkv_workspace_bytes": ([I, I, I, I, I, I], ctypes.c_size_t),
+    "fa_fwd_splitkv": ([P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P], I),
     "fa_status_string": ([I], ctypes.c_char_p),
     "fa_last_launch_count": ([], I),
     "fa_last_cuda_error": ([], I),
@@ -126,6 +128,35 @@ def fwd_raw(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> int:
     B, H, N, d = _shape(q)
     return _lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale), int(causal),
                        _stream(stream))
+
+
+def splitkv_workspace_bytes(B: int, H: int, Nq: int, Nk: int, d: int, n_split: int = 0) -> int:
+    return int(_lib.fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, int(n_split)))
+
+
+def fwd_splitkv_raw(q, k, v, o, lse, workspace, scale: float, causal: bool, n_split: int = 0, stream=None) -> int:
+    """Enqueue the split-KV forward on preallocated tensors; returns the status code."""
+    B, H, Nq, d = (int(x) for x in q.shape)
+    return _lib.fa_fwd_splitkv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(workspace), B, H, Nq,
+                               int(k.shape[2]), d, float(scale), int(bool(causal)), int(n_split), _stream(stream))
+
+
+def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, n_split: int = 0, stream=None):
+    """O, LSE for Nq queries against Nk keys: q bf16 [B,H,Nq,d], k and v bf16
+    [B,H,Nk,d].  Causal: query i sees keys j <= Nk - Nq + i.  n_split key
+    ranges are processed in parallel and merged (0: the library picks)."""
+    _same(q, k, v, dtype=torch.bfloat16)
+    B, H, Nq, d = (int(x) for x in q.shape)
+    Nk = int(k.shape[2])
+    if tuple(k.shape) != (B, H, Nk, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must be [B, H, Nk, d] with q's B, H, d")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    ws = torch.empty(max(splitkv_workspace_bytes(B, H, Nq, Nk, d, n_split), 16), dtype=torch.uint8,
+                     device=q.device)
+    _check(fwd_splitkv_raw(q, k, v, o, lse, ws, scale, causal, n_split, stream), "fa_fwd_splitkv")
+    return o, lse
 
 
 def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None, stream=None):

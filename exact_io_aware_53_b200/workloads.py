@@ -58,6 +58,50 @@ WORKLOADS = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class DecodeWorkload:
+    """Nq queries per head against a resident cache of Nk keys and values."""
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def bytes_min(self) -> float:
+        """Bytes a split-KV forward must move at least: read q, k, v (bf16),
+        write o (bf16) and lse (fp32)."""
+        BH = self.B * self.H
+        return BH * (2.0 * self.Nq * self.d * 2 + 2.0 * self.Nk * self.d * 2 + 4.0 * self.Nq)
+
+
+# Decoding shapes (one query per head against a long cache).
+DECODE_WORKLOADS = {
+    "decode_bf16_8x16x1x16384x128_causal": DecodeWorkload("decode_bf16_8x16x1x16384x128_causal", 8, 16, 1, 16384, 128,
+                                                          True, seed=2001),
+}
+
+
+def make_decode_inputs(w: DecodeWorkload, seed: int | None = None, B: int | None = None, H: int | None = None):
+    """Draw (q, k, v) on the CPU for decode workload ``w``: fp32 standard
+    normals in the order q [B,H,Nq,d], k [B,H,Nk,d], v [B,H,Nk,d], rounded to
+    bf16."""
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    q = torch.randn((B, H, w.Nq, w.d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, H, w.Nk, w.d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, w.Nk, w.d), generator=g, dtype=torch.float32)
+    return {"q": q.to(torch.bfloat16), "k": k.to(torch.bfloat16), "v": v.to(torch.bfloat16)}
+
+
 def make_inputs(w: Workload, seed: int | None = None, B: int | None = None, H: int | None = None,
                 N: int | None = None):
     """Draw (q, k, v, dO) on the CPU for workload ``w`` (shape overrides allowed).

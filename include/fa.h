@@ -170,6 +170,28 @@ int fa_check_device_status(void* stream);
  * library (default 2e9).  Values below 1e6 are raised to 1e6.  Process-wide. */
 void fa_set_wait_limit_ns(unsigned long long ns);
 
+/*
+ * Split-KV forward, bf16: Nq queries against Nk keys, the shape of decoding
+ * against a key/value cache (no counterpart as an interface on the pages; the
+ * operation is the same exact attention, "Tiling and the online softmax").
+ *   q: bf16 [B][H][Nq][d]; k, v: bf16 [B][H][Nk][d]; o: bf16 [B][H][Nq][d];
+ *   lse: fp32 [B][H][Nq] (natural log).  d = 64 or 128; Nq, Nk >= 1.
+ *   causal: the queries are the last Nq positions, query i sees keys
+ *   j <= Nk - Nq + i; requires Nk >= Nq.
+ *   The Nk keys are split into n_split ranges of whole 128-key tiles processed
+ *   in parallel (0: the library picks about two CTAs per SM); each range's
+ *   (O, LSE) goes to `workspace` and a second kernel merges them by the
+ *   online-softmax rule.  workspace: device, 16-byte aligned, at least
+ *   fa_fwd_splitkv_workspace_bytes(B, H, Nq, Nk, d, n_split) bytes, computed
+ *   with the same device current (0 for an invalid shape); caller-owned,
+ *   needs no initialisation.  Errors as for fa_fwd, plus FA_ERR_INVALID_ARG
+ *   for causal with Nk < Nq or n_split < 0, and FA_ERR_UNSUPPORTED for
+ *   B*H > 65535.  Two kernels are enqueued on `stream`.
+ */
+size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_split);
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B, int H,
+                   int Nq, int Nk, int d, float scale, int causal, int n_split, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* fa_status_string(int status);
 

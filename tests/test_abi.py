@@ -110,3 +110,31 @@ def test_selftest_argument_errors(lib):
     assert f(P(16), P(16), P(16), 64, 64, 64, 0, 0, 0, 0, P(0)) == lib.FA_ERR_UNSUPPORTED
     assert f(P(16), P(16), P(16), 128, 64, 64, 1, 0, 1, 0, P(0)) == lib.FA_ERR_UNSUPPORTED
     assert f(P(0), P(16), P(16), 128, 64, 64, 0, 0, 0, 0, P(0)) == lib.FA_ERR_INVALID_ARG
+
+
+def test_splitkv_argument_errors(lib):
+    f = lib._lib.fa_fwd_splitkv
+    P = ctypes.c_void_p
+    ptrs = [P(16)] * 6
+
+    def call(B=1, H=1, Nq=1, Nk=256, d=128, scale=0.1, causal=0, n_split=0):
+        return f(*ptrs, B, H, Nq, Nk, d, scale, causal, n_split, P(0))
+
+    assert f(P(0), *ptrs[1:], 1, 1, 1, 256, 128, 0.1, 0, 0, P(0)) == lib.FA_ERR_INVALID_ARG
+    assert call(Nq=0) == lib.FA_ERR_INVALID_ARG
+    assert call(Nk=0) == lib.FA_ERR_INVALID_ARG
+    assert call(n_split=-1) == lib.FA_ERR_INVALID_ARG
+    assert call(causal=1, Nq=300, Nk=299) == lib.FA_ERR_INVALID_ARG
+    assert call(causal=2) == lib.FA_ERR_INVALID_ARG
+    assert call(d=96) == lib.FA_ERR_UNSUPPORTED
+    assert call(B=300, H=300) == lib.FA_ERR_UNSUPPORTED
+    assert f(*ptrs[:5], P(8), 1, 1, 1, 256, 128, 0.1, 0, 0, P(0)) == lib.FA_ERR_MISALIGNED
+
+
+def test_splitkv_workspace_size(lib):
+    ws = lib._lib.fa_fwd_splitkv_workspace_bytes
+    # explicit n_split needs no device: ranges are clipped to the 128-key tiles
+    assert ws(2, 3, 5, 1000, 128, 4) == ((4 * 2 * 3 * 5 * 128 * 4 + 255) // 256 + (4 * 2 * 3 * 5 * 4 + 255) // 256) * 256
+    assert ws(1, 1, 1, 100, 64, 8) == ws(1, 1, 1, 100, 64, 1)  # one tile: one range
+    assert ws(1, 1, 0, 100, 64, 1) == 0
+    assert ws(1, 1, 1, 100, 64, -1) == 0
