@@ -67,6 +67,9 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __grid_constant__ DecodeParams p)
 {
     using C = Cfg<D>;
+    // the merge kernel may be scheduled once every range CTA is running; it
+    // still waits for this grid's completion before it reads anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int split = blockIdx.x, qt = blockIdx.y, bh = blockIdx.z;
     const int Nq = p.Nq, Nk = p.Nk;
     const int n_kv = (Nk + BN - 1) / BN;
@@ -316,29 +319,53 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
 }
 
 // One warp per query row: L = ln sum_s e^{L_s}, O = sum_s e^{L_s - L} O_s.
+// Lane t holds the LSE of ranges t, t+32, ...; the weights are broadcast and
+// every lane accumulates D/32 columns over all ranges.  Launched as a
+// programmatic dependent of the range kernel: it waits for that grid's
+// results before the first read.
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p)
 {
     constexpr int PER = D / 32;  // columns per lane
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int lane = static_cast<int>(threadIdx.x & 31);
     const long long rid = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
     if (rid >= static_cast<long long>(p.BH) * p.Nq) return;
-    const size_t stride = static_cast<size_t>(p.BH) * p.Nq;  // between splits
+    const size_t stride = static_cast<size_t>(p.BH) * p.Nq;  // between ranges
     float M = -INFINITY;
-    for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, p.lse_part[s * stride + rid]);
+    for (int s = lane; s < p.n_split; s += 32) M = fmaxf(M, p.lse_part[s * stride + rid]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float acc[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) acc[e] = 0.f;
     float W = 0.f;
-    for (int s = 0; s < p.n_split; ++s) {
-        const float L = p.lse_part[s * stride + rid];
-        if (L == -INFINITY) continue;
-        const float w = __expf(L - M);
+    for (int s0 = 0; s0 < p.n_split; s0 += 32) {
+        const int s = s0 + lane;
+        const float L = s < p.n_split ? p.lse_part[s * stride + rid] : -INFINITY;
+        // a range no key of which the row may see has L = -inf and O_s = 0
+        const float w = L == -INFINITY ? 0.f : __expf(L - M);
         W += w;
-        const float* op = p.o_part + (s * stride + rid) * D + lane * PER;
-#pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, op[e], acc[e]);
+        const int cnt = min(32, p.n_split - s0);
+#pragma unroll 8
+        for (int jn = 0; jn < cnt; ++jn) {
+            const float wj = __shfl_sync(0xffffffffu, w, jn);
+            const float* op = p.o_part + ((s0 + jn) * stride + rid) * D + lane * PER;
+            if constexpr (PER == 4) {
+                const float4 x = *reinterpret_cast<const float4*>(op);
+                acc[0] = fmaf(wj, x.x, acc[0]);
+                acc[1] = fmaf(wj, x.y, acc[1]);
+                acc[2] = fmaf(wj, x.z, acc[2]);
+                acc[3] = fmaf(wj, x.w, acc[3]);
+            } else {
+                const float2 x = *reinterpret_cast<const float2*>(op);
+                acc[0] = fmaf(wj, x.x, acc[0]);
+                acc[1] = fmaf(wj, x.y, acc[1]);
+            }
+        }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
     const float inv = W > 0.f ? 1.f / W : 0.f;
     __nv_bfloat16* out = p.o + rid * D + lane * PER;
 #pragma unroll
@@ -357,8 +384,17 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t stream)
     kern<<<grid, NTHREADS, C::SMEM_BYTES, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const long long rows = static_cast<long long>(p.BH) * p.Nq;
-    decode_combine_kernel<D><<<static_cast<unsigned int>((rows + 3) / 4), 128, 0, stream>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned int>((rows + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
 }
 
 }  // namespace deck

@@ -259,8 +259,10 @@ int splitkv_ranges(int B, int H, int Nq, int Nk, int n_split)
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm < 1)
         return 0;
+    // as many ranges as keep every range CTA in one wave (two fit on an SM):
+    // a second, partly filled wave costs more than the longer ranges do
     const long long base = static_cast<long long>(B) * H * ((Nq + 127) / 128);
-    const long long want = (2ll * n_sm + base - 1) / base;
+    const long long want = (2ll * n_sm) / base;
     return static_cast<int>(std::max(1ll, std::min<long long>(want, n_kv)));
 }
 

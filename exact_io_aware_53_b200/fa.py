@@ -145,7 +145,8 @@ def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, n_spl
     """O, LSE for Nq queries against Nk keys: q bf16 [B,H,Nq,d], k and v bf16
     [B,H,Nk,d].  Causal: query i sees keys j <= Nk - Nq + i.  n_split key
     ranges are processed in parallel and merged (0: the library picks)."""
-    _same(q, k, v, dtype=torch.bfloat16)
+    _same(q, dtype=torch.bfloat16)
+    _same(k, v, dtype=torch.bfloat16)
     B, H, Nq, d = (int(x) for x in q.shape)
     Nk = int(k.shape[2])
     if tuple(k.shape) != (B, H, Nk, d) or tuple(v.shape) != tuple(k.shape):
