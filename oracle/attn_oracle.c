@@ -201,6 +201,72 @@ int oracle_attn_fwd_rect(const double* q, const double* k, const double* v, doub
 }
 
 /*
+ * Block-sparse forward: the square problem restricted to the (query block, key
+ * block) pairs a block mask allows.  The pages name block-sparse FlashAttention
+ * as the approximate extension of the method (guide, "Prerequisites"); the
+ * approximation is the mask itself, and over the allowed pairs this is the
+ * definition above with every other score at -inf (weight exactly 0).
+ *   mask: uint8 [Hm][nqb][nkb], nqb = ceil(N / br), nkb = ceil(N / bc); the
+ *   head h of row block bh uses mask + (bh % H) * mask_h_stride (stride 0: one
+ *   mask for every head).  Key j is allowed for query i iff
+ *   mask[(i / br) * nkb + j / bc] != 0 and, when causal, j <= i.
+ * A row that no key is allowed for gets O = 0 and LSE = -inf (a reading: the
+ * pages do not say).  Returns 0, or -1 on bad sizes / no memory.
+ */
+int oracle_attn_fwd_blockmask(const double* q, const double* k, const double* v, double* o,
+                              double* lse, long BH, long H, long N, long d, double scale,
+                              int causal, const unsigned char* mask, long mask_h_stride,
+                              long br, long bc)
+{
+    if (BH < 0 || H < 1 || N < 0 || d < 1 || br < 1 || bc < 1 || mask_h_stride < 0 || !mask)
+        return -1;
+    const long nkb = (N + bc - 1) / bc;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* srow = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+        if (!srow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 16) collapse(2)
+        for (long h = 0; h < BH; ++h)
+            for (long i = 0; i < N; ++i) {
+                if (!srow) continue;
+                const unsigned char* mrow = mask + (h % H) * mask_h_stride + (i / br) * nkb;
+                const double* qi = q + (h * N + i) * d;
+                const double* kh = k + h * N * d;
+                const double* vh = v + h * N * d;
+                double* oi = o + (h * N + i) * d;
+                double m = -INFINITY;
+                for (long j = 0; j < N; ++j) {
+                    const int allowed = mrow[j / bc] != 0 && (!causal || j <= i);
+                    srow[j] = allowed ? scale * dot(qi, kh + j * d, d) : -INFINITY;
+                    if (srow[j] > m) m = srow[j];
+                }
+                for (long t = 0; t < d; ++t) oi[t] = 0.0;
+                if (m == -INFINITY) {
+                    lse[h * N + i] = -INFINITY;
+                    continue;
+                }
+                double l = 0.0;
+                for (long j = 0; j < N; ++j) {
+                    srow[j] = srow[j] == -INFINITY ? 0.0 : exp(srow[j] - m);
+                    l += srow[j];
+                }
+                for (long j = 0; j < N; ++j) {
+                    if (srow[j] == 0.0) continue;
+                    const double pj = srow[j] / l;
+                    for (long t = 0; t < d; ++t) oi[t] += pj * vh[j * d + t];
+                }
+                lse[h * N + i] = m + log(l);
+            }
+        free(srow);
+    }
+    return err;
+}
+
+/*
  * Forward for rows [i0, i1) of ONE head (q, k, v point at that head's [N][d]
  * block; o / lse receive i1 - i0 rows).  Used to check sampled rows of
  * workloads too large to run whole.

@@ -51,6 +51,8 @@ def _load():
         lib.oracle_attn_fwd_rows.restype = I
         lib.oracle_attn_fwd_rect.argtypes = [P, P, P, P, P, L, L, L, L, D, I]
         lib.oracle_attn_fwd_rect.restype = I
+        lib.oracle_attn_fwd_blockmask.argtypes = [P, P, P, P, P, L, L, L, L, D, I, P, L, L, L]
+        lib.oracle_attn_fwd_blockmask.restype = I
         lib.oracle_attn_fwd_tiled.argtypes = [P, P, P, P, P, L, L, L, D, I, L]
         lib.oracle_attn_fwd_tiled.restype = I
         lib.oracle_attn_bwd.argtypes = [P, P, P, P, P, P, P, L, L, L, D, I]
@@ -128,6 +130,29 @@ def attn_fwd_rect(q, k, v, scale: float, causal: bool):
                                       B * H, Nq, Nk, d, float(scale), int(bool(causal)))
     if rc != 0:
         raise RuntimeError("oracle_attn_fwd_rect failed (%d)" % rc)
+    return o, lse
+
+
+def attn_fwd_blockmask(q, k, v, scale: float, causal: bool, mask, br: int = 128, bc: int = 128):
+    """Square attention restricted to a block mask: q, k, v [B,H,N,d]; mask
+    uint8-like [Hm, ceil(N/br), ceil(N/bc)] with Hm = 1 (shared) or H.  Key j is
+    allowed for query i iff mask[h, i // br, j // bc] and (not causal or
+    j <= i).  Rows with no allowed key: O = 0, LSE = -inf.  Returns (O, LSE)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    assert k.shape == q.shape and v.shape == q.shape
+    m = np.ascontiguousarray(np.asarray(mask.cpu() if hasattr(mask, "cpu") else mask) != 0, dtype=np.uint8)
+    if m.ndim == 2:
+        m = m[None]
+    nqb, nkb = -(-N // br), -(-N // bc)
+    assert m.shape[1:] == (nqb, nkb) and m.shape[0] in (1, H), m.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, H, N))
+    rc = _load().oracle_attn_fwd_blockmask(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B * H, H, N, d,
+                                           float(scale), int(bool(causal)), m.ctypes.data_as(ctypes.c_void_p),
+                                           0 if m.shape[0] == 1 else nqb * nkb, br, bc)
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd_blockmask failed (%d)" % rc)
     return o, lse
 
 

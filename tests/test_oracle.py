@@ -334,3 +334,84 @@ def test_rect_key_splits_combine_by_the_rescale_rule():
     L = np.log(sum(np.exp(p[1]) for p in parts))
     O = sum(np.exp(p[1] - L)[..., None] * p[0] for p in parts)
     assert np.max(np.abs(L - lse)) < 1e-12 and np.max(np.abs(O - o)) < 1e-12
+
+
+# ---------------------------------------------------------------- block-sparse
+# Square attention restricted to the (query block, key block) pairs a block
+# mask allows; rows with no allowed key give O = 0, LSE = -inf.
+
+def _torch_attention_blockmask(q, k, v, scale, causal, mask, br, bc):
+    """Library brute force: the block mask expanded to an element mask with
+    torch.repeat_interleave, then fp64 softmax(Q K^T scale + mask) V."""
+    q, k, v = (torch.as_tensor(np.asarray(t, dtype=np.float64)) for t in (q, k, v))
+    N = q.shape[-2]
+    m = torch.as_tensor(np.asarray(mask) != 0)
+    if m.dim() == 2:
+        m = m[None]
+    keep = m.repeat_interleave(br, dim=1)[:, :N].repeat_interleave(bc, dim=2)[:, :, :N]  # [Hm, N, N]
+    if causal:
+        keep = keep & torch.tril(torch.ones(N, N, dtype=torch.bool))
+    s = (torch.matmul(q, k.transpose(-1, -2)) * scale).masked_fill(~keep, float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    p = torch.softmax(s, dim=-1).nan_to_num(0.0)  # a row with no allowed key: all -inf
+    return torch.matmul(p, v).numpy(), lse.numpy()
+
+
+@pytest.mark.parametrize("N,br,bc", [(7, 2, 3), (12, 4, 4), (13, 5, 2), (9, 9, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("per_head", [False, True])
+def test_blockmask_matches_library_bruteforce(N, br, bc, causal, per_head):
+    H = 3
+    q, k, v = (_rand((2, H, N, 5), seed=N * 7 + br + 10 * s) for s in range(3))
+    nqb, nkb = -(-N // br), -(-N // bc)
+    rng = np.random.default_rng(N * 13 + bc)
+    mask = (rng.random((H if per_head else 1, nqb, nkb)) < 0.5).astype(np.uint8)
+    mask[0, 0, :] = 0  # the first query block of head 0 sees nothing
+    o, lse = oracle.attn_fwd_blockmask(q, k, v, 0.6, causal, mask, br, bc)
+    ro, rlse = _torch_attention_blockmask(q, k, v, 0.6, causal, mask, br, bc)
+    assert np.max(np.abs(o - ro)) < 1e-12
+    assert np.array_equal(np.isinf(lse), np.isinf(rlse))
+    fin = np.isfinite(rlse)
+    assert np.max(np.abs(lse[fin] - rlse[fin]), initial=0.0) < 1e-12
+    assert np.all(o[0, 0, :br] == 0.0) and np.all(lse[0, 0, :br] == -np.inf)
+
+
+def test_blockmask_zero_queries_give_the_mean_of_the_chosen_key_block():
+    """Q = 0 and one key block per query block: uniform weights over that
+    block's keys, so O_i is their mean and LSE_i = ln(block size)."""
+    N, br, bc = 20, 4, 6
+    q = np.zeros((1, 1, N, 3))
+    k, v = _rand((1, 1, N, 3), 31), _rand((1, 1, N, 3), 32)
+    nqb, nkb = N // br, -(-N // bc)
+    mask = np.zeros((1, nqb, nkb), dtype=np.uint8)
+    for qb in range(nqb):
+        mask[0, qb, (3 * qb + 1) % nkb] = 1
+    o, lse = oracle.attn_fwd_blockmask(q, k, v, 1.0, False, mask, br, bc)
+    for i in range(N):
+        kb = (3 * (i // br) + 1) % nkb
+        keys = v[0, 0, kb * bc:min(N, (kb + 1) * bc)]
+        assert np.allclose(o[0, 0, i], keys.mean(axis=0), atol=1e-14)
+        assert abs(lse[0, 0, i] - math.log(len(keys))) < 1e-14
+
+
+def test_blockmask_all_ones_and_lower_triangle_reduce_to_dense():
+    q, k, v = (_rand((1, 2, 23, 4), 40 + s) for s in range(3))
+    ones = np.ones((1, 3, 3), dtype=np.uint8)
+    lower = np.tril(ones[0])[None]
+    for causal, mask in ((False, ones), (True, ones), (True, lower)):
+        o, lse = oracle.attn_fwd_blockmask(q, k, v, 0.5, causal, mask, 8, 8)
+        ro, rlse = _torch_attention(q, k, v, 0.5, causal)
+        assert np.max(np.abs(o - ro)) < 1e-12 and np.max(np.abs(lse - rlse)) < 1e-12
+
+
+def test_blockmask_block_diagonal_is_independent_blocks():
+    """A block-diagonal mask splits the problem into independent attentions,
+    one per block (computed here by slicing the inputs)."""
+    N, b = 18, 6
+    q, k, v = (_rand((1, 1, N, 4), 50 + s) for s in range(3))
+    mask = np.eye(N // b, dtype=np.uint8)[None]
+    o, lse = oracle.attn_fwd_blockmask(q, k, v, 0.8, False, mask, b, b)
+    for t in range(N // b):
+        sl = slice(t * b, (t + 1) * b)
+        ro, rlse = _torch_attention(q[:, :, sl], k[:, :, sl], v[:, :, sl], 0.8, False)
+        assert np.max(np.abs(o[:, :, sl] - ro)) < 1e-12 and np.max(np.abs(lse[:, :, sl] - rlse)) < 1e-12
