@@ -14,6 +14,13 @@
 // Causal reading for Nq != Nk: the queries are the last Nq positions, so query
 // i sees keys j <= Nk - Nq + i.
 //
+// Block-sparse variant (SPARSE): the square problem restricted to the (query
+// tile, key tile) pairs a block mask allows, the approximate extension the
+// pages name ("Block-sparse FlashAttention").  The CTA of Q tile i compacts
+// row i of the mask into a key-tile list in shared memory and runs the same
+// loop over the listed tiles only; one range per Q tile, output written
+// directly.
+//
 // The work is bound by reading K and V.  A CTA keeps one Q tile, so S and P
 // share TMEM without a second tile to ping-pong with; instead two CTAs share
 // an SM (96 KB shared memory, 256 TMEM columns each) and one's softmax runs
@@ -36,7 +43,7 @@ constexpr int LOAD_WARP = 5;
 constexpr float RESCALE_LOG2 = 8.0f;  // move the running max only when it grows by more
 constexpr float LN2 = 0.6931471805599453f;
 
-template <int D>
+template <int D, bool SPARSE>
 struct Cfg {
     static constexpr int NDC = D / 64;
     static constexpr int BOX_BYTES = 128 * 128;  // 128 rows x 64 bf16
@@ -46,7 +53,9 @@ struct Cfg {
     static constexpr int KV_OFF = TILE_BYTES;
     static constexpr int BAR_OFF = KV_OFF + STAGES * TILE_BYTES;
     static constexpr int NBARS = 1 + 2 * STAGES + 3 + 1;  // q, kv full/empty, s, p, o, drain
-    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;
+    static constexpr int LIST_OFF = BAR_OFF + NBARS * 8 + 16;  // key-tile list (SPARSE)
+    static constexpr int LIST_BYTES = SPARSE ? kMaxMaskKeyTiles * 2 : 0;
+    static constexpr int SMEM_BYTES = LIST_OFF + LIST_BYTES + 1024;
     static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t O_COL = 128;
 };
@@ -63,31 +72,56 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __grid_constant__ DecodeParams p)
+// Writes the rows of Q tile qt that see no key of this range: O = 0, LSE = -inf.
+template <int D>
+__device__ void write_empty_rows(const DecodeParams& p, int qt, int bh, size_t part_row0)
 {
-    using C = Cfg<D>;
-    // the merge kernel may be scheduled once every range CTA is running; it
-    // still waits for this grid's completion before it reads anything
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int split = blockIdx.x, qt = blockIdx.y, bh = blockIdx.z;
-    const int Nq = p.Nq, Nk = p.Nk;
-    const int n_kv = (Nk + BN - 1) / BN;
-    // key tiles of this split, clipped to those the tile's last query row sees
-    const int j0 = split * p.tiles_per_split;
-    int j1 = min(n_kv, j0 + p.tiles_per_split);
-    const int row_last = min(Nq, (qt + 1) * BM) - 1;
-    if (CAUSAL) j1 = min(j1, (Nk - Nq + row_last) / BN + 1);
-    const size_t part_row0 = (static_cast<size_t>(split) * p.BH + bh) * Nq;
-    if (j0 >= j1) {
-        // no key of this range reaches this Q tile
-        for (int r = threadIdx.x; r < BM; r += NTHREADS) {
-            const int row = qt * BM + r;
-            if (row >= Nq) continue;
+    for (int r = threadIdx.x; r < BM; r += NTHREADS) {
+        const int row = qt * BM + r;
+        if (row >= p.Nq) continue;
+        if (p.direct) {
+            const size_t g = static_cast<size_t>(bh) * p.Nq + row;
+            p.lse[g] = -INFINITY;
+            uint4* op = reinterpret_cast<uint4*>(p.o + g * D);
+            for (int c = 0; c < D / 8; ++c) op[c] = make_uint4(0u, 0u, 0u, 0u);
+        } else {
             p.lse_part[part_row0 + row] = -INFINITY;
             float4* op = reinterpret_cast<float4*>(p.o_part + (part_row0 + row) * D);
             for (int c = 0; c < D / 4; ++c) op[c] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
+    }
+}
+
+template <int D, bool CAUSAL, bool SPARSE>
+__global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __grid_constant__ DecodeParams p)
+{
+    using C = Cfg<D, SPARSE>;
+    // the merge kernel may be scheduled once every range CTA is running; it
+    // still waits for this grid's completion before it reads anything
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int split = blockIdx.x, bh = blockIdx.z;
+    // block-sparse causal rows grow with the tile index: start the longest first
+    const int qt = (SPARSE && CAUSAL) ? static_cast<int>(gridDim.y - 1 - blockIdx.y) : static_cast<int>(blockIdx.y);
+    const int Nq = p.Nq, Nk = p.Nk;
+    const int n_kv = (Nk + BN - 1) / BN;
+    const int row_last = min(Nq, (qt + 1) * BM) - 1;
+    // key tiles the tile's last query row may see
+    const int j_lim = CAUSAL ? min(n_kv, (Nk - Nq + row_last) / BN + 1) : n_kv;
+    const uint8_t* mrow = nullptr;
+    int n_list = j_lim;  // positions in the key-tile list (tile j itself when dense)
+    if constexpr (SPARSE) {
+        mrow = p.mask + static_cast<size_t>(bh % p.H) * p.mask_h_stride + static_cast<size_t>(qt) * p.n_kt;
+        int cnt = 0;
+        for (int j = static_cast<int>(lane_id()); j < j_lim; j += 32) cnt += mrow[j] != 0;
+        n_list = __reduce_add_sync(0xffffffffu, cnt);
+    }
+    // this range's positions in the list
+    const int j0 = split * p.tiles_per_split;
+    const int j1 = min(n_list, j0 + p.tiles_per_split);
+    const size_t part_row0 = (static_cast<size_t>(split) * p.BH + bh) * Nq;
+    if (j0 >= j1) {
+        // no key of this range reaches this Q tile
+        write_empty_rows<D>(p, qt, bh, part_row0);
         return;
     }
     const int nj = j1 - j0;
@@ -105,8 +139,22 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
     uint64_t* o_full = p_full + 1;
     uint64_t* drain = o_full + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint16_t* jlist = reinterpret_cast<uint16_t*>(smem + C::LIST_OFF);
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
+    if (SPARSE && warp == 0) {
+        // compact the mask row into the ascending list of allowed key tiles
+        int base = 0;
+        for (int c0 = 0; c0 < j_lim; c0 += 32) {
+            const int j = c0 + lane;
+            const bool on = j < j_lim && mrow[j] != 0;
+            const uint32_t b = __ballot_sync(0xffffffffu, on);
+            if (on) jlist[base + __popc(b & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
+            base += __popc(b);
+        }
+    }
+    // key tile at position jj of this range
+    auto tile_of = [&](int jj) -> int { return SPARSE ? static_cast<int>(jlist[j0 + jj]) : j0 + jj; };
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -151,9 +199,10 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
                     }
                     mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
                     const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
+                    const int krow = tile_of(jj) * BN;
                     for (int c = 0; c < C::NDC; ++c)
-                        tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64,
-                                    (j0 + jj) * BN, bh);
+                        tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64, krow,
+                                    bh);
                     ++it;
                 }
             }
@@ -241,7 +290,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
 #pragma unroll
             for (int c = 0; c < BN; c += 32) tmem_ld32(s_addr + c, reinterpret_cast<uint32_t*>(s + c));
             tmem_wait_ld();
-            const int limit = key_max - (j0 + jj) * BN;  // columns c <= limit are allowed
+            const int limit = key_max - tile_of(jj) * BN;  // columns c <= limit are allowed
             if (limit < BN - 1) {
 #pragma unroll
                 for (int c = 0; c < BN; ++c)
@@ -291,22 +340,49 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
             tc_fence_after();
             const bool any = l > 0.f;
             const float inv_l = any ? 1.f / l : 0.f;
-            float* op = p.o_part + (part_row0 + row) * D;
+            const float lse_row = any ? (m + __log2f(l)) * LN2 : -INFINITY;
+            if (p.direct) {
+                // the only range: O / l as bf16 and the LSE go straight to the outputs
+                const size_t g = static_cast<size_t>(bh) * Nq + row;
+                __nv_bfloat16* op = p.o + g * D;
 #pragma unroll
-            for (int cc = 0; cc < D; cc += 32) {
-                uint32_t o[32];
-                tmem_ld32(o_addr + cc, o);
-                tmem_wait_ld();
-                if (row < Nq) {
-                    float4* d4 = reinterpret_cast<float4*>(op + cc);
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + cc, o);
+                    tmem_wait_ld();
+                    if (row < Nq) {
+                        uint4* d4 = reinterpret_cast<uint4*>(op + cc);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        d4[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
-                                            __uint_as_float(o[4 * e + 2]) * inv_l,
-                                            __uint_as_float(o[4 * e + 3]) * inv_l);
+                        for (int e = 0; e < 4; ++e) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t)
+                                w[t] = pack_bf16x2(__uint_as_float(o[8 * e + 2 * t]) * inv_l,
+                                                   __uint_as_float(o[8 * e + 2 * t + 1]) * inv_l);
+                            d4[e] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
                 }
+                if (row < Nq) p.lse[g] = lse_row;
+            } else {
+                float* op = p.o_part + (part_row0 + row) * D;
+#pragma unroll
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + cc, o);
+                    tmem_wait_ld();
+                    if (row < Nq) {
+                        float4* d4 = reinterpret_cast<float4*>(op + cc);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            d4[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l,
+                                                __uint_as_float(o[4 * e + 1]) * inv_l,
+                                                __uint_as_float(o[4 * e + 2]) * inv_l,
+                                                __uint_as_float(o[4 * e + 3]) * inv_l);
+                    }
+                }
+                if (row < Nq) p.lse_part[part_row0 + row] = lse_row;
             }
-            if (row < Nq) p.lse_part[part_row0 + row] = any ? (m + __log2f(l)) * LN2 : -INFINITY;
         }
     }
 
@@ -373,16 +449,16 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
     if (lane == 0) p.lse[rid] = W > 0.f ? M + __logf(W) : -INFINITY;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE>
 cudaError_t launch(const DecodeParams& p, cudaStream_t stream)
 {
-    using C = Cfg<D>;
-    auto kern = decode_partial_kernel<D, CAUSAL>;
+    using C = Cfg<D, SPARSE>;
+    auto kern = decode_partial_kernel<D, CAUSAL, SPARSE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_split, (p.Nq + BM - 1) / BM, p.BH);
     kern<<<grid, NTHREADS, C::SMEM_BYTES, stream>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaGetLastError()) != cudaSuccess || p.direct) return e;
     const long long rows = static_cast<long long>(p.BH) * p.Nq;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned int>((rows + 3) / 4));
@@ -401,8 +477,17 @@ cudaError_t launch(const DecodeParams& p, cudaStream_t stream)
 
 cudaError_t launch_decode_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream)
 {
-    if (d == 128) return causal ? deck::launch<128, true>(p, stream) : deck::launch<128, false>(p, stream);
-    return causal ? deck::launch<64, true>(p, stream) : deck::launch<64, false>(p, stream);
+    if (d == 128)
+        return causal ? deck::launch<128, true, false>(p, stream) : deck::launch<128, false, false>(p, stream);
+    return causal ? deck::launch<64, true, false>(p, stream) : deck::launch<64, false, false>(p, stream);
+}
+
+cudaError_t launch_blocksparse_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream)
+{
+    if (!p.direct || p.n_split != 1) return cudaErrorInvalidValue;
+    if (d == 128)
+        return causal ? deck::launch<128, true, true>(p, stream) : deck::launch<128, false, true>(p, stream);
+    return causal ? deck::launch<64, true, true>(p, stream) : deck::launch<64, false, true>(p, stream);
 }
 
 }  // namespace fa

@@ -320,8 +320,51 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
     p.Nq = Nq;
     p.Nk = Nk;
     p.scale_log2 = scale * kLog2e;
+    p.direct = p.n_split == 1 ? 1 : 0;  // one range: no merge kernel
     st = cuda_status(launch_decode_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
-    if (st == FA_OK) g_last_launches = 2;
+    if (st == FA_OK) g_last_launches = p.direct ? 1 : 2;
+    return st;
+}
+
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, const void* block_mask,
+                       long long mask_head_stride, int B, int H, int N, int d, float scale, int causal, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse || !block_mask) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    const int n_t = (N + 127) / 128;
+    if (mask_head_stride < 0) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (n_t > kMaxMaskKeyTiles || static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+    if ((st = get_encoder()) != FA_OK) return st;
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.BH = static_cast<int>(BH);
+    p.Nq = N;
+    p.Nk = N;
+    p.n_split = 1;
+    p.tiles_per_split = n_t;
+    p.scale_log2 = scale * kLog2e;
+    p.direct = 1;
+    p.mask = static_cast<const uint8_t*>(block_mask);
+    p.mask_h_stride = mask_head_stride;
+    p.H = H;
+    p.n_kt = n_t;
+    st = cuda_status(launch_blocksparse_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
     return st;
 }
 

@@ -53,10 +53,22 @@ struct DecodeParams {
     int n_split;
     int tiles_per_split;  // 128-key tiles per range
     float scale_log2;
+    int direct;           // 1: one range; the range kernel writes o (bf16) and lse itself
+    // block-sparse only: uint8 [.][n_qt][n_kt] mask of (query tile, key tile)
+    // pairs, head h = bh % H at mask + h * mask_h_stride
+    const uint8_t* mask;
+    long long mask_h_stride;
+    int H;
+    int n_kt;
     WaitCtl ctl;
 };
-// Partial kernel over (range, Q tile, head) plus the combine kernel.
+// Maximum key tiles per row of a block mask (the kernel's tile list lives in
+// shared memory).
+constexpr int kMaxMaskKeyTiles = 2048;
+// Range kernel over (range, Q tile, head), plus the merge kernel unless direct.
 cudaError_t launch_decode_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream);
+// Block-sparse forward: one range per Q tile, direct output.
+cudaError_t launch_blocksparse_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream);
 
 // ---------------------------------------------------------------- bf16 backward
 struct BwdPreParams {

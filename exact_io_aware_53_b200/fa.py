@@ -42,6 +42,7 @@ _SIGS = {
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
     "fa_fwd_splitkv_workspace_bytes": ([I, I, I, I, I, I], ctypes.c_size_t),
     "fa_fwd_splitkv": ([P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P], I),
+    "fa_fwd_blocksparse": ([P, P, P, P, P, P, ctypes.c_longlong, I, I, I, I, ctypes.c_float, I, P], I),
     "fa_status_string": ([I], ctypes.c_char_p),
     "fa_last_launch_count": ([], I),
     "fa_last_cuda_error": ([], I),
@@ -157,6 +158,34 @@ def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, n_spl
     ws = torch.empty(max(splitkv_workspace_bytes(B, H, Nq, Nk, d, n_split), 16), dtype=torch.uint8,
                      device=q.device)
     _check(fwd_splitkv_raw(q, k, v, o, lse, ws, scale, causal, n_split, stream), "fa_fwd_splitkv")
+    return o, lse
+
+
+def fwd_blocksparse_raw(q, k, v, o, lse, block_mask, scale: float, causal: bool, stream=None) -> int:
+    """Enqueue the block-sparse forward on preallocated tensors; block_mask is
+    a CUDA uint8 tensor [T, T] (shared by every head) or [H, T, T], T = ceil(N/128)."""
+    B, H, N, d = _shape(q)
+    stride = 0 if block_mask.dim() == 2 or block_mask.shape[0] == 1 else int(block_mask.stride(0))
+    return _lib.fa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_mask), stride,
+                                   B, H, N, d, float(scale), int(bool(causal)), _stream(stream))
+
+
+def fwd_blocksparse(q, k, v, block_mask, causal: bool = False, scale: float | None = None, stream=None):
+    """O, LSE of attention restricted to the allowed (128-query, 128-key) tile
+    pairs of block_mask (bool or uint8, [T, T] or [H, T, T], T = ceil(N/128))."""
+    _same(q, k, v, dtype=torch.bfloat16)
+    B, H, N, d = _shape(q)
+    T = (N + 127) // 128
+    m = block_mask
+    if m.dim() == 2:
+        m = m.unsqueeze(0)
+    if m.dim() != 3 or tuple(m.shape[1:]) != (T, T) or m.shape[0] not in (1, H):
+        raise ValueError("block_mask must be [T, T] or [H, T, T] with T = ceil(N / 128) = %d" % T)
+    m = m.to(device=q.device, dtype=torch.uint8).contiguous()
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check(fwd_blocksparse_raw(q, k, v, o, lse, m, scale, causal, stream), "fa_fwd_blocksparse")
     return o, lse
 
 

@@ -88,6 +88,55 @@ DECODE_WORKLOADS = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class BlockSparseWorkload:
+    """Square attention restricted to a seeded block mask over 128 x 128
+    (query tile, key tile) pairs: each pair is kept with probability
+    ``density``, the diagonal pairs always (no empty row), one mask shared by
+    every head and batch entry."""
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    density: float
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def tiles(self) -> int:
+        return (self.N + 127) // 128
+
+    def flops(self, mask) -> float:
+        """4 * 128 * 128 * d per allowed (query tile, key tile) pair and head
+        (N a multiple of 128; with causal, the diagonal pairs count half)."""
+        m = mask.to(torch.bool)
+        if self.causal:
+            m = torch.tril(m)
+        pairs = float(m.sum()) - (0.5 * self.tiles if self.causal else 0.0)
+        return 4.0 * 128 * 128 * self.d * pairs * self.B * self.H
+
+
+BLOCKSPARSE_WORKLOADS = {
+    "blocksparse_bf16_4x16x4096x128_d50": BlockSparseWorkload("blocksparse_bf16_4x16x4096x128_d50", 4, 16, 4096, 128,
+                                                              False, 0.5, seed=3001),
+}
+
+
+def make_block_mask(w: BlockSparseWorkload, seed: int | None = None):
+    """uint8 [T, T] mask: Bernoulli(density) from a torch CPU Generator, diagonal set."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    T = w.tiles
+    m = torch.rand((T, T), generator=g) < w.density
+    m |= torch.eye(T, dtype=torch.bool)
+    return m.to(torch.uint8)
+
+
 def make_decode_inputs(w: DecodeWorkload, seed: int | None = None, B: int | None = None, H: int | None = None):
     """Draw (q, k, v) on the CPU for decode workload ``w``: fp32 standard
     normals in the order q [B,H,Nq,d], k [B,H,Nk,d], v [B,H,Nk,d], rounded to

@@ -186,11 +186,32 @@ void fa_set_wait_limit_ns(unsigned long long ns);
  *   with the same device current (0 for an invalid shape); caller-owned,
  *   needs no initialisation.  Errors as for fa_fwd, plus FA_ERR_INVALID_ARG
  *   for causal with Nk < Nq or n_split < 0, and FA_ERR_UNSUPPORTED for
- *   B*H > 65535.  Two kernels are enqueued on `stream`.
+ *   B*H > 65535.  Two kernels are enqueued on `stream`, one when a single
+ *   range is used (it then writes o and lse itself).
  */
 size_t fa_fwd_splitkv_workspace_bytes(int B, int H, int Nq, int Nk, int d, int n_split);
 int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B, int H,
                    int Nq, int Nk, int d, float scale, int causal, int n_split, void* stream);
+
+/*
+ * Block-sparse forward, bf16: the square problem restricted to the (query
+ * tile, key tile) pairs a block mask allows, the approximate extension of the
+ * method ("Block-sparse FlashAttention", guide "Prerequisites").  Tiles are
+ * 128 rows by 128 keys; only the allowed key tiles are read and computed.
+ *   q, k, v, o: bf16 [B][H][N][d]; lse: fp32 [B][H][N] (natural log);
+ *   d = 64 or 128.
+ *   block_mask: device uint8 [.][T][T], T = ceil(N / 128); key tile j is
+ *   allowed for query tile i of head h iff
+ *   block_mask[h * mask_head_stride + i * T + j] != 0 (mask_head_stride 0: one
+ *   mask for every head; T*T: one per head).  The batch shares the masks.
+ *   causal additionally keeps key j <= query i.
+ *   A query row that no key is allowed for gets O = 0 and LSE = -inf.
+ * One kernel is enqueued on `stream`; nothing is allocated.  Errors as for
+ * fa_fwd, plus FA_ERR_UNSUPPORTED for T > 2048 (N > 262144) or B*H > 65535.
+ */
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, const void* block_mask,
+                       long long mask_head_stride, int B, int H, int N, int d, float scale, int causal,
+                       void* stream);
 
 /* Human-readable name of a status code (static string). */
 const char* fa_status_string(int status);

@@ -138,3 +138,20 @@ def test_splitkv_workspace_size(lib):
     assert ws(1, 1, 1, 100, 64, 8) == ws(1, 1, 1, 100, 64, 1)  # one tile: one range
     assert ws(1, 1, 0, 100, 64, 1) == 0
     assert ws(1, 1, 1, 100, 64, -1) == 0
+
+
+def test_blocksparse_argument_errors(lib):
+    f = lib._lib.fa_fwd_blocksparse
+    P = ctypes.c_void_p
+
+    def call(B=1, H=1, N=256, d=128, scale=0.1, causal=0, stride=0, mask=P(16), q=P(16)):
+        return f(q, P(16), P(16), P(16), P(16), mask, stride, B, H, N, d, scale, causal, P(0))
+
+    assert call(q=P(0)) == lib.FA_ERR_INVALID_ARG
+    assert call(mask=P(0)) == lib.FA_ERR_INVALID_ARG
+    assert call(N=0) == lib.FA_ERR_INVALID_ARG
+    assert call(stride=-1) == lib.FA_ERR_INVALID_ARG
+    assert call(causal=3) == lib.FA_ERR_INVALID_ARG
+    assert call(d=32) == lib.FA_ERR_UNSUPPORTED
+    assert call(N=2048 * 128 + 1, d=64) == lib.FA_ERR_UNSUPPORTED   # more than 2048 key tiles
+    assert call(q=P(24)) == lib.FA_ERR_MISALIGNED
