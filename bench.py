@@ -737,6 +737,162 @@ def run_blocksparse(args, w):
     return line
 
 
+# ------------------------------------------------------------------ e4m3 forward
+
+FP8_METRIC = "FP8 (e4m3) attention forward TFLOPS on 1 B200 and fraction of the FP8 tensor peak"
+FP8_OVER_BF16 = 4.5 / 2.25  # nominal dense fp8 : bf16 tensor throughput
+
+
+def fp8_oracle_sample(w, heads: int, seed: int):
+    """fp64 oracle forward on `heads` heads of the dequantized e4m3 inputs; returns (seconds, flops, threads)."""
+    from exact_io_aware_53_b200.workloads import make_fp8_inputs
+    from oracle import oracle
+    x = make_fp8_inputs((1, heads, w.N, w.d), seed=seed)
+    q, k, v = (x[n].double() * s for n, s in zip(("q", "k", "v"), x["descales"]))
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, w.scale, w.causal)
+    dt = time.perf_counter() - t0
+    return dt, w.flops() / (w.B * w.H) * heads, oracle.num_threads()
+
+
+def run_reference_fp8(args, w):
+    rank, world, _ = rank_env()
+    if rank != 0:
+        return 0
+    for i in range(args.warmup):
+        fp8_oracle_sample(w, 1, w.seed + i)
+    times, fl, thr = [], 0.0, 1
+    for i in range(args.steps):
+        dt, fl, thr = fp8_oracle_sample(w, 1, w.seed + 100 + i)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = fl / (ms / 1e3) / 1e12
+    line = {"impl": "reference", "metric": FP8_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": 1, "H": 1, "N": w.N, "d": w.d, "causal": w.causal,
+                       "sample": "one head per step (dequantized e4m3 inputs)", "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                             "sample": "one head of %s per step (fp64)" % w.name},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_fp8(args, w):
+    """One step = fa_fwd_fp8 over the whole batch, e4m3 inputs resident in device memory."""
+    import torch
+    from exact_io_aware_53_b200 import fa
+    from exact_io_aware_53_b200.workloads import make_fp8_inputs
+
+    rank, world, local = rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        init_dist(world, "nccl", torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    B, H, N, d = w.B, w.H, w.N, w.d
+    x = make_fp8_inputs((B, H, N, d), seed=rank_seed(w.seed, rank))
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    launches = [0]
+
+    def step():
+        rc = fa.fwd_fp8_raw(q, k, v, o, lse, x["descales"], w.scale, w.causal)
+        launches[0] += fa.last_launch_count()
+        if rc:
+            raise fa.FAError(rc, "fa_fwd_fp8")
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after warm-up: %s" % fa.status_string(st))
+    # inputs are 100 MB: flush L2 between timed calls by writing 2x its size
+    flush = torch.empty(2 * 126 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    launches[0] = 0
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after timing: %s" % fa.status_string(st))
+    ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ms = max_over_ranks(ms_local, world, dev)
+    fl = w.flops()
+    value = world * fl / (ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak = bf16 * FP8_OVER_BF16
+    achieved = fl / (ms_local / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "decode_partial_kernel (e4m3, direct output)", "achieved": achieved,
+                "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                "peak_source": "bf16_tflops %s x %.1f (nominal fp8 : bf16 ratio)" % (peak_src, FP8_OVER_BF16),
+                "frac_of_bf16_peak": achieved / bf16, "algorithmic_flops_per_launch": fl, "ms_per_launch": ms_local,
+                "traffic": measured_traffic("fp8", w.name), "traffic_unit": "bytes per launch (ncu dram read+write)"}
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x[n].pin_memory() for n in ("q", "k", "v"))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        steps = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
+        e2e = {"value": world * fl / (ems / 1e3) / 1e12, "unit": UNIT, "ms_per_step": ems,
+               "h2d_bytes_per_step": 3 * hq.numel(), "d2h_bytes_per_step": ho.numel() * 2 + hl.numel() * 4,
+               "steps": steps, "api": "fa.fwd_fp8_raw with q, k, v from and o, lse to pinned host memory"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, cfl, thr = fp8_oracle_sample(w, 1, w.seed)
+        cpu = {"value": cfl / dt / 1e12, "unit": UNIT, "cores": thr, "kind": "oracle",
+               "sample": "1 of %d heads (N=%d, d=%d, causal=%s, dequantized e4m3), fp64, %.1f s" % (
+                   B * H, N, d, w.causal, dt)}
+    line = {"metric": FP8_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate, bf16 out)", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
+                       "parallelism": "dp%d (independent batches per GPU, no collective)" % world,
+                       "l2": "flushed before each timed call (q, k, v = %.0f MB per GPU)" % (3 * B * H * N * d / 1e6)},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches[0], "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return line
+
+
 def probe_mma_rate():
     """Cycles per tcgen05 MMA instruction for the shapes the kernels issue
     (fa_selftest_umma_rate, one CTA per SM); printed as JSON lines."""
@@ -776,14 +932,21 @@ def main(argv=None):
     if args.probe_mma_rate:
         probe_mma_rate()
         return 0
-    from exact_io_aware_53_b200.workloads import BLOCKSPARSE_WORKLOADS, DECODE_WORKLOADS, WORKLOADS
-    known = list(WORKLOADS) + list(DECODE_WORKLOADS) + list(BLOCKSPARSE_WORKLOADS)
+    from exact_io_aware_53_b200.workloads import BLOCKSPARSE_WORKLOADS, DECODE_WORKLOADS, FP8_WORKLOADS, WORKLOADS
+    known = list(WORKLOADS) + list(DECODE_WORKLOADS) + list(BLOCKSPARSE_WORKLOADS) + list(FP8_WORKLOADS)
     if args.workload != "all" and args.workload not in known:
         ap.error("unknown workload %s (choose from %s)" % (args.workload, ", ".join(known)))
     names = known if args.workload == "all" else [args.workload]
     rc = 0
     try:
         for name in names:
+            if name in FP8_WORKLOADS:
+                w = FP8_WORKLOADS[name]
+                if args.impl == "reference":
+                    rc |= run_reference_fp8(args, w)
+                else:
+                    run_fp8(args, w)
+                continue
             if name in BLOCKSPARSE_WORKLOADS:
                 w = BLOCKSPARSE_WORKLOADS[name]
                 if args.impl == "reference":

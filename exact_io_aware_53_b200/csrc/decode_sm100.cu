@@ -21,6 +21,13 @@
 // loop over the listed tiles only; one range per Q tile, output written
 // directly.
 //
+// FP8 variant (FP8): q, k, v in e4m3 with per-tensor descale factors (the
+// FP8 support of the FlashAttention-3 line, "Lineage"), d = 128, square, one
+// range per Q tile.  S = Q K^T and O += P V run as tcgen05 kind::f8f6f4 MMAs
+// (K = 32 per instruction); the softmax writes P back to TMEM as e4m3, four
+// per 32-bit column.  The descales fold into the exponent scale (q, k) and
+// the epilogue factor (v).
+//
 // The work is bound by reading K and V.  A CTA keeps one Q tile, so S and P
 // share TMEM without a second tile to ping-pong with; instead two CTAs share
 // an SM (96 KB shared memory, 256 TMEM columns each) and one's softmax runs
@@ -43,12 +50,12 @@ constexpr int LOAD_WARP = 5;
 constexpr float RESCALE_LOG2 = 8.0f;  // move the running max only when it grows by more
 constexpr float LN2 = 0.6931471805599453f;
 
-template <int D, bool SPARSE>
+template <int D, bool SPARSE, bool FP8>
 struct Cfg {
-    static constexpr int NDC = D / 64;
-    static constexpr int BOX_BYTES = 128 * 128;  // 128 rows x 64 bf16
+    static constexpr int NDC = FP8 ? 1 : D / 64;  // 128-byte column chunks per row
+    static constexpr int BOX_BYTES = 128 * 128;   // 128 rows x 128 bytes (64 bf16 or 128 e4m3)
     static constexpr int TILE_BYTES = NDC * BOX_BYTES;
-    static constexpr int STAGES = (D == 128) ? 2 : 4;
+    static constexpr int STAGES = (FP8 || D == 64) ? 4 : 2;
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = TILE_BYTES;
     static constexpr int BAR_OFF = KV_OFF + STAGES * TILE_BYTES;
@@ -59,6 +66,52 @@ struct Cfg {
     static constexpr uint32_t TMEM_COLS = 256;
     static constexpr uint32_t O_COL = 128;
 };
+
+// Instruction descriptor, kind::f8f6f4 with e4m3 A and B (format code 0) and
+// an f32 accumulator; field positions as for kind::f16 (idesc_bf16).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4)  // D format: f32; A, B format fields 0: e4m3
+           | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem], 8-bit operands, issued by the elected lane.
+__device__ __forceinline__ void mma_ss_f8_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem], 8-bit operands (A: four elements per
+// 32-bit column, lowest K in the low byte).
+__device__ __forceinline__ void mma_ts_f8_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Four floats -> four e4m3 bytes (round to nearest even, saturating), p0 in
+// the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3)
+{
+    uint16_t lo, hi;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(p1), "f"(p0));
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(p3), "f"(p2));
+    return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
 {
@@ -92,16 +145,16 @@ __device__ void write_empty_rows(const DecodeParams& p, int qt, int bh, size_t p
     }
 }
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool FP8>
 __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __grid_constant__ DecodeParams p)
 {
-    using C = Cfg<D, SPARSE>;
+    using C = Cfg<D, SPARSE, FP8>;
     // the merge kernel may be scheduled once every range CTA is running; it
     // still waits for this grid's completion before it reads anything
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int split = blockIdx.x, bh = blockIdx.z;
-    // block-sparse causal rows grow with the tile index: start the longest first
-    const int qt = (SPARSE && CAUSAL) ? static_cast<int>(gridDim.y - 1 - blockIdx.y) : static_cast<int>(blockIdx.y);
+    // causal rows grow with the tile index: start the longest first
+    const int qt = CAUSAL ? static_cast<int>(gridDim.y - 1 - blockIdx.y) : static_cast<int>(blockIdx.y);
     const int Nq = p.Nq, Nk = p.Nk;
     const int n_kv = (Nk + BN - 1) / BN;
     const int row_last = min(Nq, (qt + 1) * BM) - 1;
@@ -217,24 +270,32 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
         // ------------------------------------------------------------ MMA issuer
         // S and P share TMEM columns 0..127, so S of the next key tile is
         // issued after the P V that reads this one's P
-        constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
-        constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
+        constexpr uint32_t idesc_s = FP8 ? idesc_e4m3(BM, BN, false, false) : idesc_bf16(BM, BN, false, false);
+        constexpr uint32_t idesc_o = FP8 ? idesc_e4m3(BM, D, false, true) : idesc_bf16(BM, D, false, true);
+        // K per instruction: 16 bf16 or 32 e4m3, i.e. 32 bytes of a K-major row
+        // and 8 TMEM columns of P either way
+        constexpr int KI = FP8 ? 32 : 16;
         const uint32_t qa = smem_u32(sQ), kva = smem_u32(sKV);
         auto issue_s = [&](int stage) {
             const uint32_t kb = kva + stage * C::TILE_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
+            for (int kk = 0; kk < D / KI; ++kk) {
                 const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                mma_ss_elect(tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idesc_s,
-                             kk > 0 ? 1u : 0u);
+                const uint64_t ad = sdesc_sw128(qa + off, 16, 1024), bd = sdesc_sw128(kb + off, 16, 1024);
+                if constexpr (FP8) mma_ss_f8_elect(tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                else mma_ss_elect(tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
             }
         };
         auto issue_o = [&](int stage, int jj) {
             const uint32_t vb = kva + stage * C::TILE_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)
-                mma_ts_elect(tmem + C::O_COL, tmem + kk * 8, sdesc_sw128(vb + kk * 2048, C::BOX_BYTES, 1024),
-                             idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / KI; ++kk) {
+                // V is MN-major: KI key rows of 128 bytes per instruction
+                const uint64_t bd = sdesc_sw128(vb + kk * KI * 128, C::BOX_BYTES, 1024);
+                const uint32_t acc = (jj > 0 || kk > 0) ? 1u : 0u;
+                if constexpr (FP8) mma_ts_f8_elect(tmem + C::O_COL, tmem + kk * 8, bd, idesc_o, acc);
+                else mma_ts_elect(tmem + C::O_COL, tmem + kk * 8, bd, idesc_o, acc);
+            }
         };
         int it = 0;
         bool ok = warp_wait(q_full, 0, p.ctl);
@@ -308,14 +369,22 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
             }
             // while no key has been allowed m is -inf and every p is 0
             const float m_use = (m == -INFINITY) ? 0.f : m;
-            uint32_t pk[BN / 2];
+            constexpr int PER_WORD = FP8 ? 4 : 2;  // P elements per TMEM column
+            uint32_t pk[BN / PER_WORD];
             float sum = 0.f;
 #pragma unroll
-            for (int c = 0; c < BN; c += 2) {
+            for (int c = 0; c < BN; c += PER_WORD) {
                 const float p0 = ex2_approx(fmaf(s[c], cl2, -m_use));
                 const float p1 = ex2_approx(fmaf(s[c + 1], cl2, -m_use));
-                sum += p0 + p1;
-                pk[c / 2] = pack_bf16x2(p0, p1);
+                if constexpr (FP8) {
+                    const float p2 = ex2_approx(fmaf(s[c + 2], cl2, -m_use));
+                    const float p3 = ex2_approx(fmaf(s[c + 3], cl2, -m_use));
+                    sum += (p0 + p1) + (p2 + p3);
+                    pk[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
+                } else {
+                    sum += p0 + p1;
+                    pk[c / 2] = pack_bf16x2(p0, p1);
+                }
             }
             l = l * alpha + sum;
             if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
@@ -331,7 +400,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
                 }
             }
             tmem_st32(s_addr, pk);
-            tmem_st32(s_addr + BN / 4, pk + BN / 4);
+            if constexpr (!FP8) tmem_st32(s_addr + BN / 4, pk + BN / 4);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_full);
@@ -339,7 +408,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
         if (ok && warp_wait(o_full, 0, p.ctl)) {
             tc_fence_after();
             const bool any = l > 0.f;
-            const float inv_l = any ? 1.f / l : 0.f;
+            // e4m3 V carries its descale factor into the output
+            const float inv_l = any ? (FP8 ? p.o_scale : 1.f) / l : 0.f;
             const float lse_row = any ? (m + __log2f(l)) * LN2 : -INFINITY;
             if (p.direct) {
                 // the only range: O / l as bf16 and the LSE go straight to the outputs
@@ -449,11 +519,11 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
     if (lane == 0) p.lse[rid] = W > 0.f ? M + __logf(W) : -INFINITY;
 }
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool FP8 = false>
 cudaError_t launch(const DecodeParams& p, cudaStream_t stream)
 {
-    using C = Cfg<D, SPARSE>;
-    auto kern = decode_partial_kernel<D, CAUSAL, SPARSE>;
+    using C = Cfg<D, SPARSE, FP8>;
+    auto kern = decode_partial_kernel<D, CAUSAL, SPARSE, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_split, (p.Nq + BM - 1) / BM, p.BH);
@@ -488,6 +558,12 @@ cudaError_t launch_blocksparse_sm100(const DecodeParams& p, int d, bool causal, 
     if (d == 128)
         return causal ? deck::launch<128, true, true>(p, stream) : deck::launch<128, false, true>(p, stream);
     return causal ? deck::launch<64, true, true>(p, stream) : deck::launch<64, false, true>(p, stream);
+}
+
+cudaError_t launch_fp8_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream)
+{
+    if (!p.direct || p.n_split != 1 || d != 128) return cudaErrorInvalidValue;
+    return causal ? deck::launch<128, true, false, true>(p, stream) : deck::launch<128, false, false, true>(p, stream);
 }
 
 }  // namespace fa

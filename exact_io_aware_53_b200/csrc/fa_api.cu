@@ -368,6 +368,47 @@ int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, flo
     return st;
 }
 
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, float q_descale, float k_descale,
+               float v_descale, int B, int H, int N, int d, float scale, int causal, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    for (float f : {q_descale, k_descale, v_descale})
+        if (!(f > 0.f) || !std::isfinite(f)) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale * q_descale * k_descale * kLog2e)) return FA_ERR_INVALID_ARG;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+    if ((st = get_encoder()) != FA_OK) return st;
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    // e4m3 rows of d = 128 bytes: one 128-byte swizzled box of 128 rows per tile
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, d, N, BH, 128, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, d, N, BH, 128, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, v, d, N, BH, 128, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.BH = static_cast<int>(BH);
+    p.Nq = N;
+    p.Nk = N;
+    p.n_split = 1;
+    p.tiles_per_split = (N + 127) / 128;
+    p.scale_log2 = scale * q_descale * k_descale * kLog2e;
+    p.o_scale = v_descale;
+    p.direct = 1;
+    st = cuda_status(launch_fp8_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d)
 {
     if (B < 1 || H < 1 || N < 1 || d < 1) return 0;

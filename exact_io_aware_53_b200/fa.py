@@ -43,6 +43,8 @@ _SIGS = {
     "fa_fwd_splitkv_workspace_bytes": ([I, I, I, I, I, I], ctypes.c_size_t),
     "fa_fwd_splitkv": ([P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P], I),
     "fa_fwd_blocksparse": ([P, P, P, P, P, P, ctypes.c_longlong, I, I, I, I, ctypes.c_float, I, P], I),
+    "fa_fwd_fp8": ([P, P, P, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_float, I, I, I, I, ctypes.c_float, I, P],
+                   I),
     "fa_status_string": ([I], ctypes.c_char_p),
     "fa_last_launch_count": ([], I),
     "fa_last_cuda_error": ([], I),
@@ -186,6 +188,25 @@ def fwd_blocksparse(q, k, v, block_mask, causal: bool = False, scale: float | No
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     _check(fwd_blocksparse_raw(q, k, v, o, lse, m, scale, causal, stream), "fa_fwd_blocksparse")
+    return o, lse
+
+
+def fwd_fp8_raw(q, k, v, o, lse, descales, scale: float, causal: bool, stream=None) -> int:
+    """Enqueue the e4m3 forward on preallocated tensors; descales = (q, k, v) factors."""
+    B, H, N, d = _shape(q)
+    qd, kd, vd = (float(x) for x in descales)
+    return _lib.fa_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), qd, kd, vd, B, H, N, d, float(scale),
+                           int(bool(causal)), _stream(stream))
+
+
+def fwd_fp8(q, k, v, descales=(1.0, 1.0, 1.0), causal: bool = False, scale: float | None = None, stream=None):
+    """O (bf16), LSE for e4m3 q, k, v [B,H,N,128] whose values are x * descale."""
+    _same(q, k, v, dtype=torch.float8_e4m3fn)
+    B, H, N, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check(fwd_fp8_raw(q, k, v, o, lse, descales, scale, causal, stream), "fa_fwd_fp8")
     return o, lse
 
 

@@ -137,6 +137,55 @@ def make_block_mask(w: BlockSparseWorkload, seed: int | None = None):
     return m.to(torch.uint8)
 
 
+@dataclasses.dataclass(frozen=True)
+class Fp8Workload:
+    """Square attention with e4m3 q, k, v (one descale factor per tensor)."""
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """4*B*H*N^2*d, halved under the causal mask (the bf16 convention)."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+
+FP8_WORKLOADS = {
+    "fp8_e4m3_4x16x4096x128_causal": Fp8Workload("fp8_e4m3_4x16x4096x128_causal", 4, 16, 4096, 128, True, seed=4001),
+}
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-tensor e4m3 quantization of an fp32 tensor: descale = amax / 448
+    (448 is e4m3's largest finite value), x8 = (x / descale) rounded to
+    float8_e4m3fn.  Returns (x8, descale); x8 * descale are the values the
+    attention sees."""
+    amax = float(x.abs().max())
+    descale = amax / 448.0 if amax > 0 else 1.0
+    return (x / descale).to(torch.float8_e4m3fn), descale
+
+
+def make_fp8_inputs(shape, seed: int, gain: float = 1.0):
+    """q, k, v as fp32 standard normals (q, k times ``gain``) from a torch CPU
+    Generator in the order q, k, v, each quantized by ``quantize_e4m3``.
+    Returns {"q": q8, "k": k8, "v": v8, "descales": (dq, dk, dv)}."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn(shape, generator=g, dtype=torch.float32) * gain
+    k = torch.randn(shape, generator=g, dtype=torch.float32) * gain
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    (q8, dq), (k8, dk), (v8, dv) = quantize_e4m3(q), quantize_e4m3(k), quantize_e4m3(v)
+    return {"q": q8, "k": k8, "v": v8, "descales": (dq, dk, dv)}
+
+
 def make_decode_inputs(w: DecodeWorkload, seed: int | None = None, B: int | None = None, H: int | None = None):
     """Draw (q, k, v) on the CPU for decode workload ``w``: fp32 standard
     normals in the order q [B,H,Nq,d], k [B,H,Nk,d], v [B,H,Nk,d], rounded to

@@ -213,6 +213,23 @@ int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, flo
                        long long mask_head_stride, int B, int H, int N, int d, float scale, int causal,
                        void* stream);
 
+/*
+ * FP8 forward: q, k, v in e4m3 (OCP FP8, 1-4-3, no infinities) with one
+ * descale factor per tensor, so the values are q8 * q_descale and so on; the
+ * FP8 support of the FlashAttention-3 line ("Lineage" in the explainer).
+ *   q, k, v: e4m3 bytes [B][H][N][d]; o: bf16 [B][H][N][d]; lse: fp32
+ *   [B][H][N] (natural log of the sum of e^{scale * <q_i, k_j>} over the
+ *   dequantized values).  d = 128.  causal: key j <= query i.
+ *   Scores are exact products accumulated in fp32; the softmax weights P are
+ *   rounded to e4m3 (relative error <= 2^-4) before P V, so O carries an
+ *   error up to 2^-4 * sum_j P_ij |v_j| beyond the bf16 path's.
+ * One kernel is enqueued on `stream`; nothing is allocated.  Errors as for
+ * fa_fwd, plus FA_ERR_INVALID_ARG for a descale that is not finite and
+ * positive, FA_ERR_UNSUPPORTED for d != 128 or B*H > 65535.
+ */
+int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, float q_descale, float k_descale,
+               float v_descale, int B, int H, int N, int d, float scale, int causal, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* fa_status_string(int status);
 

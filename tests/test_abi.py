@@ -155,3 +155,20 @@ def test_blocksparse_argument_errors(lib):
     assert call(d=32) == lib.FA_ERR_UNSUPPORTED
     assert call(N=2048 * 128 + 1, d=64) == lib.FA_ERR_UNSUPPORTED   # more than 2048 key tiles
     assert call(q=P(24)) == lib.FA_ERR_MISALIGNED
+
+
+def test_fp8_argument_errors(lib):
+    f = lib._lib.fa_fwd_fp8
+    P = ctypes.c_void_p
+
+    def call(B=1, H=1, N=256, d=128, scale=0.1, causal=0, ds=(1.0, 1.0, 1.0), q=P(16)):
+        return f(q, P(16), P(16), P(16), P(16), ds[0], ds[1], ds[2], B, H, N, d, scale, causal, P(0))
+
+    assert call(q=P(0)) == lib.FA_ERR_INVALID_ARG
+    assert call(N=0) == lib.FA_ERR_INVALID_ARG
+    assert call(ds=(0.0, 1.0, 1.0)) == lib.FA_ERR_INVALID_ARG
+    assert call(ds=(1.0, float("inf"), 1.0)) == lib.FA_ERR_INVALID_ARG
+    assert call(ds=(1.0, 1.0, -2.0)) == lib.FA_ERR_INVALID_ARG
+    assert call(ds=(1e30, 1e30, 1.0)) == lib.FA_ERR_INVALID_ARG   # scale * descales overflows
+    assert call(d=64) == lib.FA_ERR_UNSUPPORTED
+    assert call(q=P(8)) == lib.FA_ERR_MISALIGNED
