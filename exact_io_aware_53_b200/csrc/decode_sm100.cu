@@ -357,10 +357,18 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
                 for (int c = 0; c < BN; ++c)
                     if (c > limit) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row max over four independent chains of three-input max (a
+            // single chain would serialise 127 dependent instructions)
+            float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]), mx2 = fmaxf(s[4], s[5]),
+                  mx3 = fmaxf(s[6], s[7]);
 #pragma unroll
-            for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-            const float m_blk = mx * cl2;
+            for (int c = 8; c < BN; c += 8) {
+                mx0 = fmax3(mx0, s[c], s[c + 1]);
+                mx1 = fmax3(mx1, s[c + 2], s[c + 3]);
+                mx2 = fmax3(mx2, s[c + 4], s[c + 5]);
+                mx3 = fmax3(mx3, s[c + 6], s[c + 7]);
+            }
+            const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cl2;
             float alpha = 1.f;
             if (m_blk > m + RESCALE_LOG2) {
                 // also the first tile with an allowed key (m = -inf gives alpha = 0)
@@ -371,21 +379,23 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
             const float m_use = (m == -INFINITY) ? 0.f : m;
             constexpr int PER_WORD = FP8 ? 4 : 2;  // P elements per TMEM column
             uint32_t pk[BN / PER_WORD];
-            float sum = 0.f;
+            float sum0 = 0.f, sum1 = 0.f;  // two accumulation chains
 #pragma unroll
-            for (int c = 0; c < BN; c += PER_WORD) {
+            for (int c = 0; c < BN; c += 4) {
                 const float p0 = ex2_approx(fmaf(s[c], cl2, -m_use));
                 const float p1 = ex2_approx(fmaf(s[c + 1], cl2, -m_use));
+                const float p2 = ex2_approx(fmaf(s[c + 2], cl2, -m_use));
+                const float p3 = ex2_approx(fmaf(s[c + 3], cl2, -m_use));
+                sum0 += p0 + p1;
+                sum1 += p2 + p3;
                 if constexpr (FP8) {
-                    const float p2 = ex2_approx(fmaf(s[c + 2], cl2, -m_use));
-                    const float p3 = ex2_approx(fmaf(s[c + 3], cl2, -m_use));
-                    sum += (p0 + p1) + (p2 + p3);
                     pk[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
                 } else {
-                    sum += p0 + p1;
                     pk[c / 2] = pack_bf16x2(p0, p1);
+                    pk[c / 2 + 1] = pack_bf16x2(p2, p3);
                 }
             }
+            const float sum = sum0 + sum1;
             l = l * alpha + sum;
             if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 // O holds the earlier tiles' P V (their MMA precedes this S)
