@@ -43,6 +43,7 @@
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
+#include <stdint.h>
 #endif
 
 int oracle_num_threads(void)
@@ -535,4 +536,196 @@ int oracle_attn_bwd_kv_rows(const double* q, const double* k, const double* v, c
     free(prow);
     free(dprow);
     return 0;
+}
+
+/* ------------------------------------------------------------------ dropout
+ *
+ * The pages name dropout among the settings of the kernel benchmarks (guide,
+ * "What to inspect") and give no generator.  Contract (a reading): the keep
+ * decision for (head bh, query i, key j) is a byte of a counter-based
+ * generator, Philox4x64-10 (J. K. Salmon, M. A. Moraes, R. O. Dror and D. E.
+ * Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011), so the
+ * backward pass regenerates the forward's mask from (seed, offset) alone:
+ *   counter = (j / 32, i, bh, 0), key = (seed, offset)
+ *   the 4 output words are 32 bytes, little-endian; key j uses byte j % 32
+ *   keep iff that byte < t, t in [0, 256] (keep probability t / 256)
+ *   kept weights are scaled by 256 / t.
+ * Forward:  O_i = (256 / t) * sum_j P_ij Z_ij v_j, LSE_i unchanged (P is the
+ * softmax of the undropped scores).
+ * Backward (softmax calculus with the fixed mask Z, s = 256 / t):
+ *   dV_j = s sum_i P_ij Z_ij dO_i,   dP_ij = s Z_ij <dO_i, v_j>,
+ *   D_i = sum_j P_ij dP_ij (= <dO_i, O_i>),  dS = P o (dP - D),
+ *   dQ = scale dS K,  dK = scale dS^T Q.
+ */
+
+/* Philox4x64-10: ten rounds of the Philox S-box on a 4-word counter, the
+ * 2-word key bumped by the Weyl constants between rounds (the paper's
+ * Philox-4x64 parameters). */
+void oracle_philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4])
+{
+    const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+    uint64_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint64_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += W0;
+            k1 += W1;
+        }
+        const unsigned __int128 p0 = (unsigned __int128)M0 * x0;
+        const unsigned __int128 p1 = (unsigned __int128)M1 * x2;
+        const uint64_t hi0 = (uint64_t)(p0 >> 64), lo0 = (uint64_t)p0;
+        const uint64_t hi1 = (uint64_t)(p1 >> 64), lo1 = (uint64_t)p1;
+        const uint64_t y0 = hi1 ^ x1 ^ k0, y2 = hi0 ^ x3 ^ k1;
+        x0 = y0;
+        x1 = lo1;
+        x2 = y2;
+        x3 = lo0;
+    }
+    out[0] = x0;
+    out[1] = x1;
+    out[2] = x2;
+    out[3] = x3;
+}
+
+/* Keep bit Z for (bh, i, j) under the contract above. */
+static int dropout_keep(uint64_t seed, uint64_t offset, long bh, long i, long j, int t)
+{
+    const uint64_t ctr[4] = {(uint64_t)(j / 32), (uint64_t)i, (uint64_t)bh, 0};
+    const uint64_t key[2] = {seed, offset};
+    uint64_t w[4];
+    oracle_philox4x64_10(ctr, key, w);
+    const long b = j % 32;
+    const unsigned byte = (unsigned)((w[b / 8] >> (8 * (b % 8))) & 0xFFu);
+    return (int)byte < t;
+}
+
+/* The keep mask of one head: z[i * N + j] in {0, 1} for all i, j < N. */
+int oracle_dropout_mask(unsigned char* z, long bh, long N, int t, uint64_t seed, uint64_t offset)
+{
+    if (N < 0 || t < 0 || t > 256) return -1;
+    for (long i = 0; i < N; ++i)
+        for (long j = 0; j < N; ++j) z[i * N + j] = (unsigned char)dropout_keep(seed, offset, bh, i, j, t);
+    return 0;
+}
+
+/* Forward with dropout (definition above).  t = 256 is plain attention;
+ * t = 0 drops everything (O = 0). */
+int oracle_attn_fwd_dropout(const double* q, const double* k, const double* v, double* o,
+                            double* lse, long BH, long N, long d, double scale, int causal,
+                            int t, uint64_t seed, uint64_t offset)
+{
+    if (BH < 0 || N < 0 || d < 1 || t < 0 || t > 256) return -1;
+    const double s_keep = t > 0 ? 256.0 / t : 0.0;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* srow = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+        if (!srow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 16) collapse(2)
+        for (long h = 0; h < BH; ++h)
+            for (long i = 0; i < N; ++i) {
+                if (!srow) continue;
+                const long base = h * N * d;
+                const double* qi = q + base + i * d;
+                double* oi = o + base + i * d;
+                const long nk = n_allowed(i, N, causal);
+                double m = -INFINITY;
+                for (long j = 0; j < nk; ++j) {
+                    srow[j] = scale * dot(qi, k + base + j * d, d);
+                    if (srow[j] > m) m = srow[j];
+                }
+                double l = 0.0;
+                for (long j = 0; j < nk; ++j) {
+                    srow[j] = exp(srow[j] - m);
+                    l += srow[j];
+                }
+                for (long t2 = 0; t2 < d; ++t2) oi[t2] = 0.0;
+                for (long j = 0; j < nk; ++j) {
+                    if (!dropout_keep(seed, offset, h, i, j, t)) continue;
+                    const double pj = s_keep * srow[j] / l;
+                    const double* vj = v + base + j * d;
+                    for (long t2 = 0; t2 < d; ++t2) oi[t2] += pj * vj[t2];
+                }
+                lse[h * N + i] = m + log(l);
+            }
+        free(srow);
+    }
+    return err;
+}
+
+/* Backward with dropout (definition above), the mask regenerated per element. */
+int oracle_attn_bwd_dropout(const double* q, const double* k, const double* v, const double* dO,
+                            double* dq, double* dk, double* dv, long BH, long N, long d,
+                            double scale, int causal, int t, uint64_t seed, uint64_t offset)
+{
+    if (BH < 0 || N < 0 || d < 1 || t < 0 || t > 256) return -1;
+    const double s_keep = t > 0 ? 256.0 / t : 0.0;
+    int err = 0;
+#pragma omp parallel
+    {
+        double* prow = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+        double* dprow = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+        double* zrow = (double*)malloc((size_t)(N > 0 ? N : 1) * sizeof(double));
+        if (!prow || !dprow || !zrow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long h = 0; h < BH; ++h) {
+            if (!prow || !dprow || !zrow) continue;
+            const long base = h * N * d;
+            const double *qh = q + base, *kh = k + base, *vh = v + base, *doh = dO + base;
+            double *dqh = dq + base, *dkh = dk + base, *dvh = dv + base;
+            memset(dkh, 0, (size_t)(N * d) * sizeof(double));
+            memset(dvh, 0, (size_t)(N * d) * sizeof(double));
+            for (long i = 0; i < N; ++i) {
+                const double* qi = qh + i * d;
+                const double* doi = doh + i * d;
+                const long nk = n_allowed(i, N, causal);
+                double m = -INFINITY;
+                for (long j = 0; j < nk; ++j) {
+                    prow[j] = scale * dot(qi, kh + j * d, d);
+                    if (prow[j] > m) m = prow[j];
+                }
+                double l = 0.0;
+                for (long j = 0; j < nk; ++j) {
+                    prow[j] = exp(prow[j] - m);
+                    l += prow[j];
+                }
+                for (long j = 0; j < nk; ++j) {
+                    prow[j] /= l;
+                    zrow[j] = dropout_keep(seed, offset, h, i, j, t) ? s_keep : 0.0;
+                }
+                double D = 0.0;
+                for (long j = 0; j < nk; ++j) {
+                    dprow[j] = zrow[j] * dot(doi, vh + j * d, d);
+                    D += prow[j] * dprow[j];
+                }
+                double* dqi = dqh + i * d;
+                for (long t2 = 0; t2 < d; ++t2) dqi[t2] = 0.0;
+                for (long j = 0; j < nk; ++j) {
+                    const double ds = prow[j] * (dprow[j] - D);
+                    const double pz = prow[j] * zrow[j];
+                    const double* kj = kh + j * d;
+                    double* dkj = dkh + j * d;
+                    double* dvj = dvh + j * d;
+                    for (long t2 = 0; t2 < d; ++t2) {
+                        dqi[t2] += ds * kj[t2];
+                        dkj[t2] += ds * qi[t2];
+                        dvj[t2] += pz * doi[t2];
+                    }
+                }
+                for (long t2 = 0; t2 < d; ++t2) dqi[t2] *= scale;
+            }
+            for (long e = 0; e < N * d; ++e) dkh[e] *= scale;
+        }
+        free(prow);
+        free(dprow);
+        free(zrow);
+    }
+    return err;
 }

@@ -51,6 +51,15 @@ def _load():
         lib.oracle_attn_fwd_rows.restype = I
         lib.oracle_attn_fwd_rect.argtypes = [P, P, P, P, P, L, L, L, L, D, I]
         lib.oracle_attn_fwd_rect.restype = I
+        U = ctypes.c_uint64
+        lib.oracle_philox4x64_10.argtypes = [P, P, P]
+        lib.oracle_philox4x64_10.restype = None
+        lib.oracle_dropout_mask.argtypes = [P, L, L, I, U, U]
+        lib.oracle_dropout_mask.restype = I
+        lib.oracle_attn_fwd_dropout.argtypes = [P, P, P, P, P, L, L, L, D, I, I, U, U]
+        lib.oracle_attn_fwd_dropout.restype = I
+        lib.oracle_attn_bwd_dropout.argtypes = [P, P, P, P, P, P, P, L, L, L, D, I, I, U, U]
+        lib.oracle_attn_bwd_dropout.restype = I
         lib.oracle_attn_fwd_blockmask.argtypes = [P, P, P, P, P, L, L, L, L, D, I, P, L, L, L]
         lib.oracle_attn_fwd_blockmask.restype = I
         lib.oracle_attn_fwd_tiled.argtypes = [P, P, P, P, P, L, L, L, D, I, L]
@@ -154,6 +163,51 @@ def attn_fwd_blockmask(q, k, v, scale: float, causal: bool, mask, br: int = 128,
     if rc != 0:
         raise RuntimeError("oracle_attn_fwd_blockmask failed (%d)" % rc)
     return o, lse
+
+
+def philox4x64_10(counter, key):
+    """Philox4x64-10 of a 4-word counter under a 2-word key -> 4 uint64 words."""
+    c = np.ascontiguousarray(counter, dtype=np.uint64)
+    k = np.ascontiguousarray(key, dtype=np.uint64)
+    out = np.zeros(4, dtype=np.uint64)
+    _load().oracle_philox4x64_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def dropout_mask(bh: int, N: int, keep_t: int, seed: int, offset: int):
+    """uint8 [N, N] keep mask of head bh (1 = kept) under the dropout contract."""
+    z = np.zeros((N, N), dtype=np.uint8)
+    rc = _load().oracle_dropout_mask(_ptr(z), bh, N, int(keep_t), int(seed), int(offset))
+    if rc != 0:
+        raise RuntimeError("oracle_dropout_mask failed (%d)" % rc)
+    return z
+
+
+def attn_fwd_dropout(q, k, v, scale: float, causal: bool, keep_t: int, seed: int, offset: int):
+    """Forward with dropout: keep probability keep_t / 256, kept weights x 256 / keep_t.
+    Returns (O, LSE); LSE is that of the undropped softmax."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, H, N))
+    rc = _load().oracle_attn_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B * H, N, d,
+                                         float(scale), int(bool(causal)), int(keep_t), int(seed), int(offset))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd_dropout failed (%d)" % rc)
+    return o, lse
+
+
+def attn_bwd_dropout(q, k, v, do, scale: float, causal: bool, keep_t: int, seed: int, offset: int):
+    """(dQ, dK, dV) of L = sum(O * dO) for the dropout forward above."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, H, N, d = q.shape
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    rc = _load().oracle_attn_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
+                                         B * H, N, d, float(scale), int(bool(causal)), int(keep_t), int(seed),
+                                         int(offset))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_bwd_dropout failed (%d)" % rc)
+    return dq, dk, dv
 
 
 def attn_fwd_rows(q, k, v, i0: int, i1: int, scale: float, causal: bool):

@@ -415,3 +415,98 @@ def test_blockmask_block_diagonal_is_independent_blocks():
         sl = slice(t * b, (t + 1) * b)
         ro, rlse = _torch_attention(q[:, :, sl], k[:, :, sl], v[:, :, sl], 0.8, False)
         assert np.max(np.abs(o[:, :, sl] - ro)) < 1e-12 and np.max(np.abs(lse[:, :, sl] - rlse)) < 1e-12
+
+
+# ---------------------------------------------------------------- dropout
+# Keep decisions from Philox4x64-10 (counter (j // 32, i, bh, 0), key (seed,
+# offset), byte j % 32 of the 32 output bytes < t), weights scaled by 256 / t.
+
+def test_philox_matches_numpy_bit_generator():
+    """numpy.random.Philox is Philox4x64-10; it advances its counter before each
+    block, so its first block under counter c is the function at c + 1."""
+    rng = np.random.default_rng(0)
+    for _ in range(20):
+        c = rng.integers(0, 2 ** 63, size=4, dtype=np.uint64)
+        c[0] = c[0] // 2  # no carry out of word 0
+        k = rng.integers(0, 2 ** 63, size=2, dtype=np.uint64) * np.uint64(2) + np.uint64(1)
+        ref = np.random.Philox(counter=c, key=k).random_raw(4)
+        c1 = c.copy()
+        c1[0] += np.uint64(1)
+        assert np.array_equal(oracle.philox4x64_10(c1, k), ref)
+
+
+def _numpy_block(counter, key):
+    """The Philox4x64-10 block at `counter` from numpy's bit generator, which
+    advances its 256-bit counter by one before each block: start one below."""
+    value = sum(int(w) << (64 * n) for n, w in enumerate(counter))
+    value = (value - 1) % (1 << 256)
+    below = np.array([(value >> (64 * n)) & (2 ** 64 - 1) for n in range(4)], dtype=np.uint64)
+    return np.random.Philox(counter=below, key=np.asarray(key, dtype=np.uint64)).random_raw(4)
+
+
+def _numpy_keep_mask(bh, N, t, seed, offset):
+    """The keep mask derived from numpy's Philox outputs directly."""
+    z = np.zeros((N, N), dtype=np.uint8)
+    for i in range(N):
+        for jb in range((N + 31) // 32):
+            w = _numpy_block([jb, i, bh, 0], [seed, offset])
+            b = np.frombuffer(np.asarray(w, dtype="<u8").tobytes(), dtype=np.uint8)
+            for jj in range(min(32, N - jb * 32)):
+                z[i, jb * 32 + jj] = b[jj] < t
+    return z
+
+
+@pytest.mark.parametrize("bh,N,t,seed,offset", [(0, 40, 230, 7, 0), (3, 70, 128, 2 ** 40 + 5, 9), (1, 33, 1, 1, 1)])
+def test_dropout_mask_matches_numpy_philox_bytes(bh, N, t, seed, offset):
+    assert np.array_equal(oracle.dropout_mask(bh, N, t, seed, offset), _numpy_keep_mask(bh, N, t, seed, offset))
+
+
+def test_dropout_keep_rate_is_t_over_256():
+    for t in (26, 128, 230):
+        z = oracle.dropout_mask(2, 300, t, 1234, 5)
+        p = t / 256
+        n = z.size
+        assert abs(z.mean() - p) <= 5 * math.sqrt(p * (1 - p) / n)
+
+
+def _torch_dropout_reference(q, k, v, do, scale, causal, z, t):
+    """torch fp64: O = (256/t) (softmax(S) o Z) V and its autograd gradients."""
+    q, k, v, do = (torch.tensor(np.asarray(x, dtype=np.float64), requires_grad=True) for x in (q, k, v, do))
+    s = torch.matmul(q, k.transpose(-1, -2)) * scale
+    if causal:
+        N = s.shape[-1]
+        s = s.masked_fill(~torch.tril(torch.ones(N, N, dtype=torch.bool)), float("-inf"))
+    p = torch.softmax(s, dim=-1)
+    o = torch.matmul(p * torch.as_tensor(z, dtype=torch.float64) * (256.0 / t), v)
+    (o * do).sum().backward()
+    return o.detach().numpy(), torch.logsumexp(s, dim=-1).detach().numpy(), q.grad.numpy(), k.grad.numpy(), \
+        v.grad.numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("t", [230, 100])
+def test_dropout_forward_and_backward_match_torch_with_the_mask(causal, t):
+    B, H, N, d = 1, 2, 37, 5
+    q, k, v, do = (_rand((B, H, N, d), seed=60 + s) for s in range(4))
+    seed, offset = 99, 3
+    z = np.stack([oracle.dropout_mask(h, N, t, seed, offset) for h in range(H)])[None]
+    o, lse = oracle.attn_fwd_dropout(q, k, v, 0.5, causal, t, seed, offset)
+    dq, dk, dv = oracle.attn_bwd_dropout(q, k, v, do, 0.5, causal, t, seed, offset)
+    ro, rlse, rdq, rdk, rdv = _torch_dropout_reference(q, k, v, do, 0.5, causal, z, t)
+    for a, b in ((o, ro), (lse, rlse), (dq, rdq), (dk, rdk), (dv, rdv)):
+        assert np.max(np.abs(a - b)) < 1e-12
+
+
+def test_dropout_with_t256_is_plain_attention_and_t0_is_zero():
+    q, k, v, do = (_rand((1, 2, 29, 4), seed=70 + s) for s in range(4))
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd_dropout(q, k, v, 0.7, causal, 256, 5, 6)
+        ro, rlse = oracle.attn_fwd(q, k, v, 0.7, causal)
+        assert np.array_equal(o, ro) and np.array_equal(lse, rlse)
+        g = oracle.attn_bwd_dropout(q, k, v, do, 0.7, causal, 256, 5, 6)
+        rg = oracle.attn_bwd(q, k, v, do, 0.7, causal)
+        for a, b in zip(g, rg):
+            assert np.max(np.abs(a - b)) < 1e-14
+        o0, lse0 = oracle.attn_fwd_dropout(q, k, v, 0.7, causal, 0, 5, 6)
+        assert np.all(o0 == 0) and np.array_equal(lse0, rlse)
+        assert all(np.all(x == 0) for x in oracle.attn_bwd_dropout(q, k, v, do, 0.7, causal, 0, 5, 6))
