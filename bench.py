@@ -893,6 +893,155 @@ def run_fp8(args, w):
     return line
 
 
+# ------------------------------------------------------------------ forward with dropout
+
+DROPOUT_METRIC = "attention forward with dropout TFLOPS on 1 B200 and fraction of dense BF16 tensor peak"
+
+
+def dropout_oracle_sample(w, heads: int, seed: int):
+    """fp64 oracle dropout forward on `heads` heads; returns (seconds, flops, threads)."""
+    from exact_io_aware_53_b200.workloads import random_tensors
+    from oracle import oracle
+    q, k, v, _ = random_tensors((1, heads, w.N, w.d), torch_bf16(), seed=seed)
+    t0 = time.perf_counter()
+    oracle.attn_fwd_dropout(q, k, v, w.scale, w.causal, w.keep_t, w.seed, w.offset)
+    dt = time.perf_counter() - t0
+    return dt, w.flops() / (w.B * w.H) * heads, oracle.num_threads()
+
+
+def run_reference_dropout(args, w):
+    rank, world, _ = rank_env()
+    if rank != 0:
+        return 0
+    for i in range(args.warmup):
+        dropout_oracle_sample(w, 1, w.seed + i)
+    times, fl, thr = [], 0.0, 1
+    for i in range(args.steps):
+        dt, fl, thr = dropout_oracle_sample(w, 1, w.seed + 100 + i)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = fl / (ms / 1e3) / 1e12
+    line = {"impl": "reference", "metric": DROPOUT_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": 1, "H": 1, "N": w.N, "d": w.d, "causal": w.causal,
+                       "keep_t": w.keep_t, "sample": "one head per step", "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                             "sample": "one head of %s per step (fp64)" % w.name},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_dropout(args, w):
+    """One step = fa_fwd_dropout over the whole batch, inputs resident in device memory."""
+    import torch
+    from exact_io_aware_53_b200 import fa
+    from exact_io_aware_53_b200.workloads import random_tensors
+
+    rank, world, local = rank_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        init_dist(world, "nccl", torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    B, H, N, d = w.B, w.H, w.N, w.d
+    hq, hk, hv, _ = random_tensors((B, H, N, d), torch.bfloat16, seed=rank_seed(w.seed, rank))
+    q, k, v = (t.to(dev) for t in (hq, hk, hv))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    launches = [0]
+
+    def step():
+        rc = fa.fwd_dropout_raw(q, k, v, o, lse, w.scale, w.causal, w.keep_t, w.seed, w.offset)
+        launches[0] += fa.last_launch_count()
+        if rc:
+            raise fa.FAError(rc, "fa_fwd_dropout")
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after warm-up: %s" % fa.status_string(st))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid)
+    sampler.start()
+    time.sleep(0.3)
+    launches[0] = 0
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    st = fa.check_device_status()
+    if st:
+        raise RuntimeError("device status after timing: %s" % fa.status_string(st))
+    ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ms = max_over_ranks(ms_local, world, dev)
+    fl = w.flops()
+    value = world * fl / (ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = fl / (ms_local / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "decode_partial_kernel (dropout, direct output)", "achieved": achieved,
+                "peak": peak, "unit": UNIT, "frac": achieved / peak, "peak_source": "bf16_tflops %s" % peak_src,
+                "algorithmic_flops_per_launch": fl, "ms_per_launch": ms_local,
+                "traffic": measured_traffic("dropout", w.name), "traffic_unit": "bytes per launch (ncu dram read+write)"}
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (t.pin_memory() for t in (hq, hk, hv))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        steps = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        a.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
+        e2e = {"value": world * fl / (ems / 1e3) / 1e12, "unit": UNIT, "ms_per_step": ems,
+               "h2d_bytes_per_step": 3 * hq.numel() * 2, "d2h_bytes_per_step": ho.numel() * 2 + hl.numel() * 4,
+               "steps": steps, "api": "fa.fwd_dropout_raw with q, k, v from and o, lse to pinned host memory"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, cfl, thr = dropout_oracle_sample(w, 1, w.seed)
+        cpu = {"value": cfl / dt / 1e12, "unit": UNIT, "cores": thr, "kind": "oracle",
+               "sample": "1 of %d heads (N=%d, d=%d, causal=%s, keep %d/256), fp64, %.1f s" % (
+                   B * H, N, d, w.causal, w.keep_t, dt)}
+    line = {"metric": DROPOUT_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal, "keep_t": w.keep_t,
+                       "parallelism": "dp%d (independent batches per GPU, no collective)" % world,
+                       "l2": "inputs larger than L2 (q, k, v = %.0f MB per GPU)" % (3 * B * H * N * d * 2 / 1e6)},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches[0], "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return line
+
+
 def probe_mma_rate():
     """Cycles per tcgen05 MMA instruction for the shapes the kernels issue
     (fa_selftest_umma_rate, one CTA per SM); printed as JSON lines."""
@@ -932,14 +1081,23 @@ def main(argv=None):
     if args.probe_mma_rate:
         probe_mma_rate()
         return 0
-    from exact_io_aware_53_b200.workloads import BLOCKSPARSE_WORKLOADS, DECODE_WORKLOADS, FP8_WORKLOADS, WORKLOADS
-    known = list(WORKLOADS) + list(DECODE_WORKLOADS) + list(BLOCKSPARSE_WORKLOADS) + list(FP8_WORKLOADS)
+    from exact_io_aware_53_b200.workloads import (BLOCKSPARSE_WORKLOADS, DECODE_WORKLOADS, DROPOUT_WORKLOADS,
+                                                  FP8_WORKLOADS, WORKLOADS)
+    known = (list(WORKLOADS) + list(DECODE_WORKLOADS) + list(BLOCKSPARSE_WORKLOADS) + list(FP8_WORKLOADS) +
+             list(DROPOUT_WORKLOADS))
     if args.workload != "all" and args.workload not in known:
         ap.error("unknown workload %s (choose from %s)" % (args.workload, ", ".join(known)))
     names = known if args.workload == "all" else [args.workload]
     rc = 0
     try:
         for name in names:
+            if name in DROPOUT_WORKLOADS:
+                w = DROPOUT_WORKLOADS[name]
+                if args.impl == "reference":
+                    rc |= run_reference_dropout(args, w)
+                else:
+                    run_dropout(args, w)
+                continue
             if name in FP8_WORKLOADS:
                 w = FP8_WORKLOADS[name]
                 if args.impl == "reference":

@@ -28,6 +28,14 @@
 // per 32-bit column.  The descales fold into the exponent scale (q, k) and
 // the epilogue factor (v).
 //
+// Dropout variant (DROPOUT): the square problem with each weight P_ij kept
+// with probability t / 256 and scaled by 256 / t.  The keep bit is byte
+// j % 32 of Philox4x64-10 (Salmon, Moraes, Dror and Shaw, "Parallel random
+// numbers: as easy as 1, 2, 3", SC 2011) at counter (j / 32, i, bh, 0) under
+// key (seed, offset), compared with t; so the mask is a pure function of its
+// position and can be regenerated anywhere.  The row sum l and the LSE use the
+// undropped weights.
+//
 // The work is bound by reading K and V.  A CTA keeps one Q tile, so S and P
 // share TMEM without a second tile to ping-pong with; instead two CTAs share
 // an SM (96 KB shared memory, 256 TMEM columns each) and one's softmax runs
@@ -113,6 +121,29 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, fl
     return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
+// Philox4x64-10 on (x0, x1, x2, x3) under key (k0, k1), in place: ten rounds
+// of the two 64 x 64 -> 128-bit multiplies with the paper's Philox-4x64
+// multipliers, the key bumped by its Weyl constants between rounds.
+__device__ __forceinline__ void philox4x64_10(uint64_t& x0, uint64_t& x1, uint64_t& x2, uint64_t& x3, uint64_t k0,
+                                              uint64_t k1)
+{
+    constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += W0;
+            k1 += W1;
+        }
+        const uint64_t hi0 = __umul64hi(M0, x0), lo0 = M0 * x0;
+        const uint64_t hi1 = __umul64hi(M1, x2), lo1 = M1 * x2;
+        x0 = hi1 ^ x1 ^ k0;
+        x1 = lo1;
+        x2 = hi0 ^ x3 ^ k1;
+        x3 = lo0;
+    }
+}
+
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
 {
     uintptr_t a = reinterpret_cast<uintptr_t>(p);
@@ -145,7 +176,7 @@ __device__ void write_empty_rows(const DecodeParams& p, int qt, int bh, size_t p
     }
 }
 
-template <int D, bool CAUSAL, bool SPARSE, bool FP8>
+template <int D, bool CAUSAL, bool SPARSE, bool FP8, bool DROPOUT>
 __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __grid_constant__ DecodeParams p)
 {
     using C = Cfg<D, SPARSE, FP8>;
@@ -380,14 +411,31 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
             constexpr int PER_WORD = FP8 ? 4 : 2;  // P elements per TMEM column
             uint32_t pk[BN / PER_WORD];
             float sum0 = 0.f, sum1 = 0.f;  // two accumulation chains
+            uint64_t rw[4] = {0, 0, 0, 0};  // DROPOUT: the 32 random bytes of the current 32 columns
 #pragma unroll
             for (int c = 0; c < BN; c += 4) {
-                const float p0 = ex2_approx(fmaf(s[c], cl2, -m_use));
-                const float p1 = ex2_approx(fmaf(s[c + 1], cl2, -m_use));
-                const float p2 = ex2_approx(fmaf(s[c + 2], cl2, -m_use));
-                const float p3 = ex2_approx(fmaf(s[c + 3], cl2, -m_use));
+                float p0 = ex2_approx(fmaf(s[c], cl2, -m_use));
+                float p1 = ex2_approx(fmaf(s[c + 1], cl2, -m_use));
+                float p2 = ex2_approx(fmaf(s[c + 2], cl2, -m_use));
+                float p3 = ex2_approx(fmaf(s[c + 3], cl2, -m_use));
                 sum0 += p0 + p1;
                 sum1 += p2 + p3;
+                if constexpr (DROPOUT) {
+                    if (c % 32 == 0) {
+                        rw[0] = static_cast<uint64_t>(tile_of(jj)) * (BN / 32) + c / 32;
+                        rw[1] = static_cast<uint64_t>(row);
+                        rw[2] = static_cast<uint64_t>(bh);
+                        rw[3] = 0;
+                        philox4x64_10(rw[0], rw[1], rw[2], rw[3], p.seed, p.offset);
+                    }
+                    // bytes (c % 32) .. +3 of the block, little-endian
+                    const uint32_t b4 = static_cast<uint32_t>(rw[(c % 32) / 8] >> (8 * (c % 8)));
+                    const uint32_t t = static_cast<uint32_t>(p.keep_t);
+                    p0 = (b4 & 0xFFu) < t ? p0 : 0.f;
+                    p1 = ((b4 >> 8) & 0xFFu) < t ? p1 : 0.f;
+                    p2 = ((b4 >> 16) & 0xFFu) < t ? p2 : 0.f;
+                    p3 = (b4 >> 24) < t ? p3 : 0.f;
+                }
                 if constexpr (FP8) {
                     pk[c / 4] = pack_e4m3x4(p0, p1, p2, p3);
                 } else {
@@ -418,8 +466,8 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
         if (ok && warp_wait(o_full, 0, p.ctl)) {
             tc_fence_after();
             const bool any = l > 0.f;
-            // e4m3 V carries its descale factor into the output
-            const float inv_l = any ? (FP8 ? p.o_scale : 1.f) / l : 0.f;
+            // e4m3 V carries its descale factor into the output, dropout its 256 / t
+            const float inv_l = any ? ((FP8 || DROPOUT) ? p.o_scale : 1.f) / l : 0.f;
             const float lse_row = any ? (m + __log2f(l)) * LN2 : -INFINITY;
             if (p.direct) {
                 // the only range: O / l as bf16 and the LSE go straight to the outputs
@@ -529,11 +577,11 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
     if (lane == 0) p.lse[rid] = W > 0.f ? M + __logf(W) : -INFINITY;
 }
 
-template <int D, bool CAUSAL, bool SPARSE, bool FP8 = false>
+template <int D, bool CAUSAL, bool SPARSE, bool FP8 = false, bool DROPOUT = false>
 cudaError_t launch(const DecodeParams& p, cudaStream_t stream)
 {
     using C = Cfg<D, SPARSE, FP8>;
-    auto kern = decode_partial_kernel<D, CAUSAL, SPARSE, FP8>;
+    auto kern = decode_partial_kernel<D, CAUSAL, SPARSE, FP8, DROPOUT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_split, (p.Nq + BM - 1) / BM, p.BH);
@@ -568,6 +616,16 @@ cudaError_t launch_blocksparse_sm100(const DecodeParams& p, int d, bool causal, 
     if (d == 128)
         return causal ? deck::launch<128, true, true>(p, stream) : deck::launch<128, false, true>(p, stream);
     return causal ? deck::launch<64, true, true>(p, stream) : deck::launch<64, false, true>(p, stream);
+}
+
+cudaError_t launch_dropout_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream)
+{
+    if (!p.direct || p.n_split != 1) return cudaErrorInvalidValue;
+    if (d == 128)
+        return causal ? deck::launch<128, true, false, false, true>(p, stream)
+                      : deck::launch<128, false, false, false, true>(p, stream);
+    return causal ? deck::launch<64, true, false, false, true>(p, stream)
+                  : deck::launch<64, false, false, false, true>(p, stream);
 }
 
 cudaError_t launch_fp8_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream)

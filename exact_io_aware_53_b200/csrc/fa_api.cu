@@ -368,6 +368,48 @@ int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, flo
     return st;
 }
 
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                   float scale, int causal, int keep_t, unsigned long long seed, unsigned long long offset,
+                   void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (keep_t < 0 || keep_t > 256) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+    if ((st = get_encoder()) != FA_OK) return st;
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.BH = static_cast<int>(BH);
+    p.Nq = N;
+    p.Nk = N;
+    p.n_split = 1;
+    p.tiles_per_split = (N + 127) / 128;
+    p.scale_log2 = scale * kLog2e;
+    p.direct = 1;
+    p.keep_t = keep_t;
+    p.o_scale = keep_t > 0 ? 256.0f / static_cast<float>(keep_t) : 0.0f;
+    p.seed = seed;
+    p.offset = offset;
+    st = cuda_status(launch_dropout_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    if (st == FA_OK) g_last_launches = 1;
+    return st;
+}
+
 int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, float q_descale, float k_descale,
                float v_descale, int B, int H, int N, int d, float scale, int causal, void* stream)
 {

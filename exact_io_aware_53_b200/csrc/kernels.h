@@ -54,7 +54,10 @@ struct DecodeParams {
     int tiles_per_split;  // 128-key tiles per range
     float scale_log2;
     int direct;           // 1: one range; the range kernel writes o (bf16) and lse itself
-    float o_scale;        // e4m3 only: factor on O (the V descale)
+    float o_scale;        // e4m3: factor on O (the V descale); dropout: 256 / keep_t
+    int keep_t;           // dropout: keep iff the element's random byte < keep_t
+    uint64_t seed;        // dropout: Philox key (seed, offset)
+    uint64_t offset;
     // block-sparse only: uint8 [.][n_qt][n_kt] mask of (query tile, key tile)
     // pairs, head h = bh % H at mask + h * mask_h_stride
     const uint8_t* mask;
@@ -70,6 +73,8 @@ constexpr int kMaxMaskKeyTiles = 2048;
 cudaError_t launch_decode_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream);
 // Block-sparse forward: one range per Q tile, direct output.
 cudaError_t launch_blocksparse_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream);
+// Forward with dropout (Philox4x64-10 keep mask): one range per Q tile, direct output.
+cudaError_t launch_dropout_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream);
 // e4m3 forward (d = 128): tm_q / tm_k / tm_v are uint8 maps with a {128, 128}
 // box; one range per Q tile, direct output.
 cudaError_t launch_fp8_sm100(const DecodeParams& p, int d, bool causal, cudaStream_t stream);

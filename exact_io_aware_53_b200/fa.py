@@ -45,6 +45,8 @@ _SIGS = {
     "fa_fwd_blocksparse": ([P, P, P, P, P, P, ctypes.c_longlong, I, I, I, I, ctypes.c_float, I, P], I),
     "fa_fwd_fp8": ([P, P, P, P, P, ctypes.c_float, ctypes.c_float, ctypes.c_float, I, I, I, I, ctypes.c_float, I, P],
                    I),
+    "fa_fwd_dropout": ([P, P, P, P, P, I, I, I, I, ctypes.c_float, I, I, ctypes.c_ulonglong, ctypes.c_ulonglong, P],
+                       I),
     "fa_status_string": ([I], ctypes.c_char_p),
     "fa_last_launch_count": ([], I),
     "fa_last_cuda_error": ([], I),
@@ -188,6 +190,27 @@ def fwd_blocksparse(q, k, v, block_mask, causal: bool = False, scale: float | No
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     _check(fwd_blocksparse_raw(q, k, v, o, lse, m, scale, causal, stream), "fa_fwd_blocksparse")
+    return o, lse
+
+
+def fwd_dropout_raw(q, k, v, o, lse, scale: float, causal: bool, keep_t: int, seed: int, offset: int = 0,
+                    stream=None) -> int:
+    """Enqueue the dropout forward on preallocated tensors (keep probability keep_t / 256)."""
+    B, H, N, d = _shape(q)
+    return _lib.fa_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, N, d, float(scale),
+                               int(bool(causal)), int(keep_t), int(seed), int(offset), _stream(stream))
+
+
+def fwd_dropout(q, k, v, keep_t: int, seed: int, offset: int = 0, causal: bool = False, scale: float | None = None,
+                stream=None):
+    """O, LSE with dropout: weights kept with probability keep_t / 256 (Philox4x64-10
+    mask from (seed, offset)) and scaled by 256 / keep_t; LSE of the undropped softmax."""
+    _same(q, k, v, dtype=torch.bfloat16)
+    B, H, N, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _check(fwd_dropout_raw(q, k, v, o, lse, scale, causal, keep_t, seed, offset, stream), "fa_fwd_dropout")
     return o, lse
 
 

@@ -163,6 +163,36 @@ FP8_WORKLOADS = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class DropoutWorkload:
+    """Square attention with dropout: keep probability keep_t / 256 from the
+    Philox4x64-10 contract, generator key (seed, offset)."""
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    keep_t: int
+    seed: int = 0
+    offset: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    def flops(self) -> float:
+        """4*B*H*N^2*d, halved under the causal mask (dropped weights are still computed)."""
+        f = 4.0 * self.B * self.H * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+
+DROPOUT_WORKLOADS = {
+    "dropout_bf16_4x16x4096x128_causal_keep230": DropoutWorkload("dropout_bf16_4x16x4096x128_causal_keep230", 4, 16,
+                                                                 4096, 128, True, 230, seed=5001, offset=0),
+}
+
+
 def quantize_e4m3(x: torch.Tensor):
     """Per-tensor e4m3 quantization of an fp32 tensor: descale = amax / 448
     (448 is e4m3's largest finite value), x8 = (x / descale) rounded to

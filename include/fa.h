@@ -214,6 +214,26 @@ int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, flo
                        void* stream);
 
 /*
+ * Forward with dropout, bf16: each softmax weight P_ij is kept with
+ * probability keep_t / 256 and kept weights are scaled by 256 / keep_t, so
+ *   O_i = (256 / keep_t) * sum_j P_ij Z_ij v_j,  LSE_i of the undropped P.
+ * The pages list dropout among the kernel benchmark settings (guide, "What to
+ * inspect"); the generator is this library's contract: Z_ij = 1 iff byte
+ * j % 32 of Philox4x64-10 (Salmon et al., SC 2011) at counter
+ * (j / 32, i, b * H + h, 0) under key (seed, offset), little-endian, is below
+ * keep_t.  The mask is a pure function of (seed, offset, position), so a
+ * backward pass can regenerate it.
+ *   q, k, v, o: bf16 [B][H][N][d]; lse: fp32 [B][H][N]; d = 64 or 128;
+ *   keep_t in [0, 256] (256: no dropout; 0: O = 0).
+ * One kernel is enqueued on `stream`; nothing is allocated.  Errors as for
+ * fa_fwd, plus FA_ERR_INVALID_ARG for keep_t outside [0, 256] and
+ * FA_ERR_UNSUPPORTED for B*H > 65535.
+ */
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                   float scale, int causal, int keep_t, unsigned long long seed, unsigned long long offset,
+                   void* stream);
+
+/*
  * FP8 forward: q, k, v in e4m3 (OCP FP8, 1-4-3, no infinities) with one
  * descale factor per tensor, so the values are q8 * q_descale and so on; the
  * FP8 support of the FlashAttention-3 line ("Lineage" in the explainer).

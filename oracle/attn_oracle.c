@@ -610,10 +610,11 @@ int oracle_dropout_mask(unsigned char* z, long bh, long N, int t, uint64_t seed,
 }
 
 /* Forward with dropout (definition above).  t = 256 is plain attention;
- * t = 0 drops everything (O = 0). */
+ * t = 0 drops everything (O = 0).  The heads given are heads bh0 .. bh0 + BH - 1
+ * of the whole problem (their index enters the generator's counter). */
 int oracle_attn_fwd_dropout(const double* q, const double* k, const double* v, double* o,
                             double* lse, long BH, long N, long d, double scale, int causal,
-                            int t, uint64_t seed, uint64_t offset)
+                            int t, uint64_t seed, uint64_t offset, long bh0)
 {
     if (BH < 0 || N < 0 || d < 1 || t < 0 || t > 256) return -1;
     const double s_keep = t > 0 ? 256.0 / t : 0.0;
@@ -645,7 +646,7 @@ int oracle_attn_fwd_dropout(const double* q, const double* k, const double* v, d
                 }
                 for (long t2 = 0; t2 < d; ++t2) oi[t2] = 0.0;
                 for (long j = 0; j < nk; ++j) {
-                    if (!dropout_keep(seed, offset, h, i, j, t)) continue;
+                    if (!dropout_keep(seed, offset, bh0 + h, i, j, t)) continue;
                     const double pj = s_keep * srow[j] / l;
                     const double* vj = v + base + j * d;
                     for (long t2 = 0; t2 < d; ++t2) oi[t2] += pj * vj[t2];

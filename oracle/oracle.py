@@ -56,7 +56,7 @@ def _load():
         lib.oracle_philox4x64_10.restype = None
         lib.oracle_dropout_mask.argtypes = [P, L, L, I, U, U]
         lib.oracle_dropout_mask.restype = I
-        lib.oracle_attn_fwd_dropout.argtypes = [P, P, P, P, P, L, L, L, D, I, I, U, U]
+        lib.oracle_attn_fwd_dropout.argtypes = [P, P, P, P, P, L, L, L, D, I, I, U, U, L]
         lib.oracle_attn_fwd_dropout.restype = I
         lib.oracle_attn_bwd_dropout.argtypes = [P, P, P, P, P, P, P, L, L, L, D, I, I, U, U]
         lib.oracle_attn_bwd_dropout.restype = I
@@ -183,15 +183,17 @@ def dropout_mask(bh: int, N: int, keep_t: int, seed: int, offset: int):
     return z
 
 
-def attn_fwd_dropout(q, k, v, scale: float, causal: bool, keep_t: int, seed: int, offset: int):
+def attn_fwd_dropout(q, k, v, scale: float, causal: bool, keep_t: int, seed: int, offset: int, bh0: int = 0):
     """Forward with dropout: keep probability keep_t / 256, kept weights x 256 / keep_t.
+    The heads given are heads bh0, bh0 + 1, ... (b * H + h) of the whole problem.
     Returns (O, LSE); LSE is that of the undropped softmax."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, d = q.shape
     o = np.empty_like(q)
     lse = np.empty((B, H, N))
     rc = _load().oracle_attn_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B * H, N, d,
-                                         float(scale), int(bool(causal)), int(keep_t), int(seed), int(offset))
+                                         float(scale), int(bool(causal)), int(keep_t), int(seed), int(offset),
+                                         int(bh0))
     if rc != 0:
         raise RuntimeError("oracle_attn_fwd_dropout failed (%d)" % rc)
     return o, lse

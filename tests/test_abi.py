@@ -172,3 +172,18 @@ def test_fp8_argument_errors(lib):
     assert call(ds=(1e30, 1e30, 1.0)) == lib.FA_ERR_INVALID_ARG   # scale * descales overflows
     assert call(d=64) == lib.FA_ERR_UNSUPPORTED
     assert call(q=P(8)) == lib.FA_ERR_MISALIGNED
+
+
+def test_dropout_argument_errors(lib):
+    f = lib._lib.fa_fwd_dropout
+    P = ctypes.c_void_p
+
+    def call(B=1, H=1, N=256, d=128, scale=0.1, causal=0, t=230, q=P(16)):
+        return f(q, P(16), P(16), P(16), P(16), B, H, N, d, scale, causal, t, 1, 0, P(0))
+
+    assert call(q=P(0)) == lib.FA_ERR_INVALID_ARG
+    assert call(t=-1) == lib.FA_ERR_INVALID_ARG
+    assert call(t=257) == lib.FA_ERR_INVALID_ARG
+    assert call(N=0) == lib.FA_ERR_INVALID_ARG
+    assert call(d=80) == lib.FA_ERR_UNSUPPORTED
+    assert call(q=P(4)) == lib.FA_ERR_MISALIGNED

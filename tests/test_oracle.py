@@ -510,3 +510,13 @@ def test_dropout_with_t256_is_plain_attention_and_t0_is_zero():
         o0, lse0 = oracle.attn_fwd_dropout(q, k, v, 0.7, causal, 0, 5, 6)
         assert np.all(o0 == 0) and np.array_equal(lse0, rlse)
         assert all(np.all(x == 0) for x in oracle.attn_bwd_dropout(q, k, v, do, 0.7, causal, 0, 5, 6))
+
+
+def test_dropout_head_offset_selects_the_heads_generator_stream():
+    """Heads given alone with bh0 = their index reproduce the whole problem's rows."""
+    q, k, v = (_rand((2, 3, 40, 4), seed=80 + s) for s in range(3))
+    o, lse = oracle.attn_fwd_dropout(q, k, v, 0.6, True, 200, 11, 2)
+    for b, h in ((0, 2), (1, 0), (1, 2)):
+        oh, lh = oracle.attn_fwd_dropout(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], 0.6, True,
+                                         200, 11, 2, bh0=b * 3 + h)
+        assert np.array_equal(oh[0, 0], o[b, h]) and np.array_equal(lh[0, 0], lse[b, h])
