@@ -34,6 +34,11 @@
  * size; they exist only to pin the "block size never changes the answer" and
  * "online softmax == naive softmax" assertions ("Solve it yourself").
  *
+ * Further functions, each with its own comment: Nq queries against Nk keys
+ * (oracle_attn_fwd_rect), a block mask (oracle_attn_fwd_blockmask), and
+ * dropout with a Philox4x64-10 keep mask (oracle_attn_fwd_dropout /
+ * oracle_attn_bwd_dropout).
+ *
  * Layout: every tensor is [BH][N][d] row-major fp64 (BH = batch * heads);
  * lse is [BH][N].  Masking convention (not fixed by the pages): square,
  * top-left aligned causal mask, key j allowed iff j <= i.
