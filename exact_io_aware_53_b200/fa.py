@@ -165,10 +165,24 @@ def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, n_spl
     return o, lse
 
 
+def _check_mask(m, H: int, N: int):
+    """The kernel reads mask row i of head h at h * stride + i * T: the mask must be
+    a CUDA uint8 tensor [T, T] or [1 or H, T, T] whose last two dimensions are dense."""
+    T = (N + 127) // 128
+    shape = tuple(m.shape)
+    ok = (m.dtype == torch.uint8 and m.is_cuda and
+          (shape == (T, T) or (m.dim() == 3 and shape[1:] == (T, T) and shape[0] in (1, H))) and
+          m.stride(-1) == 1 and m.stride(-2) == T)
+    if not ok:
+        raise ValueError("block_mask must be a CUDA uint8 tensor [T, T] or [1 or H, T, T] with dense rows, "
+                         "T = ceil(N / 128) = %d; got %s %s strides %s" % (T, m.dtype, shape, tuple(m.stride())))
+
+
 def fwd_blocksparse_raw(q, k, v, o, lse, block_mask, scale: float, causal: bool, stream=None) -> int:
     """Enqueue the block-sparse forward on preallocated tensors; block_mask is
     a CUDA uint8 tensor [T, T] (shared by every head) or [H, T, T], T = ceil(N/128)."""
     B, H, N, d = _shape(q)
+    _check_mask(block_mask, H, N)
     stride = 0 if block_mask.dim() == 2 or block_mask.shape[0] == 1 else int(block_mask.stride(0))
     return _lib.fa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_mask), stride,
                                    B, H, N, d, float(scale), int(bool(causal)), _stream(stream))

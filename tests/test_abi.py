@@ -187,3 +187,16 @@ def test_dropout_argument_errors(lib):
     assert call(N=0) == lib.FA_ERR_INVALID_ARG
     assert call(d=80) == lib.FA_ERR_UNSUPPORTED
     assert call(q=P(4)) == lib.FA_ERR_MISALIGNED
+
+
+def test_blocksparse_mask_layout_is_checked(lib):
+    """A mask whose rows are not dense (a transposed view) or of the wrong dtype
+    or shape is refused before the library is called."""
+    import torch
+    m = torch.ones((4, 4), dtype=torch.uint8)
+    for bad in (m.t().contiguous().t()[:, :3], m.to(torch.int32), torch.ones((2, 4, 4), dtype=torch.uint8).transpose(1, 2),
+                torch.ones((3, 3), dtype=torch.uint8)):
+        with pytest.raises(ValueError):
+            lib._check_mask(bad, 2, 512)
+    with pytest.raises(ValueError):  # not on a GPU
+        lib._check_mask(m, 2, 512)
