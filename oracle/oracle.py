@@ -6,6 +6,10 @@ shares no code with the CUDA path.  The C source states what each function
 computes and which passage of the FlashAttention pages it follows.
 
 All arrays are float64, laid out [B, H, N, d] (lse: [B, H, N]).
+
+ORACLE_LIB, when set, names a prebuilt library to load instead of building
+``attn_oracle.c``: the mutation tests point it at deliberately broken builds to
+check that the pins catch each mistake.
 """
 from __future__ import annotations
 
@@ -22,22 +26,32 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 _lib = None
 
 
+GCC_FLAGS = ["-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC"]
+
+
+def compile_source(src: str, out: str) -> None:
+    """gcc `src` into the shared library `out` with the oracle's flags."""
+    tmp = out + ".tmp.%d" % os.getpid()
+    subprocess.check_call(["gcc", *GCC_FLAGS, src, "-o", tmp, "-lm"])
+    os.replace(tmp, out)
+
+
 def build(force: bool = False) -> str:
     """Compile ``liboracle.so`` with gcc (OpenMP, no fast-math, no FMA contraction)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp.%d" % os.getpid()
-        subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
-             "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"])
-        os.replace(tmp, _LIB)
+        compile_source(_SRC, _LIB)
     return _LIB
 
 
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(_LIB)
+        override = os.environ.get("ORACLE_LIB")
+        if override:
+            lib = ctypes.CDLL(override)
+        else:
+            build()
+            lib = ctypes.CDLL(_LIB)
         P = ctypes.c_void_p
         L = ctypes.c_long
         D = ctypes.c_double
