@@ -36,10 +36,11 @@
 // position and can be regenerated anywhere.  The row sum l and the LSE use the
 // undropped weights.
 //
-// The work is bound by reading K and V.  A CTA keeps one Q tile, so S and P
-// share TMEM without a second tile to ping-pong with; instead two CTAs share
-// an SM (96 KB shared memory, 256 TMEM columns each) and one's softmax runs
-// while the other's loads and MMAs do.
+// Decoding is bound by reading K and V; the square variants by the softmax's
+// exponentials (and, with dropout, the generator).  A CTA keeps one Q tile,
+// so S and P share TMEM without a second tile to ping-pong with; instead two
+// CTAs share an SM (up to 104 KB shared memory, 256 TMEM columns each) and
+// one's softmax runs while the other's loads and MMAs do.
 //
 //   warp 5      TMA producer: Q tile, then K_j, V_j through a smem ring
 //   warp 4      MMA issuer (converged warp, elected lane)
