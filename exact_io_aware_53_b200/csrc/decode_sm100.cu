@@ -582,6 +582,9 @@ template <int D, bool CAUSAL, bool SPARSE, bool FP8 = false, bool DROPOUT = fals
 cudaError_t launch(const DecodeParams& p, cudaStream_t stream)
 {
     using C = Cfg<D, SPARSE, FP8>;
+    // two CTAs per SM: shared memory (228 KB per SM, 1 KB reserved per CTA) and TMEM
+    static_assert(2 * (C::SMEM_BYTES + 1024) <= 228 * 1024, "two range CTAs must fit one SM's shared memory");
+    static_assert(2 * C::TMEM_COLS <= 512, "two range CTAs must fit one SM's tensor memory");
     auto kern = decode_partial_kernel<D, CAUSAL, SPARSE, FP8, DROPOUT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
