@@ -200,3 +200,29 @@ def test_blocksparse_mask_layout_is_checked(lib):
             lib._check_mask(bad, 2, 512)
     with pytest.raises(ValueError):  # not on a GPU
         lib._check_mask(m, 2, 512)
+
+
+def test_blocksparse_mask_layout_accepts_dense_device_masks(lib):
+    """The accepting side of the check, with stand-ins that report a device
+    tensor's dtype, shape and strides (no GPU here)."""
+    import torch
+
+    class DeviceView:
+        def __init__(self, t):
+            self._t, self.dtype, self.is_cuda = t, t.dtype, True
+            self.shape = t.shape
+
+        def dim(self):
+            return self._t.dim()
+
+        def stride(self, i=None):
+            return self._t.stride() if i is None else self._t.stride(i)
+
+    T = 4  # N = 512
+    for good in (torch.ones((T, T), dtype=torch.uint8), torch.ones((1, T, T), dtype=torch.uint8),
+                 torch.ones((3, T, T), dtype=torch.uint8), torch.ones((6, T, T), dtype=torch.uint8)[::2]):
+        lib._check_mask(DeviceView(good), 3, 512)
+    with pytest.raises(ValueError):
+        lib._check_mask(DeviceView(torch.ones((2, T, T), dtype=torch.uint8)), 3, 512)  # 2 heads of 3
+    with pytest.raises(ValueError):
+        lib._check_mask(DeviceView(torch.ones((T, T), dtype=torch.uint8)), 3, 640)    # T = 5
