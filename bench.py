@@ -293,6 +293,15 @@ def run_ours(args, w, print_line=True):
     if st:
         raise RuntimeError("device status after warm-up: %s" % fa.status_string(st))
 
+    # inputs smaller than twice L2 would stay cached from one step to the next:
+    # then L2 is flushed (a write of twice its size) before each timed step,
+    # outside that step's events, and the step time is the mean of the steps'
+    # own event intervals
+    in_bytes = (4 if w.backward else 3) * B * H * N * d * 2
+    l2_bytes = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20))
+    flush = None
+    if in_bytes < 2 * l2_bytes:
+        flush = torch.empty(2 * l2_bytes // 4, dtype=torch.float32, device=dev)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -305,6 +314,8 @@ def run_ours(args, w, print_line=True):
     torch.cuda.synchronize()
     t_start.record(stream)
     for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(float(i))
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -315,7 +326,11 @@ def run_ours(args, w, print_line=True):
         raise RuntimeError("device status after timing: %s" % fa.status_string(st))
     timed_launches = launches[0]
 
-    ms_local = t_start.elapsed_time(t_end) / args.steps
+    if flush is None:
+        ms_local = t_start.elapsed_time(t_end) / args.steps
+    else:
+        last = 3 if w.backward else 1
+        ms_local = statistics.mean(e[0].elapsed_time(e[last]) for e in evs)
     ms = max_over_ranks(ms_local, world, dev)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     prep_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) if w.backward else 0.0
@@ -354,14 +369,18 @@ def run_ours(args, w, print_line=True):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, seed=w.seed)
 
-    in_bytes = 4 * B * H * N * d * 2
+    if flush is None:
+        l2_note = "inputs larger than L2 (q,k,v,dO = %.0f MB per GPU)" % (in_bytes / 1e6)
+    else:
+        l2_note = ("L2 flushed before each timed step (inputs %.0f MB per GPU, below twice L2); step time = "
+                   "mean of the steps' own event intervals" % (in_bytes / 1e6))
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal,
                        "backward": w.backward, "global_batch": B * world, "seq_len": N,
                        "parallelism": "dp%d (independent batches per GPU, no collective)" % world,
-                       "l2": "inputs larger than L2 (q,k,v,dO = %.0f MB per GPU)" % (in_bytes / 1e6)},
+                       "l2": l2_note},
             "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": timed_launches, "clocks": clocks}
     if rank == 0 and print_line:
@@ -1052,30 +1071,6 @@ def run_dropout(args, w):
     return line
 
 
-def probe_mma_rate():
-    """Cycles per tcgen05 MMA instruction for the shapes the kernels issue
-    (fa_selftest_umma_rate, one CTA per SM); printed as JSON lines."""
-    from exact_io_aware_53_b200 import fa
-    cases = [  # (N, K, a_mn, b_mn, a_tmem, use)
-        (128, 128, 0, 0, 0, "forward QK^T / backward S^T, dP^T (128x128)"),
-        (64, 128, 0, 0, 0, "backward d=64 S^T, dP^T (128x64)"),
-        (256, 128, 0, 0, 0, "reference: 128x256"),
-        (128, 128, 0, 1, 1, "forward PV / backward dV (A in TMEM)"),
-        (128, 64, 0, 1, 1, "backward d=64 dV, dK (A in TMEM, K=64)"),
-        (64, 128, 1, 1, 0, "backward d=64 dQ^T (both MN-major)"),
-    ]
-    for (N, K, amn, bmn, at, use) in cases:
-        for conv in (False, True):
-            tot, iss = fa.selftest_umma_rate(N, K, amn, bmn, at, reps=2048, n_acc=2 if N <= 128 else 1,
-                                             ctas=148, converged=conv)
-            cyc = float(tot.median())
-            ideal = 2 * 128 * N * 16 / 8192
-            print(json.dumps({"probe": "tcgen05_mma_rate", "shape": "128x%dx16" % N, "K": K, "a_mn": amn,
-                              "b_mn": bmn, "a_tmem": at, "issue": "elected lane of converged warp" if conv
-                              else "one lane of a diverged warp", "clk_per_instr": round(cyc, 1),
-                              "ideal_clk": ideal, "frac_of_ideal": round(ideal / cyc, 3), "use": use}), flush=True)
-
-
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1086,11 +1081,7 @@ def main(argv=None):
     ap.add_argument("--n-split", type=int, default=0, help="key ranges for the decode workloads (0: library choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--probe-mma-rate", action="store_true", help="print the tcgen05 issue-rate table and exit")
     args = ap.parse_args(argv)
-    if args.probe_mma_rate:
-        probe_mma_rate()
-        return 0
     from exact_io_aware_53_b200.workloads import (BLOCKSPARSE_WORKLOADS, DECODE_WORKLOADS, DROPOUT_WORKLOADS,
                                                   FP8_WORKLOADS, WORKLOADS)
     known = (list(WORKLOADS) + list(DECODE_WORKLOADS) + list(BLOCKSPARSE_WORKLOADS) + list(FP8_WORKLOADS) +

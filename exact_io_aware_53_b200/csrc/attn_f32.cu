@@ -114,7 +114,10 @@ __global__ void __launch_bounds__(WARPS * 32) bwd_pre_f32_kernel(const F32Params
     if (lane == 0) p.delta[static_cast<size_t>(bh) * p.N + i] = D;
 }
 
-// dQ_i = scale * sum_j P_ij (dP_ij - D_i) k_j; one warp per query row.
+// dQ_i = scale * sum_j P_ij (dP_ij - D_i) k_j; one warp per query row.  The
+// keys are walked in blocks of block_k: each block's terms are summed apart and
+// the block sum is added to the row's total, so the block size changes only
+// the order of the additions.
 __global__ void __launch_bounds__(WARPS * 32) bwd_dq_f32_kernel(const F32Params p)
 {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -131,17 +134,23 @@ __global__ void __launch_bounds__(WARPS * 32) bwd_dq_f32_kernel(const F32Params 
     const float lse = p.lse[static_cast<size_t>(bh) * N + i];
     const float D = p.delta[static_cast<size_t>(bh) * N + i];
     const int nk = p.causal ? i + 1 : N;
-    for (int j = 0; j < nk; ++j) {
-        const float* kj = p.k + base + static_cast<size_t>(j) * d;
-        const float s = p.scale * row_dot(q, kj, d, lane);
-        const float pij = expf(s - lse);
-        const float dp = row_dot(dO, p.v + base + static_cast<size_t>(j) * d, d, lane);
-        const float ds = pij * (dp - D);
+    for (int b0 = 0; b0 < nk; b0 += p.block_k) {
+        const int b1 = min(b0 + p.block_k, nk);
+        float blk[PER_LANE] = {};
+        for (int j = b0; j < b1; ++j) {
+            const float* kj = p.k + base + static_cast<size_t>(j) * d;
+            const float s = p.scale * row_dot(q, kj, d, lane);
+            const float pij = expf(s - lse);
+            const float dp = row_dot(dO, p.v + base + static_cast<size_t>(j) * d, d, lane);
+            const float ds = pij * (dp - D);
 #pragma unroll
-        for (int e = 0; e < PER_LANE; ++e) {
-            const int t = lane + 32 * e;
-            if (t < d) acc[e] = fmaf(ds, kj[t], acc[e]);
+            for (int e = 0; e < PER_LANE; ++e) {
+                const int t = lane + 32 * e;
+                if (t < d) blk[e] = fmaf(ds, kj[t], blk[e]);
+            }
         }
+#pragma unroll
+        for (int e = 0; e < PER_LANE; ++e) acc[e] += blk[e];
     }
     float* dq = p.dq + base + static_cast<size_t>(i) * d;
 #pragma unroll
@@ -152,6 +161,7 @@ __global__ void __launch_bounds__(WARPS * 32) bwd_dq_f32_kernel(const F32Params 
 }
 
 // dV_j = sum_i P_ij dO_i,  dK_j = scale * sum_i P_ij (dP_ij - D_i) q_i; one warp per key row.
+// The query rows are walked in blocks of block_k, summed apart per block.
 __global__ void __launch_bounds__(WARPS * 32) bwd_dkdv_f32_kernel(const F32Params p)
 {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -165,20 +175,29 @@ __global__ void __launch_bounds__(WARPS * 32) bwd_dkdv_f32_kernel(const F32Param
     load_row(p.v + base + static_cast<size_t>(j) * d, d, lane, v);
 #pragma unroll
     for (int e = 0; e < PER_LANE; ++e) ak[e] = av[e] = 0.f;
-    for (int i = p.causal ? j : 0; i < N; ++i) {
-        const float* qi = p.q + base + static_cast<size_t>(i) * d;
-        const float* doi = p.dO + base + static_cast<size_t>(i) * d;
-        const float s = p.scale * row_dot(k, qi, d, lane);
-        const float pij = expf(s - p.lse[static_cast<size_t>(bh) * N + i]);
-        const float dp = row_dot(v, doi, d, lane);
-        const float ds = pij * (dp - p.delta[static_cast<size_t>(bh) * N + i]);
+    for (int b0 = p.causal ? j : 0; b0 < N; b0 += p.block_k) {
+        const int b1 = min(b0 + p.block_k, N);
+        float bk[PER_LANE] = {}, bv[PER_LANE] = {};
+        for (int i = b0; i < b1; ++i) {
+            const float* qi = p.q + base + static_cast<size_t>(i) * d;
+            const float* doi = p.dO + base + static_cast<size_t>(i) * d;
+            const float s = p.scale * row_dot(k, qi, d, lane);
+            const float pij = expf(s - p.lse[static_cast<size_t>(bh) * N + i]);
+            const float dp = row_dot(v, doi, d, lane);
+            const float ds = pij * (dp - p.delta[static_cast<size_t>(bh) * N + i]);
+#pragma unroll
+            for (int e = 0; e < PER_LANE; ++e) {
+                const int t = lane + 32 * e;
+                if (t < d) {
+                    bv[e] = fmaf(pij, doi[t], bv[e]);
+                    bk[e] = fmaf(ds, qi[t], bk[e]);
+                }
+            }
+        }
 #pragma unroll
         for (int e = 0; e < PER_LANE; ++e) {
-            const int t = lane + 32 * e;
-            if (t < d) {
-                av[e] = fmaf(pij, doi[t], av[e]);
-                ak[e] = fmaf(ds, qi[t], ak[e]);
-            }
+            av[e] += bv[e];
+            ak[e] += bk[e];
         }
     }
     float* dk = p.dk + base + static_cast<size_t>(j) * d;

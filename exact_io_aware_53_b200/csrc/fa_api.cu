@@ -30,6 +30,10 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 unsigned int* g_status_ptr[kMaxDevices] = {};
 std::atomic<unsigned long long> g_limit_ns{2000000000ull};
+// forward launches per device (work-queue tickets) and the number of queue
+// words in use (64; fewer only to exercise shared words in tests)
+std::atomic<unsigned int> g_fwd_tickets[kMaxDevices];
+std::atomic<int> g_fwd_queue_slots{64};
 thread_local int g_last_launches = 0;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -121,6 +125,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 }  // namespace
 
+void set_last_launch_count(int n) { g_last_launches = n; }
+
 int cuda_status(cudaError_t e)
 {
     if (e == cudaSuccess) return FA_OK;
@@ -189,6 +195,13 @@ const char* fa_cuda_error_string(int code) { return cudaGetErrorString(static_ca
 
 void fa_set_wait_limit_ns(unsigned long long ns) { g_limit_ns.store(ns < 1000000ull ? 1000000ull : ns); }
 
+int fa_set_fwd_queue_words(int n)
+{
+    if (n < 1 || n > 64) return FA_ERR_INVALID_ARG;
+    g_fwd_queue_slots.store(n);
+    return FA_OK;
+}
+
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, float scale,
            int causal, void* stream)
 {
@@ -217,15 +230,19 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     p.n_pairs = (N + 255) / 256;
     {
         // persistent grid: one CTA per SM, no more than there are work items;
-        // each launch takes the next work-queue slot in turn (a slot is reused
-        // only after 63 other forward launches)
+        // each launch gets a ticket (its number on this device, never 0) and
+        // the work-queue word ticket % 64
         int dev = 0, n_sm = 0;
         if ((st = cuda_status(cudaGetDevice(&dev))) != FA_OK) return st;
+        if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
         if ((st = cuda_status(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev))) != FA_OK) return st;
         const long long items = static_cast<long long>(BH) * p.n_pairs;
+        if (items >= (1ll << 24) - 1) return FA_ERR_UNSUPPORTED;  // the queue counter has 24 bits
         p.n_ctas = static_cast<int>(std::max<long long>(1, std::min<long long>(n_sm, items)));
-        static std::atomic<unsigned int> launches{0};
-        p.queue_slot = static_cast<int>(launches.fetch_add(1) % 64u);
+        unsigned int t = g_fwd_tickets[dev].fetch_add(1u) + 1u;
+        if (t == 0u) t = g_fwd_tickets[dev].fetch_add(1u) + 1u;
+        p.ticket = t;
+        p.queue_slot = static_cast<int>(t % static_cast<unsigned int>(g_fwd_queue_slots.load()));
     }
     p.group_heads = 1;
     if (causal) {
@@ -594,13 +611,15 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
 
 int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* lse, const float* dO,
                float* dq, float* dk, float* dv, void* workspace, int B, int H, int N, int d, float scale, int causal,
-               void* stream)
+               int block_k, void* stream)
 {
     g_last_launches = 0;
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
     int st = check_shape(B, H, N, d, scale, causal);
     if (st != FA_OK) return st;
     if (d > 128) return FA_ERR_UNSUPPORTED;
+    if (block_k == 0) block_k = 64;
+    if (block_k < 1 || block_k > 1024) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
         return FA_ERR_MISALIGNED;
@@ -620,6 +639,7 @@ int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, c
     p.N = N;
     p.d = d;
     p.causal = causal;
+    p.block_k = block_k;
     p.scale = scale;
     st = cuda_status(launch_bwd_f32(p, static_cast<cudaStream_t>(stream)));
     if (st == FA_OK) g_last_launches = 3;
@@ -762,25 +782,6 @@ int fa_selftest_exp2(const float* x, float* y, int n, int mode, void* stream)
     if (!x || !y || n < 1 || (mode != 0 && mode != 1)) return FA_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(y)) return FA_ERR_MISALIGNED;
     const int st = cuda_status(launch_exp2_selftest(x, y, n, mode, static_cast<cudaStream_t>(stream)));
-    if (st == FA_OK) g_last_launches = 1;
-    return st;
-}
-
-int fa_selftest_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem, int reps, int n_acc, int ctas,
-                          long long* cycles, void* stream)
-{
-    g_last_launches = 0;
-    if (!cycles || reps == 0 || ctas < 1 || n_acc < 1) return FA_ERR_INVALID_ARG;
-    const bool shape_ok = M == 128 && ((K == 128 && !a_mn && !b_mn && !a_tmem && (N == 64 || N == 128 || N == 256)) ||
-                                       (K == 128 && !a_mn && b_mn && a_tmem && (N == 128 || N == 256)) ||
-                                       (K == 64 && !a_mn && b_mn && a_tmem && N == 128) ||
-                                       (K == 128 && a_mn && b_mn && !a_tmem && N == 64));
-    if (!shape_ok || n_acc * N > (a_tmem ? 384 : 512)) return FA_ERR_UNSUPPORTED;
-    WaitCtl ctl;
-    int st = get_ctl(&ctl);
-    if (st != FA_OK) return st;
-    st = cuda_status(launch_umma_rate(M, N, K, a_mn, b_mn, a_tmem, reps, n_acc, ctas, cycles, ctl,
-                                      static_cast<cudaStream_t>(stream)));
     if (st == FA_OK) g_last_launches = 1;
     return st;
 }

@@ -57,6 +57,7 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
                               const void* dO, float* dq, float* dk, float* dv, int B, int H, int N, int d,
                               float scale, int causal, void* stream)
 {
+    fa::set_last_launch_count(0);  // the rejections below enqueue nothing
     if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
     if (B < 1 || H < 1 || N < 1 || d < 1) return FA_ERR_INVALID_ARG;
     const size_t need = fa_bwd_workspace_bytes(B, H, N, d);
@@ -67,5 +68,7 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
     if (st != FA_OK) return st;
     st = fa_bwd_prep(o, lse, dO, dq, ws, B, H, N, d, stream);
     if (st != FA_OK) return st;
-    return fa_bwd_main(q, k, v, dO, dq, dk, dv, ws, B, H, N, d, scale, causal, stream);
+    st = fa_bwd_main(q, k, v, dO, dq, dk, dv, ws, B, H, N, d, scale, causal, stream);
+    fa::set_last_launch_count(st == FA_OK ? 2 : 1);  // the pre-pass ran in either case
+    return st;
 }

@@ -5,7 +5,9 @@
 // "Tiling and the online softmax", vibeengines.com/paper/flash-attention).
 // The kernel is persistent: one CTA per SM takes items from a queue in the
 // grouped longest-first order until none are left, and one item's Q load and
-// first S overlap the previous item's last softmax and epilogue.
+// first S overlap the previous item's last softmax and epilogue.  The queue
+// (below) keeps no per-launch state to reset, so launches on any number of
+// streams, and replays of a captured launch, need no ordering between them.
 //
 //   warp 17     TMA producer: takes the next item from the queue and hands it
 //               to the other warps through a two-slot ring; Q tiles once per
@@ -60,12 +62,89 @@ constexpr int MAX_REGS = 96;
 constexpr float SUM_LIMIT = 65536.0f;
 constexpr float LN2 = 0.6931471805599453f;
 
-// Work queues: slot k holds {next item, CTAs finished} for one launch in
-// flight.  The host gives each launch the next slot in turn; a launch's last
-// CTA returns its slot to {0, 0} (device memory starts zeroed), so launches
-// allocate nothing.
+// Work queue.  Each CTA's first item is item blockIdx.x (the first gridDim.x
+// items are the longest, so that is what a queue would hand out anyway); the
+// rest come from a counter in one of QUEUE_SLOTS 64-bit words, picked by the
+// launch's ticket (a per-device launch number, never 0).  A word holds
+//   [63:32] ticket of the launch that claimed it  [31:24] claim epoch
+//   [23:0]  next item, or QMARK once every item has been handed out.
+// A word is free when it is zero or its counter is QMARK.  The first CTA of a
+// launch to want a second item claims a free word for its ticket (compare and
+// swap, epoch + 1, counter = gridDim.x + 1: it takes item gridDim.x); the
+// launch's other CTAs see their ticket with a live counter and take items by
+// compare and swap; the CTA that takes the last item writes QMARK, after which
+// no CTA of the launch writes the word again.  While another launch holds the
+// word (a foreign ticket, counter live), a CTA takes its items from the static
+// sequence blockIdx.x + s * gridDim.x instead, so concurrent launches that land
+// on one word (more than QUEUE_SLOTS in flight, or replays of one captured
+// launch on two streams) still process every item, some of them twice with
+// identical results, and never take each other's items.  A free word showing
+// the launch's own ticket is either what an earlier run of the same launch (a
+// graph replay) left, when it equals what the CTA read at its start, or the
+// end of this run's own hand-out, when it does not.  Nothing is ever reset.
 constexpr int QUEUE_SLOTS = 64;
-__device__ unsigned int g_queue[QUEUE_SLOTS][2];
+constexpr unsigned int QMARK = 0xFFFFFFu;
+__device__ unsigned long long g_queue[QUEUE_SLOTS];
+
+struct QueueCursor {
+    unsigned long long snap;  // the word as this CTA first read it
+    int next_static;          // next item of the static sequence
+    bool joined;              // taking items from the word's counter
+};
+
+__device__ __forceinline__ unsigned long long queue_read(const unsigned long long* w)
+{
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(w) : "memory");
+    return v;
+}
+
+// Next work item of this CTA, or -1 when the launch has none left for it.
+__device__ int queue_next(unsigned long long* word, unsigned int ticket, int total, QueueCursor& qc,
+                          const WaitCtl& ctl)
+{
+    const int P = static_cast<int>(gridDim.x);
+    for (int tries = 0; tries < (1 << 16); ++tries) {
+        const unsigned long long w = queue_read(word);
+        const unsigned int own = static_cast<unsigned int>(w >> 32);
+        const unsigned int ep = static_cast<unsigned int>(w >> 24) & 0xFFu;
+        const unsigned int c = static_cast<unsigned int>(w) & 0xFFFFFFu;
+        const bool live = (w != 0ull) && (c != QMARK);
+        unsigned long long want;
+        int item;
+        if (own == ticket && live) {
+            // this run is handing items out: take the next one
+            qc.joined = true;
+            item = static_cast<int>(c);
+            want = (c + 1u >= static_cast<unsigned int>(total)) ? ((w & ~0xFFFFFFull) | QMARK) : w + 1ull;
+        } else if (own == ticket && w != qc.snap) {
+            // this run's hand-out is over (it began after this CTA started)
+            return -1;
+        } else if (qc.joined) {
+            // the hand-out this CTA took part in is over and the word moved on
+            return -1;
+        } else if (!live) {
+            // free: claim it for this run and take item P
+            item = P;
+            const unsigned int c1 = static_cast<unsigned int>(P) + 1u;
+            want = (static_cast<unsigned long long>(ticket) << 32) |
+                   (static_cast<unsigned long long>((ep + 1u) & 0xFFu) << 24) |
+                   (c1 >= static_cast<unsigned int>(total) ? QMARK : c1);
+        } else {
+            // another launch holds the word: static sequence
+            const int it = qc.next_static;
+            qc.next_static += P;
+            return it < total ? it : -1;
+        }
+        if (atomicCAS(word, w, want) == w) {
+            qc.joined = true;
+            return item;
+        }
+    }
+    // not reached in practice: each failed swap means another CTA took an item
+    raise_status(ctl, FA_DEV_TIMEOUT);
+    return -1;
+}
 
 template <int D>
 struct Cfg {
@@ -153,7 +232,7 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     const int lane = static_cast<int>(lane_id());
     const int N = p.N;
     const int total = p.BH * p.n_pairs;
-    unsigned int* queue = g_queue[p.queue_slot];
+    unsigned long long* queue = &g_queue[p.queue_slot];
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -192,10 +271,15 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
         if (lane == 0) {
             int it = 0, nq = 0;  // K/V ring slots and Q tiles issued so far
             bool ok = true;
+            QueueCursor qc;
+            qc.snap = queue_read(queue);
+            qc.next_static = static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x);
+            qc.joined = false;
             for (int n = 0; ok; ++n) {
                 const int slot = n & 1;
-                const int raw = static_cast<int>(atomicAdd(&queue[0], 1u));
-                const int item = raw < total ? raw : -1;
+                const int item = (n == 0) ? static_cast<int>(blockIdx.x)
+                                          : (total > static_cast<int>(gridDim.x) ? queue_next(queue, p.ticket, total, qc, p.ctl)
+                                                                                 : -1);
                 if (!(ok = mbar_wait(&item_empty[slot], ((n >> 1) & 1) ^ 1, p.ctl))) break;
                 item_buf[slot] = item;
                 mbar_arrive(&item_full[slot]);  // release: the waiters see item_buf
@@ -524,12 +608,6 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     if (warp == MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
-    }
-    // every CTA has taken its last item by now; the last one to get here
-    // returns the queue slot to {0, 0} for a later launch
-    if (threadIdx.x == 0 && atomicAdd(&queue[1], 1u) == gridDim.x - 1) {
-        atomicExch(&queue[0], 0u);
-        atomicExch(&queue[1], 0u);
     }
 }
 

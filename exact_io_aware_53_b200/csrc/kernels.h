@@ -14,6 +14,9 @@ namespace fa {
 // error (fa_last_cuda_error) and returns FA_ERR_CUDA.  Host code (fa_api.cu).
 int cuda_status(cudaError_t e);
 
+// Sets what fa_last_launch_count reports on the calling thread.  Host code.
+void set_last_launch_count(int n);
+
 // ---------------------------------------------------------------- bf16 forward
 struct FwdParams {
     CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle
@@ -26,7 +29,8 @@ struct FwdParams {
     int n_pairs;       // ceil(N / 256)
     int group_heads;   // grouping of the (pair, head) work items, >= 1 (grouped_order)
     int n_ctas;        // persistent CTAs, <= min(SMs, B*H*n_pairs)
-    int queue_slot;    // work queue slot of this launch, < 64
+    int queue_slot;    // work queue word of this launch, < 64
+    unsigned int ticket;  // launch number on this device (never 0)
     float scale_log2;  // scale * log2(e)
     WaitCtl ctl;
 };
@@ -154,7 +158,5 @@ struct UmmaTestParams {
 cudaError_t launch_umma_selftest(const UmmaTestParams& p, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(WaitCtl ctl, unsigned int* gave_up, cudaStream_t stream);
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, int mode, cudaStream_t stream);
-cudaError_t launch_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem, int reps, int n_acc, int ctas,
-                             long long* cycles, WaitCtl ctl, cudaStream_t stream);
 
 }  // namespace fa

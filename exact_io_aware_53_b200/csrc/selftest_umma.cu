@@ -149,138 +149,6 @@ cudaError_t launch_umma_selftest(const UmmaTestParams& p, cudaStream_t stream)
 }  // namespace fa
 
 namespace fa {
-namespace umma_rate {
-
-// Issue-rate probe: operands staged once (contents irrelevant), then `reps`
-// back-to-back copies of the K/16-instruction MMA sequence are issued into
-// `n_acc` rotating TMEM accumulators, with the same unrolled, inline-descriptor
-// issue pattern the attention kernels use.  Issued either by one lane of a
-// diverged warp or by a converged warp with an elected lane per instruction.
-// cycles[2 cta] = first issue -> completion, cycles[2 cta + 1] = first -> last issue.
-template <int N, int K, bool AMN, bool BMN, bool ATMEM, bool CONV>
-__global__ void __launch_bounds__(128, 1) umma_rate_kernel(int reps, int n_acc, long long* cycles, WaitCtl ctl)
-{
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = smem;
-    uint8_t* sB = smem + 32 * 1024;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 96 * 1024);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
-    const int warp = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < 96 * 1024 / 16; i += 128)
-        reinterpret_cast<uint4*>(smem)[i] = make_uint4(0x3f803f80u, 0u, 0x3f803f80u, 0u);
-    fence_proxy_async_smem();
-    if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    constexpr uint32_t idesc = idesc_bf16(128, N, AMN, BMN);
-    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
-    // CONV: the whole warp runs the loop and elect.sync picks the issuing lane;
-    // otherwise lane 0 alone.  A compile-time choice: a run-time branch around
-    // every MMA would itself slow the issue stream.
-    auto issue = [&](uint32_t d) {
-#pragma unroll
-        for (int kk = 0; kk < K / 16; ++kk) {
-            const uint32_t acc = kk > 0 ? 1u : 0u;
-            const uint64_t bdesc = BMN ? sdesc_sw128(b0 + kk * 2048, K * 128, 1024)
-                                       : sdesc_sw128(b0 + (kk >> 2) * N * 128 + (kk & 3) * 32, 16, 1024);
-            if constexpr (ATMEM) {
-                if constexpr (CONV) mma_ts_elect(d, tmem + 384 + kk * 8, bdesc, idesc, acc);
-                else mma_ts(d, tmem + 384 + kk * 8, bdesc, idesc, acc);
-            } else {
-                const uint64_t adesc = AMN ? sdesc_sw128(a0 + kk * 2048, K * 128, 1024)
-                                           : sdesc_sw128(a0 + (kk >> 2) * 128 * 128 + (kk & 3) * 32, 16, 1024);
-                if constexpr (CONV) mma_ss_elect(d, adesc, bdesc, idesc, acc);
-                else mma_ss(d, adesc, bdesc, idesc, acc);
-            }
-        }
-    };
-    if (CONV ? (warp == 0) : (threadIdx.x == 0)) {
-        const long long t0 = clock64();
-        int a = 0;
-        for (int r = 0; r < reps; ++r) {
-            issue(tmem + static_cast<uint32_t>(a * N));
-            a = (a + 1 == n_acc) ? 0 : a + 1;
-        }
-        const long long t1 = clock64();
-        if constexpr (CONV)
-            mma_commit_elect(bar);
-        else
-            mma_commit(bar);
-        mbar_wait(bar, 0, ctl);
-        const long long t2 = clock64();
-        if (threadIdx.x == 0) {
-            cycles[2 * blockIdx.x] = t2 - t0;
-            cycles[2 * blockIdx.x + 1] = t1 - t0;
-        }
-    }
-    __syncwarp();
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
-    }
-}
-
-template <int N, int K, bool AMN, bool BMN, bool ATMEM, bool CONV>
-cudaError_t launch_rate_as(int reps, int n_acc, int ctas, long long* cycles, WaitCtl ctl, cudaStream_t stream)
-{
-    const int smem = 96 * 1024 + 64 + 1024;
-    auto kern = umma_rate_kernel<N, K, AMN, BMN, ATMEM, CONV>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    kern<<<ctas, 128, smem, stream>>>(reps, n_acc, cycles, ctl);
-    return cudaGetLastError();
-}
-
-template <int N, int K, bool AMN, bool BMN, bool ATMEM>
-cudaError_t launch_rate(int reps, int n_acc, int converged, int ctas, long long* cycles, WaitCtl ctl,
-                        cudaStream_t stream)
-{
-    return converged ? launch_rate_as<N, K, AMN, BMN, ATMEM, true>(reps, n_acc, ctas, cycles, ctl, stream)
-                     : launch_rate_as<N, K, AMN, BMN, ATMEM, false>(reps, n_acc, ctas, cycles, ctl, stream);
-}
-
-}  // namespace umma_rate
-
-// Shapes the attention kernels issue: QK^T / S^T (SS, K-major), PV / dV / dK
-// (TMEM A, MN-major B), dQ^T (SS, both MN-major), plus N = 256 for reference.
-cudaError_t launch_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem, int reps, int n_acc, int ctas,
-                             long long* cycles, WaitCtl ctl, cudaStream_t stream)
-{
-    (void)M;
-    const int conv = reps < 0 ? 1 : 0;
-    const int r = reps < 0 ? -reps : reps;
-    using namespace umma_rate;
-    if (K == 128 && !a_mn && !b_mn && !a_tmem) {
-        if (N == 64) return launch_rate<64, 128, false, false, false>(r, n_acc, conv, ctas, cycles, ctl, stream);
-        if (N == 128) return launch_rate<128, 128, false, false, false>(r, n_acc, conv, ctas, cycles, ctl, stream);
-        if (N == 256) return launch_rate<256, 128, false, false, false>(r, n_acc, conv, ctas, cycles, ctl, stream);
-    }
-    if (K == 128 && !a_mn && b_mn && a_tmem) {
-        if (N == 128) return launch_rate<128, 128, false, true, true>(r, n_acc, conv, ctas, cycles, ctl, stream);
-        if (N == 256) return launch_rate<256, 128, false, true, true>(r, n_acc, conv, ctas, cycles, ctl, stream);
-    }
-    if (K == 64 && !a_mn && b_mn && a_tmem && N == 128)
-        return launch_rate<128, 64, false, true, true>(r, n_acc, conv, ctas, cycles, ctl, stream);
-    if (K == 128 && a_mn && b_mn && !a_tmem && N == 64)
-        return launch_rate<64, 128, true, true, false>(r, n_acc, conv, ctas, cycles, ctl, stream);
-    return cudaErrorInvalidValue;
-}
-
-}  // namespace fa
-
-namespace fa {
 namespace exp2_test {
 
 // y[i] = 2^x[i] by the FMA-pipe polynomial (mode 0) or ex2.approx (mode 1).

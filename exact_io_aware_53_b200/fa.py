@@ -35,11 +35,12 @@ _SIGS = {
     "fa_bwd_main": ([P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
     "fa_bwd_noalloc": ([P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
     "fa_fwd_f32": ([P, P, P, P, P, I, I, I, I, F, I, I, P], I),
-    "fa_bwd_f32": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, P], I),
+    "fa_bwd_f32": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, F, I, I, P], I),
     "fa_attention_host_arena_bytes": ([I, I, I, I], SZ),
     "fa_attention_host": ([P, P, P, P, P, P, P, P, P, P, SZ, I, I, I, I, F, I, P], I),
     "fa_check_device_status": ([P], I),
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
+    "fa_set_fwd_queue_words": ([I], I),
     "fa_fwd_splitkv_workspace_bytes": ([I, I, I, I, I, I], ctypes.c_size_t),
     "fa_fwd_splitkv": ([P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P], I),
     "fa_fwd_blocksparse": ([P, P, P, P, P, P, ctypes.c_longlong, I, I, I, I, ctypes.c_float, I, P], I),
@@ -54,7 +55,6 @@ _SIGS = {
     "fa_selftest_umma": ([P, P, P, I, I, I, I, I, I, I, P], I),
     "fa_selftest_exp2": ([P, P, I, I, P], I),
     "fa_selftest_wait_timeout": ([ctypes.c_ulonglong, P, P], I),
-    "fa_selftest_umma_rate": ([I, I, I, I, I, I, I, I, I, P, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -165,24 +165,26 @@ def fwd_splitkv(q, k, v, causal: bool = False, scale: float | None = None, n_spl
     return o, lse
 
 
-def _check_mask(m, H: int, N: int):
+def _check_mask(m, H: int, N: int, device):
     """The kernel reads mask row i of head h at h * stride + i * T: the mask must be
-    a CUDA uint8 tensor [T, T] or [1 or H, T, T] whose last two dimensions are dense."""
+    a uint8 tensor [T, T] or [1 or H, T, T] on the same GPU as q whose last two
+    dimensions are dense."""
     T = (N + 127) // 128
     shape = tuple(m.shape)
-    ok = (m.dtype == torch.uint8 and m.is_cuda and
+    ok = (m.dtype == torch.uint8 and m.is_cuda and m.device == device and
           (shape == (T, T) or (m.dim() == 3 and shape[1:] == (T, T) and shape[0] in (1, H))) and
           m.stride(-1) == 1 and m.stride(-2) == T)
     if not ok:
-        raise ValueError("block_mask must be a CUDA uint8 tensor [T, T] or [1 or H, T, T] with dense rows, "
-                         "T = ceil(N / 128) = %d; got %s %s strides %s" % (T, m.dtype, shape, tuple(m.stride())))
+        raise ValueError("block_mask must be a uint8 tensor [T, T] or [1 or H, T, T] with dense rows on %s, "
+                         "T = ceil(N / 128) = %d; got %s %s strides %s on %s"
+                         % (device, T, m.dtype, shape, tuple(m.stride()), m.device))
 
 
 def fwd_blocksparse_raw(q, k, v, o, lse, block_mask, scale: float, causal: bool, stream=None) -> int:
     """Enqueue the block-sparse forward on preallocated tensors; block_mask is
     a CUDA uint8 tensor [T, T] (shared by every head) or [H, T, T], T = ceil(N/128)."""
     B, H, N, d = _shape(q)
-    _check_mask(block_mask, H, N)
+    _check_mask(block_mask, H, N, q.device)
     stride = 0 if block_mask.dim() == 2 or block_mask.shape[0] == 1 else int(block_mask.stride(0))
     return _lib.fa_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_mask), stride,
                                    B, H, N, d, float(scale), int(bool(causal)), _stream(stream))
@@ -313,7 +315,8 @@ def fwd_f32(q, k, v, causal: bool = False, scale: float | None = None, block_k: 
     return o, lse
 
 
-def bwd_f32(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, stream=None):
+def bwd_f32(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, block_k: int = 0,
+            stream=None):
     _same(q, k, v, o, do, dtype=torch.float32)
     B, H, N, d = _shape(q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
@@ -322,7 +325,8 @@ def bwd_f32(q, k, v, o, lse, do, causal: bool = False, scale: float | None = Non
     dv = torch.empty_like(q)
     ws = torch.empty(bwd_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=q.device)
     _check(_lib.fa_bwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
-                           _ptr(ws), B, H, N, d, float(scale), int(causal), _stream(stream)), "fa_bwd_f32")
+                           _ptr(ws), B, H, N, d, float(scale), int(causal), int(block_k), _stream(stream)),
+           "fa_bwd_f32")
     return dq, dk, dv
 
 
@@ -353,16 +357,6 @@ def selftest_umma(a, b, M, N, K, a_mn, b_mn, a_tmem=False, b_manual=False, strea
     return d
 
 
-def selftest_umma_rate(N, K, a_mn=0, b_mn=0, a_tmem=0, reps=256, n_acc=1, ctas=1, M=128, converged=True,
-                       stream=None):
-    """(cycles per MMA instruction to completion, cycles per instruction to issue), per CTA."""
-    cyc = torch.zeros(2 * ctas, dtype=torch.int64, device="cuda")
-    r = -int(reps) if converged else int(reps)
-    _check(_lib.fa_selftest_umma_rate(M, N, K, int(a_mn), int(b_mn), int(a_tmem), r, int(n_acc), int(ctas),
-                                      _ptr(cyc), _stream(stream)), "fa_selftest_umma_rate")
-    torch.cuda.synchronize()
-    c = (cyc.double() / (reps * K / 16)).cpu().view(ctas, 2)
-    return c[:, 0], c[:, 1]
 
 
 def selftest_exp2(x, mode: int, stream=None):

@@ -54,11 +54,14 @@ typedef enum {
  * reading of the pages' standard attention is 1/sqrt(d)).  causal: 0 or 1.
  * All pointers 16-byte aligned.  q/k/v may alias each other, o and lse must
  * not overlap any input.
- * The kernel is persistent: one CTA per SM takes work items from a queue in
- * the library's device memory (64 slots, one per launch in turn, returned to
- * zero by each launch's last CTA).  Launches may run concurrently on several
- * streams as long as fewer than 64 forward launches are in flight on a device
- * at once.
+ * The kernel is persistent: one CTA per SM takes work items (256 query rows
+ * of one head) from a queue.  The queue is one of 64 counter words in the
+ * library's device memory, claimed per launch with a launch ticket and never
+ * reset; a launch that finds its word held by another launch in flight takes
+ * its items in a fixed order instead.  So launches may run concurrently on any
+ * number of streams, and a captured launch may be replayed, with every output
+ * element written by this launch's own arithmetic (at worst some items twice,
+ * with identical results).  FA_ERR_UNSUPPORTED if B*H*ceil(N/256) >= 2^24-1.
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, void* stream);
@@ -135,10 +138,13 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
 /*
  * Backward, fp32.  Inputs as fa_fwd_f32 plus o, lse (from it) and dO; outputs
  * dq, dk, dv fp32 [B][H][N][d].  workspace: fa_bwd_workspace_bytes bytes.
+ * block_k (1 .. 1024; 0 selects 64) is the block size of the walks over keys
+ * (for dQ) and over queries (for dK, dV): each block's terms are summed apart,
+ * so, as in the forward, the block size changes only the rounding order.
  */
 int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* lse,
                const float* dO, float* dq, float* dk, float* dv, void* workspace, int B, int H, int N, int d,
-               float scale, int causal, void* stream);
+               float scale, int causal, int block_k, void* stream);
 
 /*
  * Bytes of device arena fa_attention_host needs for B,H,N,d (bf16 path).
@@ -169,6 +175,12 @@ int fa_check_device_status(void* stream);
 /* Upper bound, in nanoseconds, on any single wait inside a kernel of this
  * library (default 2e9).  Values below 1e6 are raised to 1e6.  Process-wide. */
 void fa_set_wait_limit_ns(unsigned long long ns);
+
+/* Diagnostics: how many of the forward's 64 work-queue words launches are
+ * spread over (1 .. 64; default 64).  1 puts every forward launch on one word,
+ * so that concurrent launches share it; tests use this to check the shared
+ * case.  Process-wide.  FA_ERR_INVALID_ARG outside 1 .. 64. */
+int fa_set_fwd_queue_words(int n);
 
 /*
  * Split-KV forward, bf16: Nq queries against Nk keys, the shape of decoding

@@ -47,23 +47,6 @@ int fa_selftest_wait_timeout(unsigned long long limit_ns, unsigned int* gave_up,
  */
 int fa_selftest_exp2(const float* x, float* y, int n, int mode, void* stream);
 
-/*
- * Tensor-core issue-rate probe: `ctas` CTAs (one per SM when ctas <= SM count)
- * each stage dummy operands once and issue `reps` back-to-back copies of the
- * K/16-instruction 128 x N x K MMA sequence (same operand kinds as
- * fa_selftest_umma), rotating over `n_acc` TMEM accumulators of N columns.
- * cycles (device buffer of 2 * ctas int64) receives per CTA the SM clock
- * cycles from first issue to completion, then from first to last issue.
- * Shapes (M = 128): K-major A and B with K = 128 and N in {64, 128, 256};
- * A in TMEM with MN-major B, K = 128 and N in {128, 256}, or K = 64 and
- * N = 128; MN-major A and B with K = 128 and N = 64.  Others return
- * FA_ERR_UNSUPPORTED.  n_acc * N <= 512 (384 with a_tmem).  reps > 0 issues
- * from one lane of a diverged warp; reps < 0 issues |reps| copies from a
- * converged warp with an elected lane per instruction.
- */
-int fa_selftest_umma_rate(int M, int N, int K, int a_mn, int b_mn, int a_tmem, int reps, int n_acc, int ctas,
-                          long long* cycles, void* stream);
-
 #ifdef __cplusplus
 }
 #endif

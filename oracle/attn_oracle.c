@@ -44,11 +44,11 @@
  * top-left aligned causal mask, key j allowed iff j <= i.
  */
 #include <math.h>
+#include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
-#include <stdint.h>
 #endif
 
 int oracle_num_threads(void)
@@ -663,10 +663,11 @@ int oracle_attn_fwd_dropout(const double* q, const double* k, const double* v, d
     return err;
 }
 
-/* Backward with dropout (definition above), the mask regenerated per element. */
+/* Backward with dropout (definition above), the mask regenerated per element.
+ * The heads given are heads bh0 .. bh0 + BH - 1 of the whole problem. */
 int oracle_attn_bwd_dropout(const double* q, const double* k, const double* v, const double* dO,
                             double* dq, double* dk, double* dv, long BH, long N, long d,
-                            double scale, int causal, int t, uint64_t seed, uint64_t offset)
+                            double scale, int causal, int t, uint64_t seed, uint64_t offset, long bh0)
 {
     if (BH < 0 || N < 0 || d < 1 || t < 0 || t > 256) return -1;
     const double s_keep = t > 0 ? 256.0 / t : 0.0;
@@ -704,7 +705,7 @@ int oracle_attn_bwd_dropout(const double* q, const double* k, const double* v, c
                 }
                 for (long j = 0; j < nk; ++j) {
                     prow[j] /= l;
-                    zrow[j] = dropout_keep(seed, offset, h, i, j, t) ? s_keep : 0.0;
+                    zrow[j] = dropout_keep(seed, offset, bh0 + h, i, j, t) ? s_keep : 0.0;
                 }
                 double D = 0.0;
                 for (long j = 0; j < nk; ++j) {
@@ -734,4 +735,117 @@ int oracle_attn_bwd_dropout(const double* q, const double* k, const double* v, c
         free(zrow);
     }
     return err;
+}
+
+/*
+ * Backward of ONE head, with the work spread over threads, for heads too long
+ * for oracle_attn_bwd's one-thread-per-head loop (N = 16384).  Same definition
+ * as oracle_attn_bwd, and as oracle_attn_bwd_dropout when t < 256 (t = 256 is
+ * plain attention: every key kept, factor 1); bh is the head's index b * H + h
+ * in the whole problem, which only enters the dropout generator.
+ *
+ * Two passes, each parallel over independent outputs, so every sum still runs
+ * in one thread in a fixed order:
+ *   rows:  for each query i, the materialised row s_i, m_i = max s_i,
+ *          l_i = sum e^{s_ij - m_i}, P_ij = e^{s_ij - m_i} / l_i, dP_ij and
+ *          D_i = sum_j P_ij dP_ij, then dQ_i = scale sum_j P_ij (dP_ij - D_i) k_j
+ *          (exactly the row loop of oracle_attn_bwd); m_i, l_i, D_i are kept.
+ *   keys:  for each key j, every query i that sees it in row order: P_ij from the
+ *          same s_ij, m_i, l_i, then dV_j = sum_i P_ij Z_ij dO_i and
+ *          dK_j = scale sum_i P_ij (dP_ij - D_i) q_i.
+ */
+int oracle_attn_bwd_head(const double* q, const double* k, const double* v, const double* dO,
+                         double* dq, double* dk, double* dv, long N, long d, double scale, int causal,
+                         int t, uint64_t seed, uint64_t offset, long bh)
+{
+    if (N < 1 || d < 1 || t < 0 || t > 256) return -1;
+    const double s_keep = t > 0 ? 256.0 / t : 0.0;
+    double* rm = (double*)malloc((size_t)N * sizeof(double));
+    double* rl = (double*)malloc((size_t)N * sizeof(double));
+    double* rD = (double*)malloc((size_t)N * sizeof(double));
+    if (!rm || !rl || !rD) {
+        free(rm);
+        free(rl);
+        free(rD);
+        return -1;
+    }
+    int err = 0;
+#pragma omp parallel
+    {
+        double* prow = (double*)malloc((size_t)N * sizeof(double));
+        double* dprow = (double*)malloc((size_t)N * sizeof(double));
+        if (!prow || !dprow) {
+#pragma omp atomic write
+            err = -1;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (long i = 0; i < N; ++i) {
+            if (!prow || !dprow) continue;
+            const double* qi = q + i * d;
+            const double* doi = dO + i * d;
+            const long nk = n_allowed(i, N, causal);
+            double m = -INFINITY;
+            for (long j = 0; j < nk; ++j) {
+                prow[j] = scale * dot(qi, k + j * d, d);
+                if (prow[j] > m) m = prow[j];
+            }
+            double l = 0.0;
+            for (long j = 0; j < nk; ++j) {
+                prow[j] = exp(prow[j] - m);
+                l += prow[j];
+            }
+            for (long j = 0; j < nk; ++j) prow[j] /= l;
+            double D = 0.0;
+            for (long j = 0; j < nk; ++j) {
+                const double z = (t == 256) ? 1.0 : (dropout_keep(seed, offset, bh, i, j, t) ? s_keep : 0.0);
+                dprow[j] = z * dot(doi, v + j * d, d);
+                D += prow[j] * dprow[j];
+            }
+            double* dqi = dq + i * d;
+            for (long e = 0; e < d; ++e) dqi[e] = 0.0;
+            for (long j = 0; j < nk; ++j) {
+                const double ds = prow[j] * (dprow[j] - D);
+                const double* kj = k + j * d;
+                for (long e = 0; e < d; ++e) dqi[e] += ds * kj[e];
+            }
+            for (long e = 0; e < d; ++e) dqi[e] *= scale;
+            rm[i] = m;
+            rl[i] = l;
+            rD[i] = D;
+        }
+        free(prow);
+        free(dprow);
+    }
+    if (err) {
+        free(rm);
+        free(rl);
+        free(rD);
+        return err;
+    }
+#pragma omp parallel for schedule(dynamic, 8)
+    for (long j = 0; j < N; ++j) {
+        const double* kj = k + j * d;
+        const double* vj = v + j * d;
+        double* dkj = dk + j * d;
+        double* dvj = dv + j * d;
+        for (long e = 0; e < d; ++e) dkj[e] = dvj[e] = 0.0;
+        for (long i = causal ? j : 0; i < N; ++i) {
+            const double* qi = q + i * d;
+            const double* doi = dO + i * d;
+            const double p = exp(scale * dot(qi, kj, d) - rm[i]) / rl[i];
+            const double z = (t == 256) ? 1.0 : (dropout_keep(seed, offset, bh, i, j, t) ? s_keep : 0.0);
+            const double dp = z * dot(doi, vj, d);
+            const double ds = p * (dp - rD[i]);
+            const double pz = p * z;
+            for (long e = 0; e < d; ++e) {
+                dkj[e] += ds * qi[e];
+                dvj[e] += pz * doi[e];
+            }
+        }
+        for (long e = 0; e < d; ++e) dkj[e] *= scale;
+    }
+    free(rm);
+    free(rl);
+    free(rD);
+    return 0;
 }

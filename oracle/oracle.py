@@ -72,7 +72,7 @@ def _load():
         lib.oracle_dropout_mask.restype = I
         lib.oracle_attn_fwd_dropout.argtypes = [P, P, P, P, P, L, L, L, D, I, I, U, U, L]
         lib.oracle_attn_fwd_dropout.restype = I
-        lib.oracle_attn_bwd_dropout.argtypes = [P, P, P, P, P, P, P, L, L, L, D, I, I, U, U]
+        lib.oracle_attn_bwd_dropout.argtypes = [P, P, P, P, P, P, P, L, L, L, D, I, I, U, U, L]
         lib.oracle_attn_bwd_dropout.restype = I
         lib.oracle_attn_fwd_blockmask.argtypes = [P, P, P, P, P, L, L, L, L, D, I, P, L, L, L]
         lib.oracle_attn_fwd_blockmask.restype = I
@@ -84,6 +84,8 @@ def _load():
         lib.oracle_attn_bwd_dq_rows.restype = I
         lib.oracle_attn_bwd_kv_rows.argtypes = [P, P, P, P, P, P, L, L, L, L, D, I]
         lib.oracle_attn_bwd_kv_rows.restype = I
+        lib.oracle_attn_bwd_head.argtypes = [P, P, P, P, P, P, P, L, L, D, I, I, U, U, L]
+        lib.oracle_attn_bwd_head.restype = I
         _lib = lib
     return _lib
 
@@ -213,14 +215,15 @@ def attn_fwd_dropout(q, k, v, scale: float, causal: bool, keep_t: int, seed: int
     return o, lse
 
 
-def attn_bwd_dropout(q, k, v, do, scale: float, causal: bool, keep_t: int, seed: int, offset: int):
-    """(dQ, dK, dV) of L = sum(O * dO) for the dropout forward above."""
+def attn_bwd_dropout(q, k, v, do, scale: float, causal: bool, keep_t: int, seed: int, offset: int, bh0: int = 0):
+    """(dQ, dK, dV) of L = sum(O * dO) for the dropout forward above; the heads
+    given are heads bh0, bh0 + 1, ... of the whole problem."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     B, H, N, d = q.shape
     dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
     rc = _load().oracle_attn_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
                                          B * H, N, d, float(scale), int(bool(causal)), int(keep_t), int(seed),
-                                         int(offset))
+                                         int(offset), int(bh0))
     if rc != 0:
         raise RuntimeError("oracle_attn_bwd_dropout failed (%d)" % rc)
     return dq, dk, dv
@@ -291,3 +294,19 @@ def attn_bwd_kv_rows(q, k, v, do, j0: int, j1: int, scale: float, causal: bool):
     if rc != 0:
         raise RuntimeError("oracle_attn_bwd_kv_rows failed (%d)" % rc)
     return dk, dv
+
+
+def attn_bwd_head(q, k, v, do, scale: float, causal: bool, keep_t: int = 256, seed: int = 0, offset: int = 0,
+                  bh: int = 0):
+    """(dQ, dK, dV) of ONE head ([N, d] arrays), the work spread over threads
+    (rows, then keys).  keep_t = 256: plain attention, as attn_bwd; otherwise
+    the dropout backward of head index bh (b * H + h) of the whole problem."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    N, d = q.shape
+    assert k.shape == v.shape == do.shape == (N, d)
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    rc = _load().oracle_attn_bwd_head(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), N, d,
+                                      float(scale), int(bool(causal)), int(keep_t), int(seed), int(offset), int(bh))
+    if rc != 0:
+        raise RuntimeError("oracle_attn_bwd_head failed (%d)" % rc)
+    return dq, dk, dv

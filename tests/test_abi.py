@@ -197,9 +197,9 @@ def test_blocksparse_mask_layout_is_checked(lib):
     for bad in (m.t().contiguous().t()[:, :3], m.to(torch.int32), torch.ones((2, 4, 4), dtype=torch.uint8).transpose(1, 2),
                 torch.ones((3, 3), dtype=torch.uint8)):
         with pytest.raises(ValueError):
-            lib._check_mask(bad, 2, 512)
+            lib._check_mask(bad, 2, 512, torch.device("cuda", 0))
     with pytest.raises(ValueError):  # not on a GPU
-        lib._check_mask(m, 2, 512)
+        lib._check_mask(m, 2, 512, torch.device("cuda", 0))
 
 
 def test_blocksparse_mask_layout_accepts_dense_device_masks(lib):
@@ -208,9 +208,10 @@ def test_blocksparse_mask_layout_accepts_dense_device_masks(lib):
     import torch
 
     class DeviceView:
-        def __init__(self, t):
+        def __init__(self, t, index=0):
             self._t, self.dtype, self.is_cuda = t, t.dtype, True
             self.shape = t.shape
+            self.device = torch.device("cuda", index)
 
         def dim(self):
             return self._t.dim()
@@ -219,10 +220,13 @@ def test_blocksparse_mask_layout_accepts_dense_device_masks(lib):
             return self._t.stride() if i is None else self._t.stride(i)
 
     T = 4  # N = 512
+    dev = torch.device("cuda", 0)
     for good in (torch.ones((T, T), dtype=torch.uint8), torch.ones((1, T, T), dtype=torch.uint8),
                  torch.ones((3, T, T), dtype=torch.uint8), torch.ones((6, T, T), dtype=torch.uint8)[::2]):
-        lib._check_mask(DeviceView(good), 3, 512)
+        lib._check_mask(DeviceView(good), 3, 512, dev)
     with pytest.raises(ValueError):
-        lib._check_mask(DeviceView(torch.ones((2, T, T), dtype=torch.uint8)), 3, 512)  # 2 heads of 3
+        lib._check_mask(DeviceView(torch.ones((2, T, T), dtype=torch.uint8)), 3, 512, dev)  # 2 heads of 3
     with pytest.raises(ValueError):
-        lib._check_mask(DeviceView(torch.ones((T, T), dtype=torch.uint8)), 3, 640)    # T = 5
+        lib._check_mask(DeviceView(torch.ones((T, T), dtype=torch.uint8)), 3, 640, dev)    # T = 5
+    with pytest.raises(ValueError):  # on another GPU than q
+        lib._check_mask(DeviceView(torch.ones((T, T), dtype=torch.uint8), index=1), 3, 512, dev)

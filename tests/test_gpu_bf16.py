@@ -58,17 +58,19 @@ def test_small_fwd_bwd_full_compare(fa_lib, B, H, N, d, causal):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-def test_sharp_softmax_rescaling_fwd(fa_lib, d):
-    """Scores with std ~8 force the running max to move many times.  Only the
-    forward is held to 2e-2 here: O is a convex combination of V rows whatever
-    the sharpness, while the gradients grow with it (|dQ| ~ 20 at this scale,
-    where bf16 rounding of dS alone is ~2^-9 relative)."""
+def test_sharp_softmax_rescaling_fwd_bwd(fa_lib, d):
+    """Scores with std ~8 force the running max to move many times.  O is a
+    convex combination of V rows whatever the sharpness and is held to 2e-2;
+    the gradients grow with the sharpness (|dQ| ~ 20 here), so each element is
+    held to 2e-2 plus the bound on what the bf16 roundings of P, dS and O can
+    move it by (_bwd_rounding_bounds)."""
     x = _inputs((1, 2, 700, d), seed=99 + d, gain=2.8)
     scale = 1 / math.sqrt(d)
-    out = gpu_fwd_bwd(fa_lib, to_cuda(x), scale, True, backward=False)
+    out = gpu_fwd_bwd(fa_lib, to_cuda(x), scale, True)
     ro, rlse = oracle.attn_fwd(x["q"], x["k"], x["v"], scale, True)
     assert max_abs(out["o"], ro) <= BF16_TOL
     assert max_abs(out["lse"], rlse) <= LSE_TOL
+    _assert_grads_within_rounding_bound(out, x, scale, True)
 
 
 @pytest.mark.parametrize("d,causal", [(128, False), (128, True), (64, True)])
@@ -122,31 +124,113 @@ def test_forward_work_queue_survives_many_launches(fa_lib, d, causal):
         assert torch.equal(o, o0) and torch.equal(lse, lse0)
 
 
-def _d_rounding_bounds(x, scale, causal):
-    """First-order effect on dQ and dK of forming D_i = <dO_i, O_i> from the bf16
-    O the backward is given (the oracle uses D_i = sum_j P_ij dP_ij exactly).
-    |O~ - O| <= 2^-9 |O| (final rounding) + 2^-9 sum_j P_ij |v_j| (bf16 P in the
-    PV product) <= 2^-8 sum_j P_ij |v_j|; dS_ij moves by -P_ij dD_i, hence
-    |d dQ_i| <= scale |dD_i| sum_j P_ij |k_j| and |d dK_j| <= scale sum_i P_ij |dD_i| |q_i|.
-    Computed in fp64 with torch's own softmax / matmul on the inputs only."""
+@pytest.mark.parametrize("words", [1, 64])
+def test_forward_on_concurrent_streams_with_shared_queue_words(fa_lib, words):
+    """Forward launches on four streams at once.  With words = 1 every launch
+    takes its work items from the same queue word, so launches in flight
+    together meet there: a launch that finds the word held by another takes
+    its items in the fixed order instead.  Every output must equal the same
+    launch run alone, bit for bit, and the device must report no error."""
+    shapes = [((2, 3, 700, 128), True), ((1, 5, 1000, 128), False), ((3, 2, 513, 64), True),
+              ((2, 4, 900, 64), False)]
+    xs, refs = [], []
+    for n, (shape, causal) in enumerate(shapes):
+        x = to_cuda(_inputs(shape, seed=1234 + n))
+        scale = 1 / math.sqrt(shape[-1])
+        xs.append((x, scale, causal))
+        refs.append(fa_lib.fwd(x["q"], x["k"], x["v"], causal=causal, scale=scale))
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in shapes]
+    assert fa_lib._lib.fa_set_fwd_queue_words(words) == fa_lib.FA_OK
+    try:
+        outs = []
+        for _ in range(25):
+            for n, st in enumerate(streams):
+                x, scale, causal = xs[n]
+                with torch.cuda.stream(st):
+                    outs.append((n, fa_lib.fwd(x["q"], x["k"], x["v"], causal=causal, scale=scale)))
+        torch.cuda.synchronize()
+    finally:
+        fa_lib._lib.fa_set_fwd_queue_words(64)
+    assert fa_lib.check_device_status() == 0
+    for n, (o, lse) in outs:
+        assert torch.equal(o, refs[n][0]) and torch.equal(lse, refs[n][1]), n
+
+
+def test_forward_replayed_from_a_captured_graph(fa_lib):
+    """A captured forward keeps its launch ticket, so each replay finds the
+    queue word as the previous replay left it; every replay must still process
+    every item (inputs change between replays, outputs must follow)."""
+    x = to_cuda(_inputs((2, 3, 1100, 128), seed=4321))
+    scale = 1 / math.sqrt(128)
+    o = torch.empty_like(x["q"])
+    lse = torch.empty(x["q"].shape[:3], dtype=torch.float32, device="cuda")
+    fa_lib.fwd(x["q"], x["k"], x["v"], causal=True, scale=scale, out=o, lse=lse)  # warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="relaxed"):
+        fa_lib.fwd(x["q"], x["k"], x["v"], causal=True, scale=scale, out=o, lse=lse)
+    for rep in range(4):
+        fresh = _inputs((2, 3, 1100, 128), seed=5000 + rep)
+        for n in ("q", "k", "v"):
+            x[n].copy_(fresh[n])
+        o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        ro, rlse = oracle.attn_fwd(fresh["q"], fresh["k"], fresh["v"], scale, True)
+        assert max_abs(o, ro) <= BF16_TOL, rep
+        assert max_abs(lse, rlse) <= LSE_TOL, rep
+    del g
+    assert fa_lib.check_device_status() == 0
+
+
+def _bwd_rounding_bounds(x, scale, causal):
+    """Per-element bounds on how far the bf16 roundings inside the backward
+    can move dQ, dK and dV away from the exact gradients, to first order.
+
+    The kernels keep P = 2^(c s - lse2) in bf16 (|dP| <= 2^-9 P) as the dV
+    operand and for dS, form D_i = <dO_i, O~_i> from the bf16 output O~ of the
+    forward, and round dS = P (dP - D) to bf16 (2^-9 relative) before the dK and
+    dQ products; every sum is fp32 (2^-24 relative per term, negligible here).
+      |O~ - O|_i <= 2^-9 |O_i| + 2^-9 sum_j P_ij |v_j| <= 2^-8 sum_j P_ij |v_j|
+      |dD_i|     <= sum_t |dO_it| |O~ - O|_it
+      |d dS_ij|  <= 2^-8 |dS_ij| + P_ij |dD_i|       (P and dS rounded, D moved)
+      |d dQ_i|   <= scale sum_j |d dS_ij| |k_j|,  |d dK_j| <= scale sum_i |d dS_ij| |q_i|
+      |d dV_j|   <= 2^-9 sum_i P_ij |dO_i|
+    Computed in fp64 with torch's own softmax and matmul on the inputs only."""
     q, k, v, do = (x[n].double() for n in ("q", "k", "v", "do"))
     s = scale * q @ k.transpose(-1, -2)
     if causal:
         N = s.shape[-1]
         s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
     P = torch.softmax(s, -1)
-    bound_d = (2.0 ** -8) * 1.01 * (do.abs() * (P @ v.abs())).sum(-1, keepdim=True)
-    tq = scale * bound_d * (P @ k.abs())
-    tk = scale * (P.transpose(-1, -2) @ (bound_d * q.abs()))
-    return tq.numpy(), tk.numpy()
+    dP = do @ v.transpose(-1, -2)
+    D = (P * dP).sum(-1, keepdim=True)
+    dS = P * (dP - D)
+    u = 1.02  # room for the fp32 sums and ex2.approx
+    bound_d = u * (2.0 ** -8) * (do.abs() * (P @ v.abs())).sum(-1, keepdim=True)
+    e_ds = u * (2.0 ** -8) * dS.abs() + P * bound_d
+    tq = scale * (e_ds @ k.abs())
+    tk = scale * (e_ds.transpose(-1, -2) @ q.abs())
+    tv = u * (2.0 ** -9) * (P.transpose(-1, -2) @ do.abs())
+    return tq.numpy(), tk.numpy(), tv.numpy()
+
+
+def _assert_grads_within_rounding_bound(out, x, scale, causal):
+    rdq, rdk, rdv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], scale, causal)
+    tq, tk, tv = _bwd_rounding_bounds(x, scale, causal)
+    for n, r, t in (("dq", rdq, tq), ("dk", rdk, tk), ("dv", rdv, tv)):
+        err = np.abs(out[n].double().cpu().numpy() - r)
+        assert np.all(err <= BF16_TOL + t), (n, float(err.max()), float((err - t).max()))
 
 
 @pytest.mark.parametrize("d,causal", [(64, True), (128, True), (128, False)])
 def test_long_context_distribution_fwd_bwd(fa_lib, d, causal):
     """The long-context workload's distribution (q, k ~ 2 N(0,1)) at N = 777,
     compared in full.  With few keys per row the softmax is sharp, so in
-    dS = P (dP - D) the two terms nearly cancel and the bf16 rounding of O
-    (through D) shows up in dQ and dK; their bar adds that term's bound."""
+    dS = P (dP - D) the two terms nearly cancel and the bf16 roundings (of O
+    through D, of P and of dS) show up in dQ and dK; their bar adds the bound
+    of _bwd_rounding_bounds.  dV is held to the plain 2e-2."""
     x = _inputs((1, 2, 777, d), seed=5 + d + causal, gain=2.0)
     scale = 1 / math.sqrt(d)
     out = gpu_fwd_bwd(fa_lib, to_cuda(x), scale, causal)
@@ -155,10 +239,7 @@ def test_long_context_distribution_fwd_bwd(fa_lib, d, causal):
     assert max_abs(out["o"], ro) <= BF16_TOL
     assert max_abs(out["lse"], rlse) <= LSE_TOL
     assert max_abs(out["dv"], rdv) <= BF16_TOL
-    tq, tk = _d_rounding_bounds(x, scale, causal)
-    for n, r, t in (("dq", rdq, tq), ("dk", rdk, tk)):
-        err = np.abs(out[n].double().cpu().numpy() - r)
-        assert np.all(err <= BF16_TOL + t), (n, float(err.max()), float((err - t).max()))
+    _assert_grads_within_rounding_bound(out, x, scale, causal)
 
 
 def test_worked_row_bf16():
@@ -238,10 +319,11 @@ def _check_sampled(w, x, out, heads, full_bwd_heads, last_keys):
         assert max_abs(gdv[h, N - last_keys:], rdv) <= BF16_TOL, ("dv", h)
     for h in full_bwd_heads:
         xs = {n: flat[n][h][None, None] for n in ("q", "k", "v", "do")}
-        rdq, rdk, rdv = oracle.attn_bwd(xs["q"], xs["k"], xs["v"], xs["do"], w.scale, w.causal)
-        assert max_abs(gdq[h][None, None], rdq) <= BF16_TOL, ("dq full", h)
-        assert max_abs(gdk[h][None, None], rdk) <= BF16_TOL, ("dk full", h)
-        assert max_abs(gdv[h][None, None], rdv) <= BF16_TOL, ("dv full", h)
+        rdq, rdk, rdv = oracle.attn_bwd_head(flat["q"][h], flat["k"][h], flat["v"][h], flat["do"][h], w.scale,
+                                             w.causal)
+        assert max_abs(gdq[h], rdq) <= BF16_TOL, ("dq full", h)
+        assert max_abs(gdk[h], rdk) <= BF16_TOL, ("dk full", h)
+        assert max_abs(gdv[h], rdv) <= BF16_TOL, ("dv full", h)
         ro, rlse = oracle.attn_fwd(xs["q"], xs["k"], xs["v"], w.scale, w.causal)
         assert max_abs(go[h][None, None], ro) <= BF16_TOL, ("o full", h)
         assert max_abs(glse[h][None, None], rlse) <= LSE_TOL, ("lse full", h)
@@ -254,8 +336,11 @@ def test_workload4_sampled(fa_lib):
     _check_sampled(w, x, out, heads=[0, 21, 63], full_bwd_heads=[42], last_keys=256)
 
 
-def test_workload5_sampled(fa_lib):
+def test_workload5_sampled_and_whole_heads(fa_lib):
+    """The long-context workload: sampled rows and the last keys of heads 0 and
+    15, and heads 6 and 11 compared whole (every dQ, dK, dV element, including
+    the first keys, which every query row sees and where |dK| peaks)."""
     w = WORKLOADS["c5_bf16_1x16x16384x128_causal_qk2"]
     x = make_inputs(w)
     out = gpu_fwd_bwd(fa_lib, to_cuda(x), w.scale, w.causal)
-    _check_sampled(w, x, out, heads=[0, 15], full_bwd_heads=[], last_keys=128)
+    _check_sampled(w, x, out, heads=[0, 15], full_bwd_heads=[6, 11], last_keys=128)

@@ -19,7 +19,7 @@ GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 def _run(fa, x, causal, scale, block_k=0):
     q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
     o, lse = fa.fwd_f32(q, k, v, causal=causal, scale=scale, block_k=block_k)
-    dq, dk, dv = fa.bwd_f32(q, k, v, o, lse, do, causal=causal, scale=scale)
+    dq, dk, dv = fa.bwd_f32(q, k, v, o, lse, do, causal=causal, scale=scale, block_k=block_k)
     torch.cuda.synchronize()
     return o, lse, dq, dk, dv
 
@@ -48,13 +48,20 @@ def test_ragged_and_edge_shapes(fa_lib, shape, causal):
 
 
 @pytest.mark.parametrize("block_k", [1, 2, 3, 7, 64, 256])
-def test_block_size_never_changes_the_answer(fa_lib, block_k):
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_size_never_changes_the_answer(fa_lib, block_k, causal):
+    """Forward and backward walk keys (and, for dK / dV, queries) in blocks of
+    block_k; every block size, divisors of N or not, gives the oracle's answer."""
     w = WORKLOADS["c1_f32_1x2x256x64"]
     x = make_inputs(w)
-    o, lse, *_ = _run(fa_lib, x, False, w.scale, block_k)
-    ro, rlse = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, False)
+    o, lse, dq, dk, dv = _run(fa_lib, x, causal, w.scale, block_k)
+    ro, rlse = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, causal)
+    rdq, rdk, rdv = oracle.attn_bwd(x["q"], x["k"], x["v"], x["do"], w.scale, causal)
     assert max_abs(o, ro) <= F32_TOL
     assert max_abs(lse, rlse) <= F32_TOL
+    assert max_abs(dq, rdq) <= F32_TOL
+    assert max_abs(dk, rdk) <= F32_TOL
+    assert max_abs(dv, rdv) <= F32_TOL
 
 
 def test_worked_row_through_the_gpu():

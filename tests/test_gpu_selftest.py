@@ -45,8 +45,10 @@ def test_fma_pipe_exp2_within_its_fitted_bound(fa_lib):
     """The polynomial exp2 the kernels use beside ex2.approx: relative error
     against float64 2^x within the Remez fit's bound (exp2_poly.h) plus float32
     evaluation rounding, over the range the kernels feed it."""
+    import os
     import re
-    hdr = open("exact_io_aware_53_b200/csrc/exp2_poly.h").read()
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    hdr = open(os.path.join(root, "exact_io_aware_53_b200", "csrc", "exp2_poly.h")).read()
     bound = float(re.search(r"MAX_REL_ERR = ([0-9.e+-]+)f", hdr).group(1))
     g = torch.Generator().manual_seed(3)
     x = torch.cat([torch.linspace(-124.0, 64.0, 1 << 20), torch.rand(1 << 20, generator=g) * 20 - 16,

@@ -520,3 +520,72 @@ def test_dropout_head_offset_selects_the_heads_generator_stream():
         oh, lh = oracle.attn_fwd_dropout(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], 0.6, True,
                                          200, 11, 2, bh0=b * 3 + h)
         assert np.array_equal(oh[0, 0], o[b, h]) and np.array_equal(lh[0, 0], lse[b, h])
+
+
+# ---------------------------------------------------------------- per-head threaded backward
+
+
+def _torch_grads(q, k, v, g, scale, causal, z=None, t=256):
+    """torch fp64 autograd of L = sum(O * G), O = (256/t) (softmax(S) o Z) V (Z = 1: plain)."""
+    tq, tk, tv = (torch.from_numpy(np.asarray(x, dtype=np.float64)).requires_grad_(True) for x in (q, k, v))
+    s = scale * tq @ tk.transpose(-1, -2)
+    N = s.shape[-1]
+    if causal:
+        s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+    p = torch.softmax(s, -1)
+    if z is not None:
+        p = p * torch.as_tensor(z, dtype=torch.float64) * (256.0 / t)
+    ((p @ tv) * torch.from_numpy(np.asarray(g, dtype=np.float64))).sum().backward()
+    return tq.grad.numpy(), tk.grad.numpy(), tv.grad.numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(1, 3), (23, 5), (70, 8)])
+def test_head_backward_matches_torch_autograd(N, d, causal):
+    q, k, v, g = (_rand((N, d), seed=s, gain=1.3) for s in (121, 122, 123, 124))
+    dq, dk, dv = oracle.attn_bwd_head(q, k, v, g, 0.55, causal)
+    for a, b in zip((dq, dk, dv), _torch_grads(q, k, v, g, 0.55, causal)):
+        assert np.max(np.abs(a - b)) < 1e-12
+    # the same definition as the per-head-threaded backward
+    for a, b in zip((dq, dk, dv), oracle.attn_bwd(q[None, None], k[None, None], v[None, None], g[None, None],
+                                                  0.55, causal)):
+        assert np.max(np.abs(a - b[0, 0])) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_backward_invariants(causal):
+    N, d = 90, 6
+    q, k, v, g = (_rand((N, d), seed=s, gain=1.5) for s in (131, 132, 133, 134))
+    dq, dk, dv = oracle.attn_bwd_head(q, k, v, g, 0.4, causal)
+    assert np.max(np.abs(dk.sum(0))) < 1e-12          # rows of dS sum to zero
+    assert np.max(np.abs(dv.sum(0) - g.sum(0))) < 1e-12  # rows of P sum to one
+    if causal:
+        # key 0 is seen by every query and the first query sees only key 0
+        o, lse = oracle.attn_fwd(q[None, None], k[None, None], v[None, None], 0.4, True)
+        assert np.max(np.abs(dq[0])) < 1e-15          # P_00 = 1, dS_00 = dP_00 - D_0 = 0
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("bh,t", [(0, 200), (5, 77)])
+def test_head_backward_with_dropout_matches_torch_with_numpy_mask(bh, t, causal):
+    N, d = 45, 4
+    q, k, v, g = (_rand((N, d), seed=s) for s in (141, 142, 143, 144))
+    seed, offset = 2 ** 33 + 17, 4
+    z = _numpy_keep_mask(bh, N, t, seed, offset)
+    dq, dk, dv = oracle.attn_bwd_head(q, k, v, g, 0.5, causal, keep_t=t, seed=seed, offset=offset, bh=bh)
+    for a, b in zip((dq, dk, dv), _torch_grads(q, k, v, g, 0.5, causal, z, t)):
+        assert np.max(np.abs(a - b)) < 1e-12
+
+
+def test_dropout_backward_head_offset_selects_the_heads_generator_stream():
+    """Heads given alone with bh0 = their index reproduce the whole problem's gradients."""
+    q, k, v, g = (_rand((2, 3, 33, 4), seed=150 + s) for s in range(4))
+    full = oracle.attn_bwd_dropout(q, k, v, g, 0.6, True, 190, 8, 1)
+    for b, h in ((0, 1), (1, 2)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        part = oracle.attn_bwd_dropout(q[sl], k[sl], v[sl], g[sl], 0.6, True, 190, 8, 1, bh0=b * 3 + h)
+        head = oracle.attn_bwd_head(q[b, h], k[b, h], v[b, h], g[b, h], 0.6, True, keep_t=190, seed=8, offset=1,
+                                    bh=b * 3 + h)
+        for a, p, hh in zip(full, part, head):
+            assert np.array_equal(p[0, 0], a[b, h])
+            assert np.max(np.abs(hh - a[b, h])) < 1e-13

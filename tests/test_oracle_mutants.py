@@ -40,6 +40,10 @@ MUTANTS = [
      "const double s_keep = t > 0 ? 255.0 / t : 0.0;", "dropout"),
     ("dropout dV from the undropped weights", "const double pz = prow[j] * zrow[j];", "const double pz = prow[j];",
      "dropout"),
+    ("head backward: key pass skips the diagonal query", "for (long i = causal ? j : 0; i < N; ++i) {",
+     "for (long i = causal ? j + 1 : 0; i < N; ++i) {", "head"),
+    ("head backward: weight from the key's row statistics", "- rm[i]) / rl[i];", "- rm[j]) / rl[i];", "head"),
+    ("head backward: dV ignores the dropout mask", "const double pz = p * z;", "const double pz = p;", "head"),
 ]
 
 
