@@ -719,18 +719,22 @@ def run_blocksparse(args, w):
                 "traffic_unit": "bytes per launch (ncu dram read+write)"}
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv = (t.pin_memory() for t in (hq, hk, hv))
+        hq, hk, hv, hdo = (t.pin_memory() for t in (hq, hk, hv, hdo))
         ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        hg = [torch.empty(dq.shape, dtype=dq.dtype).pin_memory() for _ in range(3)]
         steps = max(3, min(args.steps, 20))
 
         def e2e_step():
             q.copy_(hq, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
+            do.copy_(hdo, non_blocking=True)
             step()
             ho.copy_(o, non_blocking=True)
             hl.copy_(lse, non_blocking=True)
+            for h_, g_ in zip(hg, (dq, dk, dv)):
+                h_.copy_(g_, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -924,18 +928,22 @@ def run_fp8(args, w):
 
 # ------------------------------------------------------------------ forward with dropout
 
-DROPOUT_METRIC = "attention forward with dropout TFLOPS on 1 B200 and fraction of dense BF16 tensor peak"
+DROPOUT_METRIC = "attention fwd/bwd with dropout TFLOPS on 1 B200 and fraction of dense BF16 tensor peak"
 
 
 def dropout_oracle_sample(w, heads: int, seed: int):
-    """fp64 oracle dropout forward on `heads` heads; returns (seconds, flops, threads)."""
+    """fp64 oracle dropout forward and backward on `heads` heads; returns
+    (seconds, flops under the fwd + 2.5 x fwd convention, threads)."""
     from exact_io_aware_53_b200.workloads import random_tensors
     from oracle import oracle
-    q, k, v, _ = random_tensors((1, heads, w.N, w.d), torch_bf16(), seed=seed)
+    q, k, v, do = random_tensors((1, heads, w.N, w.d), torch_bf16(), seed=seed)
     t0 = time.perf_counter()
     oracle.attn_fwd_dropout(q, k, v, w.scale, w.causal, w.keep_t, w.seed, w.offset)
+    for h in range(heads):
+        oracle.attn_bwd_head(q[0, h], k[0, h], v[0, h], do[0, h], w.scale, w.causal, keep_t=w.keep_t, seed=w.seed,
+                             offset=w.offset, bh=h)
     dt = time.perf_counter() - t0
-    return dt, w.flops() / (w.B * w.H) * heads, oracle.num_threads()
+    return dt, 3.5 * w.flops() / (w.B * w.H) * heads, oracle.num_threads()
 
 
 def run_reference_dropout(args, w):
@@ -964,7 +972,9 @@ def run_reference_dropout(args, w):
 
 
 def run_dropout(args, w):
-    """One step = fa_fwd_dropout over the whole batch, inputs resident in device memory."""
+    """One step = fa_fwd_dropout then fa_bwd_dropout over the whole batch, inputs
+    resident in device memory; FLOPs: forward 4 B H N^2 d (halved causal),
+    backward 2.5 times that."""
     import torch
     from exact_io_aware_53_b200 import fa
     from exact_io_aware_53_b200.workloads import random_tensors
@@ -976,17 +986,31 @@ def run_dropout(args, w):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     B, H, N, d = w.B, w.H, w.N, w.d
-    hq, hk, hv, _ = random_tensors((B, H, N, d), torch.bfloat16, seed=rank_seed(w.seed, rank))
-    q, k, v = (t.to(dev) for t in (hq, hk, hv))
+    hq, hk, hv, hdo = random_tensors((B, H, N, d), torch.bfloat16, seed=rank_seed(w.seed, rank))
+    q, k, v, do = (t.to(dev) for t in (hq, hk, hv, hdo))
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty_like(dq)
+    dv = torch.empty_like(dq)
+    ws = torch.empty(max(1, fa.bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8, device=dev)
     launches = [0]
 
-    def step():
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
         rc = fa.fwd_dropout_raw(q, k, v, o, lse, w.scale, w.causal, w.keep_t, w.seed, w.offset)
         launches[0] += fa.last_launch_count()
         if rc:
             raise fa.FAError(rc, "fa_fwd_dropout")
+        if ev is not None:
+            ev[1].record(stream)
+        rc = fa.bwd_dropout_raw(q, k, v, o, lse, do, dq, dk, dv, ws, w.scale, w.causal, w.keep_t, w.seed, w.offset)
+        launches[0] += fa.last_launch_count()
+        if rc:
+            raise fa.FAError(rc, "fa_bwd_dropout")
+        if ev is not None:
+            ev[2].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -994,7 +1018,9 @@ def run_dropout(args, w):
     st = fa.check_device_status()
     if st:
         raise RuntimeError("device status after warm-up: %s" % fa.status_string(st))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
     uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(uuid)
     sampler.start()
@@ -1002,41 +1028,56 @@ def run_dropout(args, w):
     launches[0] = 0
     barrier(world)
     torch.cuda.synchronize()
+    t_start.record(stream)
     for i in range(args.steps):
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
+        step(evs[i])
+    t_end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clocks = sampler.stop()
     st = fa.check_device_status()
     if st:
         raise RuntimeError("device status after timing: %s" % fa.status_string(st))
-    ms_local = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    timed_launches = launches[0]
+    ms_local = t_start.elapsed_time(t_end) / args.steps
     ms = max_over_ranks(ms_local, world, dev)
-    fl = w.flops()
-    value = world * fl / (ms / 1e3) / 1e12
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    fl_fwd = w.flops()
+    fl_bwd = 2.5 * fl_fwd
+    value = world * (fl_fwd + fl_bwd) / (ms / 1e3) / 1e12
     peaks, peak_src = load_peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = fl / (ms_local / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "decode_partial_kernel (dropout, direct output)", "achieved": achieved,
-                "peak": peak, "unit": UNIT, "frac": achieved / peak, "peak_source": "bf16_tflops %s" % peak_src,
-                "algorithmic_flops_per_launch": fl, "ms_per_launch": ms_local,
-                "traffic": measured_traffic("dropout", w.name), "traffic_unit": "bytes per launch (ncu dram read+write)"}
+    long_region = ms * args.steps > 500.0
+    peak_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+    peak = float(peaks.get(peak_key, FALLBACK_PEAKS[peak_key]))
+    achieved = fl_bwd / (bwd_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "fa_bwd_dropout (pre-pass + bwd_kernel<128, causal, dropout>)",
+                "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                "peak_source": "%s %s" % (peak_key, peak_src), "algorithmic_flops_per_launch": fl_bwd,
+                "ms_per_launch": bwd_ms, "traffic": measured_traffic("bwd_dropout", w.name),
+                "traffic_unit": "bytes per launch (ncu dram read+write)"}
+    fwd_tf = fl_fwd / (fwd_ms / 1e3) / 1e12
+    kernels = {"fwd_dropout": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
+               "bwd_dropout": {"ms": bwd_ms, "tflops": achieved, "frac": achieved / peak}}
+    fl = fl_fwd + fl_bwd
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv = (t.pin_memory() for t in (hq, hk, hv))
+        hq, hk, hv, hdo = (t.pin_memory() for t in (hq, hk, hv, hdo))
         ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        hg = [torch.empty(dq.shape, dtype=dq.dtype).pin_memory() for _ in range(3)]
         steps = max(3, min(args.steps, 20))
 
         def e2e_step():
             q.copy_(hq, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
+            do.copy_(hdo, non_blocking=True)
             step()
             ho.copy_(o, non_blocking=True)
             hl.copy_(lse, non_blocking=True)
+            for h_, g_ in zip(hg, (dq, dk, dv)):
+                h_.copy_(g_, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -1051,8 +1092,10 @@ def run_dropout(args, w):
         barrier(world)
         ems = max_over_ranks(a.elapsed_time(b) / steps, world, dev)
         e2e = {"value": world * fl / (ems / 1e3) / 1e12, "unit": UNIT, "ms_per_step": ems,
-               "h2d_bytes_per_step": 3 * hq.numel() * 2, "d2h_bytes_per_step": ho.numel() * 2 + hl.numel() * 4,
-               "steps": steps, "api": "fa.fwd_dropout_raw with q, k, v from and o, lse to pinned host memory"}
+               "h2d_bytes_per_step": 4 * hq.numel() * 2,
+               "d2h_bytes_per_step": ho.numel() * 2 + hl.numel() * 4 + 3 * dq.numel() * 4, "steps": steps,
+               "api": "fa.fwd_dropout_raw + fa.bwd_dropout_raw with q, k, v, dO from and o, lse, dq, dk, dv to "
+                      "pinned host memory"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, cfl, thr, nh = sized_oracle_sample(lambda h: dropout_oracle_sample(w, h, w.seed), B * H)
@@ -1063,9 +1106,11 @@ def run_dropout(args, w):
             "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d, "causal": w.causal, "keep_t": w.keep_t,
+                       "backward": True,
                        "parallelism": "dp%d (independent batches per GPU, no collective)" % world,
-                       "l2": "inputs larger than L2 (q, k, v = %.0f MB per GPU)" % (3 * B * H * N * d * 2 / 1e6)},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches[0], "clocks": clocks}
+                       "l2": "inputs larger than L2 (q, k, v, dO = %.0f MB per GPU)" % (4 * B * H * N * d * 2 / 1e6)},
+            "roofline": roofline, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": timed_launches, "clocks": clocks}
     if rank == 0:
         print(json.dumps(line), flush=True)
     return line

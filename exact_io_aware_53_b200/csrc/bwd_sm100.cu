@@ -1,72 +1,93 @@
-// Backward attention for head dimension 64, bf16 in / fp32 gradients, sm_100a
-// (head dimension 128 has its own kernel, bwd128_sm100.cu).
+// Backward attention, bf16 in / fp32 gradients, sm_100a, head dimension 64 or
+// 128, optionally with dropout.
 //
-// The attention weights are never stored: each CTA owns one tile of 128 keys
-// (K_j, V_j resident in shared memory) and walks the 64-row query tiles that
-// see it, recomputing the transposed weights from the saved log-sum-exp
-// (the recomputation of "What it did not solve", vibeengines.com/paper/
-// flash-attention).  With c = scale * log2(e) and lse2 = lse * log2(e):
+// The attention weights are never stored: they are rebuilt per tile from the
+// saved log-sum-exp ("What it did not solve", vibeengines.com/paper/
+// flash-attention).  With c = scale * log2 e and lse2 = lse * log2 e:
 //
-//   S^T  = K Q_i^T                      (tensor core, TMEM)
-//   P^T  = 2^(c S^T - lse2_i)           (softmax warps; masked entries 0)
-//   dP^T = V dO_i^T                     (tensor core, TMEM)
-//   dS^T = P^T o (dP^T - D_i)           (softmax warps; D_i = <dO_i, O_i>)
-//   dV  += P^T dO_i,   dK += dS^T Q_i   (A operand from TMEM, accumulate in TMEM)
-//   dQ_i^T = K^T dS^T                   (tensor core) -> fp32 TMA reduce-add into dQ
+//   S^T  = K Q_t^T,  P^T = 2^(c S^T - lse2_t)      dP^T = V dO_t^T
+//   dS^T = P^T o (dP^T - D_t)                        D_t = <dO, O> per query row
+//   dV += P^T dO_t,  dK += dS^T Q_t,  dQ_t = dS K_j   (dK, dQ times scale)
 //
-// and dK is multiplied by `scale` at the end, dQ by `scale` before the add.
+// One CTA owns 128 keys (K_j, V_j stay in shared memory) and walks the
+// 128-row query tiles t that see them, so every tensor-core instruction is
+// 128 rows by 128 (or by d) columns.
+//
+// TMEM (512 columns): two 128-column regions R0, R1, then dV and dK (d columns
+// each) and, for d = 64, dQ (64 columns).  Tile t uses X = R[t & 1] for
+// S^T -> P^T (bf16 pairs in its first 64 columns) and Y = R[(t + 1) & 1] for
+// dP^T.  dS^T goes to shared memory only, where it is the K-major A operand
+// of dK and the MN-major operand of the dQ product; so Y is free once the
+// softmax has read dP^T, and S^T of tile t + 1 is issued there before dK and
+// dQ of tile t, overlapping the next softmax with them.  dP^T of tile t + 1
+// then goes to X.
+//   d = 128: dQ_t^T = K^T dS^T (lanes = head-dim index) is written into X
+//            after dS^T, so dP^T of tile t + 1 waits for the dQ warps to have
+//            read it; staged as fp32 [64 query][128 d] tiles, two per tile.
+//   d = 64:  dQ_t = dS K (lanes = query rows, 64 columns) has its own region;
+//            the next dQ waits for the dQ warps instead.  Staged as one fp32
+//            [128 query][64 d] tile.
+// Staged tiles are TMA reduce-added (fp32) into dQ.
+//
+// Dropout (DROPOUT): the forward kept weight P_ij with probability keep_t / 256
+// and scaled kept weights by 256 / keep_t; the keep bit is byte j % 32 of
+// Philox4x64-10 at counter (j / 32, i, bh, 0) under key (seed, offset), kept
+// iff it is below keep_t.  With Z the keep mask and z = 256 / keep_t:
+//   dV = z (P o Z)^T dO,   dS = P o (z Z o dP - D)       (D from the dropped O)
+// A warp's 32 key rows are one 32-key group of the generator, so each lane
+// draws the block of one query (32 bytes: the keep bytes of all 32 keys for
+// that query) and a 32 x 32 bit transpose across the warp hands every lane its
+// own key's bits: four blocks per thread per tile, as in the forward.  X then
+// holds bf16(P o Z) in columns 0-63 (the dV operand; the factor z is applied
+// to dV at the end) and bf16(P) in columns 64-127 for dS.
 //
 // Warp roles (320 threads):
-//   warps 0-3  softmax: thread = key row = TMEM lane; writes P^T, dS^T as bf16
-//              pairs into TMEM and dS^T into swizzled shared memory
-//   warps 4-7  dQ: thread = head-dim row of dQ^T; scales it, stages it in
-//              shared memory, one thread issues the TMA reduce-add
+//   warps 0-3  softmax: thread = key row = TMEM lane
+//   warps 4-7  dQ: read dQ (or dQ^T) out of TMEM, scale, stage, reduce-add
 //   warp 8     MMA issuer (one thread)
-//   warp 9     TMA producer (K, V once; Q_i, dO_i, lse2_i, D_i through a 3-stage ring)
-//
-// TMEM columns: dV [0, D), dK [D, 2D), S^T x2 [2D, 2D+128), dP^T [2D+128,
-// 2D+192), dQ^T [2D+192, 2D+256).  P^T overwrites the first 32 columns of its
-// S^T buffer, dS^T the first 32 columns of dP^T.  For D = 64 the dQ^T MMA
-// still has M = 128: K^T's second 64-row half reads a zero block, and the
-// rows it produces are ignored.
+//   warp 9     TMA producer: K, V once; {Q_t, lse2_t, D_t} in a 2-stage ring,
+//              dO_t in one buffer (its last reader, dV, runs early in a tile
+//              and its next reader, dP^T, late in the previous one)
 #include "kernels.h"
 #include "sm100.cuh"
 
 namespace fa {
 namespace bwdk {
 
-constexpr int BKV = 128;  // keys per CTA
-constexpr int BQ = 64;    // query rows per step
+constexpr int BKV = 128;
+constexpr int BQ = 128;
 constexpr int NTHREADS = 320;
 constexpr int MMA_WARP = 8;
 constexpr int LOAD_WARP = 9;
-constexpr int QSTAGES = 3;
+constexpr int QSTAGES = 2;
+constexpr int BOX = 128 * 128;  // 128 rows x 128 B (64 bf16)
 
 template <int D>
 struct Cfg {
-    static constexpr int NDC = D / 64;                 // 64-column boxes per row
-    static constexpr int KBOX = BKV * 128;             // 128 rows x 128 B
-    static constexpr int QBOX = BQ * 128;              // 64 rows x 128 B
-    static constexpr int K_OFF = 0;                    // K (+ zero block when D = 64): 2 boxes
-    static constexpr int V_OFF = K_OFF + 2 * KBOX;
-    static constexpr int QS_OFF = V_OFF + NDC * KBOX;  // stages of {Q_i, dO_i}
-    static constexpr int QSTAGE_BYTES = 2 * NDC * QBOX;
-    static constexpr int DS_OFF = QS_OFF + QSTAGES * QSTAGE_BYTES;  // 2 x (128 x 64 bf16)
-    static constexpr int DS_BYTES = BKV * BQ * 2;
-    static constexpr int DQ_OFF = DS_OFF + 2 * DS_BYTES;            // fp32 [D/32 chunks][BQ rows][128 B]
-    static constexpr int DQ_CHUNK = BQ * 128;
-    static constexpr int VEC_OFF = DQ_OFF + (D / 32) * DQ_CHUNK;    // [QSTAGES][lse2 64 | delta 64]
+    static constexpr int NDC = D / 64;  // 128-byte column boxes per row
+    static constexpr int TILE = NDC * BOX;
+    static constexpr int K_OFF = 0;
+    static constexpr int V_OFF = K_OFF + TILE;
+    static constexpr int Q_OFF = V_OFF + TILE;             // Q_t, 2 stages
+    static constexpr int DO_OFF = Q_OFF + QSTAGES * TILE;  // dO_t, 1 stage
+    static constexpr int DS_OFF = DO_OFF + TILE;           // dS^T: 2 boxes of 64 query columns
+    static constexpr int STG_OFF = DS_OFF + 2 * BOX;       // dQ staging
+    // fp32 staging tile: D / 32 chunks of [STG_ROWS query rows][32 d], 128-byte swizzled
+    static constexpr int STG_ROWS = (D == 128) ? 64 : 128;
+    static constexpr int STG_CHUNK = STG_ROWS * 128;
+    static constexpr int VEC_OFF = STG_OFF + (D / 32) * STG_CHUNK;  // [stage][lse2 128 | delta 128]
     static constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
-    static constexpr int NBARS = 19;
+    static constexpr int NBARS = 17;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static constexpr uint32_t DV_COL = 0;
-    static constexpr uint32_t DK_COL = D;
-    static constexpr uint32_t S_COL = 2 * D;
-    static constexpr uint32_t DP_COL = 2 * D + 128;
-    static constexpr uint32_t DQ_COL = 2 * D + 192;
+    static constexpr uint32_t DV_COL = 256;
+    static constexpr uint32_t DK_COL = 256 + D;
+    static constexpr uint32_t DQ_COL = 256 + 2 * D;  // d = 64 only
     static constexpr uint32_t TMEM_COLS = 512;
 };
+
+// TMEM column of region R[t & 1]
+__device__ __forceinline__ uint32_t rcol(int t) { return 128u * static_cast<uint32_t>(t & 1); }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c)
 {
@@ -74,39 +95,77 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
     return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, bool CAUSAL>
+// 32 x 32 bit-matrix transpose across a warp: lane l holds row l on entry and
+// column l on return (bit b of lane l's result = bit l of lane b's row), by
+// swapping the off-diagonal blocks of size 16, 8, 4, 2, 1 in turn.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane)
+{
+    const uint32_t masks[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const int s = 16 >> k;
+        const uint32_t m = masks[k];
+        const uint32_t other = __shfl_xor_sync(0xffffffffu, x, s);
+        x = (lane & s) ? ((x & ~m) | ((other & ~m) >> s)) : ((x & m) | ((other & m) << s));
+    }
+    return x;
+}
+
+// Keep bits of one query row for the 32 keys of one generator block: bit b is
+// set iff byte b of Philox4x64-10 at (key_group, query, bh, 0) is below keep_t.
+__device__ __noinline__ uint32_t keep_bits(uint64_t key_group, uint64_t query, uint64_t bh, int keep_t,
+                                         uint64_t seed, uint64_t offset)
+{
+    if (keep_t >= 256) return 0xFFFFFFFFu;
+    uint64_t x0 = key_group, x1 = query, x2 = bh, x3 = 0;
+    philox4x64_10(x0, x1, x2, x3, seed, offset);
+    const uint64_t w[4] = {x0, x1, x2, x3};
+    const uint32_t t4 = static_cast<uint32_t>(keep_t) * 0x01010101u;
+    uint32_t m = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t word = static_cast<uint32_t>(w[k >> 1] >> (32 * (k & 1)));
+        const uint32_t lt = __vcmpltu4(word, t4);  // 0xFF in each byte below keep_t
+        m |= (((lt & 0x01010101u) * 0x01020408u) >> 24) << (4 * k);
+    }
+    return m;
+}
+
+template <int D, bool CAUSAL, bool DROPOUT>
 __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant__ BwdParams p)
 {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t smem[];
-    uint8_t* sK = smem + C::K_OFF;
-    uint8_t* sV = smem + C::V_OFF;
-    uint8_t* sQS = smem + C::QS_OFF;
-    uint8_t* sDS = smem + C::DS_OFF;
-    uint8_t* sDQ = smem + C::DQ_OFF;
-    float* sVec = reinterpret_cast<float*>(smem + C::VEC_OFF);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
-    uint64_t* kv_full = bars + 0;
-    uint64_t* qdo_full = bars + 1;   // [3]
-    uint64_t* qdo_empty = bars + 4;  // [3]
-    uint64_t* s_full = bars + 7;     // [2]
-    uint64_t* dp_full = bars + 9;
-    uint64_t* p_ready = bars + 10;
-    uint64_t* ds_ready = bars + 11;
-    uint64_t* ds_free = bars + 12;   // [2]
-    uint64_t* dq_full = bars + 14;
-    uint64_t* dq_empty = bars + 15;
-    uint64_t* dkdv_done = bars + 16;
-    uint64_t* drain = bars + 17;
-    uint64_t* dqw_bar = bars + 18;  // the 4 dQ warps (128 threads)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
-
     // the 128-byte-swizzled tiles need a 1024-byte aligned base; the layout
     // leaves no slack, so a misaligned base is reported instead of used
     if ((smem_u32(smem) & 1023u) != 0u) {
         if (threadIdx.x == 0) raise_status(p.ctl, FA_DEV_BAD_TILE);
         return;
     }
+    uint8_t* sK = smem + C::K_OFF;
+    uint8_t* sV = smem + C::V_OFF;
+    uint8_t* sQ = smem + C::Q_OFF;
+    uint8_t* sDO = smem + C::DO_OFF;
+    uint8_t* sDS = smem + C::DS_OFF;
+    uint8_t* sSTG = smem + C::STG_OFF;
+    float* sVec = reinterpret_cast<float*>(smem + C::VEC_OFF);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+    uint64_t* kv_full = bars + 0;
+    uint64_t* q_full = bars + 1;   // [2]
+    uint64_t* q_empty = bars + 3;  // [2]
+    uint64_t* do_full = bars + 5;
+    uint64_t* do_empty = bars + 6;
+    uint64_t* s_full = bars + 7;
+    uint64_t* dp_full = bars + 8;
+    uint64_t* p_ready = bars + 9;
+    uint64_t* ds_ready = bars + 10;
+    uint64_t* dq_full = bars + 11;
+    uint64_t* dq_empty = bars + 12;
+    uint64_t* dkdv_done = bars + 13;
+    uint64_t* drain = bars + 14;
+    uint64_t* dqw_bar = bars + 15;  // the 4 dQ warps (128 threads)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
     // grouped longest-first order over (key tile, head): key tile 0 sees the
@@ -115,35 +174,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
     grouped_order(static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x), p.BH, p.n_kv_tiles, p.group_heads, bh, j);
     const int N = p.N;
     const int n_pad = p.n_kv_tiles * BKV;
-    const int n_q_all = (N + BQ - 1) / BQ;
-    const int i_first = CAUSAL ? (j * BKV) / BQ : 0;
-    const int n_it = n_q_all - i_first;  // >= 1
+    const int n_q = (N + BQ - 1) / BQ;
+    const int i_first = CAUSAL ? j : 0;
+    const int n_it = n_q - i_first;  // >= 1
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
         for (int s = 0; s < QSTAGES; ++s) {
-            mbar_init(&qdo_full[s], 1);
-            mbar_init(&qdo_empty[s], 1);
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
         }
-        mbar_init(&s_full[0], 1);
-        mbar_init(&s_full[1], 1);
+        mbar_init(do_full, 1);
+        mbar_init(do_empty, 1);
+        mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
         mbar_init(p_ready, 128);
         mbar_init(ds_ready, 128);
-        mbar_init(&ds_free[0], 1);
-        mbar_init(&ds_free[1], 1);
         mbar_init(dq_full, 1);
         mbar_init(dq_empty, 128);
         mbar_init(dkdv_done, 1);
         mbar_init(drain, 1);
         mbar_init(dqw_bar, 128);
         fence_mbar_init();
-    }
-    if (D == 64) {
-        // zero block read as rows 64..127 of K^T by the dQ^T MMA
-        uint4* z = reinterpret_cast<uint4*>(sK + C::KBOX);
-        for (int i = threadIdx.x; i < C::KBOX / 16; i += NTHREADS) z[i] = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
     }
     if (warp == MMA_WARP) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -164,115 +216,135 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
     if (warp == LOAD_WARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(kv_full, 2 * C::NDC * C::KBOX);
+            mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
             for (int c = 0; c < C::NDC; ++c) {
-                tma_load_3d(sK + c * C::KBOX, &p.tm_k, kv_full, c * 64, j * BKV, bh);
-                tma_load_3d(sV + c * C::KBOX, &p.tm_v, kv_full, c * 64, j * BKV, bh);
+                tma_load_3d(sK + c * BOX, &p.tm_k, kv_full, c * 64, j * BKV, bh);
+                tma_load_3d(sV + c * BOX, &p.tm_v, kv_full, c * 64, j * BKV, bh);
             }
             const float* lse2_h = p.lse2 + static_cast<size_t>(bh) * n_pad;
             const float* delta_h = p.delta + static_cast<size_t>(bh) * n_pad;
-            int t = 0;
-            for (; t < n_it; ++t) {
-                const int s = t % QSTAGES;
-                if (!mbar_wait(&qdo_empty[s], ((t / QSTAGES) & 1) ^ 1, p.ctl)) break;
+            int nq = 0, ndo = 0;  // tiles issued: Q (with its row vectors), dO
+            bool ok = true;
+            for (int t = 0; t < n_it && ok; ++t) {
+                const int s = t & 1;
                 const int i = i_first + t;
-                mbar_arrive_expect_tx(&qdo_full[s], C::QSTAGE_BYTES + 2 * BQ * 4);
-                uint8_t* st = sQS + s * C::QSTAGE_BYTES;
-                for (int c = 0; c < C::NDC; ++c) {
-                    tma_load_3d(st + c * C::QBOX, &p.tm_q, &qdo_full[s], c * 64, i * BQ, bh);
-                    tma_load_3d(st + (C::NDC + c) * C::QBOX, &p.tm_do, &qdo_full[s], c * 64, i * BQ, bh);
-                }
-                bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &qdo_full[s]);
-                bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &qdo_full[s]);
+                if (!(ok = mbar_wait(&q_empty[s], ((t >> 1) & 1) ^ 1, p.ctl))) break;
+                mbar_arrive_expect_tx(&q_full[s], C::TILE + 2 * BQ * 4);
+                for (int c = 0; c < C::NDC; ++c)
+                    tma_load_3d(sQ + s * C::TILE + c * BOX, &p.tm_q, &q_full[s], c * 64, i * BQ, bh);
+                bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &q_full[s]);
+                bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &q_full[s]);
+                ++nq;
+                if (!(ok = mbar_wait(do_empty, (t & 1) ^ 1, p.ctl))) break;
+                mbar_arrive_expect_tx(do_full, C::TILE);
+                for (int c = 0; c < C::NDC; ++c) tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, bh);
+                ++ndo;
             }
-            if (t < n_it) {
+            if (!ok) {
                 mbar_wait_drain(kv_full, 0, p.ctl.limit_ns);
-                for (int u = max(0, t - QSTAGES); u < t; ++u)
-                    mbar_wait_drain(&qdo_full[u % QSTAGES], (u / QSTAGES) & 1, p.ctl.limit_ns);
+                for (int u = max(0, nq - QSTAGES); u < nq; ++u)
+                    mbar_wait_drain(&q_full[u & 1], (u >> 1) & 1, p.ctl.limit_ns);
+                if (ndo > 0) mbar_wait_drain(do_full, (ndo - 1) & 1, p.ctl.limit_ns);
             }
         }
         __syncwarp();
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
-        // The whole warp runs this loop in step and elect.sync picks the lane
-        // that issues each tcgen05 instruction (from one lane of a diverged warp
-        // the same MMAs measured ~92 cycles each instead of ~65, B200).
-        {
-            constexpr uint32_t idesc_st = idesc_bf16(BKV, BQ, false, false);
-            constexpr uint32_t idesc_dkv = idesc_bf16(BKV, D, false, true);
-            constexpr uint32_t idesc_dq = idesc_bf16(128, BQ, true, true);
-            const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQS = smem_u32(sQS), aDS = smem_u32(sDS);
-            // S^T or dP^T = (K or V) x (Q or dO)^T; both K-major
-            auto issue_sT = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_kk = idesc_bf16(128, 128, false, false);  // S^T, dP^T
+            constexpr uint32_t idesc_tm = idesc_bf16(128, D, false, true);     // dV (A in TMEM), dK
+            constexpr uint32_t idesc_dq = idesc_bf16(128, D, true, true);      // dQ^T (d = 128) / dQ (d = 64)
+            const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
+                           aDS = smem_u32(sDS);
+            auto q_base = [&](int t) { return aQ + (t & 1) * C::TILE; };
+            // (K or V) x (Q or dO)^T, both K-major over the head dimension
+            auto issue_kk = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ka = (kk >> 2) * C::KBOX + (kk & 3) * 32;
-                    const uint32_t kb = (kk >> 2) * C::QBOX + (kk & 3) * 32;
-                    mma_ss_elect(tmem + d_col, sdesc_sw128(a_base + ka, 16, 1024), sdesc_sw128(b_base + kb, 16, 1024),
-                           idesc_st, kk > 0 ? 1u : 0u);
+                    const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
+                    mma_ss(tmem + d_col, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
+                           idesc_kk, kk > 0 ? 1u : 0u);
                 }
             };
-            // dV or dK += (P^T or dS^T from TMEM) x (dO or Q, MN-major)
-            auto issue_dkv = [&](uint32_t d_col, uint32_t a_col, uint32_t b_base, bool acc0) {
+            // dV += P^T (TMEM) x dO (MN-major over d)
+            auto issue_dv = [&](uint32_t a_col, bool acc0) {
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    mma_ts_elect(tmem + d_col, tmem + a_col + kk * 8, sdesc_sw128(b_base + kk * 2048, C::QBOX, 1024),
-                           idesc_dkv, (acc0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + C::DV_COL, tmem + a_col + kk * 8, sdesc_sw128(aDO + kk * 2048, BOX, 1024),
+                           idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
             };
-            // dQ^T = K^T (MN-major) x dS^T (MN-major, software-swizzled)
-            auto issue_dq = [&](uint32_t ds_base) {
+            // dK += dS^T (shared, K-major) x Q (MN-major over d)
+            auto issue_dk = [&](uint32_t b_base, bool acc0) {
 #pragma unroll
-                for (int kk = 0; kk < BKV / 16; ++kk)
-                    mma_ss_elect(tmem + C::DQ_COL, sdesc_sw128(aK + kk * 2048, C::KBOX, 1024),
-                           sdesc_sw128(ds_base + kk * 2048, C::KBOX, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < BQ / 16; ++kk)
+                    mma_ss(tmem + C::DK_COL, sdesc_sw128(aDS + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024),
+                           sdesc_sw128(b_base + kk * 2048, BOX, 1024), idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
             };
-            auto q_base = [&](int t) { return aQS + (t % QSTAGES) * C::QSTAGE_BYTES; };
-            auto do_base = [&](int t) { return aQS + (t % QSTAGES) * C::QSTAGE_BYTES + C::NDC * C::QBOX; };
+            // d = 128: dQ^T = K^T x dS^T into X; d = 64: dQ = dS x K into its own
+            // region.  Both operands MN-major, walking the 128 keys.
+            auto issue_dq = [&](uint32_t d_col) {
+#pragma unroll
+                for (int kk = 0; kk < BKV / 16; ++kk) {
+                    const uint64_t k_desc = sdesc_sw128(aK + kk * 2048, BOX, 1024);
+                    const uint64_t ds_desc = sdesc_sw128(aDS + kk * 2048, BOX, 1024);
+                    if constexpr (D == 128)
+                        mma_ss(tmem + d_col, k_desc, ds_desc, idesc_dq, kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss(tmem + d_col, ds_desc, k_desc, idesc_dq, kk > 0 ? 1u : 0u);
+                }
+            };
 
-            bool ok = warp_wait(kv_full, 0, p.ctl);
-            if (ok) ok = warp_wait(&qdo_full[0], 0, p.ctl);
+            bool ok = mbar_wait(kv_full, 0, p.ctl) && mbar_wait(&q_full[0], 0, p.ctl);
             if (ok) {
                 tc_fence_after();
-                issue_sT(C::S_COL, aK, q_base(0));
-                mma_commit_elect(&s_full[0]);
-                issue_sT(C::DP_COL, aV, do_base(0));
-                mma_commit_elect(dp_full);
-                if (n_it > 1) {
-                    ok = warp_wait(&qdo_full[1], 0, p.ctl);
-                    if (ok) {
-                        tc_fence_after();
-                        issue_sT(C::S_COL + 64, aK, q_base(1));
-                        mma_commit_elect(&s_full[1]);
-                    }
+                issue_kk(rcol(0), aK, q_base(0));
+                mma_commit(s_full);
+                ok = mbar_wait(do_full, 0, p.ctl);
+                if (ok) {
+                    tc_fence_after();
+                    issue_kk(rcol(1), aV, aDO);
+                    mma_commit(dp_full);
                 }
             }
             for (int t = 0; t < n_it && ok; ++t) {
-                const uint32_t sb = C::S_COL + 64 * (t & 1);
-                if (!(ok = warp_wait(p_ready, t & 1, p.ctl))) break;
+                const uint32_t X = rcol(t), Y = rcol(t + 1);
+                if (!(ok = mbar_wait(p_ready, t & 1, p.ctl))) break;
                 tc_fence_after();
-                issue_dkv(C::DV_COL, sb, do_base(t), t > 0);
-                if (!(ok = warp_wait(ds_ready, t & 1, p.ctl))) break;
+                issue_dv(X, t > 0);
+                mma_commit(do_empty);
+                if (!(ok = mbar_wait(ds_ready, t & 1, p.ctl))) break;
                 tc_fence_after();
-                issue_dkv(C::DK_COL, C::DP_COL, q_base(t), t > 0);
-                mma_commit_elect(&qdo_empty[t % QSTAGES]);
                 if (t + 1 < n_it) {
-                    issue_sT(C::DP_COL, aV, do_base(t + 1));
-                    mma_commit_elect(dp_full);
-                }
-                if (t > 0 && !(ok = warp_wait(dq_empty, (t - 1) & 1, p.ctl))) break;
-                tc_fence_after();
-                issue_dq(aDS + (t & 1) * C::DS_BYTES);
-                mma_commit_elect(dq_full);
-                mma_commit_elect(&ds_free[t & 1]);
-                if (t + 2 < n_it) {
-                    if (!(ok = warp_wait(&qdo_full[(t + 2) % QSTAGES], ((t + 2) / QSTAGES) & 1, p.ctl))) break;
+                    // Y held dP^T of tile t, already read by the softmax
+                    if (!(ok = mbar_wait(&q_full[(t + 1) & 1], ((t + 1) >> 1) & 1, p.ctl))) break;
                     tc_fence_after();
-                    issue_sT(sb, aK, q_base(t + 2));
-                    mma_commit_elect(&s_full[t & 1]);
+                    issue_kk(Y, aK, q_base(t + 1));
+                    mma_commit(s_full);
+                }
+                issue_dk(q_base(t), t > 0);
+                mma_commit(&q_empty[t & 1]);
+                if constexpr (D == 128) {
+                    issue_dq(X);
+                } else {
+                    // the dQ warps must have read the previous tile's dQ out
+                    if (t > 0 && !(ok = mbar_wait(dq_empty, (t - 1) & 1, p.ctl))) break;
+                    tc_fence_after();
+                    issue_dq(C::DQ_COL);
+                }
+                mma_commit(dq_full);
+                if (t + 1 < n_it) {
+                    if (!(ok = mbar_wait(do_full, (t + 1) & 1, p.ctl))) break;
+                    if constexpr (D == 128) {
+                        // X holds dQ^T of tile t until the dQ warps have read it
+                        if (!(ok = mbar_wait(dq_empty, t & 1, p.ctl))) break;
+                    }
+                    tc_fence_after();
+                    issue_kk(X, aV, aDO);
+                    mma_commit(dp_full);
                 }
             }
-            if (ok) mma_commit_elect(dkdv_done);
-            mma_commit_elect(drain);
+            if (ok) mma_commit(dkdv_done);
+            mma_commit(drain);
             mbar_wait_drain(drain, 0, p.ctl.limit_ns);
         }
         __syncwarp();
@@ -284,73 +356,152 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
         const float cl2 = p.scale_log2;
         bool ok = true;
         for (int t = 0; t < n_it && ok; ++t) {
+            const int s = t & 1;
             const int i = i_first + t;
-            const int s = t % QSTAGES;
             const float* lse2 = sVec + s * 2 * BQ;
             const float* delta = lse2 + BQ;
-            const uint32_t sb = tmem + lane_off + C::S_COL + 64 * (t & 1);
-            if (!(ok = warp_wait(&s_full[t & 1], (t >> 1) & 1, p.ctl))) break;
-            if (!(ok = warp_wait(&qdo_full[s], (t / QSTAGES) & 1, p.ctl))) break;
+            const uint32_t xa = tmem + lane_off + rcol(t);
+            const uint32_t ya = tmem + lane_off + rcol(t + 1);
+            // keep bits of this key row for the tile's 128 queries (bit c of zq[q4]:
+            // query 32 q4 + c), drawn while S^T is still being computed
+            uint32_t zq[DROPOUT ? 4 : 1];
+            if constexpr (DROPOUT) {
+                const uint64_t key_group = static_cast<uint64_t>(j) * 4 + static_cast<uint64_t>(warp);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    zq[q4] = warp_transpose32(keep_bits(key_group, static_cast<uint64_t>(i * BQ + q4 * 32 + lane),
+                                                        static_cast<uint64_t>(bh), p.keep_t, p.seed, p.offset),
+                                              lane);
+            }
+            if (!(ok = warp_wait(s_full, t & 1, p.ctl))) break;
+            if (!(ok = warp_wait(&q_full[s], (t >> 1) & 1, p.ctl))) break;
             tc_fence_after();
-            float pv[BQ];
-            tmem_ld32(sb, reinterpret_cast<uint32_t*>(pv));
-            tmem_ld32(sb + 32, reinterpret_cast<uint32_t*>(pv + 32));
-            tmem_wait_ld();
+            // causal: query (t-th tile, column c) sees this key iff key <= query; only
+            // the first (diagonal) tile has such pairs.  Keys past N carry no weight.
+            const bool masked = (CAUSAL && t == 0) || (j * BKV + BKV > N);  // CTA-uniform
+            const int lim = (key >= N) ? BQ : ((CAUSAL && t == 0) ? r : 0);   // zero columns c < lim
+            const float2 c2 = make_float2(cl2, cl2);
+            if constexpr (!DROPOUT) {
 #pragma unroll
-            for (int c = 0; c < BQ; c += 4) {
-                const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c);
-                pv[c] = ex2_approx(fmaf(pv[c], cl2, -l4.x));
-                pv[c + 1] = ex2_approx(fmaf(pv[c + 1], cl2, -l4.y));
-                pv[c + 2] = ex2_approx(fmaf(pv[c + 2], cl2, -l4.z));
-                pv[c + 3] = ex2_approx(fmaf(pv[c + 3], cl2, -l4.w));
+                for (int h = 0; h < 2; ++h) {
+                    float pv[64];
+                    tmem_ld32(xa + h * 64, reinterpret_cast<uint32_t*>(pv));
+                    tmem_ld32(xa + h * 64 + 32, reinterpret_cast<uint32_t*>(pv + 32));
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 64; c += 4) {
+                        // x = c s - lse2, two at a time
+                        const float4 l4 = *reinterpret_cast<const float4*>(lse2 + h * 64 + c);
+                        const float2 xa2 = ffma2(make_float2(pv[c], pv[c + 1]), c2, make_float2(-l4.x, -l4.y));
+                        const float2 xb2 = ffma2(make_float2(pv[c + 2], pv[c + 3]), c2, make_float2(-l4.z, -l4.w));
+                        pv[c] = ex2_approx(xa2.x);
+                        pv[c + 1] = ex2_approx(xa2.y);
+                        pv[c + 2] = ex2_approx(xb2.x);
+                        pv[c + 3] = ex2_approx(xb2.y);
+                    }
+                    if (masked) {
+#pragma unroll
+                        for (int c = 0; c < 64; ++c)
+                            if (h * 64 + c < lim) pv[c] = 0.f;
+                    }
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) pk[c / 2] = pack_bf16x2(pv[c], pv[c + 1]);
+                    tmem_st32(xa + h * 32, pk);
+                }
+            } else {
+                // quarters of 32 query columns; bf16(P o Z) packs of quarter q go
+                // to columns 16 q .. 16 q + 15 (S of queries 0-63, already read),
+                // bf16(P) packs to 64 + 16 q once those S columns have been read
+                // (quarters 0, 1 at quarter 2; quarter 2 at quarter 3)
+                uint32_t held[32];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float pv[32];
+                    tmem_ld32(xa + q4 * 32, reinterpret_cast<uint32_t*>(pv));
+                    tmem_wait_ld();
+                    if (q4 == 2) tmem_st32(xa + 64, held);
+                    if (q4 == 3) tmem_st16(xa + 96, held);
+                    const uint32_t z = zq[q4];
+#pragma unroll
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4*>(lse2 + q4 * 32 + c);
+                        const float2 xa2 = ffma2(make_float2(pv[c], pv[c + 1]), c2, make_float2(-l4.x, -l4.y));
+                        const float2 xb2 = ffma2(make_float2(pv[c + 2], pv[c + 3]), c2, make_float2(-l4.z, -l4.w));
+                        pv[c] = ex2_approx(xa2.x);
+                        pv[c + 1] = ex2_approx(xa2.y);
+                        pv[c + 2] = ex2_approx(xb2.x);
+                        pv[c + 3] = ex2_approx(xb2.y);
+                    }
+                    if (masked) {
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (q4 * 32 + c < lim) pv[c] = 0.f;
+                    }
+                    uint32_t pk[16], pu[16];
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        pu[c / 2] = pack_bf16x2(pv[c], pv[c + 1]);
+                        pk[c / 2] = pack_bf16x2(((z >> c) & 1u) ? pv[c] : 0.f, ((z >> (c + 1)) & 1u) ? pv[c + 1] : 0.f);
+                    }
+                    tmem_st16(xa + q4 * 16, pk);
+                    if (q4 < 3) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) held[(q4 & 1) * 16 + e] = pu[e];
+                    } else {
+                        tmem_st16(xa + 112, pu);
+                    }
+                }
             }
-            // causal: query (i*BQ + c) sees this key iff key <= query; keys past N carry no weight
-            if (key >= N) {
-#pragma unroll
-                for (int c = 0; c < BQ; ++c) pv[c] = 0.f;
-            } else if (CAUSAL && i * BQ < (j + 1) * BKV) {
-                const int lim = key - i * BQ;  // mask c < lim
-#pragma unroll
-                for (int c = 0; c < BQ; ++c)
-                    if (c < lim) pv[c] = 0.f;
-            }
-            uint32_t pk[BQ / 2];
-#pragma unroll
-            for (int c = 0; c < BQ; c += 2) pk[c / 2] = pack_bf16x2(pv[c], pv[c + 1]);
-            tmem_st32(sb, pk);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(p_ready);
 
+            // dP^T of this tile was issued after the dK and dQ MMAs of the previous
+            // one, so once it is complete they have read the old dS^T
             if (!(ok = warp_wait(dp_full, t & 1, p.ctl))) break;
             tc_fence_after();
-            float dp[BQ];
-            const uint32_t dpa = tmem + lane_off + C::DP_COL;
-            tmem_ld32(dpa, reinterpret_cast<uint32_t*>(dp));
-            tmem_ld32(dpa + 32, reinterpret_cast<uint32_t*>(dp + 32));
-            tmem_wait_ld();
+            // dS^T = P^T (dP^T - D), with the bf16 P^T read back from TMEM (it stays in
+            // X until this tile's dS^T is written), to shared memory: row r, query
+            // columns in 2 chunks of 64 (128-byte swizzled rows)
 #pragma unroll
-            for (int c = 0; c < BQ; c += 4) {
-                const float4 d4 = *reinterpret_cast<const float4*>(delta + c);
-                pk[c / 2] = pack_bf16x2(pv[c] * (dp[c] - d4.x), pv[c + 1] * (dp[c + 1] - d4.y));
-                pk[c / 2 + 1] = pack_bf16x2(pv[c + 2] * (dp[c + 2] - d4.z), pv[c + 3] * (dp[c + 3] - d4.w));
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float dp[32];
+                uint32_t pq[16];
+                tmem_ld32(ya + q4 * 32, reinterpret_cast<uint32_t*>(dp));
+                tmem_ld16(xa + (DROPOUT ? 64 : 0) + q4 * 16, pq);
+                tmem_wait_ld();
+                if constexpr (DROPOUT) {
+                    // dropped weights contribute no dP: z Z dP
+                    const uint32_t z = zq[q4];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) dp[c] = ((z >> c) & 1u) ? dp[c] * p.keep_scale : 0.f;
+                }
+                uint32_t ds[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(delta + q4 * 32 + c);
+                    const float2 pa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pq[c / 2]));
+                    const float2 pb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pq[c / 2 + 1]));
+                    const float2 ga = fmul2(pa, fadd2(make_float2(dp[c], dp[c + 1]), make_float2(-d4.x, -d4.y)));
+                    const float2 gb = fmul2(pb, fadd2(make_float2(dp[c + 2], dp[c + 3]), make_float2(-d4.z, -d4.w)));
+                    ds[c / 2] = pack_bf16x2(ga.x, ga.y);
+                    ds[c / 2 + 1] = pack_bf16x2(gb.x, gb.y);
+                }
+                uint8_t* chunk = sDS + (q4 >> 1) * BOX;
+#pragma unroll
+                for (int pc = 0; pc < 4; ++pc)
+                    *reinterpret_cast<uint4*>(chunk + sw128_offset(r, (q4 & 1) * 4 + pc)) =
+                        make_uint4(ds[4 * pc], ds[4 * pc + 1], ds[4 * pc + 2], ds[4 * pc + 3]);
             }
-            tmem_st32(dpa, pk);
-            // dS^T row r into the swizzled shared buffer read by the dQ^T MMA
-            if (t >= 2 && !(ok = warp_wait(&ds_free[t & 1], ((t >> 1) + 1) & 1, p.ctl))) break;
-            uint8_t* dsrow = sDS + (t & 1) * C::DS_BYTES;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4*>(dsrow + sw128_offset(r, c)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
             fence_proxy_async_smem();
-            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(ds_ready);
         }
-        // epilogue: dV rows
+        // epilogue: dV rows (times 256 / keep_t under dropout)
         if (ok && warp_wait(dkdv_done, 0, p.ctl)) {
             tc_fence_after();
+            const float f = DROPOUT ? p.keep_scale : 1.f;
             float* dst = p.dv + (static_cast<size_t>(bh) * N + key) * D;
 #pragma unroll
             for (int cc = 0; cc < D; cc += 32) {
@@ -361,19 +512,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
                     float4* d4 = reinterpret_cast<float4*>(dst + cc);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                            __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+                        d4[e] = make_float4(__uint_as_float(v[4 * e]) * f, __uint_as_float(v[4 * e + 1]) * f,
+                                            __uint_as_float(v[4 * e + 2]) * f, __uint_as_float(v[4 * e + 3]) * f);
                 }
             }
         }
     } else {
         // ------------------------------------------------------------ dQ (warps 4-7)
         const int wq = warp - 4;
-        const int dr = wq * 32 + lane;  // row of dQ^T = head-dim index
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-        const bool has_rows = (wq * 32) < D;  // warp-uniform
         const bool issuer = (threadIdx.x == 4 * 32);
-        bool ok = true;
         // thread barrier on an mbarrier with the bounded wait (never bar.sync), so a
         // warp that gives up on a wait cannot strand the others at a barrier
         int bar_uses = 0;
@@ -381,35 +529,71 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             mbar_arrive(dqw_bar);
             return warp_wait(dqw_bar, (bar_uses++) & 1, p.ctl);
         };
+        bool ok = true;
         for (int t = 0; t < n_it && ok; ++t) {
             const int i = i_first + t;
             if (!(ok = warp_wait(dq_full, t & 1, p.ctl))) break;
             tc_fence_after();
-            float q[BQ];
-            if (has_rows) {
+            if constexpr (D == 128) {
+                // thread = head-dim index dr (TMEM lane of dQ^T), 128 query columns;
+                // element (query c, dim dr) of a [64][128] staging tile: 32-column
+                // chunk dr / 32, row c, 16-byte piece (dr % 32) / 4 swizzled with c % 8
+                const int dr = wq * 32 + lane;
+                uint8_t* stg = sSTG + (dr >> 5) * C::STG_CHUNK;
+                const uint32_t piece = (dr & 31) >> 2, word = (dr & 3) * 4;
+                float q[BQ];
+                const uint32_t xa = tmem + lane_off + rcol(t);
+#pragma unroll
+                for (int c = 0; c < BQ; c += 32) tmem_ld32(xa + c, reinterpret_cast<uint32_t*>(q + c));
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(dq_empty);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    // the previous reduce-add must have read the staging tile
+                    if (issuer) bulk_wait_group_read0();
+                    if (!(ok = sync_dq())) break;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        *reinterpret_cast<float*>(stg + c * 128 + ((piece ^ (c & 7)) << 4) + word) =
+                            q[half * 64 + c] * p.scale;
+                    fence_proxy_async_smem();
+                    if (!(ok = sync_dq())) break;
+                    if (issuer) {
+#pragma unroll
+                        for (int ch = 0; ch < D / 32; ++ch)
+                            tma_reduce_add_3d(&p.tm_dq, sSTG + ch * C::STG_CHUNK, ch * 32, i * BQ + half * 64, bh);
+                        bulk_commit_group();
+                    }
+                }
+            } else {
+                // thread = query row qr (TMEM lane of dQ), 64 head-dim columns;
+                // row qr of the [128][64] staging tile: 32-column chunk d / 32,
+                // 16-byte piece (d % 32) / 4 swizzled with qr % 8
+                const int qr = wq * 32 + lane;
+                float q[D];
                 tmem_ld32(tmem + lane_off + C::DQ_COL, reinterpret_cast<uint32_t*>(q));
                 tmem_ld32(tmem + lane_off + C::DQ_COL + 32, reinterpret_cast<uint32_t*>(q + 32));
                 tmem_wait_ld();
-            }
-            tc_fence_before();
-            mbar_arrive(dq_empty);
-            // staging is free once the previous reduce-add has read it
-            if (issuer) bulk_wait_group_read0();
-            if (!(ok = sync_dq())) break;
-            if (has_rows) {
-                // element (query c, dim dr) of a [BQ][D] fp32 tile in 32-column swizzled chunks
-                uint8_t* chunk = sDQ + (dr >> 5) * C::DQ_CHUNK;
-                const uint32_t piece = (dr & 31) >> 2, word = (dr & 3) * 4;
+                tc_fence_before();
+                mbar_arrive(dq_empty);
+                if (issuer) bulk_wait_group_read0();
+                if (!(ok = sync_dq())) break;
 #pragma unroll
-                for (int c = 0; c < BQ; ++c)
-                    *reinterpret_cast<float*>(chunk + c * 128 + ((piece ^ (c & 7)) << 4) + word) = q[c] * p.scale;
-            }
-            fence_proxy_async_smem();
-            if (!(ok = sync_dq())) break;
-            if (issuer) {
-                for (int ch = 0; ch < D / 32; ++ch)
-                    tma_reduce_add_3d(&p.tm_dq, sDQ + ch * C::DQ_CHUNK, ch * 32, i * BQ, bh);
-                bulk_commit_group();
+                for (int d4 = 0; d4 < D / 4; ++d4) {
+                    uint8_t* row = sSTG + (d4 >> 3) * C::STG_CHUNK + qr * 128;
+                    *reinterpret_cast<float4*>(row + (((d4 & 7) ^ (qr & 7)) << 4)) =
+                        make_float4(q[4 * d4] * p.scale, q[4 * d4 + 1] * p.scale, q[4 * d4 + 2] * p.scale,
+                                    q[4 * d4 + 3] * p.scale);
+                }
+                fence_proxy_async_smem();
+                if (!(ok = sync_dq())) break;
+                if (issuer) {
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ++ch)
+                        tma_reduce_add_3d(&p.tm_dq, sSTG + ch * C::STG_CHUNK, ch * 32, i * BQ, bh);
+                    bulk_commit_group();
+                }
             }
         }
         if (issuer) bulk_wait_group0();
@@ -443,24 +627,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
     }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DROPOUT>
 cudaError_t launch(const BwdParams& p, cudaStream_t stream)
 {
-    using C = Cfg<D>;
-    auto kern = bwd_kernel<D, CAUSAL>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    auto kern = bwd_kernel<D, CAUSAL, DROPOUT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_kv_tiles, p.BH);
-    kern<<<grid, NTHREADS, C::SMEM_BYTES, stream>>>(p);
+    kern<<<grid, NTHREADS, Cfg<D>::SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const BwdParams& p, bool causal, bool dropout, cudaStream_t stream)
+{
+    if (dropout) return causal ? launch<D, true, true>(p, stream) : launch<D, false, true>(p, stream);
+    return causal ? launch<D, true, false>(p, stream) : launch<D, false, false>(p, stream);
 }
 
 }  // namespace bwdk
 
-cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, cudaStream_t stream)
+cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, bool dropout, cudaStream_t stream)
 {
-    if (d == 128) return launch_bwd128_sm100(p, causal, stream);
-    return causal ? bwdk::launch<64, true>(p, stream) : bwdk::launch<64, false>(p, stream);
+    return d == 128 ? bwdk::launch_d<128>(p, causal, dropout, stream) : bwdk::launch_d<64>(p, causal, dropout, stream);
 }
+
+int bwd_dq_tile_rows(int d) { return d == 128 ? bwdk::Cfg<128>::STG_ROWS : bwdk::Cfg<64>::STG_ROWS; }
 
 }  // namespace fa

@@ -122,29 +122,6 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, fl
     return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// Philox4x64-10 on (x0, x1, x2, x3) under key (k0, k1), in place: ten rounds
-// of the two 64 x 64 -> 128-bit multiplies with the paper's Philox-4x64
-// multipliers, the key bumped by its Weyl constants between rounds.
-__device__ __forceinline__ void philox4x64_10(uint64_t& x0, uint64_t& x1, uint64_t& x2, uint64_t& x3, uint64_t k0,
-                                              uint64_t k1)
-{
-    constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
-    constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
-#pragma unroll
-    for (int r = 0; r < 10; ++r) {
-        if (r > 0) {
-            k0 += W0;
-            k1 += W1;
-        }
-        const uint64_t hi0 = __umul64hi(M0, x0), lo0 = M0 * x0;
-        const uint64_t hi1 = __umul64hi(M1, x2), lo1 = M1 * x2;
-        x0 = hi1 ^ x1 ^ k0;
-        x1 = lo1;
-        x2 = hi0 ^ x3 ^ k1;
-        x3 = lo0;
-    }
-}
-
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p)
 {
     uintptr_t a = reinterpret_cast<uintptr_t>(p);

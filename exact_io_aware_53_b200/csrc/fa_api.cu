@@ -220,28 +220,29 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
         (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
         (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, o, d, N, BH, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
         return st;
     if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
-    p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     p.BH = static_cast<int>(BH);
     p.N = N;
     p.n_pairs = (N + 255) / 256;
     {
         // persistent grid: one CTA per SM, no more than there are work items;
-        // each launch gets a ticket (its number on this device, never 0) and
-        // the work-queue word ticket % 64
+        // each launch gets a ticket (its number on this device, 16 bits kept)
+        // and the work-queue word ticket % 64
         int dev = 0, n_sm = 0;
         if ((st = cuda_status(cudaGetDevice(&dev))) != FA_OK) return st;
         if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
         if ((st = cuda_status(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev))) != FA_OK) return st;
         const long long items = static_cast<long long>(BH) * p.n_pairs;
-        if (items >= (1ll << 24) - 1) return FA_ERR_UNSUPPORTED;  // the queue counter has 24 bits
+        if (items >= (1ll << 29)) return FA_ERR_UNSUPPORTED;  // the queue counter has 30 bits
         p.n_ctas = static_cast<int>(std::max<long long>(1, std::min<long long>(n_sm, items)));
-        unsigned int t = g_fwd_tickets[dev].fetch_add(1u) + 1u;
-        if (t == 0u) t = g_fwd_tickets[dev].fetch_add(1u) + 1u;
-        p.ticket = t;
+        if (p.n_ctas > 511) return FA_ERR_UNSUPPORTED;  // the queue word counts takers in 9 bits
+        const unsigned int t = g_fwd_tickets[dev].fetch_add(1u);
+        p.ticket = t & 0xFFFFu;
         p.queue_slot = static_cast<int>(t % static_cast<unsigned int>(g_fwd_queue_slots.load()));
     }
     p.group_heads = 1;
@@ -504,13 +505,20 @@ int fa_bwd_prep(const void* o, const float* lse, const void* dO, float* dq, void
     return st;
 }
 
-int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, float* dq, float* dk, float* dv,
-                const void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream)
+}  // extern "C"
+
+namespace {
+
+// The tensor-core backward proper (fa_bwd_main), plain or with dropout.
+int bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, float* dq, float* dk, float* dv,
+                  const void* workspace, int B, int H, int N, int d, float scale, int causal, bool dropout, int keep_t,
+                  unsigned long long seed, unsigned long long offset, void* stream)
 {
     g_last_launches = 0;
     if (!q || !k || !v || !dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
     int st = check_shape(B, H, N, d, scale, causal);
     if (st != FA_OK) return st;
+    if (dropout && (keep_t < 0 || keep_t > 256)) return FA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
         !aligned16(dv) || !aligned16(workspace))
@@ -521,17 +529,17 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, flo
     const size_t vec_bytes = (static_cast<size_t>(BH) * n_pad * sizeof(float) + 255) & ~size_t(255);
     BwdParams p;
     std::memset(&p, 0, sizeof(p));
-    const uint32_t bq = d == 128 ? 128 : 64;  // query rows per backward step
-    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, bq,
+    // 128-row query tiles and 128-key CTAs for both head dimensions
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dO, d, N, BH, 64, bq,
+        (st = encode_3d(&p.tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dO, d, N, BH, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
         (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
         (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq, d, N, BH, 32, 64,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        (st = encode_3d(&p.tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq, d, N, BH, 32,
+                        static_cast<uint32_t>(bwd_dq_tile_rows(d)), CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
         return st;
     if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
     p.delta = static_cast<const float*>(workspace);
@@ -545,18 +553,30 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, flo
     p.group_heads = 1;
     if (causal) {
         // key tile j runs the query tiles from its diagonal on (levels = key tiles)
-        const int n_q = (N + static_cast<int>(bq) - 1) / static_cast<int>(bq);
-        const int per_kv = 128 / static_cast<int>(bq);
         std::vector<double> work(p.n_kv_tiles);
-        for (int j = 0; j < p.n_kv_tiles; ++j) work[j] = static_cast<double>(n_q - j * per_kv) / per_kv;
+        for (int jt = 0; jt < p.n_kv_tiles; ++jt) work[jt] = static_cast<double>(p.n_kv_tiles - jt);
         // Q, dO (bf16) and the fp32 dQ accumulator of a head
         p.group_heads = choose_group_heads(p.BH, p.n_kv_tiles, work.data(), static_cast<size_t>(N) * d * 8);
     }
     p.scale = scale;
     p.scale_log2 = scale * kLog2e;
-    st = cuda_status(launch_bwd_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    p.keep_t = dropout ? keep_t : 256;
+    p.keep_scale = (dropout && keep_t > 0) ? 256.0f / static_cast<float>(keep_t) : (dropout ? 0.0f : 1.0f);
+    p.seed = seed;
+    p.offset = offset;
+    st = cuda_status(launch_bwd_sm100(p, d, causal != 0, dropout, static_cast<cudaStream_t>(stream)));
     if (st == FA_OK) g_last_launches = 1;
     return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, float* dq, float* dk, float* dv,
+                const void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream)
+{
+    return bwd_main_impl(q, k, v, dO, dq, dk, dv, workspace, B, H, N, d, scale, causal, false, 256, 0, 0, stream);
 }
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO, float* dq,
@@ -573,6 +593,32 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
     if ((st = get_encoder()) != FA_OK) return st;
     if ((st = fa_bwd_prep(o, lse, dO, dq, workspace, B, H, N, d, stream)) != FA_OK) return st;
     if ((st = fa_bwd_main(q, k, v, dO, dq, dk, dv, workspace, B, H, N, d, scale, causal, stream)) != FA_OK) {
+        g_last_launches = 1;
+        return st;
+    }
+    g_last_launches = 2;
+    return FA_OK;
+}
+
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   float* dq, float* dk, float* dv, void* workspace, int B, int H, int N, int d, float scale,
+                   int causal, int keep_t, unsigned long long seed, unsigned long long offset, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (keep_t < 0 || keep_t > 256) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dO) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+        return FA_ERR_MISALIGNED;
+    if ((st = get_encoder()) != FA_OK) return st;
+    // D_i = <dO_i, O_i> with the dropped O the forward returned
+    if ((st = fa_bwd_prep(o, lse, dO, dq, workspace, B, H, N, d, stream)) != FA_OK) return st;
+    if ((st = bwd_main_impl(q, k, v, dO, dq, dk, dv, workspace, B, H, N, d, scale, causal, true, keep_t, seed, offset,
+                            stream)) != FA_OK) {
         g_last_launches = 1;
         return st;
     }

@@ -65,31 +65,37 @@ constexpr float LN2 = 0.6931471805599453f;
 // Work queue.  Each CTA's first item is item blockIdx.x (the first gridDim.x
 // items are the longest, so that is what a queue would hand out anyway); the
 // rest come from a counter in one of QUEUE_SLOTS 64-bit words, picked by the
-// launch's ticket (a per-device launch number, never 0).  A word holds
-//   [63:32] ticket of the launch that claimed it  [31:24] claim epoch
-//   [23:0]  next item, or QMARK once every item has been handed out.
-// A word is free when it is zero or its counter is QMARK.  The first CTA of a
-// launch to want a second item claims a free word for its ticket (compare and
-// swap, epoch + 1, counter = gridDim.x + 1: it takes item gridDim.x); the
-// launch's other CTAs see their ticket with a live counter and take items by
-// compare and swap; the CTA that takes the last item writes QMARK, after which
-// no CTA of the launch writes the word again.  While another launch holds the
-// word (a foreign ticket, counter live), a CTA takes its items from the static
-// sequence blockIdx.x + s * gridDim.x instead, so concurrent launches that land
-// on one word (more than QUEUE_SLOTS in flight, or replays of one captured
-// launch on two streams) still process every item, some of them twice with
-// identical results, and never take each other's items.  A free word showing
-// the launch's own ticket is either what an earlier run of the same launch (a
-// graph replay) left, when it equals what the CTA read at its start, or the
-// end of this run's own hand-out, when it does not.  Nothing is ever reset.
+// launch's ticket (a per-device launch number).  A word holds
+//   [63:48] ticket of the launch that claimed it   [47:40] claim epoch
+//   [39]    DONE: every item has been handed out   [38:30] CTAs taking items
+//   [29:0]  counter of the next item
+// and is free when it is zero or DONE with no CTA taking items.  The first CTA
+// of a launch to want a second item claims a free word (compare and swap:
+// ticket, epoch + 1, one taker, counter gridDim.x + 1, taking item gridDim.x);
+// the launch's other CTAs join it (+1 taker, checked afterwards) and then take
+// items by atomic add until the counter passes the last item; the one that
+// draws exactly the item count sets DONE, and each leaves (-1 taker) after its
+// first draw past the end.  While a CTA takes items the word cannot be freed,
+// so no draw lands in another launch's counter.  A CTA that finds the word held
+// by another launch (more than QUEUE_SLOTS launches in flight, or replays of
+// one captured launch on two streams) takes items blockIdx.x + s * gridDim.x
+// instead, so every item is processed, some twice with identical results.  A
+// free word with the launch's own ticket is what an earlier run of the same
+// launch left (a graph replay) when it equals what the CTA read at its start,
+// else the end of this run's own hand-out.  Nothing is ever reset.
 constexpr int QUEUE_SLOTS = 64;
-constexpr unsigned int QMARK = 0xFFFFFFu;
+constexpr unsigned long long Q_COUNT = (1ull << 30) - 1;
+constexpr unsigned long long Q_TAKER = 1ull << 30;
+constexpr unsigned long long Q_TAKERS = 0x1FFull << 30;
+constexpr unsigned long long Q_DONE = 1ull << 39;
 __device__ unsigned long long g_queue[QUEUE_SLOTS];
+
+enum QueueMode { Q_UNDECIDED = 0, Q_TAKING = 1, Q_FIXED = 2, Q_FINISHED = 3 };
 
 struct QueueCursor {
     unsigned long long snap;  // the word as this CTA first read it
-    int next_static;          // next item of the static sequence
-    bool joined;              // taking items from the word's counter
+    int mode;                 // QueueMode
+    int next_fixed;           // next item of the fixed sequence (Q_FIXED)
 };
 
 __device__ __forceinline__ unsigned long long queue_read(const unsigned long long* w)
@@ -99,50 +105,78 @@ __device__ __forceinline__ unsigned long long queue_read(const unsigned long lon
     return v;
 }
 
+__device__ __forceinline__ bool queue_free(unsigned long long w)
+{
+    return w == 0ull || ((w & Q_DONE) != 0ull && (w & Q_TAKERS) == 0ull);
+}
+
+__device__ __forceinline__ void queue_leave(unsigned long long* word) { atomicAdd(word, ~Q_TAKER + 1ull); }
+
 // Next work item of this CTA, or -1 when the launch has none left for it.
+// `ticket` is the launch's 16-bit ticket; total > gridDim.x.
 __device__ int queue_next(unsigned long long* word, unsigned int ticket, int total, QueueCursor& qc,
                           const WaitCtl& ctl)
 {
-    const int P = static_cast<int>(gridDim.x);
-    for (int tries = 0; tries < (1 << 16); ++tries) {
+    const unsigned int P = gridDim.x;
+    for (int tries = 0; qc.mode == Q_UNDECIDED; ++tries) {
+        if (tries == 4096) {  // not reached in practice: each failed step means progress elsewhere
+            raise_status(ctl, FA_DEV_TIMEOUT);
+            qc.mode = Q_FINISHED;
+            break;
+        }
         const unsigned long long w = queue_read(word);
-        const unsigned int own = static_cast<unsigned int>(w >> 32);
-        const unsigned int ep = static_cast<unsigned int>(w >> 24) & 0xFFu;
-        const unsigned int c = static_cast<unsigned int>(w) & 0xFFFFFFu;
-        const bool live = (w != 0ull) && (c != QMARK);
-        unsigned long long want;
-        int item;
-        if (own == ticket && live) {
-            // this run is handing items out: take the next one
-            qc.joined = true;
-            item = static_cast<int>(c);
-            want = (c + 1u >= static_cast<unsigned int>(total)) ? ((w & ~0xFFFFFFull) | QMARK) : w + 1ull;
-        } else if (own == ticket && w != qc.snap) {
-            // this run's hand-out is over (it began after this CTA started)
-            return -1;
-        } else if (qc.joined) {
-            // the hand-out this CTA took part in is over and the word moved on
-            return -1;
-        } else if (!live) {
-            // free: claim it for this run and take item P
-            item = P;
-            const unsigned int c1 = static_cast<unsigned int>(P) + 1u;
-            want = (static_cast<unsigned long long>(ticket) << 32) |
-                   (static_cast<unsigned long long>((ep + 1u) & 0xFFu) << 24) |
-                   (c1 >= static_cast<unsigned int>(total) ? QMARK : c1);
-        } else {
-            // another launch holds the word: static sequence
-            const int it = qc.next_static;
-            qc.next_static += P;
-            return it < total ? it : -1;
+        const bool own = w != 0ull && static_cast<unsigned int>(w >> 48) == ticket;
+        if (queue_free(w)) {
+            if (own && w != qc.snap) {
+                qc.mode = Q_FINISHED;  // this run's own hand-out is over
+                break;
+            }
+            // claim it for this run and take item P
+            const unsigned long long ep = ((w >> 40) + 1ull) & 0xFFull;
+            const unsigned long long want =
+                (static_cast<unsigned long long>(ticket) << 48) | (ep << 40) | Q_TAKER | static_cast<unsigned long long>(P + 1u);
+            if (atomicCAS(word, w, want) != w) continue;
+            qc.mode = Q_TAKING;
+            if (P + 1u >= static_cast<unsigned int>(total)) {
+                // item P is the last one: the hand-out ends with this draw
+                atomicOr(word, Q_DONE);
+                queue_leave(word);
+                qc.mode = Q_FINISHED;
+            }
+            return static_cast<int>(P);
         }
-        if (atomicCAS(word, w, want) == w) {
-            qc.joined = true;
-            return item;
+        if (own) {
+            if ((w & Q_DONE) != 0ull) {
+                qc.mode = Q_FINISHED;  // this run's hand-out is finishing
+                break;
+            }
+            // join; while this CTA counts as a taker the word stays this run's
+            const unsigned long long old = atomicAdd(word, Q_TAKER);
+            if (old != 0ull && static_cast<unsigned int>(old >> 48) == ticket && (old & Q_DONE) == 0ull) {
+                qc.mode = Q_TAKING;
+            } else {
+                queue_leave(word);  // it changed under us: undo and look again
+            }
+            continue;
         }
+        // another launch holds the word: keep to the fixed sequence
+        qc.mode = Q_FIXED;
+        qc.next_fixed = static_cast<int>(blockIdx.x + P);
     }
-    // not reached in practice: each failed swap means another CTA took an item
-    raise_status(ctl, FA_DEV_TIMEOUT);
+    if (qc.mode == Q_TAKING) {
+        const unsigned long long c = atomicAdd(word, 1ull) & Q_COUNT;
+        if (c < static_cast<unsigned long long>(total)) return static_cast<int>(c);
+        if (c == static_cast<unsigned long long>(total)) atomicOr(word, Q_DONE);
+        queue_leave(word);
+        qc.mode = Q_FINISHED;
+        return -1;
+    }
+    if (qc.mode == Q_FIXED) {
+        const int it = qc.next_fixed;
+        qc.next_fixed += static_cast<int>(P);
+        if (it < total) return it;
+        qc.mode = Q_FINISHED;
+    }
     return -1;
 }
 
@@ -154,11 +188,13 @@ struct Cfg {
     static constexpr int STAGES = (D == 128) ? 4 : 8;
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = 2 * TILE_BYTES;
-    static constexpr int BAR_OFF = KV_OFF + STAGES * TILE_BYTES;
+    static constexpr int STG_OFF = KV_OFF + STAGES * TILE_BYTES;  // O staging tile (bf16, as Q's boxes)
+    static constexpr int BAR_OFF = STG_OFF + TILE_BYTES;
     // q_full, q_empty, kv_full/empty[S], s_full, p_full, o_full, o_free [2],
-    // item_full, item_empty [2], drain
-    static constexpr int NBARS = 2 + 2 * STAGES + 4 * 2 + 2 * 2 + 1;
+    // item_full, item_empty [2], drain, stg_full, stg_free
+    static constexpr int NBARS = 2 + 2 * STAGES + 4 * 2 + 2 * 2 + 1 + 2;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;  // + TMEM slot and item ring
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t O_COL = 256;
 };
@@ -225,7 +261,10 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     uint64_t* item_full = o_free + 2;         // [2]
     uint64_t* item_empty = item_full + 2;     // [2]
     uint64_t* drain = item_empty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* stg_full = drain + 1;  // the 256 threads of a Q tile have written O into staging
+    uint64_t* stg_free = drain + 2;  // the TMA store has read the staging tile
+    uint8_t* sSTG = smem + C::STG_OFF;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
     int* item_buf = reinterpret_cast<int*>(tmem_slot + 1);  // [2]
 
     const int warp = static_cast<int>(warp_id());
@@ -250,6 +289,8 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
             mbar_init(&item_empty[t], 1 + 16);  // the MMA warp and the 16 softmax warps
         }
         mbar_init(drain, 1);
+        mbar_init(stg_full, 256);
+        mbar_init(stg_free, 1);
         fence_mbar_init();
     }
     if (warp == MMA_WARP) {
@@ -260,6 +301,7 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
         tma_prefetch_desc(&p.tm_q);
         tma_prefetch_desc(&p.tm_k);
         tma_prefetch_desc(&p.tm_v);
+        tma_prefetch_desc(&p.tm_o);
     }
     tc_fence_before();
     __syncthreads();
@@ -273,8 +315,8 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
             bool ok = true;
             QueueCursor qc;
             qc.snap = queue_read(queue);
-            qc.next_static = static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x);
-            qc.joined = false;
+            qc.mode = Q_UNDECIDED;  // the first access decides
+            qc.next_fixed = 0;
             for (int n = 0; ok; ++n) {
                 const int slot = n & 1;
                 const int item = (n == 0) ? static_cast<int>(blockIdx.x)
@@ -426,6 +468,11 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
         int pc = 0;       // key tiles of this Q tile done over all items (s_full / p_full phases)
         int oc = 0;       // items in which this Q tile was present (o_full phases)
         int ring0 = 0;    // K/V ring slots used by earlier items
+        // O leaves through one staging tile that the two Q tiles take in turn, in
+        // the order their O is complete: tile 0 then tile 1 within an item (tile 0
+        // never has more key tiles), item after item; stg_seq counts the uses
+        // before the current item, in both tile groups alike
+        uint32_t stg_seq = 0;
         bool ok = true;
         for (int n = 0; ok; ++n) {
             const int slot = n & 1;
@@ -561,8 +608,10 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                 ++pc;
             }
             if (ok && nk > 0) {
+                const uint32_t seq = stg_seq + ((t == 1 && w.n_kv[0] > 0) ? 1u : 0u);
                 ok = warp_wait(&o_full[t], oc & 1, p.ctl);
                 ++oc;
+                if (ok) ok = warp_wait(stg_free, (seq & 1) ^ 1, p.ctl);
                 if (ok) {
                     tc_fence_after();
                     // each row's sum is split over its four threads
@@ -571,9 +620,19 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
                     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
                     const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-                    const int row0 = w.q0 + t * BM + rr0, row1 = row0 + 8;
-                    __nv_bfloat16* orow0 = p.o + (static_cast<size_t>(w.bh) * N + row0) * D;
-                    __nv_bfloat16* orow1 = orow0 + 8 * D;
+                    {
+                        // LSE of the warp's 16 rows as one contiguous 64-byte store: lane L
+                        // (< 16) writes row base + L, held by lane 4 (L % 8)
+                        const float lse0 = (m0 + __log2f(l0)) * LN2, lse1 = (m1 + __log2f(l1)) * LN2;
+                        const float a = __shfl_sync(0xffffffffu, lse0, 4 * (lane & 7));
+                        const float b = __shfl_sync(0xffffffffu, lse1, 4 * (lane & 7));
+                        const int lrow = w.q0 + t * BM + base + lane;
+                        if (lane < 16 && lrow < N) p.lse[static_cast<size_t>(w.bh) * N + lrow] = lane < 8 ? a : b;
+                    }
+                    // O / l as bf16 into the staging tile: box col / 64, row rr0 (and
+                    // rr0 + 8), 16-byte chunk (col % 64) / 8 swizzled with the row; a
+                    // warp's 32-bit stores of one column group cover 8 rows x 16 bytes
+                    // in distinct bank groups
     #pragma unroll
                     for (int cc = 0; cc < D; cc += 32) {
                         uint32_t o[16];
@@ -582,27 +641,37 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     #pragma unroll
                         for (int n = 0; n < 4; ++n) {
                             const int col = cc + 8 * n + cg;
-                            if (row0 < N)
-                                *reinterpret_cast<uint32_t*>(orow0 + col) =
-                                    pack_bf16x2(__uint_as_float(o[4 * n]) * inv0, __uint_as_float(o[4 * n + 1]) * inv0);
-                            if (row1 < N)
-                                *reinterpret_cast<uint32_t*>(orow1 + col) = pack_bf16x2(
-                                    __uint_as_float(o[4 * n + 2]) * inv1, __uint_as_float(o[4 * n + 3]) * inv1);
+                            uint8_t* box = sSTG + (col >> 6) * C::BOX_BYTES + (col & 7) * 2;
+                            const uint32_t chunk = static_cast<uint32_t>(col & 63) >> 3;
+                            *reinterpret_cast<uint32_t*>(box + sw128_offset(rr0, chunk)) =
+                                pack_bf16x2(__uint_as_float(o[4 * n]) * inv0, __uint_as_float(o[4 * n + 1]) * inv0);
+                            *reinterpret_cast<uint32_t*>(box + sw128_offset(rr0 + 8, chunk)) =
+                                pack_bf16x2(__uint_as_float(o[4 * n + 2]) * inv1, __uint_as_float(o[4 * n + 3]) * inv1);
                         }
-                    }
-                    if ((lane & 3) == 0) {
-                        if (row0 < N) p.lse[static_cast<size_t>(w.bh) * N + row0] = (m0 + __log2f(l0)) * LN2;
-                        if (row1 < N) p.lse[static_cast<size_t>(w.bh) * N + row1] = (m1 + __log2f(l1)) * LN2;
                     }
                     // O_t has been read: the next item's first P V may overwrite it
                     tc_fence_before();
                     mbar_arrive(&o_free[t]);
+                    fence_proxy_async_smem();
+                    mbar_arrive(stg_full);
+                    if (warp == 8 * t && lane == 0) {
+                        // one TMA tile store per 64-column box; rows past N are clipped
+                        if (mbar_wait(stg_full, seq & 1, p.ctl)) {
+                            for (int c = 0; c < C::NDC; ++c)
+                                tma_store_3d(&p.tm_o, sSTG + c * C::BOX_BYTES, c * 64, w.q0 + t * BM, w.bh);
+                            bulk_commit_group();
+                            bulk_wait_group_read0();
+                        }
+                        mbar_arrive(stg_free);
+                    }
                 }
             }
+            stg_seq += (w.n_kv[0] > 0 ? 1u : 0u) + (w.n_kv[1] > 0 ? 1u : 0u);
             ring0 += 2 * w.n_kv_max;
         }
     }
 
+    if (warp < MMA_WARP && (warp & 7) == 0 && lane == 0) bulk_wait_group0();  // this thread's O stores
     tc_fence_before();
     __syncthreads();
     if (warp == MMA_WARP) {

@@ -22,7 +22,7 @@ struct FwdParams {
     CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle
     CUtensorMap tm_k;
     CUtensorMap tm_v;
-    __nv_bfloat16* o;  // [B*H][N][d]
+    CUtensorMap tm_o;  // the output, same layout; TMA store target
     float* lse;        // [B*H][N]
     int BH;
     int N;
@@ -30,7 +30,7 @@ struct FwdParams {
     int group_heads;   // grouping of the (pair, head) work items, >= 1 (grouped_order)
     int n_ctas;        // persistent CTAs, <= min(SMs, B*H*n_pairs)
     int queue_slot;    // work queue word of this launch, < 64
-    unsigned int ticket;  // launch number on this device (never 0)
+    unsigned int ticket;  // launch number on this device, low 16 bits
     float scale_log2;  // scale * log2(e)
     WaitCtl ctl;
 };
@@ -99,11 +99,11 @@ struct BwdPreParams {
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t stream);
 
 struct BwdParams {
-    CUtensorMap tm_q;    // {d, N, B*H}, box {64, BQ, 1} (BQ = 64 for d = 64, 128 for d = 128)
-    CUtensorMap tm_do;   // {d, N, B*H}, box {64, BQ, 1}
+    CUtensorMap tm_q;    // {d, N, B*H}, box {64, 128, 1}
+    CUtensorMap tm_do;   // {d, N, B*H}, box {64, 128, 1}
     CUtensorMap tm_k;    // {d, N, B*H}, box {64, 128, 1}
     CUtensorMap tm_v;    // {d, N, B*H}, box {64, 128, 1}
-    CUtensorMap tm_dq;   // fp32 {d, N, B*H}, box {32, 64, 1}, 128-byte swizzle, reduce-add target
+    CUtensorMap tm_dq;   // fp32 {d, N, B*H}, box {32, bwd_dq_tile_rows(d), 1}, 128-byte swizzle, reduce-add target
     const float* lse2;   // [B*H][n_kv_tiles * 128]; +inf past N
     const float* delta;  // [B*H][n_kv_tiles * 128]; 0 past N
     float* dq;           // [B*H][N][d], accumulated into (zeroed by the pre-pass)
@@ -115,10 +115,16 @@ struct BwdParams {
     int group_heads;  // dispatch grouping of the (key tile, head) grid, >= 1 (grouped_order)
     float scale;
     float scale_log2;
+    // dropout (the launch's dropout flag): keep iff the element's random byte < keep_t
+    int keep_t;
+    float keep_scale;  // 256 / keep_t (0 when keep_t = 0)
+    uint64_t seed;     // Philox key (seed, offset)
+    uint64_t offset;
     WaitCtl ctl;
 };
-cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, cudaStream_t stream);
-cudaError_t launch_bwd128_sm100(const BwdParams& p, bool causal, cudaStream_t stream);
+cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, bool dropout, cudaStream_t stream);
+// Query rows of the fp32 dQ tile the backward reduce-adds (box height of tm_dq).
+int bwd_dq_tile_rows(int d);
 
 // ---------------------------------------------------------------- fp32 path
 struct F32Params {

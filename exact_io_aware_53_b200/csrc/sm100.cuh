@@ -528,6 +528,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Philox4x64-10 on (x0, x1, x2, x3) under key (k0, k1), in place: ten rounds
+// of the two 64 x 64 -> 128-bit multiplies with the paper's Philox-4x64
+// multipliers, the key bumped by its Weyl constants between rounds.
+__device__ __forceinline__ void philox4x64_10(uint64_t& x0, uint64_t& x1, uint64_t& x2, uint64_t& x3, uint64_t k0,
+                                              uint64_t k1)
+{
+    constexpr uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    constexpr uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += W0;
+            k1 += W1;
+        }
+        const uint64_t hi0 = __umul64hi(M0, x0), lo0 = M0 * x0;
+        const uint64_t hi1 = __umul64hi(M1, x2), lo1 = M1 * x2;
+        x0 = hi1 ^ x1 ^ k0;
+        x1 = lo1;
+        x2 = hi0 ^ x3 ^ k1;
+        x3 = lo0;
+    }
+}
+
 // Byte offset of 16-byte chunk `c` (0..7) of row `r` inside a 128-byte-swizzled
 // tile whose rows are 128 bytes (tile base 1024-byte aligned).
 __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c)

@@ -48,6 +48,8 @@ _SIGS = {
                    I),
     "fa_fwd_dropout": ([P, P, P, P, P, I, I, I, I, ctypes.c_float, I, I, ctypes.c_ulonglong, ctypes.c_ulonglong, P],
                        I),
+    "fa_bwd_dropout": ([P, P, P, P, P, P, P, P, P, P, I, I, I, I, ctypes.c_float, I, I, ctypes.c_ulonglong,
+                        ctypes.c_ulonglong, P], I),
     "fa_status_string": ([I], ctypes.c_char_p),
     "fa_last_launch_count": ([], I),
     "fa_last_cuda_error": ([], I),
@@ -228,6 +230,31 @@ def fwd_dropout(q, k, v, keep_t: int, seed: int, offset: int = 0, causal: bool =
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     _check(fwd_dropout_raw(q, k, v, o, lse, scale, causal, keep_t, seed, offset, stream), "fa_fwd_dropout")
     return o, lse
+
+
+def bwd_dropout_raw(q, k, v, o, lse, do, dq, dk, dv, ws, scale: float, causal: bool, keep_t: int, seed: int,
+                    offset: int = 0, stream=None) -> int:
+    """Enqueue the dropout backward on preallocated tensors (ws: bwd_workspace_bytes)."""
+    B, H, N, d = _shape(q)
+    return _lib.fa_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                               _ptr(dv), _ptr(ws), B, H, N, d, float(scale), int(bool(causal)), int(keep_t),
+                               int(seed), int(offset), _stream(stream))
+
+
+def bwd_dropout(q, k, v, o, lse, do, keep_t: int, seed: int, offset: int = 0, causal: bool = False,
+                scale: float | None = None, stream=None):
+    """dQ, dK, dV (fp32) of L = sum(O * dO) for fwd_dropout's O with the same
+    keep_t, seed and offset; the keep mask is regenerated, not stored."""
+    _same(q, k, v, o, do, dtype=torch.bfloat16)
+    B, H, N, d = _shape(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dk = torch.empty_like(dq)
+    dv = torch.empty_like(dq)
+    ws = torch.empty(max(1, bwd_workspace_bytes(B, H, N, d)), dtype=torch.uint8, device=q.device)
+    _check(bwd_dropout_raw(q, k, v, o, lse, do, dq, dk, dv, ws, scale, causal, keep_t, seed, offset, stream),
+           "fa_bwd_dropout")
+    return dq, dk, dv
 
 
 def fwd_fp8_raw(q, k, v, o, lse, descales, scale: float, causal: bool, stream=None) -> int:

@@ -61,7 +61,7 @@ typedef enum {
  * its items in a fixed order instead.  So launches may run concurrently on any
  * number of streams, and a captured launch may be replayed, with every output
  * element written by this launch's own arithmetic (at worst some items twice,
- * with identical results).  FA_ERR_UNSUPPORTED if B*H*ceil(N/256) >= 2^24-1.
+ * with identical results).
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, void* stream);
@@ -244,6 +244,23 @@ int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, flo
 int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
                    float scale, int causal, int keep_t, unsigned long long seed, unsigned long long offset,
                    void* stream);
+
+/*
+ * Backward of fa_fwd_dropout: gradients of L = sum(O * dO) for
+ *   O_i = (256 / keep_t) * sum_j P_ij Z_ij v_j
+ * with the same keep mask Z, regenerated from (seed, offset) and each
+ * element's position by the contract of fa_fwd_dropout (the forward stores no
+ * mask).  With z = 256 / keep_t:  dV = z (P o Z)^T dO,
+ * dS = P o (z Z o dP - D) with dP = dO V^T and D_i = <dO_i, O_i>,
+ * dQ = scale dS K, dK = scale dS^T Q.  Arguments as fa_bwd (o, lse: what
+ * fa_fwd_dropout returned for the same q, k, v, keep_t, seed, offset) plus
+ * keep_t, seed, offset.  Two kernels are enqueued on `stream`; nothing is
+ * allocated.  Errors as for fa_bwd, plus FA_ERR_INVALID_ARG for keep_t
+ * outside [0, 256] and FA_ERR_UNSUPPORTED for B*H > 65535.
+ */
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                   float* dq, float* dk, float* dv, void* workspace, int B, int H, int N, int d, float scale,
+                   int causal, int keep_t, unsigned long long seed, unsigned long long offset, void* stream);
 
 /*
  * FP8 forward: q, k, v in e4m3 (OCP FP8, 1-4-3, no infinities) with one

@@ -230,3 +230,41 @@ def test_blocksparse_mask_layout_accepts_dense_device_masks(lib):
         lib._check_mask(DeviceView(torch.ones((T, T), dtype=torch.uint8)), 3, 640, dev)    # T = 5
     with pytest.raises(ValueError):  # on another GPU than q
         lib._check_mask(DeviceView(torch.ones((T, T), dtype=torch.uint8), index=1), 3, 512, dev)
+
+
+def test_dropout_backward_argument_errors(lib):
+    f = lib._lib.fa_bwd_dropout
+    P = ctypes.c_void_p
+
+    def call(B=1, H=1, N=256, d=128, scale=0.1, causal=0, t=230, q=P(16), ws=P(16)):
+        return f(q, P(16), P(16), P(16), P(16), P(16), P(16), P(16), P(16), ws, B, H, N, d, scale, causal, t, 1, 0,
+                 P(0))
+
+    assert call(q=P(0)) == lib.FA_ERR_INVALID_ARG
+    assert call(ws=P(0)) == lib.FA_ERR_INVALID_ARG
+    assert call(t=-1) == lib.FA_ERR_INVALID_ARG
+    assert call(t=257) == lib.FA_ERR_INVALID_ARG
+    assert call(N=0) == lib.FA_ERR_INVALID_ARG
+    assert call(scale=0.0) == lib.FA_ERR_INVALID_ARG
+    assert call(d=96) == lib.FA_ERR_UNSUPPORTED
+    assert call(B=300, H=300) == lib.FA_ERR_UNSUPPORTED   # more than 65535 heads
+    assert call(q=P(4)) == lib.FA_ERR_MISALIGNED
+    assert lib.last_launch_count() == 0
+
+
+def test_fp32_backward_block_size_is_checked(lib):
+    f = lib._lib.fa_bwd_f32
+    P = ctypes.c_void_p
+
+    def call(block_k):
+        return f(P(16), P(16), P(16), P(16), P(16), P(16), P(16), P(16), P(16), P(16), 1, 1, 64, 64, 0.1, 0, block_k,
+                 P(0))
+
+    assert call(-1) == lib.FA_ERR_INVALID_ARG
+    assert call(1025) == lib.FA_ERR_INVALID_ARG
+
+
+def test_forward_queue_word_count_is_checked(lib):
+    f = lib._lib.fa_set_fwd_queue_words
+    assert f(0) == lib.FA_ERR_INVALID_ARG and f(65) == lib.FA_ERR_INVALID_ARG
+    assert f(64) == lib.FA_OK
