@@ -1126,7 +1126,12 @@ def main(argv=None):
     ap.add_argument("--n-split", type=int, default=0, help="key ranges for the decode workloads (0: library choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bwd-softmax-warps", type=int, default=0, choices=[0, 4, 8],
+                    help="softmax warps per backward CTA (0: the library's choice)")
     args = ap.parse_args(argv)
+    if args.bwd_softmax_warps and args.impl == "ours":
+        from exact_io_aware_53_b200 import fa
+        fa._lib.fa_set_bwd_softmax_warps(args.bwd_softmax_warps)
     from exact_io_aware_53_b200.workloads import (BLOCKSPARSE_WORKLOADS, DECODE_WORKLOADS, DROPOUT_WORKLOADS,
                                                   FP8_WORKLOADS, WORKLOADS)
     known = (list(WORKLOADS) + list(DECODE_WORKLOADS) + list(BLOCKSPARSE_WORKLOADS) + list(FP8_WORKLOADS) +

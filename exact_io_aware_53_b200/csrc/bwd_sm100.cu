@@ -15,8 +15,10 @@
 //
 // TMEM (512 columns): two 128-column regions R0, R1, then dV and dK (d columns
 // each) and, for d = 64, dQ (64 columns).  Tile t uses X = R[t & 1] for
-// S^T -> P^T (bf16 pairs in its first 64 columns) and Y = R[(t + 1) & 1] for
-// dP^T.  dS^T goes to shared memory only, where it is the K-major A operand
+// S^T -> P^T and Y = R[(t + 1) & 1] for dP^T.  P^T of query half h (queries
+// 64 h .. 64 h + 63) goes, as bf16 pairs, to columns 64 h .. 64 h + 31 of X,
+// inside the S^T columns that half has just read, so the two halves never
+// write where the other still has to read.  dS^T goes to shared memory only, where it is the K-major A operand
 // of dK and the MN-major operand of the dQ product; so Y is free once the
 // softmax has read dP^T, and S^T of tile t + 1 is issued there before dK and
 // dQ of tile t, overlapping the next softmax with them.  dP^T of tile t + 1
@@ -37,17 +39,21 @@
 // A warp's 32 key rows are one 32-key group of the generator, so each lane
 // draws the block of one query (32 bytes: the keep bytes of all 32 keys for
 // that query) and a 32 x 32 bit transpose across the warp hands every lane its
-// own key's bits: four blocks per thread per tile, as in the forward.  X then
-// holds bf16(P o Z) in columns 0-63 (the dV operand; the factor z is applied
-// to dV at the end) and bf16(P) in columns 64-127 for dS.
+// own key's bits: four blocks per key row per tile, as in the forward.  Half
+// h of X then holds bf16(P o Z) in columns 64 h .. 64 h + 31 (the dV operand;
+// the factor z is applied to dV at the end) and bf16(P) in 64 h + 32 .. 64 h
+// + 63 for dS.
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax: thread = key row = TMEM lane
-//   warps 4-7  dQ: read dQ (or dQ^T) out of TMEM, scale, stage, reduce-add
-//   warp 8     MMA issuer (one thread)
-//   warp 9     TMA producer: K, V once; {Q_t, lse2_t, D_t} in a 2-stage ring,
-//              dO_t in one buffer (its last reader, dV, runs early in a tile
-//              and its next reader, dP^T, late in the previous one)
+// Warp roles (SMW softmax warps, 4 or 8):
+//   warps 0 .. SMW-1   softmax: thread = key row = TMEM lane of quadrant w % 4;
+//                      with 8 warps, warp w takes query half w / 4 (two warps
+//                      per SM sub-partition overlap their exponentials with
+//                      the other's FMA-pipe work), with 4 both halves
+//   next 4 warps       dQ: read dQ (or dQ^T) out of TMEM, scale, stage, reduce-add
+//   next warp          MMA issuer (one thread)
+//   last warp          TMA producer: K, V once; {Q_t, lse2_t, D_t} in a 2-stage
+//                      ring, dO_t in one buffer (its last reader, dV, runs early
+//                      in a tile and its next reader, dP^T, late in the previous one)
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -56,10 +62,18 @@ namespace bwdk {
 
 constexpr int BKV = 128;
 constexpr int BQ = 128;
-constexpr int NTHREADS = 320;
-constexpr int MMA_WARP = 8;
-constexpr int LOAD_WARP = 9;
 constexpr int QSTAGES = 2;
+
+// Warp layout for SMW softmax warps.  14 warps put four on two of the SM's
+// sub-partitions, whose 16K registers then allow 128 per thread.
+template <int SMW>
+struct Roles {
+    static constexpr int DQ_WARP0 = SMW;
+    static constexpr int MMA_WARP = SMW + 4;
+    static constexpr int LOAD_WARP = SMW + 5;
+    static constexpr int NTHREADS = 32 * (SMW + 6);
+    static constexpr int MAX_REGS = SMW == 8 ? 128 : 168;
+};
 constexpr int BOX = 128 * 128;  // 128 rows x 128 B (64 bf16)
 
 template <int D>
@@ -113,8 +127,8 @@ __device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane)
 
 // Keep bits of one query row for the 32 keys of one generator block: bit b is
 // set iff byte b of Philox4x64-10 at (key_group, query, bh, 0) is below keep_t.
-__device__ __noinline__ uint32_t keep_bits(uint64_t key_group, uint64_t query, uint64_t bh, int keep_t,
-                                         uint64_t seed, uint64_t offset)
+__device__ __forceinline__ uint32_t keep_bits(uint64_t key_group, uint64_t query, uint64_t bh, int keep_t,
+                                             uint64_t seed, uint64_t offset)
 {
     if (keep_t >= 256) return 0xFFFFFFFFu;
     uint64_t x0 = key_group, x1 = query, x2 = bh, x3 = 0;
@@ -131,10 +145,15 @@ __device__ __noinline__ uint32_t keep_bits(uint64_t key_group, uint64_t query, u
     return m;
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
-__global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant__ BwdParams p)
+template <int D, bool CAUSAL, bool DROPOUT, int SMW>
+__global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW>::MAX_REGS)
+    bwd_kernel(const __grid_constant__ BwdParams p)
 {
     using C = Cfg<D>;
+    using R = Roles<SMW>;
+    constexpr int MMA_WARP = R::MMA_WARP;
+    constexpr int LOAD_WARP = R::LOAD_WARP;
+    constexpr int HALVES = SMW == 8 ? 1 : 2;  // query halves per softmax warp
     extern __shared__ __align__(1024) uint8_t smem[];
     // the 128-byte-swizzled tiles need a 1024-byte aligned base; the layout
     // leaves no slack, so a misaligned base is reported instead of used
@@ -188,8 +207,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
         mbar_init(do_empty, 1);
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(p_ready, 128);
-        mbar_init(ds_ready, 128);
+        mbar_init(p_ready, 32 * SMW);
+        mbar_init(ds_ready, 32 * SMW);
         mbar_init(dq_full, 1);
         mbar_init(dq_empty, 128);
         mbar_init(dkdv_done, 1);
@@ -266,12 +285,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
                            idesc_kk, kk > 0 ? 1u : 0u);
                 }
             };
-            // dV += P^T (TMEM) x dO (MN-major over d)
+            // dV += P^T (TMEM: queries 16 kk .. 16 kk + 15 in half kk / 4) x dO (MN-major over d)
             auto issue_dv = [&](uint32_t a_col, bool acc0) {
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    mma_ts(tmem + C::DV_COL, tmem + a_col + kk * 8, sdesc_sw128(aDO + kk * 2048, BOX, 1024),
-                           idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
+                    mma_ts(tmem + C::DV_COL, tmem + a_col + (kk >> 2) * 64 + (kk & 3) * 8,
+                           sdesc_sw128(aDO + kk * 2048, BOX, 1024), idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
             };
             // dK += dS^T (shared, K-major) x Q (MN-major over d)
             auto issue_dk = [&](uint32_t b_base, bool acc0) {
@@ -348,11 +367,13 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             mbar_wait_drain(drain, 0, p.ctl.limit_ns);
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else if (warp < SMW) {
         // ------------------------------------------------------------ softmax (key rows)
-        const int r = warp * 32 + lane;
+        const int quad = warp & 3;
+        const int h0 = (SMW == 8) ? (warp >> 2) : 0;  // first query half of this warp
+        const int r = quad * 32 + lane;
         const int key = j * BKV + r;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const float cl2 = p.scale_log2;
         bool ok = true;
         for (int t = 0; t < n_it && ok; ++t) {
@@ -362,16 +383,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             const float* delta = lse2 + BQ;
             const uint32_t xa = tmem + lane_off + rcol(t);
             const uint32_t ya = tmem + lane_off + rcol(t + 1);
-            // keep bits of this key row for the tile's 128 queries (bit c of zq[q4]:
-            // query 32 q4 + c), drawn while S^T is still being computed
-            uint32_t zq[DROPOUT ? 4 : 1];
+            // keep bits of this key row for the warp's query quarters (bit c of
+            // zq[q]: query 32 (2 h0 + q) + c), drawn while S^T is being computed
+            uint32_t zq[DROPOUT ? 2 * HALVES : 1];
             if constexpr (DROPOUT) {
-                const uint64_t key_group = static_cast<uint64_t>(j) * 4 + static_cast<uint64_t>(warp);
+                const uint64_t key_group = static_cast<uint64_t>(j) * 4 + static_cast<uint64_t>(quad);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    zq[q4] = warp_transpose32(keep_bits(key_group, static_cast<uint64_t>(i * BQ + q4 * 32 + lane),
-                                                        static_cast<uint64_t>(bh), p.keep_t, p.seed, p.offset),
-                                              lane);
+                for (int q = 0; q < 2 * HALVES; ++q)
+                    zq[q] = warp_transpose32(
+                        keep_bits(key_group, static_cast<uint64_t>(i * BQ + (2 * h0 + q) * 32 + lane),
+                                  static_cast<uint64_t>(bh), p.keep_t, p.seed, p.offset),
+                        lane);
             }
             if (!(ok = warp_wait(s_full, t & 1, p.ctl))) break;
             if (!(ok = warp_wait(&q_full[s], (t >> 1) & 1, p.ctl))) break;
@@ -381,76 +403,48 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             const bool masked = (CAUSAL && t == 0) || (j * BKV + BKV > N);  // CTA-uniform
             const int lim = (key >= N) ? BQ : ((CAUSAL && t == 0) ? r : 0);   // zero columns c < lim
             const float2 c2 = make_float2(cl2, cl2);
-            if constexpr (!DROPOUT) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    float pv[64];
-                    tmem_ld32(xa + h * 64, reinterpret_cast<uint32_t*>(pv));
-                    tmem_ld32(xa + h * 64 + 32, reinterpret_cast<uint32_t*>(pv + 32));
-                    tmem_wait_ld();
+            for (int hh = 0; hh < HALVES; ++hh) {
+                const int h = h0 + hh;
+                float pv[64];
+                tmem_ld32(xa + h * 64, reinterpret_cast<uint32_t*>(pv));
+                tmem_ld32(xa + h * 64 + 32, reinterpret_cast<uint32_t*>(pv + 32));
+                tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 64; c += 4) {
-                        // x = c s - lse2, two at a time
-                        const float4 l4 = *reinterpret_cast<const float4*>(lse2 + h * 64 + c);
-                        const float2 xa2 = ffma2(make_float2(pv[c], pv[c + 1]), c2, make_float2(-l4.x, -l4.y));
-                        const float2 xb2 = ffma2(make_float2(pv[c + 2], pv[c + 3]), c2, make_float2(-l4.z, -l4.w));
-                        pv[c] = ex2_approx(xa2.x);
-                        pv[c + 1] = ex2_approx(xa2.y);
-                        pv[c + 2] = ex2_approx(xb2.x);
-                        pv[c + 3] = ex2_approx(xb2.y);
-                    }
-                    if (masked) {
+                for (int c = 0; c < 64; c += 4) {
+                    // x = c s - lse2, two at a time
+                    const float4 l4 = *reinterpret_cast<const float4*>(lse2 + h * 64 + c);
+                    const float2 xa2 = ffma2(make_float2(pv[c], pv[c + 1]), c2, make_float2(-l4.x, -l4.y));
+                    const float2 xb2 = ffma2(make_float2(pv[c + 2], pv[c + 3]), c2, make_float2(-l4.z, -l4.w));
+                    pv[c] = ex2_approx(xa2.x);
+                    pv[c + 1] = ex2_approx(xa2.y);
+                    pv[c + 2] = ex2_approx(xb2.x);
+                    pv[c + 3] = ex2_approx(xb2.y);
+                }
+                if (masked) {
 #pragma unroll
-                        for (int c = 0; c < 64; ++c)
-                            if (h * 64 + c < lim) pv[c] = 0.f;
-                    }
-                    uint32_t pk[32];
+                    for (int c = 0; c < 64; ++c)
+                        if (h * 64 + c < lim) pv[c] = 0.f;
+                }
+                // bf16 pairs into this half's own S^T columns (already read)
+                uint32_t pk[32];
+                if constexpr (!DROPOUT) {
 #pragma unroll
                     for (int c = 0; c < 64; c += 2) pk[c / 2] = pack_bf16x2(pv[c], pv[c + 1]);
-                    tmem_st32(xa + h * 32, pk);
-                }
-            } else {
-                // quarters of 32 query columns; bf16(P o Z) packs of quarter q go
-                // to columns 16 q .. 16 q + 15 (S of queries 0-63, already read),
-                // bf16(P) packs to 64 + 16 q once those S columns have been read
-                // (quarters 0, 1 at quarter 2; quarter 2 at quarter 3)
-                uint32_t held[32];
+                    tmem_st32(xa + h * 64, pk);
+                } else {
+                    // bf16(P) for dS, then bf16(P o Z) for dV: the same pairs with the
+                    // dropped halves cleared (so pv is dead before the second store)
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    float pv[32];
-                    tmem_ld32(xa + q4 * 32, reinterpret_cast<uint32_t*>(pv));
-                    tmem_wait_ld();
-                    if (q4 == 2) tmem_st32(xa + 64, held);
-                    if (q4 == 3) tmem_st16(xa + 96, held);
-                    const uint32_t z = zq[q4];
+                    for (int c = 0; c < 64; c += 2) pk[c / 2] = pack_bf16x2(pv[c], pv[c + 1]);
+                    tmem_st32(xa + h * 64 + 32, pk);
+                    uint32_t pz[32];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4) {
-                        const float4 l4 = *reinterpret_cast<const float4*>(lse2 + q4 * 32 + c);
-                        const float2 xa2 = ffma2(make_float2(pv[c], pv[c + 1]), c2, make_float2(-l4.x, -l4.y));
-                        const float2 xb2 = ffma2(make_float2(pv[c + 2], pv[c + 3]), c2, make_float2(-l4.z, -l4.w));
-                        pv[c] = ex2_approx(xa2.x);
-                        pv[c + 1] = ex2_approx(xa2.y);
-                        pv[c + 2] = ex2_approx(xb2.x);
-                        pv[c + 3] = ex2_approx(xb2.y);
+                    for (int c = 0; c < 64; c += 2) {
+                        const uint32_t z = zq[2 * hh + (c >> 5)] >> (c & 31);
+                        pz[c / 2] = pk[c / 2] & ((z & 1u) * 0x0000FFFFu | ((z >> 1) & 1u) * 0xFFFF0000u);
                     }
-                    if (masked) {
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            if (q4 * 32 + c < lim) pv[c] = 0.f;
-                    }
-                    uint32_t pk[16], pu[16];
-#pragma unroll
-                    for (int c = 0; c < 32; c += 2) {
-                        pu[c / 2] = pack_bf16x2(pv[c], pv[c + 1]);
-                        pk[c / 2] = pack_bf16x2(((z >> c) & 1u) ? pv[c] : 0.f, ((z >> (c + 1)) & 1u) ? pv[c + 1] : 0.f);
-                    }
-                    tmem_st16(xa + q4 * 16, pk);
-                    if (q4 < 3) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) held[(q4 & 1) * 16 + e] = pu[e];
-                    } else {
-                        tmem_st16(xa + 112, pu);
-                    }
+                    tmem_st32(xa + h * 64, pz);
                 }
             }
             tmem_wait_st();
@@ -463,17 +457,19 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             tc_fence_after();
             // dS^T = P^T (dP^T - D), with the bf16 P^T read back from TMEM (it stays in
             // X until this tile's dS^T is written), to shared memory: row r, query
-            // columns in 2 chunks of 64 (128-byte swizzled rows)
+            // columns in 2 chunks of 64 (128-byte swizzled rows), chunk = half
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int qq = 0; qq < 2 * HALVES; ++qq) {
+                const int q4 = 2 * h0 + qq;  // query quarter
+                const int h = q4 >> 1;
                 float dp[32];
                 uint32_t pq[16];
                 tmem_ld32(ya + q4 * 32, reinterpret_cast<uint32_t*>(dp));
-                tmem_ld16(xa + (DROPOUT ? 64 : 0) + q4 * 16, pq);
+                tmem_ld16(xa + h * 64 + (DROPOUT ? 32 : 0) + (q4 & 1) * 16, pq);
                 tmem_wait_ld();
                 if constexpr (DROPOUT) {
                     // dropped weights contribute no dP: z Z dP
-                    const uint32_t z = zq[q4];
+                    const uint32_t z = zq[qq];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) dp[c] = ((z >> c) & 1u) ? dp[c] * p.keep_scale : 0.f;
                 }
@@ -488,7 +484,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
                     ds[c / 2] = pack_bf16x2(ga.x, ga.y);
                     ds[c / 2 + 1] = pack_bf16x2(gb.x, gb.y);
                 }
-                uint8_t* chunk = sDS + (q4 >> 1) * BOX;
+                uint8_t* chunk = sDS + h * BOX;
 #pragma unroll
                 for (int pc = 0; pc < 4; ++pc)
                     *reinterpret_cast<uint4*>(chunk + sw128_offset(r, (q4 & 1) * 4 + pc)) =
@@ -498,13 +494,15 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             tc_fence_before();
             mbar_arrive(ds_ready);
         }
-        // epilogue: dV rows (times 256 / keep_t under dropout)
+        // epilogue: dV rows (times 256 / keep_t under dropout); with 8 warps the two
+        // warps of a quadrant take half the columns each
         if (ok && warp_wait(dkdv_done, 0, p.ctl)) {
             tc_fence_after();
             const float f = DROPOUT ? p.keep_scale : 1.f;
             float* dst = p.dv + (static_cast<size_t>(bh) * N + key) * D;
+            constexpr int COLS = D / (SMW / 4);
 #pragma unroll
-            for (int cc = 0; cc < D; cc += 32) {
+            for (int cc = h0 * COLS; cc < h0 * COLS + COLS; cc += 32) {
                 uint32_t v[32];
                 tmem_ld32(tmem + lane_off + C::DV_COL + cc, v);
                 tmem_wait_ld();
@@ -518,10 +516,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
             }
         }
     } else {
-        // ------------------------------------------------------------ dQ (warps 4-7)
-        const int wq = warp - 4;
+        // ------------------------------------------------------------ dQ (4 warps)
+        const int wq = warp - R::DQ_WARP0;  // TMEM quadrant wq (warp % 4 == wq)
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-        const bool issuer = (threadIdx.x == 4 * 32);
+        const bool issuer = (threadIdx.x == R::DQ_WARP0 * 32);
         // thread barrier on an mbarrier with the bounded wait (never bar.sync), so a
         // warp that gives up on a wait cannot strand the others at a barrier
         int bar_uses = 0;
@@ -541,22 +539,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
                 const int dr = wq * 32 + lane;
                 uint8_t* stg = sSTG + (dr >> 5) * C::STG_CHUNK;
                 const uint32_t piece = (dr & 31) >> 2, word = (dr & 3) * 4;
-                float q[BQ];
                 const uint32_t xa = tmem + lane_off + rcol(t);
+                // with 4 softmax warps both halves of dQ^T are read before X is released;
+                // with 8 (128 registers) half 0 is staged first and X released after half 1
+                constexpr int LOADS = (SMW == 8) ? 1 : 2;
+                float q[64 * LOADS];
 #pragma unroll
-                for (int c = 0; c < BQ; c += 32) tmem_ld32(xa + c, reinterpret_cast<uint32_t*>(q + c));
+                for (int c = 0; c < 64 * LOADS; c += 32) tmem_ld32(xa + c, reinterpret_cast<uint32_t*>(q + c));
                 tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(dq_empty);
+                if constexpr (LOADS == 2) {
+                    tc_fence_before();
+                    mbar_arrive(dq_empty);
+                }
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
+                    if (LOADS == 1 && half == 1) {
+                        tmem_ld32(xa + 64, reinterpret_cast<uint32_t*>(q));
+                        tmem_ld32(xa + 96, reinterpret_cast<uint32_t*>(q + 32));
+                        tmem_wait_ld();
+                        tc_fence_before();
+                        mbar_arrive(dq_empty);
+                    }
                     // the previous reduce-add must have read the staging tile
                     if (issuer) bulk_wait_group_read0();
                     if (!(ok = sync_dq())) break;
 #pragma unroll
                     for (int c = 0; c < 64; ++c)
                         *reinterpret_cast<float*>(stg + c * 128 + ((piece ^ (c & 7)) << 4) + word) =
-                            q[half * 64 + c] * p.scale;
+                            q[(LOADS == 2 ? half * 64 : 0) + c] * p.scale;
                     fence_proxy_async_smem();
                     if (!(ok = sync_dq())) break;
                     if (issuer) {
@@ -627,29 +637,33 @@ __global__ void __launch_bounds__(NTHREADS, 1) bwd_kernel(const __grid_constant_
     }
 }
 
-template <int D, bool CAUSAL, bool DROPOUT>
+template <int D, bool CAUSAL, bool DROPOUT, int SMW>
 cudaError_t launch(const BwdParams& p, cudaStream_t stream)
 {
-    auto kern = bwd_kernel<D, CAUSAL, DROPOUT>;
+    auto kern = bwd_kernel<D, CAUSAL, DROPOUT, SMW>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     dim3 grid(p.n_kv_tiles, p.BH);
-    kern<<<grid, NTHREADS, Cfg<D>::SMEM_BYTES, stream>>>(p);
+    kern<<<grid, Roles<SMW>::NTHREADS, Cfg<D>::SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, int SMW>
 cudaError_t launch_d(const BwdParams& p, bool causal, bool dropout, cudaStream_t stream)
 {
-    if (dropout) return causal ? launch<D, true, true>(p, stream) : launch<D, false, true>(p, stream);
-    return causal ? launch<D, true, false>(p, stream) : launch<D, false, false>(p, stream);
+    if (dropout) return causal ? launch<D, true, true, SMW>(p, stream) : launch<D, false, true, SMW>(p, stream);
+    return causal ? launch<D, true, false, SMW>(p, stream) : launch<D, false, false, SMW>(p, stream);
 }
 
 }  // namespace bwdk
 
 cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, bool dropout, cudaStream_t stream)
 {
-    return d == 128 ? bwdk::launch_d<128>(p, causal, dropout, stream) : bwdk::launch_d<64>(p, causal, dropout, stream);
+    if (p.softmax_warps == 8)
+        return d == 128 ? bwdk::launch_d<128, 8>(p, causal, dropout, stream)
+                        : bwdk::launch_d<64, 8>(p, causal, dropout, stream);
+    return d == 128 ? bwdk::launch_d<128, 4>(p, causal, dropout, stream)
+                    : bwdk::launch_d<64, 4>(p, causal, dropout, stream);
 }
 
 int bwd_dq_tile_rows(int d) { return d == 128 ? bwdk::Cfg<128>::STG_ROWS : bwdk::Cfg<64>::STG_ROWS; }

@@ -34,6 +34,8 @@ std::atomic<unsigned long long> g_limit_ns{2000000000ull};
 // words in use (64; fewer only to exercise shared words in tests)
 std::atomic<unsigned int> g_fwd_tickets[kMaxDevices];
 std::atomic<int> g_fwd_queue_slots{64};
+// softmax warps per backward CTA (4 or 8; 0: the library's choice)
+std::atomic<int> g_bwd_softmax_warps{0};
 thread_local int g_last_launches = 0;
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -194,6 +196,13 @@ int fa_last_cuda_error(void) { return g_last_cuda_error; }
 const char* fa_cuda_error_string(int code) { return cudaGetErrorString(static_cast<cudaError_t>(code)); }
 
 void fa_set_wait_limit_ns(unsigned long long ns) { g_limit_ns.store(ns < 1000000ull ? 1000000ull : ns); }
+
+int fa_set_bwd_softmax_warps(int n)
+{
+    if (n != 0 && n != 4 && n != 8) return FA_ERR_INVALID_ARG;
+    g_bwd_softmax_warps.store(n);
+    return FA_OK;
+}
 
 int fa_set_fwd_queue_words(int n)
 {
@@ -564,6 +573,8 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, f
     p.keep_scale = (dropout && keep_t > 0) ? 256.0f / static_cast<float>(keep_t) : (dropout ? 0.0f : 1.0f);
     p.seed = seed;
     p.offset = offset;
+    const int smw = g_bwd_softmax_warps.load();
+    p.softmax_warps = smw != 0 ? smw : 8;
     st = cuda_status(launch_bwd_sm100(p, d, causal != 0, dropout, static_cast<cudaStream_t>(stream)));
     if (st == FA_OK) g_last_launches = 1;
     return st;

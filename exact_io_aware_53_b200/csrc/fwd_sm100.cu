@@ -191,9 +191,9 @@ struct Cfg {
     static constexpr int STG_OFF = KV_OFF + STAGES * TILE_BYTES;  // O staging tile (bf16, as Q's boxes)
     static constexpr int BAR_OFF = STG_OFF + TILE_BYTES;
     // q_full, q_empty, kv_full/empty[S], s_full, p_full, o_full, o_free [2],
-    // item_full, item_empty [2], drain, stg_full, stg_free
-    static constexpr int NBARS = 2 + 2 * STAGES + 4 * 2 + 2 * 2 + 1 + 2;
-    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;  // + TMEM slot and item ring
+    // item_full, item_empty [2], drain, stg_free
+    static constexpr int NBARS = 2 + 2 * STAGES + 4 * 2 + 2 * 2 + 1 + 1;
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;  // + TMEM slot, item ring, staging count
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t O_COL = 256;
@@ -261,10 +261,10 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     uint64_t* item_full = o_free + 2;         // [2]
     uint64_t* item_empty = item_full + 2;     // [2]
     uint64_t* drain = item_empty + 2;
-    uint64_t* stg_full = drain + 1;  // the 256 threads of a Q tile have written O into staging
-    uint64_t* stg_free = drain + 2;  // the TMA store has read the staging tile
+    uint64_t* stg_free = drain + 1;  // the TMA store has read the staging tile
     uint8_t* sSTG = smem + C::STG_OFF;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+    unsigned int* stg_count = tmem_slot + 3;  // warps of a Q tile done writing the staging tile
     int* item_buf = reinterpret_cast<int*>(tmem_slot + 1);  // [2]
 
     const int warp = static_cast<int>(warp_id());
@@ -289,8 +289,8 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
             mbar_init(&item_empty[t], 1 + 16);  // the MMA warp and the 16 softmax warps
         }
         mbar_init(drain, 1);
-        mbar_init(stg_full, 256);
         mbar_init(stg_free, 1);
+        *stg_count = 0u;
         fence_mbar_init();
     }
     if (warp == MMA_WARP) {
@@ -470,9 +470,9 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
         int ring0 = 0;    // K/V ring slots used by earlier items
         // O leaves through one staging tile that the two Q tiles take in turn, in
         // the order their O is complete: tile 0 then tile 1 within an item (tile 0
-        // never has more key tiles), item after item; stg_seq counts the uses
-        // before the current item, in both tile groups alike
-        uint32_t stg_seq = 0;
+        // never has more key tiles), item after item.  Use 2 n + t therefore waits
+        // for the staging tile's free phase of parity t ^ 1; an item whose tile 1
+        // lies past N still takes its turn, without writing anything.
         bool ok = true;
         for (int n = 0; ok; ++n) {
             const int slot = n & 1;
@@ -607,11 +607,15 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                 mbar_arrive(&p_full[t]);
                 ++pc;
             }
+            if (ok && nk == 0) {
+                // tile 1 past N: pass the staging tile on
+                ok = warp_wait(stg_free, 0u, p.ctl);
+                if (ok && warp == 8 && lane == 0) mbar_arrive(stg_free);
+            }
             if (ok && nk > 0) {
-                const uint32_t seq = stg_seq + ((t == 1 && w.n_kv[0] > 0) ? 1u : 0u);
                 ok = warp_wait(&o_full[t], oc & 1, p.ctl);
                 ++oc;
-                if (ok) ok = warp_wait(stg_free, (seq & 1) ^ 1, p.ctl);
+                if (ok) ok = warp_wait(stg_free, static_cast<uint32_t>(t ^ 1), p.ctl);
                 if (ok) {
                     tc_fence_after();
                     // each row's sum is split over its four threads
@@ -632,7 +636,13 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                     // O / l as bf16 into the staging tile: box col / 64, row rr0 (and
                     // rr0 + 8), 16-byte chunk (col % 64) / 8 swizzled with the row; a
                     // warp's 32-bit stores of one column group cover 8 rows x 16 bytes
-                    // in distinct bank groups
+                    // in distinct bank groups.  The addresses are formed here from an
+                    // opaque copy of the row, so that none of them is computed once
+                    // ahead of the key-tile loop and kept live through it.
+                    uint32_t srow = static_cast<uint32_t>(rr0);
+                    asm volatile("" : "+r"(srow));
+                    const uint32_t stg0 = smem_u32(sSTG) + srow * 128u + static_cast<uint32_t>(cg) * 2u;
+                    const uint32_t sx = srow & 7u;
     #pragma unroll
                     for (int cc = 0; cc < D; cc += 32) {
                         uint32_t o[16];
@@ -640,33 +650,39 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                         tmem_wait_ld();
     #pragma unroll
                         for (int n = 0; n < 4; ++n) {
-                            const int col = cc + 8 * n + cg;
-                            uint8_t* box = sSTG + (col >> 6) * C::BOX_BYTES + (col & 7) * 2;
-                            const uint32_t chunk = static_cast<uint32_t>(col & 63) >> 3;
-                            *reinterpret_cast<uint32_t*>(box + sw128_offset(rr0, chunk)) =
-                                pack_bf16x2(__uint_as_float(o[4 * n]) * inv0, __uint_as_float(o[4 * n + 1]) * inv0);
-                            *reinterpret_cast<uint32_t*>(box + sw128_offset(rr0 + 8, chunk)) =
-                                pack_bf16x2(__uint_as_float(o[4 * n + 2]) * inv1, __uint_as_float(o[4 * n + 3]) * inv1);
+                            // chunk (cc + 8 n) % 64 / 8 of box (cc + 8 n) / 64; rows rr0 and rr0 + 8
+                            // share the swizzle (8 apart)
+                            const uint32_t chunk = static_cast<uint32_t>(((cc + 8 * n) & 63) >> 3);
+                            const uint32_t a = stg0 + static_cast<uint32_t>(((cc + 8 * n) >> 6) * C::BOX_BYTES) +
+                                               ((chunk ^ sx) << 4);
+                            st_shared_u32(a, pack_bf16x2(__uint_as_float(o[4 * n]) * inv0,
+                                                         __uint_as_float(o[4 * n + 1]) * inv0));
+                            st_shared_u32(a + 8u * 128u, pack_bf16x2(__uint_as_float(o[4 * n + 2]) * inv1,
+                                                                     __uint_as_float(o[4 * n + 3]) * inv1));
                         }
                     }
                     // O_t has been read: the next item's first P V may overwrite it
                     tc_fence_before();
                     mbar_arrive(&o_free[t]);
+                    // the last of the tile's 8 warps to finish its part issues the TMA
+                    // tile stores (one per 64-column box; rows past N are clipped)
                     fence_proxy_async_smem();
-                    mbar_arrive(stg_full);
-                    if (warp == 8 * t && lane == 0) {
-                        // one TMA tile store per 64-column box; rows past N are clipped
-                        if (mbar_wait(stg_full, seq & 1, p.ctl)) {
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (atomicAdd(stg_count, 1u) == 7u) {
+                            __threadfence_block();
+                            *stg_count = 0u;
+                            fence_proxy_async_smem();
                             for (int c = 0; c < C::NDC; ++c)
                                 tma_store_3d(&p.tm_o, sSTG + c * C::BOX_BYTES, c * 64, w.q0 + t * BM, w.bh);
                             bulk_commit_group();
                             bulk_wait_group_read0();
+                            mbar_arrive(stg_free);
                         }
-                        mbar_arrive(stg_free);
                     }
+                    __syncwarp();
                 }
             }
-            stg_seq += (w.n_kv[0] > 0 ? 1u : 0u) + (w.n_kv[1] > 0 ? 1u : 0u);
             ring0 += 2 * w.n_kv_max;
         }
     }

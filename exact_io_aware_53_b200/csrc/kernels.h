@@ -120,6 +120,7 @@ struct BwdParams {
     float keep_scale;  // 256 / keep_t (0 when keep_t = 0)
     uint64_t seed;     // Philox key (seed, offset)
     uint64_t offset;
+    int softmax_warps;  // 4 or 8 softmax warps per CTA
     WaitCtl ctl;
 };
 cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, bool dropout, cudaStream_t stream);

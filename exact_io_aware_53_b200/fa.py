@@ -41,6 +41,7 @@ _SIGS = {
     "fa_check_device_status": ([P], I),
     "fa_set_wait_limit_ns": ([ctypes.c_ulonglong], None),
     "fa_set_fwd_queue_words": ([I], I),
+    "fa_set_bwd_softmax_warps": ([I], I),
     "fa_fwd_splitkv_workspace_bytes": ([I, I, I, I, I, I], ctypes.c_size_t),
     "fa_fwd_splitkv": ([P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, I, I, P], I),
     "fa_fwd_blocksparse": ([P, P, P, P, P, P, ctypes.c_longlong, I, I, I, I, ctypes.c_float, I, P], I),

@@ -182,6 +182,13 @@ void fa_set_wait_limit_ns(unsigned long long ns);
  * case.  Process-wide.  FA_ERR_INVALID_ARG outside 1 .. 64. */
 int fa_set_fwd_queue_words(int n);
 
+/* Diagnostics: softmax warps per CTA of the backward kernels, 4 or 8 (0: the
+ * library's choice, 8).  With 8, two warps share each SM sub-partition and
+ * split the 128 query columns of a tile; with 4, one warp takes them all.
+ * Both give the same results up to the order of the dQ additions; tests run
+ * both.  Process-wide.  FA_ERR_INVALID_ARG for other values. */
+int fa_set_bwd_softmax_warps(int n);
+
 /*
  * Split-KV forward, bf16: Nq queries against Nk keys, the shape of decoding
  * against a key/value cache (no counterpart as an interface on the pages; the

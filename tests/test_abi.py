@@ -268,3 +268,9 @@ def test_forward_queue_word_count_is_checked(lib):
     f = lib._lib.fa_set_fwd_queue_words
     assert f(0) == lib.FA_ERR_INVALID_ARG and f(65) == lib.FA_ERR_INVALID_ARG
     assert f(64) == lib.FA_OK
+
+
+def test_backward_softmax_warp_count_is_checked(lib):
+    f = lib._lib.fa_set_bwd_softmax_warps
+    assert f(2) == lib.FA_ERR_INVALID_ARG and f(16) == lib.FA_ERR_INVALID_ARG
+    assert f(4) == lib.FA_OK and f(8) == lib.FA_OK and f(0) == lib.FA_OK
