@@ -269,7 +269,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         __syncwarp();
     } else if (warp == MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs this loop in step and elect.sync picks the lane that
+        // issues each tcgen05 instruction: issued that way a 128 x 128 x 16 MMA
+        // takes ~65 cycles of issue, against ~92 from one lane of a diverged warp,
+        // which with 8 softmax warps would make the issue loop the bound.
+        {
             constexpr uint32_t idesc_kk = idesc_bf16(128, 128, false, false);  // S^T, dP^T
             constexpr uint32_t idesc_tm = idesc_bf16(128, D, false, true);     // dV (A in TMEM), dK
             constexpr uint32_t idesc_dq = idesc_bf16(128, D, true, true);      // dQ^T (d = 128) / dQ (d = 64)
@@ -281,7 +285,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * BOX + (kk & 3) * 32;
-                    mma_ss(tmem + d_col, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
+                    mma_ss_elect(tmem + d_col, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
                            idesc_kk, kk > 0 ? 1u : 0u);
                 }
             };
@@ -289,14 +293,14 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             auto issue_dv = [&](uint32_t a_col, bool acc0) {
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    mma_ts(tmem + C::DV_COL, tmem + a_col + (kk >> 2) * 64 + (kk & 3) * 8,
+                    mma_ts_elect(tmem + C::DV_COL, tmem + a_col + (kk >> 2) * 64 + (kk & 3) * 8,
                            sdesc_sw128(aDO + kk * 2048, BOX, 1024), idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
             };
             // dK += dS^T (shared, K-major) x Q (MN-major over d)
             auto issue_dk = [&](uint32_t b_base, bool acc0) {
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
-                    mma_ss(tmem + C::DK_COL, sdesc_sw128(aDS + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024),
+                    mma_ss_elect(tmem + C::DK_COL, sdesc_sw128(aDS + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024),
                            sdesc_sw128(b_base + kk * 2048, BOX, 1024), idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
             };
             // d = 128: dQ^T = K^T x dS^T into X; d = 64: dQ = dS x K into its own
@@ -307,63 +311,63 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     const uint64_t k_desc = sdesc_sw128(aK + kk * 2048, BOX, 1024);
                     const uint64_t ds_desc = sdesc_sw128(aDS + kk * 2048, BOX, 1024);
                     if constexpr (D == 128)
-                        mma_ss(tmem + d_col, k_desc, ds_desc, idesc_dq, kk > 0 ? 1u : 0u);
+                        mma_ss_elect(tmem + d_col, k_desc, ds_desc, idesc_dq, kk > 0 ? 1u : 0u);
                     else
-                        mma_ss(tmem + d_col, ds_desc, k_desc, idesc_dq, kk > 0 ? 1u : 0u);
+                        mma_ss_elect(tmem + d_col, ds_desc, k_desc, idesc_dq, kk > 0 ? 1u : 0u);
                 }
             };
 
-            bool ok = mbar_wait(kv_full, 0, p.ctl) && mbar_wait(&q_full[0], 0, p.ctl);
+            bool ok = warp_wait(kv_full, 0, p.ctl) && warp_wait(&q_full[0], 0, p.ctl);
             if (ok) {
                 tc_fence_after();
                 issue_kk(rcol(0), aK, q_base(0));
-                mma_commit(s_full);
-                ok = mbar_wait(do_full, 0, p.ctl);
+                mma_commit_elect(s_full);
+                ok = warp_wait(do_full, 0, p.ctl);
                 if (ok) {
                     tc_fence_after();
                     issue_kk(rcol(1), aV, aDO);
-                    mma_commit(dp_full);
+                    mma_commit_elect(dp_full);
                 }
             }
             for (int t = 0; t < n_it && ok; ++t) {
                 const uint32_t X = rcol(t), Y = rcol(t + 1);
-                if (!(ok = mbar_wait(p_ready, t & 1, p.ctl))) break;
+                if (!(ok = warp_wait(p_ready, t & 1, p.ctl))) break;
                 tc_fence_after();
                 issue_dv(X, t > 0);
-                mma_commit(do_empty);
-                if (!(ok = mbar_wait(ds_ready, t & 1, p.ctl))) break;
+                mma_commit_elect(do_empty);
+                if (!(ok = warp_wait(ds_ready, t & 1, p.ctl))) break;
                 tc_fence_after();
                 if (t + 1 < n_it) {
                     // Y held dP^T of tile t, already read by the softmax
-                    if (!(ok = mbar_wait(&q_full[(t + 1) & 1], ((t + 1) >> 1) & 1, p.ctl))) break;
+                    if (!(ok = warp_wait(&q_full[(t + 1) & 1], ((t + 1) >> 1) & 1, p.ctl))) break;
                     tc_fence_after();
                     issue_kk(Y, aK, q_base(t + 1));
-                    mma_commit(s_full);
+                    mma_commit_elect(s_full);
                 }
                 issue_dk(q_base(t), t > 0);
-                mma_commit(&q_empty[t & 1]);
+                mma_commit_elect(&q_empty[t & 1]);
                 if constexpr (D == 128) {
                     issue_dq(X);
                 } else {
                     // the dQ warps must have read the previous tile's dQ out
-                    if (t > 0 && !(ok = mbar_wait(dq_empty, (t - 1) & 1, p.ctl))) break;
+                    if (t > 0 && !(ok = warp_wait(dq_empty, (t - 1) & 1, p.ctl))) break;
                     tc_fence_after();
                     issue_dq(C::DQ_COL);
                 }
-                mma_commit(dq_full);
+                mma_commit_elect(dq_full);
                 if (t + 1 < n_it) {
-                    if (!(ok = mbar_wait(do_full, (t + 1) & 1, p.ctl))) break;
+                    if (!(ok = warp_wait(do_full, (t + 1) & 1, p.ctl))) break;
                     if constexpr (D == 128) {
                         // X holds dQ^T of tile t until the dQ warps have read it
-                        if (!(ok = mbar_wait(dq_empty, t & 1, p.ctl))) break;
+                        if (!(ok = warp_wait(dq_empty, t & 1, p.ctl))) break;
                     }
                     tc_fence_after();
                     issue_kk(X, aV, aDO);
-                    mma_commit(dp_full);
+                    mma_commit_elect(dp_full);
                 }
             }
-            if (ok) mma_commit(dkdv_done);
-            mma_commit(drain);
+            if (ok) mma_commit_elect(dkdv_done);
+            mma_commit_elect(drain);
             mbar_wait_drain(drain, 0, p.ctl.limit_ns);
         }
         __syncwarp();
