@@ -91,7 +91,7 @@ struct Cfg {
     static constexpr int STG_CHUNK = STG_ROWS * 128;
     static constexpr int VEC_OFF = STG_OFF + (D / 32) * STG_CHUNK;  // [stage][lse2 128 | delta 128]
     static constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
-    static constexpr int NBARS = 17;
+    static constexpr int NBARS = 18;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t DV_COL = 256;
@@ -154,6 +154,10 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     constexpr int MMA_WARP = R::MMA_WARP;
     constexpr int LOAD_WARP = R::LOAD_WARP;
     constexpr int HALVES = SMW == 8 ? 1 : 2;  // query halves per softmax warp
+    // With one query half per softmax warp its dP^T (64 columns) fits in registers:
+    // the warps read it first and release Y, so S^T of the next tile is computed
+    // while they still form dS^T
+    constexpr bool EARLY_DP = HALVES == 1;
     extern __shared__ __align__(1024) uint8_t smem[];
     // the 128-byte-swizzled tiles need a 1024-byte aligned base; the layout
     // leaves no slack, so a misaligned base is reported instead of used
@@ -183,6 +187,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     uint64_t* dkdv_done = bars + 13;
     uint64_t* drain = bars + 14;
     uint64_t* dqw_bar = bars + 15;  // the 4 dQ warps (128 threads)
+    uint64_t* dp_read = bars + 16;  // the softmax warps hold dP^T of the tile in registers (Y is free)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
 
     const int warp = static_cast<int>(warp_id());
@@ -209,6 +214,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         mbar_init(dp_full, 1);
         mbar_init(p_ready, 32 * SMW);
         mbar_init(ds_ready, 32 * SMW);
+        mbar_init(dp_read, 32 * SMW);
         mbar_init(dq_full, 1);
         mbar_init(dq_empty, 128);
         mbar_init(dkdv_done, 1);
@@ -335,7 +341,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 tc_fence_after();
                 issue_dv(X, t > 0);
                 mma_commit_elect(do_empty);
-                if (!(ok = warp_wait(ds_ready, t & 1, p.ctl))) break;
+                if (!(ok = warp_wait(EARLY_DP ? dp_read : ds_ready, t & 1, p.ctl))) break;
                 tc_fence_after();
                 if (t + 1 < n_it) {
                     // Y held dP^T of tile t, already read by the softmax
@@ -343,6 +349,10 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     tc_fence_after();
                     issue_kk(Y, aK, q_base(t + 1));
                     mma_commit_elect(s_full);
+                }
+                if constexpr (EARLY_DP) {
+                    if (!(ok = warp_wait(ds_ready, t & 1, p.ctl))) break;
+                    tc_fence_after();
                 }
                 issue_dk(q_base(t), t > 0);
                 mma_commit_elect(&q_empty[t & 1]);
@@ -462,15 +472,32 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             // dS^T = P^T (dP^T - D), with the bf16 P^T read back from TMEM (it stays in
             // X until this tile's dS^T is written), to shared memory: row r, query
             // columns in 2 chunks of 64 (128-byte swizzled rows), chunk = half
+            float dph[EARLY_DP ? 64 : 1];
+            uint32_t pqh[EARLY_DP ? 32 : 1];
+            if constexpr (EARLY_DP) {
+                tmem_ld32(ya + h0 * 64, reinterpret_cast<uint32_t*>(dph));
+                tmem_ld32(ya + h0 * 64 + 32, reinterpret_cast<uint32_t*>(dph + 32));
+                tmem_ld32(xa + h0 * 64 + (DROPOUT ? 32 : 0), pqh);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(dp_read);
+            }
 #pragma unroll
             for (int qq = 0; qq < 2 * HALVES; ++qq) {
                 const int q4 = 2 * h0 + qq;  // query quarter
                 const int h = q4 >> 1;
                 float dp[32];
                 uint32_t pq[16];
-                tmem_ld32(ya + q4 * 32, reinterpret_cast<uint32_t*>(dp));
-                tmem_ld16(xa + h * 64 + (DROPOUT ? 32 : 0) + (q4 & 1) * 16, pq);
-                tmem_wait_ld();
+                if constexpr (EARLY_DP) {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) dp[c] = dph[32 * qq + c];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) pq[c] = pqh[16 * qq + c];
+                } else {
+                    tmem_ld32(ya + q4 * 32, reinterpret_cast<uint32_t*>(dp));
+                    tmem_ld16(xa + h * 64 + (DROPOUT ? 32 : 0) + (q4 & 1) * 16, pq);
+                    tmem_wait_ld();
+                }
                 if constexpr (DROPOUT) {
                     // dropped weights contribute no dP: z Z dP
                     const uint32_t z = zq[qq];
