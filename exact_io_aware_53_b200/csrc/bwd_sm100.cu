@@ -23,13 +23,13 @@
 // softmax has read dP^T, and S^T of tile t + 1 is issued there before dK and
 // dQ of tile t, overlapping the next softmax with them.  dP^T of tile t + 1
 // then goes to X.
-//   d = 128: dQ_t^T = K^T dS^T (lanes = head-dim index) is written into X
-//            after dS^T, so dP^T of tile t + 1 waits for the dQ warps to have
-//            read it; staged as fp32 [64 query][128 d] tiles, two per tile.
-//   d = 64:  dQ_t = dS K (lanes = query rows, 64 columns) has its own region;
-//            the next dQ waits for the dQ warps instead.  Staged as one fp32
-//            [128 query][64 d] tile.
-// Staged tiles are TMA reduce-added (fp32) into dQ.
+// dQ_t = dS K_j (lanes = query rows, d columns; dS^T in shared memory read as
+// the MN-major A operand):
+//   d = 128: written into X after dS^T, so dP^T of tile t + 1 waits for the dQ
+//            warps to have read it out;
+//   d = 64:  in its own region; the next dQ waits for the dQ warps instead.
+// The dQ warps stage it as fp32 [128 query][64 d] tiles (one per 64 columns,
+// a row's 16-byte pieces written as float4) and TMA reduce-add them into dQ.
 //
 // Dropout (DROPOUT): the forward kept weight P_ij with probability keep_t / 256
 // and scaled kept weights by 256 / keep_t; the keep bit is byte j % 32 of
@@ -49,7 +49,7 @@
 //                      with 8 warps, warp w takes query half w / 4 (two warps
 //                      per SM sub-partition overlap their exponentials with
 //                      the other's FMA-pipe work), with 4 both halves
-//   next 4 warps       dQ: read dQ (or dQ^T) out of TMEM, scale, stage, reduce-add
+//   next 4 warps       dQ: read dQ out of TMEM, scale, stage, reduce-add
 //   next warp          MMA issuer (one thread)
 //   last warp          TMA producer: K, V once; {Q_t, lse2_t, D_t} in a 2-stage
 //                      ring, dO_t in one buffer (its last reader, dV, runs early
@@ -86,10 +86,11 @@ struct Cfg {
     static constexpr int DO_OFF = Q_OFF + QSTAGES * TILE;  // dO_t, 1 stage
     static constexpr int DS_OFF = DO_OFF + TILE;           // dS^T: 2 boxes of 64 query columns
     static constexpr int STG_OFF = DS_OFF + 2 * BOX;       // dQ staging
-    // fp32 staging tile: D / 32 chunks of [STG_ROWS query rows][32 d], 128-byte swizzled
-    static constexpr int STG_ROWS = (D == 128) ? 64 : 128;
+    // fp32 staging tile: 2 chunks of [STG_ROWS query rows][32 d], 128-byte swizzled
+    // (64 of the d columns at a time)
+    static constexpr int STG_ROWS = 128;
     static constexpr int STG_CHUNK = STG_ROWS * 128;
-    static constexpr int VEC_OFF = STG_OFF + (D / 32) * STG_CHUNK;  // [stage][lse2 128 | delta 128]
+    static constexpr int VEC_OFF = STG_OFF + 2 * STG_CHUNK;  // [stage][lse2 128 | delta 128]
     static constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
     static constexpr int NBARS = 18;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         {
             constexpr uint32_t idesc_kk = idesc_bf16(128, 128, false, false);  // S^T, dP^T
             constexpr uint32_t idesc_tm = idesc_bf16(128, D, false, true);     // dV (A in TMEM), dK
-            constexpr uint32_t idesc_dq = idesc_bf16(128, D, true, true);      // dQ^T (d = 128) / dQ (d = 64)
+            constexpr uint32_t idesc_dq = idesc_bf16(128, D, true, true);      // dQ
             const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
                            aDS = smem_u32(sDS);
             auto q_base = [&](int t) { return aQ + (t & 1) * C::TILE; };
@@ -309,18 +310,13 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     mma_ss_elect(tmem + C::DK_COL, sdesc_sw128(aDS + (kk >> 2) * BOX + (kk & 3) * 32, 16, 1024),
                            sdesc_sw128(b_base + kk * 2048, BOX, 1024), idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
             };
-            // d = 128: dQ^T = K^T x dS^T into X; d = 64: dQ = dS x K into its own
-            // region.  Both operands MN-major, walking the 128 keys.
+            // dQ = dS (shared dS^T read MN-major: 64 contiguous queries per 128-byte
+            // row) x K (MN-major over d), walking the 128 keys
             auto issue_dq = [&](uint32_t d_col) {
 #pragma unroll
-                for (int kk = 0; kk < BKV / 16; ++kk) {
-                    const uint64_t k_desc = sdesc_sw128(aK + kk * 2048, BOX, 1024);
-                    const uint64_t ds_desc = sdesc_sw128(aDS + kk * 2048, BOX, 1024);
-                    if constexpr (D == 128)
-                        mma_ss_elect(tmem + d_col, k_desc, ds_desc, idesc_dq, kk > 0 ? 1u : 0u);
-                    else
-                        mma_ss_elect(tmem + d_col, ds_desc, k_desc, idesc_dq, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < BKV / 16; ++kk)
+                    mma_ss_elect(tmem + d_col, sdesc_sw128(aDS + kk * 2048, BOX, 1024),
+                                 sdesc_sw128(aK + kk * 2048, BOX, 1024), idesc_dq, kk > 0 ? 1u : 0u);
             };
 
             bool ok = warp_wait(kv_full, 0, p.ctl) && warp_wait(&q_full[0], 0, p.ctl);
@@ -368,7 +364,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 if (t + 1 < n_it) {
                     if (!(ok = warp_wait(do_full, (t + 1) & 1, p.ctl))) break;
                     if constexpr (D == 128) {
-                        // X holds dQ^T of tile t until the dQ warps have read it
+                        // X holds dQ of tile t until the dQ warps have read it
                         if (!(ok = warp_wait(dq_empty, t & 1, p.ctl))) break;
                     }
                     tc_fence_after();
@@ -563,76 +559,48 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             const int i = i_first + t;
             if (!(ok = warp_wait(dq_full, t & 1, p.ctl))) break;
             tc_fence_after();
-            if constexpr (D == 128) {
-                // thread = head-dim index dr (TMEM lane of dQ^T), 128 query columns;
-                // element (query c, dim dr) of a [64][128] staging tile: 32-column
-                // chunk dr / 32, row c, 16-byte piece (dr % 32) / 4 swizzled with c % 8
-                const int dr = wq * 32 + lane;
-                uint8_t* stg = sSTG + (dr >> 5) * C::STG_CHUNK;
-                const uint32_t piece = (dr & 31) >> 2, word = (dr & 3) * 4;
-                const uint32_t xa = tmem + lane_off + rcol(t);
-                // with 4 softmax warps both halves of dQ^T are read before X is released;
-                // with 8 (128 registers) half 0 is staged first and X released after half 1
-                constexpr int LOADS = (SMW == 8) ? 1 : 2;
-                float q[64 * LOADS];
+            // thread = query row qr (TMEM lane of dQ), D head-dim columns in halves of
+            // 64; row qr of the [128][64] staging tile: 32-column chunk, 16-byte
+            // piece swizzled with qr % 8
+            const int qr = wq * 32 + lane;
+            const uint32_t qa = tmem + lane_off + (D == 128 ? rcol(t) : C::DQ_COL);
+            // with 4 softmax warps (168 registers) all of dQ is read before the region
+            // is released; with 8 (128 registers) the second half is read after the
+            // first has been staged
+            constexpr int HOLD = (D == 128 && SMW == 4) ? 2 : 1;  // halves held in registers
+            float q[64 * HOLD];
 #pragma unroll
-                for (int c = 0; c < 64 * LOADS; c += 32) tmem_ld32(xa + c, reinterpret_cast<uint32_t*>(q + c));
-                tmem_wait_ld();
-                if constexpr (LOADS == 2) {
+            for (int c = 0; c < 64 * HOLD; c += 32) tmem_ld32(qa + c, reinterpret_cast<uint32_t*>(q + c));
+            tmem_wait_ld();
+            if (HOLD * 64 == D) {
+                tc_fence_before();
+                mbar_arrive(dq_empty);
+            }
+#pragma unroll
+            for (int hd = 0; hd < D / 64; ++hd) {
+                if (HOLD == 1 && hd == 1) {
+                    tmem_ld32(qa + 64, reinterpret_cast<uint32_t*>(q));
+                    tmem_ld32(qa + 96, reinterpret_cast<uint32_t*>(q + 32));
+                    tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(dq_empty);
                 }
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    if (LOADS == 1 && half == 1) {
-                        tmem_ld32(xa + 64, reinterpret_cast<uint32_t*>(q));
-                        tmem_ld32(xa + 96, reinterpret_cast<uint32_t*>(q + 32));
-                        tmem_wait_ld();
-                        tc_fence_before();
-                        mbar_arrive(dq_empty);
-                    }
-                    // the previous reduce-add must have read the staging tile
-                    if (issuer) bulk_wait_group_read0();
-                    if (!(ok = sync_dq())) break;
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        *reinterpret_cast<float*>(stg + c * 128 + ((piece ^ (c & 7)) << 4) + word) =
-                            q[(LOADS == 2 ? half * 64 : 0) + c] * p.scale;
-                    fence_proxy_async_smem();
-                    if (!(ok = sync_dq())) break;
-                    if (issuer) {
-#pragma unroll
-                        for (int ch = 0; ch < D / 32; ++ch)
-                            tma_reduce_add_3d(&p.tm_dq, sSTG + ch * C::STG_CHUNK, ch * 32, i * BQ + half * 64, bh);
-                        bulk_commit_group();
-                    }
-                }
-            } else {
-                // thread = query row qr (TMEM lane of dQ), 64 head-dim columns;
-                // row qr of the [128][64] staging tile: 32-column chunk d / 32,
-                // 16-byte piece (d % 32) / 4 swizzled with qr % 8
-                const int qr = wq * 32 + lane;
-                float q[D];
-                tmem_ld32(tmem + lane_off + C::DQ_COL, reinterpret_cast<uint32_t*>(q));
-                tmem_ld32(tmem + lane_off + C::DQ_COL + 32, reinterpret_cast<uint32_t*>(q + 32));
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(dq_empty);
+                // the previous reduce-add must have read the staging tile
                 if (issuer) bulk_wait_group_read0();
                 if (!(ok = sync_dq())) break;
+                const float* qh = q + (HOLD == 2 ? hd * 64 : 0);
 #pragma unroll
-                for (int d4 = 0; d4 < D / 4; ++d4) {
+                for (int d4 = 0; d4 < 16; ++d4) {
                     uint8_t* row = sSTG + (d4 >> 3) * C::STG_CHUNK + qr * 128;
                     *reinterpret_cast<float4*>(row + (((d4 & 7) ^ (qr & 7)) << 4)) =
-                        make_float4(q[4 * d4] * p.scale, q[4 * d4 + 1] * p.scale, q[4 * d4 + 2] * p.scale,
-                                    q[4 * d4 + 3] * p.scale);
+                        make_float4(qh[4 * d4] * p.scale, qh[4 * d4 + 1] * p.scale, qh[4 * d4 + 2] * p.scale,
+                                    qh[4 * d4 + 3] * p.scale);
                 }
                 fence_proxy_async_smem();
                 if (!(ok = sync_dq())) break;
                 if (issuer) {
-#pragma unroll
-                    for (int ch = 0; ch < D / 32; ++ch)
-                        tma_reduce_add_3d(&p.tm_dq, sSTG + ch * C::STG_CHUNK, ch * 32, i * BQ, bh);
+                    tma_reduce_add_3d(&p.tm_dq, sSTG, hd * 64, i * BQ, bh);
+                    tma_reduce_add_3d(&p.tm_dq, sSTG + C::STG_CHUNK, hd * 64 + 32, i * BQ, bh);
                     bulk_commit_group();
                 }
             }
