@@ -92,7 +92,7 @@ struct Cfg {
     static constexpr int STG_CHUNK = STG_ROWS * 128;
     static constexpr int VEC_OFF = STG_OFF + 2 * STG_CHUNK;  // [stage][lse2 128 | delta 128]
     static constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
-    static constexpr int NBARS = 18;
+    static constexpr int NBARS = 19;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t DV_COL = 256;
@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     uint64_t* drain = bars + 14;
     uint64_t* dqw_bar = bars + 15;  // the 4 dQ warps (128 threads)
     uint64_t* dp_read = bars + 16;  // the softmax warps hold dP^T of the tile in registers (Y is free)
+    uint64_t* ds_free = bars + 17;  // the reduce-add staged in the dS^T buffer has read it
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
 
     const int warp = static_cast<int>(warp_id());
@@ -221,6 +222,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         mbar_init(dkdv_done, 1);
         mbar_init(drain, 1);
         mbar_init(dqw_bar, 128);
+        mbar_init(ds_free, 1);
         fence_mbar_init();
     }
     if (warp == MMA_WARP) {
@@ -462,8 +464,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             mbar_arrive(p_ready);
 
             // dP^T of this tile was issued after the dK and dQ MMAs of the previous
-            // one, so once it is complete they have read the old dS^T
+            // one, so once it is complete they have read the old dS^T; the previous
+            // tile's first dQ half was staged in the dS^T buffer, so its reduce-add
+            // must have read it too
             if (!(ok = warp_wait(dp_full, t & 1, p.ctl))) break;
+            if (t > 0 && !(ok = warp_wait(ds_free, (t - 1) & 1, p.ctl))) break;
             tc_fence_after();
             // dS^T = P^T (dP^T - D), with the bf16 P^T read back from TMEM (it stays in
             // X until this tile's dS^T is written), to shared memory: row r, query
@@ -576,8 +581,13 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 tc_fence_before();
                 mbar_arrive(dq_empty);
             }
+            // the first 64 columns are staged in the dS^T buffer, which the dK and dQ
+            // MMAs of this tile (complete) have read and the softmax rewrites only
+            // after ds_free; the second in the staging tile, once the previous
+            // tile's reduce-add from it has read it
 #pragma unroll
             for (int hd = 0; hd < D / 64; ++hd) {
+                uint8_t* stg = hd == 0 ? sDS : sSTG;
                 if (HOLD == 1 && hd == 1) {
                     tmem_ld32(qa + 64, reinterpret_cast<uint32_t*>(q));
                     tmem_ld32(qa + 96, reinterpret_cast<uint32_t*>(q + 32));
@@ -585,13 +595,16 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     tc_fence_before();
                     mbar_arrive(dq_empty);
                 }
-                // the previous reduce-add must have read the staging tile
-                if (issuer) bulk_wait_group_read0();
-                if (!(ok = sync_dq())) break;
+                if (hd == 1) {
+                    // the previous tile's reduce-add from the staging tile has read it
+                    // (at most this tile's first, from dS^T, still reading)
+                    if (issuer) bulk_wait_group_read1();
+                    if (!(ok = sync_dq())) break;
+                }
                 const float* qh = q + (HOLD == 2 ? hd * 64 : 0);
 #pragma unroll
                 for (int d4 = 0; d4 < 16; ++d4) {
-                    uint8_t* row = sSTG + (d4 >> 3) * C::STG_CHUNK + qr * 128;
+                    uint8_t* row = stg + (d4 >> 3) * C::STG_CHUNK + qr * 128;
                     *reinterpret_cast<float4*>(row + (((d4 & 7) ^ (qr & 7)) << 4)) =
                         make_float4(qh[4 * d4] * p.scale, qh[4 * d4 + 1] * p.scale, qh[4 * d4 + 2] * p.scale,
                                     qh[4 * d4 + 3] * p.scale);
@@ -599,10 +612,16 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 fence_proxy_async_smem();
                 if (!(ok = sync_dq())) break;
                 if (issuer) {
-                    tma_reduce_add_3d(&p.tm_dq, sSTG, hd * 64, i * BQ, bh);
-                    tma_reduce_add_3d(&p.tm_dq, sSTG + C::STG_CHUNK, hd * 64 + 32, i * BQ, bh);
+                    tma_reduce_add_3d(&p.tm_dq, stg, hd * 64, i * BQ, bh);
+                    tma_reduce_add_3d(&p.tm_dq, stg + C::STG_CHUNK, hd * 64 + 32, i * BQ, bh);
                     bulk_commit_group();
                 }
+            }
+            if (issuer) {
+                // the dS^T buffer is free again once its reduce-add has read it
+                if (D == 128) bulk_wait_group_read1();
+                else bulk_wait_group_read0();
+                mbar_arrive(ds_free);
             }
         }
         if (issuer) bulk_wait_group0();
