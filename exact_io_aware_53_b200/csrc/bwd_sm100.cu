@@ -159,6 +159,10 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     // the warps read it first and release Y, so S^T of the next tile is computed
     // while they still form dS^T
     constexpr bool EARLY_DP = HALVES == 1;
+    // d = 128 with 8 softmax warps: the first half of dQ is staged in the dS^T
+    // buffer (free between this tile's dQ MMA and the next tile's dS^T), so the
+    // region dQ occupies is released without waiting for the staging tile
+    constexpr bool DQ_IN_DS = (D == 128 && SMW == 8);
     extern __shared__ __align__(1024) uint8_t smem[];
     // the 128-byte-swizzled tiles need a 1024-byte aligned base; the layout
     // leaves no slack, so a misaligned base is reported instead of used
@@ -468,7 +472,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             // tile's first dQ half was staged in the dS^T buffer, so its reduce-add
             // must have read it too
             if (!(ok = warp_wait(dp_full, t & 1, p.ctl))) break;
-            if (t > 0 && !(ok = warp_wait(ds_free, (t - 1) & 1, p.ctl))) break;
+            if (DQ_IN_DS && t > 0 && !(ok = warp_wait(ds_free, (t - 1) & 1, p.ctl))) break;
             tc_fence_after();
             // dS^T = P^T (dP^T - D), with the bf16 P^T read back from TMEM (it stays in
             // X until this tile's dS^T is written), to shared memory: row r, query
@@ -581,13 +585,14 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 tc_fence_before();
                 mbar_arrive(dq_empty);
             }
-            // the first 64 columns are staged in the dS^T buffer, which the dK and dQ
-            // MMAs of this tile (complete) have read and the softmax rewrites only
-            // after ds_free; the second in the staging tile, once the previous
-            // tile's reduce-add from it has read it
+            // DQ_IN_DS: the first 64 columns are staged in the dS^T buffer, which the
+            // dK and dQ MMAs of this tile (complete) have read and the softmax
+            // rewrites only after ds_free, the second in the staging tile.
+            // Otherwise every half goes through the staging tile, once the previous
+            // reduce-add from it has read it.
 #pragma unroll
             for (int hd = 0; hd < D / 64; ++hd) {
-                uint8_t* stg = hd == 0 ? sDS : sSTG;
+                uint8_t* stg = (DQ_IN_DS && hd == 0) ? sDS : sSTG;
                 if (HOLD == 1 && hd == 1) {
                     tmem_ld32(qa + 64, reinterpret_cast<uint32_t*>(q));
                     tmem_ld32(qa + 96, reinterpret_cast<uint32_t*>(q + 32));
@@ -595,10 +600,13 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     tc_fence_before();
                     mbar_arrive(dq_empty);
                 }
-                if (hd == 1) {
-                    // the previous tile's reduce-add from the staging tile has read it
-                    // (at most this tile's first, from dS^T, still reading)
-                    if (issuer) bulk_wait_group_read1();
+                if (!DQ_IN_DS || hd == 1) {
+                    // every reduce-add from the staging tile (and, with DQ_IN_DS, this
+                    // tile's from dS^T, which then frees dS^T) has read its source
+                    if (issuer) {
+                        bulk_wait_group_read0();
+                        if (DQ_IN_DS) mbar_arrive(ds_free);
+                    }
                     if (!(ok = sync_dq())) break;
                 }
                 const float* qh = q + (HOLD == 2 ? hd * 64 : 0);
@@ -617,12 +625,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     bulk_commit_group();
                 }
             }
-            if (issuer) {
-                // the dS^T buffer is free again once its reduce-add has read it
-                if (D == 128) bulk_wait_group_read1();
-                else bulk_wait_group_read0();
-                mbar_arrive(ds_free);
-            }
+
         }
         if (issuer) bulk_wait_group0();
         // epilogue: dK rows (lanes = key rows)
