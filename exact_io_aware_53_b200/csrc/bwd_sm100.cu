@@ -601,11 +601,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     mbar_arrive(dq_empty);
                 }
                 if (!DQ_IN_DS || hd == 1) {
-                    // every reduce-add from the staging tile (and, with DQ_IN_DS, this
-                    // tile's from dS^T, which then frees dS^T) has read its source
+                    // the previous reduce-add from the staging tile has read it (with
+                    // DQ_IN_DS this tile's first, from dS^T, may still be reading)
                     if (issuer) {
-                        bulk_wait_group_read0();
-                        if (DQ_IN_DS) mbar_arrive(ds_free);
+                        if (DQ_IN_DS) bulk_wait_group_read1();
+                        else bulk_wait_group_read0();
                     }
                     if (!(ok = sync_dq())) break;
                 }
@@ -624,6 +624,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     tma_reduce_add_3d(&p.tm_dq, stg + C::STG_CHUNK, hd * 64 + 32, i * BQ, bh);
                     bulk_commit_group();
                 }
+            }
+            if (DQ_IN_DS && issuer) {
+                // dS^T is free again once the first half's reduce-add has read it
+                bulk_wait_group_read1();
+                mbar_arrive(ds_free);
             }
 
         }
