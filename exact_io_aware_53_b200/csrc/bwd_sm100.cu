@@ -468,15 +468,13 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             mbar_arrive(p_ready);
 
             // dP^T of this tile was issued after the dK and dQ MMAs of the previous
-            // one, so once it is complete they have read the old dS^T; the previous
-            // tile's first dQ half was staged in the dS^T buffer, so its reduce-add
-            // must have read it too
+            // one, so once it is complete they have read the old dS^T
             if (!(ok = warp_wait(dp_full, t & 1, p.ctl))) break;
-            if (DQ_IN_DS && t > 0 && !(ok = warp_wait(ds_free, (t - 1) & 1, p.ctl))) break;
             tc_fence_after();
             // dS^T = P^T (dP^T - D), with the bf16 P^T read back from TMEM (it stays in
             // X until this tile's dS^T is written), to shared memory: row r, query
             // columns in 2 chunks of 64 (128-byte swizzled rows), chunk = half
+            uint32_t dsk[DQ_IN_DS ? 2 : 1][16];  // packed dS^T of the warp's quarters (DQ_IN_DS)
             float dph[EARLY_DP ? 64 : 1];
             uint32_t pqh[EARLY_DP ? 32 : 1];
             if constexpr (EARLY_DP) {
@@ -509,7 +507,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
 #pragma unroll
                     for (int c = 0; c < 32; ++c) dp[c] = ((z >> c) & 1u) ? dp[c] * p.keep_scale : 0.f;
                 }
-                uint32_t ds[16];
+                uint32_t* ds = dsk[DQ_IN_DS ? qq : 0];
 #pragma unroll
                 for (int c = 0; c < 32; c += 4) {
                     const float4 d4 = *reinterpret_cast<const float4*>(delta + q4 * 32 + c);
@@ -520,11 +518,26 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     ds[c / 2] = pack_bf16x2(ga.x, ga.y);
                     ds[c / 2 + 1] = pack_bf16x2(gb.x, gb.y);
                 }
-                uint8_t* chunk = sDS + h * BOX;
+                if constexpr (!DQ_IN_DS) {
+                    uint8_t* chunk = sDS + h * BOX;
 #pragma unroll
-                for (int pc = 0; pc < 4; ++pc)
-                    *reinterpret_cast<uint4*>(chunk + sw128_offset(r, (q4 & 1) * 4 + pc)) =
-                        make_uint4(ds[4 * pc], ds[4 * pc + 1], ds[4 * pc + 2], ds[4 * pc + 3]);
+                    for (int pc = 0; pc < 4; ++pc)
+                        *reinterpret_cast<uint4*>(chunk + sw128_offset(r, (q4 & 1) * 4 + pc)) =
+                            make_uint4(ds[4 * pc], ds[4 * pc + 1], ds[4 * pc + 2], ds[4 * pc + 3]);
+                }
+            }
+            if constexpr (DQ_IN_DS) {
+                // the previous tile's first dQ half was staged in the dS^T buffer: its
+                // reduce-add must have read it before dS^T is written there (dS^T is
+                // formed in registers meanwhile)
+                if (t > 0 && !(ok = warp_wait(ds_free, (t - 1) & 1, p.ctl))) break;
+                uint8_t* chunk = sDS + h0 * BOX;
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq)
+#pragma unroll
+                    for (int pc = 0; pc < 4; ++pc)
+                        *reinterpret_cast<uint4*>(chunk + sw128_offset(r, qq * 4 + pc)) =
+                            make_uint4(dsk[qq][4 * pc], dsk[qq][4 * pc + 1], dsk[qq][4 * pc + 2], dsk[qq][4 * pc + 3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
