@@ -606,13 +606,6 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
 #pragma unroll
             for (int hd = 0; hd < D / 64; ++hd) {
                 uint8_t* stg = (DQ_IN_DS && hd == 0) ? sDS : sSTG;
-                if (HOLD == 1 && hd == 1) {
-                    tmem_ld32(qa + 64, reinterpret_cast<uint32_t*>(q));
-                    tmem_ld32(qa + 96, reinterpret_cast<uint32_t*>(q + 32));
-                    tmem_wait_ld();
-                    tc_fence_before();
-                    mbar_arrive(dq_empty);
-                }
                 if (!DQ_IN_DS || hd == 1) {
                     // the previous reduce-add from the staging tile has read it (with
                     // DQ_IN_DS this tile's first, from dS^T, may still be reading)
@@ -629,6 +622,15 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     *reinterpret_cast<float4*>(row + (((d4 & 7) ^ (qr & 7)) << 4)) =
                         make_float4(qh[4 * d4] * p.scale, qh[4 * d4 + 1] * p.scale, qh[4 * d4 + 2] * p.scale,
                                     qh[4 * d4 + 3] * p.scale);
+                }
+                if (HOLD == 1 && hd + 1 < D / 64) {
+                    // the stores above have taken the first half: read the second and
+                    // release dQ's region before this half's fence and reduce-add
+                    tmem_ld32(qa + 64, reinterpret_cast<uint32_t*>(q));
+                    tmem_ld32(qa + 96, reinterpret_cast<uint32_t*>(q + 32));
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(dq_empty);
                 }
                 fence_proxy_async_smem();
                 if (!(ok = sync_dq())) break;
