@@ -719,22 +719,18 @@ def run_blocksparse(args, w):
                 "traffic_unit": "bytes per launch (ncu dram read+write)"}
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdo = (t.pin_memory() for t in (hq, hk, hv, hdo))
+        hq, hk, hv = (t.pin_memory() for t in (hq, hk, hv))
         ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
         hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-        hg = [torch.empty(dq.shape, dtype=dq.dtype).pin_memory() for _ in range(3)]
         steps = max(3, min(args.steps, 20))
 
         def e2e_step():
             q.copy_(hq, non_blocking=True)
             k.copy_(hk, non_blocking=True)
             v.copy_(hv, non_blocking=True)
-            do.copy_(hdo, non_blocking=True)
             step()
             ho.copy_(o, non_blocking=True)
             hl.copy_(lse, non_blocking=True)
-            for h_, g_ in zip(hg, (dq, dk, dv)):
-                h_.copy_(g_, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
