@@ -193,7 +193,7 @@ def oracle_sample(w, heads: int, seed: int):
 
 def cpu_baseline(w, seed: int, budget_s: float = 10.0):
     dt1, fl1, thr = oracle_sample(w, 1, seed)
-    extra = max(0, min(int(budget_s / max(dt1, 1e-3)) - 1, 7))
+    extra = max(0, min(int(budget_s / max(dt1, 1e-3)) - 1, w.B * w.H - 1))
     dt, fl = dt1, fl1
     if extra:
         dt2, fl2, _ = oracle_sample(w, extra, seed + 1)

@@ -50,7 +50,7 @@
 //                      per SM sub-partition overlap their exponentials with
 //                      the other's FMA-pipe work), with 4 both halves
 //   next 4 warps       dQ: read dQ out of TMEM, scale, stage, reduce-add
-//   next warp          MMA issuer (one thread)
+//   next warp          MMA issuer (converged warp; an elected lane issues)
 //   last warp          TMA producer: K, V once; {Q_t, lse2_t, D_t} in a 2-stage
 //                      ring, dO_t in one buffer (its last reader, dV, runs early
 //                      in a tile and its next reader, dP^T, late in the previous one)
