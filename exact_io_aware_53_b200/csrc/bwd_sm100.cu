@@ -245,6 +245,45 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+
+    // Epilogue of dV (which = 0, staged in the K, V buffers) or dK (which = 1, in
+    // the Q buffers), both free once dkdv_done has completed.  A warp holds key
+    // rows in its lanes and 32 columns per TMEM read; it writes its own 32 rows
+    // into 128-byte-swizzled [128 rows][32 columns] fp32 boxes and reads them back
+    // with the lanes along a row, so that each store covers whole rows (512 bytes
+    // at d = 128) instead of 16 bytes of 32 rows.  No other warp touches those
+    // rows, and the stores need no shared memory once issued.
+    auto store_rows = [&](int which, uint32_t lane_off, int row0, float f) {
+        uint8_t* stg = which == 0 ? sK : sQ;
+        const uint32_t col = which == 0 ? C::DV_COL : C::DK_COL;
+        const uint32_t l = static_cast<uint32_t>(row0 + lane);
+#pragma unroll
+        for (int cc = 0; cc < D; cc += 32) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + col + cc, v);
+            tmem_wait_ld();
+            uint8_t* box = stg + (cc / 32) * (BKV * 128);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<uint4*>(box + sw128_offset(l, k)) =
+                    make_uint4(__float_as_uint(__uint_as_float(v[4 * k]) * f), __float_as_uint(__uint_as_float(v[4 * k + 1]) * f),
+                               __float_as_uint(__uint_as_float(v[4 * k + 2]) * f), __float_as_uint(__uint_as_float(v[4 * k + 3]) * f));
+        }
+        __syncwarp();
+        constexpr int LPR = D / 4;       // lanes per row (16 bytes each)
+        constexpr int RPI = 32 / LPR;    // rows per store instruction
+        const int sub = lane / LPR;
+        const int cgp = lane % LPR;      // columns 4 cgp .. 4 cgp + 3
+        const uint8_t* src = stg + (cgp / 8) * (BKV * 128);
+        float* dst = (which == 0 ? p.dv : p.dk) + static_cast<size_t>(bh) * N * D + 4 * cgp;
+#pragma unroll 4
+        for (int rr = 0; rr < 32; rr += RPI) {
+            const uint32_t r = static_cast<uint32_t>(row0 + rr + sub);
+            const int key = j * BKV + static_cast<int>(r);
+            const uint4 x = *reinterpret_cast<const uint4*>(src + sw128_offset(r, cgp % 8));
+            if (key < N) *reinterpret_cast<uint4*>(dst + static_cast<size_t>(key) * D) = x;
+        }
+    };
     if (warp == LOAD_WARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -543,26 +582,13 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             tc_fence_before();
             mbar_arrive(ds_ready);
         }
-        // epilogue: dV rows (times 256 / keep_t under dropout); with 8 warps the two
-        // warps of a quadrant take half the columns each
+        // epilogue: dV rows (times 256 / keep_t under dropout); with 8 warps the
+        // warps of query half 1 stage the dK rows (times scale) at the same time,
+        // while the dQ warps finish the last dQ
         if (ok && warp_wait(dkdv_done, 0, p.ctl)) {
             tc_fence_after();
-            const float f = DROPOUT ? p.keep_scale : 1.f;
-            float* dst = p.dv + (static_cast<size_t>(bh) * N + key) * D;
-            constexpr int COLS = D / (SMW / 4);
-#pragma unroll
-            for (int cc = h0 * COLS; cc < h0 * COLS + COLS; cc += 32) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_off + C::DV_COL + cc, v);
-                tmem_wait_ld();
-                if (key < N) {
-                    float4* d4 = reinterpret_cast<float4*>(dst + cc);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        d4[e] = make_float4(__uint_as_float(v[4 * e]) * f, __uint_as_float(v[4 * e + 1]) * f,
-                                            __uint_as_float(v[4 * e + 2]) * f, __uint_as_float(v[4 * e + 3]) * f);
-                }
-            }
+            const bool dk_rows = SMW == 8 && h0 == 1;
+            store_rows(dk_rows ? 1 : 0, lane_off, quad * 32, dk_rows ? p.scale : (DROPOUT ? p.keep_scale : 1.f));
         }
     } else {
         // ------------------------------------------------------------ dQ (4 warps)
@@ -647,26 +673,13 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             }
 
         }
-        if (issuer) bulk_wait_group0();
-        // epilogue: dK rows (lanes = key rows)
-        if (ok && warp_wait(dkdv_done, 0, p.ctl)) {
+        // the staging buffers are read: the reduce-adds themselves complete in L2
+        // before the grid does
+        if (issuer) bulk_wait_group_read0();
+        // epilogue (4 softmax warps): dK rows (lanes = key rows)
+        if (SMW == 4 && ok && warp_wait(dkdv_done, 0, p.ctl)) {
             tc_fence_after();
-            const int key = j * BKV + wq * 32 + lane;
-            float* dst = p.dk + (static_cast<size_t>(bh) * N + key) * D;
-#pragma unroll
-            for (int cc = 0; cc < D; cc += 32) {
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_off + C::DK_COL + cc, v);
-                tmem_wait_ld();
-                if (key < N) {
-                    float4* d4 = reinterpret_cast<float4*>(dst + cc);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        d4[e] = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
-                                            __uint_as_float(v[4 * e + 2]) * p.scale,
-                                            __uint_as_float(v[4 * e + 3]) * p.scale);
-                }
-            }
+            store_rows(1, lane_off, wq * 32, p.scale);
         }
     }
 
