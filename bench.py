@@ -869,7 +869,7 @@ def run_fp8(args, w):
     bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak = bf16 * FP8_OVER_BF16
     achieved = fl / (ms_local / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "decode_partial_kernel (e4m3, direct output)", "achieved": achieved,
+    roofline = {"bound": "tensor", "kernel": "fwd_kernel<128, causal, e4m3> (persistent, kind::f8f6f4)", "achieved": achieved,
                 "peak": peak, "unit": UNIT, "frac": achieved / peak,
                 "peak_source": "bf16_tflops %s x %.1f (nominal fp8 : bf16 ratio)" % (peak_src, FP8_OVER_BF16),
                 "frac_of_bf16_peak": achieved / bf16, "algorithmic_flops_per_launch": fl, "ms_per_launch": ms_local,

@@ -109,6 +109,21 @@ int encode_3d(CUtensorMap* m, CUtensorMapDataType dt, int elem_bytes, const void
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// e4m3 K of [BH][N][128] bytes (N a multiple of 16) as 5-D {128, 2, 4, 2, BH*N/16}
+// over (byte, f, q, h, b) with row = 16 b + 4 q + 2 h + f; box {128, 2, 4, 2, 8}:
+// one 128-row tile laid out as rows 16 b + 8 h + 2 q + f
+int encode_k_perm(CUtensorMap* m, const void* ptr, uint64_t BH, uint64_t N)
+{
+    cuuint64_t dims[5] = {128, 2, 4, 2, BH * N / 16};
+    cuuint64_t strides[4] = {128, 4 * 128, 2 * 128, 16 * 128};
+    cuuint32_t box[5] = {128, 2, 4, 2, 8};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_shape(int B, int H, int N, int d, float scale, int causal)
@@ -211,30 +226,11 @@ int fa_set_fwd_queue_words(int n)
     return FA_OK;
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, float scale,
-           int causal, void* stream)
+// Persistent grid, work queue and dispatch grouping of the square forward
+// (bf16 or e4m3 inputs, bytes_per_elem of each).
+static int fwd_grid(FwdParams& p, uint64_t BH, int N, int d, int causal, size_t bytes_per_elem)
 {
-    g_last_launches = 0;
-    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-    int st = check_shape(B, H, N, d, scale, causal);
-    if (st != FA_OK) return st;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
-    if ((st = get_encoder()) != FA_OK) return st;
-    FwdParams p;
-    std::memset(&p, 0, sizeof(p));
-    const uint64_t BH = static_cast<uint64_t>(B) * H;
-    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, o, d, N, BH, 64, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
-        return st;
-    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
-    p.lse = lse;
+    int st = FA_OK;
     p.BH = static_cast<int>(BH);
     p.N = N;
     p.n_pairs = (N + 255) / 256;
@@ -263,10 +259,39 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
             const int t0 = 2 * (p.n_pairs - 1 - v);
             work[v] = (t0 < n_t ? t0 + 1 : 0) + (t0 + 1 < n_t ? t0 + 2 : 0);
         }
-        p.group_heads = choose_group_heads(p.BH, p.n_pairs, work.data(), static_cast<size_t>(N) * d * 2 * 2);
+        p.group_heads = choose_group_heads(p.BH, p.n_pairs, work.data(), static_cast<size_t>(N) * d * bytes_per_elem * 2);
     }
+    return FA_OK;
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d, float scale,
+           int causal, void* stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    int st = check_shape(B, H, N, d, scale, causal);
+    if (st != FA_OK) return st;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+    if ((st = get_encoder()) != FA_OK) return st;
+    FwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    const uint64_t BH = static_cast<uint64_t>(B) * H;
+    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, o, d, N, BH, 64, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+        return st;
+    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+    p.lse = lse;
+    if ((st = fwd_grid(p, BH, N, d, causal, 2)) != FA_OK) return st;
     p.scale_log2 = scale * kLog2e;
-    st = cuda_status(launch_fwd_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    p.o_scale = 1.f;
+    st = cuda_status(launch_fwd_sm100(p, d, causal != 0, false, static_cast<cudaStream_t>(stream)));
     if (st == FA_OK) g_last_launches = 1;
     return st;
 }
@@ -448,32 +473,55 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
         if (!(f > 0.f) || !std::isfinite(f)) return FA_ERR_INVALID_ARG;
     if (!std::isfinite(scale * q_descale * k_descale * kLog2e)) return FA_ERR_INVALID_ARG;
     if (d != 128) return FA_ERR_UNSUPPORTED;
-    if (static_cast<long long>(B) * H > 65535) return FA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
     if ((st = get_encoder()) != FA_OK) return st;
-    DecodeParams p;
-    std::memset(&p, 0, sizeof(p));
     const uint64_t BH = static_cast<uint64_t>(B) * H;
-    // e4m3 rows of d = 128 bytes: one 128-byte swizzled box of 128 rows per tile
-    if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, d, N, BH, 128, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, d, N, BH, 128, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
-        (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, v, d, N, BH, 128, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
-        return st;
-    if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
-    p.o = static_cast<__nv_bfloat16*>(o);
-    p.lse = lse;
-    p.BH = static_cast<int>(BH);
-    p.Nq = N;
-    p.Nk = N;
-    p.n_split = 1;
-    p.tiles_per_split = (N + 127) / 128;
-    p.scale_log2 = scale * q_descale * k_descale * kLog2e;
-    p.o_scale = v_descale;
-    p.direct = 1;
-    st = cuda_status(launch_fp8_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    if (N % 16 == 0) {
+        // fa_fwd's persistent kernel with e4m3 MMAs; K is read through a permuted
+        // view of its rows (encode_k_perm), which needs N to be a multiple of 16
+        FwdParams p;
+        std::memset(&p, 0, sizeof(p));
+        // e4m3 rows of d = 128 bytes: one 128-byte swizzled box of 128 rows per tile;
+        // the output is bf16 as in fa_fwd
+        if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, d, N, BH, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+            (st = encode_k_perm(&p.tm_k, k, BH, N)) != FA_OK ||
+            (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, v, d, N, BH, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+            (st = encode_3d(&p.tm_o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, o, d, N, BH, 64, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+            return st;
+        if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+        p.lse = lse;
+        if ((st = fwd_grid(p, BH, N, d, causal, 1)) != FA_OK) return st;
+        p.scale_log2 = scale * q_descale * k_descale * kLog2e;
+        p.o_scale = v_descale;
+        st = cuda_status(launch_fwd_sm100(p, d, causal != 0, true, static_cast<cudaStream_t>(stream)));
+    } else {
+        // other N: the range kernel's e4m3 form, one range per Q tile
+        if (BH > 65535) return FA_ERR_UNSUPPORTED;
+        DecodeParams p;
+        std::memset(&p, 0, sizeof(p));
+        if ((st = encode_3d(&p.tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q, d, N, BH, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+            (st = encode_3d(&p.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k, d, N, BH, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+            (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, v, d, N, BH, 128, 128,
+                            CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+            return st;
+        if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
+        p.o = static_cast<__nv_bfloat16*>(o);
+        p.lse = lse;
+        p.BH = static_cast<int>(BH);
+        p.Nq = N;
+        p.Nk = N;
+        p.n_split = 1;
+        p.tiles_per_split = (N + 127) / 128;
+        p.scale_log2 = scale * q_descale * k_descale * kLog2e;
+        p.o_scale = v_descale;
+        p.direct = 1;
+        st = cuda_status(launch_fp8_sm100(p, d, causal != 0, static_cast<cudaStream_t>(stream)));
+    }
     if (st == FA_OK) g_last_launches = 1;
     return st;
 }

@@ -180,16 +180,19 @@ __device__ int queue_next(unsigned long long* word, unsigned int ticket, int tot
     return -1;
 }
 
-template <int D>
+template <int D, bool FP8>
 struct Cfg {
-    static constexpr int NDC = D / 64;              // 128-byte swizzle boxes per row
-    static constexpr int BOX_BYTES = 128 * 128;     // 128 rows x 64 bf16
+    static constexpr int NDC = FP8 ? 1 : D / 64;    // 128-byte swizzle boxes per input row
+    static constexpr int BOX_BYTES = 128 * 128;     // 128 rows x 128 bytes
     static constexpr int TILE_BYTES = NDC * BOX_BYTES;
-    static constexpr int STAGES = (D == 128) ? 4 : 8;
+    static constexpr int OUT_NDC = D / 64;          // boxes per bf16 output row
+    static constexpr int STG_BYTES = OUT_NDC * BOX_BYTES;
+    static constexpr int STAGES = (D == 128 && !FP8) ? 4 : 8;
+    static constexpr int KI = FP8 ? 32 : 16;        // K of one MMA instruction (32 bytes of a K-major row)
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = 2 * TILE_BYTES;
-    static constexpr int STG_OFF = KV_OFF + STAGES * TILE_BYTES;  // O staging tile (bf16, as Q's boxes)
-    static constexpr int BAR_OFF = STG_OFF + TILE_BYTES;
+    static constexpr int STG_OFF = KV_OFF + STAGES * TILE_BYTES;  // O staging tile (bf16)
+    static constexpr int BAR_OFF = STG_OFF + STG_BYTES;
     // q_full, q_empty, kv_full/empty[S], s_full, p_full, o_full, o_free [2],
     // item_full, item_empty [2], drain, stg_free
     static constexpr int NBARS = 2 + 2 * STAGES + 4 * 2 + 2 * 2 + 1 + 1;
@@ -241,10 +244,13 @@ __device__ __forceinline__ Item decode_item(const FwdParams& p, int item)
     return w;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8>
 __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdParams p)
 {
-    using C = Cfg<D>;
+    using C = Cfg<D, FP8>;
+    // e4m3 P must stay below its largest finite value (448): the running max is
+    // moved whenever a thread's share of a row sum passes 2^8
+    constexpr float SUM_LIM = FP8 ? 256.0f : SUM_LIMIT;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sQ = smem + C::Q_OFF;
@@ -347,9 +353,17 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                         }
                         mbar_arrive_expect_tx(&kv_full[s], C::TILE_BYTES);
                         const CUtensorMap* map = kind == 0 ? &p.tm_k : &p.tm_v;
-                        for (int c = 0; c < C::NDC; ++c)
-                            tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64,
-                                        j * BN, w.bh);
+                        if (FP8 && kind == 0) {
+                            // e4m3 K through a 5-D view of its rows (row = 16 b + 4 q + 2 h + f;
+                            // box order f, q, h, b): shared-memory row 16 b + 8 h + 2 q + f holds
+                            // key 16 b + 4 q + 2 h + f, so a thread's S columns pair up into
+                            // P words (N is a multiple of 16: blocks never straddle heads)
+                            tma_load_5d(sKV + s * C::TILE_BYTES, map, &kv_full[s], 0, 0, 0, 0, (w.bh * N + j * BN) / 16);
+                        } else {
+                            for (int c = 0; c < C::NDC; ++c)
+                                tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64,
+                                            j * BN, w.bh);
+                        }
                         ++it;
                     }
                 }
@@ -369,26 +383,32 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
         // diverged warp the same MMAs measured ~92 cycles each instead of ~65
         // (128 x 128 x 16, B200).
         {
-            constexpr uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
-            constexpr uint32_t idesc_o = idesc_bf16(BM, D, false, true);
+            constexpr uint32_t idesc_s = FP8 ? idesc_e4m3(BM, BN, false, false) : idesc_bf16(BM, BN, false, false);
+            constexpr uint32_t idesc_o = FP8 ? idesc_e4m3(BM, D, false, true) : idesc_bf16(BM, D, false, true);
             const uint32_t sQa = smem_u32(sQ);
             const uint32_t sKVa = smem_u32(sKV);
             auto issue_s = [&](int t, int stage) {
                 const uint32_t qa = sQa + t * C::TILE_BYTES;
                 const uint32_t kb = sKVa + stage * C::TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < D / C::KI; ++kk) {
                     const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                    mma_ss_elect(tmem + 128u * t, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                           idesc_s, kk > 0 ? 1u : 0u);
+                    const uint64_t ad = sdesc_sw128(qa + off, 16, 1024), bd = sdesc_sw128(kb + off, 16, 1024);
+                    if constexpr (FP8) mma_ss_f8_elect(tmem + 128u * t, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    else mma_ss_elect(tmem + 128u * t, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_o = [&](int t, int stage, int j) {
                 const uint32_t vb = sKVa + stage * C::TILE_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_ts_elect(tmem + C::O_COL + D * t, tmem + 128u * t + kk * 8,
-                           sdesc_sw128(vb + kk * 2048, C::BOX_BYTES, 1024), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < BN / C::KI; ++kk) {
+                    // V is MN-major: KI key rows of 128 bytes per instruction; P (bf16
+                    // pairs or e4m3 quadruples) takes 8 TMEM columns per instruction
+                    const uint64_t bd = sdesc_sw128(vb + kk * C::KI * 128, C::BOX_BYTES, 1024);
+                    const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (FP8) mma_ts_f8_elect(tmem + C::O_COL + D * t, tmem + 128u * t + kk * 8, bd, idesc_o, acc);
+                    else mma_ts_elect(tmem + C::O_COL + D * t, tmem + 128u * t + kk * 8, bd, idesc_o, acc);
+                }
             };
             int it = 0;                 // K/V ring slots consumed
             int pc[2] = {0, 0};         // key tiles of Q tile t done (s_full / p_full phases)
@@ -513,7 +533,8 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                         for (int n = 0; n < 16; ++n)
     #pragma unroll
                             for (int e = 0; e < 2; ++e) {
-                                const int c = 8 * n + cg + e;
+                                // the key of S column 8n + cg + e (permuted for e4m3)
+                                const int c = FP8 ? 16 * (n >> 1) + 2 * cg + 2 * (n & 1) + e : 8 * n + cg + e;
                                 if (c > lim0) s[4 * n + e] = -INFINITY;
                                 if (c > lim1) s[4 * n + 2 + e] = -INFINITY;
                             }
@@ -562,13 +583,25 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                         const float2 pb = make_float2(ex2_approx(xb.x), ex2_fma(xb.y));
                         sum0 = fadd2(sum0, pa);
                         sum1 = fadd2(sum1, pb);
-                        // packed pairs in the 16x128b layout: column 4n + i%4
-                        pk[2 * n] = pack_bf16x2(pa.x, pa.y);
-                        pk[2 * n + 1] = pack_bf16x2(pb.x, pb.y);
+                        if constexpr (FP8) {
+                            // e4m3 pairs; groups 2n', 2n' + 1 of a row make one word
+                            const uint32_t h0 = pack_e4m3x2(pa.x, pa.y), h1 = pack_e4m3x2(pb.x, pb.y);
+                            if (n & 1) {
+                                pk[n - 1] |= h0 << 16;
+                                pk[n] |= h1 << 16;
+                            } else {
+                                pk[n] = h0;
+                                pk[n + 1] = h1;
+                            }
+                        } else {
+                            // packed pairs in the 16x128b layout: column 4n + i%4
+                            pk[2 * n] = pack_bf16x2(pa.x, pa.y);
+                            pk[2 * n + 1] = pack_bf16x2(pb.x, pb.y);
+                        }
                     }
                     ts0 = sum0.x + sum0.y;
                     ts1 = sum1.x + sum1.y;
-                    if (redo || j == 0 || !__any_sync(0xffffffffu, !(ts0 <= SUM_LIMIT && ts1 <= SUM_LIMIT))) break;
+                    if (redo || j == 0 || !__any_sync(0xffffffffu, !(ts0 <= SUM_LIM && ts1 <= SUM_LIM))) break;
                     // a score far above m in some row of this warp: take the true row
                     // maxima (the whole warp, so TMEM access stays warp-wide)
                     redo = true;
@@ -601,7 +634,15 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                         tmem_st_16x256b_x4(o_addr + cc, o);
                     }
                 }
-                tmem_st_16x128b_x16(s_addr, pk);
+                if constexpr (FP8) {
+                    // TMEM column c of P holds keys 4c .. 4c + 3 (of V's rows) and
+                    // thread i writes column 4n' + i % 4 (16x128b).  K's rows are
+                    // loaded permuted (see the producer), so that this thread's
+                    // S columns of groups 2n', 2n' + 1 are exactly those four keys.
+                    tmem_st_16x128b_x8(s_addr, pk);
+                } else {
+                    tmem_st_16x128b_x16(s_addr, pk);
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&p_full[t]);
@@ -623,7 +664,7 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
                     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
                     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-                    const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+                    const float inv0 = p.o_scale / l0, inv1 = p.o_scale / l1;
                     {
                         // LSE of the warp's 16 rows as one contiguous 64-byte store: lane L
                         // (< 16) writes row base + L, held by lane 4 (L % 8)
@@ -673,7 +714,7 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                             __threadfence_block();
                             *stg_count = 0u;
                             fence_proxy_async_smem();
-                            for (int c = 0; c < C::NDC; ++c)
+                            for (int c = 0; c < C::OUT_NDC; ++c)
                                 tma_store_3d(&p.tm_o, sSTG + c * C::BOX_BYTES, c * 64, w.q0 + t * BM, w.bh);
                             bulk_commit_group();
                             bulk_wait_group_read0();
@@ -696,11 +737,11 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool FP8 = false>
 cudaError_t launch(const FwdParams& p, cudaStream_t stream)
 {
-    using C = Cfg<D>;
-    auto kern = fwd_kernel<D, CAUSAL>;
+    using C = Cfg<D, FP8>;
+    auto kern = fwd_kernel<D, CAUSAL, FP8>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     kern<<<p.n_ctas, NTHREADS, C::SMEM_BYTES, stream>>>(p);
@@ -709,8 +750,12 @@ cudaError_t launch(const FwdParams& p, cudaStream_t stream)
 
 }  // namespace fwdk
 
-cudaError_t launch_fwd_sm100(const FwdParams& p, int d, bool causal, cudaStream_t stream)
+cudaError_t launch_fwd_sm100(const FwdParams& p, int d, bool causal, bool fp8, cudaStream_t stream)
 {
+    if (fp8) {
+        if (d != 128) return cudaErrorInvalidValue;
+        return causal ? fwdk::launch<128, true, true>(p, stream) : fwdk::launch<128, false, true>(p, stream);
+    }
     if (d == 128) return causal ? fwdk::launch<128, true>(p, stream) : fwdk::launch<128, false>(p, stream);
     return causal ? fwdk::launch<64, true>(p, stream) : fwdk::launch<64, false>(p, stream);
 }

@@ -19,10 +19,12 @@ void set_last_launch_count(int n);
 
 // ---------------------------------------------------------------- bf16 forward
 struct FwdParams {
-    CUtensorMap tm_q;  // 3-D {d, N, B*H}, box {64, 128, 1}, 128-byte swizzle
+    // 3-D {d, N, B*H}, 128-byte swizzle; box {64, 128, 1} for bf16, {128, 128, 1}
+    // for e4m3 (one 128-byte box per row)
+    CUtensorMap tm_q;
     CUtensorMap tm_k;
     CUtensorMap tm_v;
-    CUtensorMap tm_o;  // the output, same layout; TMA store target
+    CUtensorMap tm_o;  // the output (bf16, box {64, 128, 1}); TMA store target
     float* lse;        // [B*H][N]
     int BH;
     int N;
@@ -31,11 +33,12 @@ struct FwdParams {
     int n_ctas;        // persistent CTAs, <= min(SMs, B*H*n_pairs)
     int queue_slot;    // work queue word of this launch, < 64
     unsigned int ticket;  // launch number on this device, low 16 bits
-    float scale_log2;  // scale * log2(e)
+    float scale_log2;  // scale * log2(e) (e4m3: times the q and k descales)
+    float o_scale;     // factor on O / l: 1, or the v descale for e4m3
     WaitCtl ctl;
 };
 
-cudaError_t launch_fwd_sm100(const FwdParams& p, int d, bool causal, cudaStream_t stream);
+cudaError_t launch_fwd_sm100(const FwdParams& p, int d, bool causal, bool fp8, cudaStream_t stream);
 
 // Heads per dispatch group for a causal grid: work[v] is the relative cost of
 // a CTA at level v (levels in dispatch order), bytes_per_head the data a head's

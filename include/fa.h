@@ -279,9 +279,12 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, c
  *   Scores are exact products accumulated in fp32; the softmax weights P are
  *   rounded to e4m3 (relative error <= 2^-4) before P V, so O carries an
  *   error up to 2^-4 * sum_j P_ij |v_j| beyond the bf16 path's.
- * One kernel is enqueued on `stream`; nothing is allocated.  Errors as for
- * fa_fwd, plus FA_ERR_INVALID_ARG for a descale that is not finite and
- * positive, FA_ERR_UNSUPPORTED for d != 128 or B*H > 65535.
+ * For N a multiple of 16 the kernel is fa_fwd's (persistent CTAs, the same
+ * work queue) with e4m3 tensor-core instructions; otherwise one CTA per
+ * 128-row query tile.  One kernel is enqueued on `stream`; nothing is
+ * allocated.  Errors as for fa_fwd, plus FA_ERR_INVALID_ARG for a descale that
+ * is not finite and positive, FA_ERR_UNSUPPORTED for d != 128 or (N not a
+ * multiple of 16) B*H > 65535.
  */
 int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, float q_descale, float k_descale,
                float v_descale, int B, int H, int N, int d, float scale, int causal, void* stream);

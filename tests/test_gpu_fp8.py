@@ -52,8 +52,14 @@ def _run(fa_lib, x, causal, scale):
 
 
 @pytest.mark.parametrize("B,H,N,causal,gain", [
-    (1, 1, 1, False, 1.0), (1, 2, 128, True, 1.0), (2, 1, 200, False, 1.0), (1, 2, 513, True, 1.0),
+    # N not a multiple of 16: one CTA per query tile
+    (1, 1, 1, False, 1.0), (2, 1, 200, False, 1.0), (1, 2, 513, True, 1.0),
     (1, 1, 1000, False, 1.0), (1, 2, 700, True, 2.0), (2, 2, 383, False, 2.0),
+    # N a multiple of 16: the persistent kernel with K read through its permuted
+    # view; 400 = 3 * 128 + 16 leaves a last key tile that reaches into the next
+    # head's rows (masked), 16 a single short tile
+    (1, 2, 128, True, 1.0), (2, 2, 400, True, 1.0), (2, 2, 400, False, 2.0), (1, 3, 16, False, 1.0),
+    (1, 1, 1024, True, 1.0), (3, 1, 768, False, 1.0),
 ])
 def test_fp8_matches_oracle_within_the_derived_bound(fa_lib, B, H, N, causal, gain):
     x = make_fp8_inputs((B, H, N, 128), seed=N * 5 + causal, gain=gain)
@@ -67,11 +73,12 @@ def test_fp8_matches_oracle_within_the_derived_bound(fa_lib, B, H, N, causal, ga
     assert np.all(err <= bound), (float(err.max()), float((err - bound).max()))
 
 
-def test_fp8_descales_are_applied(fa_lib):
+@pytest.mark.parametrize("N", [300, 320])
+def test_fp8_descales_are_applied(fa_lib, N):
     # q's descale doubled and k's halved leave every score unchanged (powers
     # of two are exact), so the result is bit for bit the same; v's descale
     # doubled doubles O exactly
-    x = make_fp8_inputs((1, 2, 300, 128), seed=3)
+    x = make_fp8_inputs((1, 2, N, 128), seed=3)
     qd, kd, vd = x["descales"]
     o1, l1 = _run(fa_lib, x, False, 0.1)
     o2, l2 = _run(fa_lib, dict(x, descales=(qd * 2.0, kd / 2.0, vd)), False, 0.1)
@@ -86,8 +93,8 @@ def test_fp8_workload_sampled_rows(fa_lib):
     o, lse = _run(fa_lib, x, w.causal, w.scale)
     assert fa_lib.last_launch_count() == 1
     dq = _dequant(x)
-    rows = [0, 1, 127, 128, 1000, 2047, 3071, 4095]
-    for b, h in ((0, 0), (3, 15)):
+    # head (0, 0) on sampled rows, head (3, 15) whole
+    for b, h, rows in ((0, 0, [0, 1, 127, 128, 1000, 2047, 3071, 4095]), (3, 15, list(range(w.N)))):
         sl = (slice(b, b + 1), slice(h, h + 1))
         qh, kh, vh = (dq[n][sl] for n in ("q", "k", "v"))
         ro, rlse = oracle.attn_fwd_rows(qh[0, 0], kh[0, 0], vh[0, 0], 0, w.N, w.scale, w.causal)
