@@ -576,11 +576,13 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                     float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
     #pragma unroll
                     for (int n = 0; n < 16; ++n) {
-                        // one exponential in four on the FMA pipe, beside MUFU
+                        // one exponential in four on the FMA pipe, beside MUFU (bf16; the
+                        // e4m3 path's conversions already load the FMA pipe, so there all
+                        // four go to MUFU: 2% faster measured)
                         const float2 xa = ffma2(make_float2(s[4 * n], s[4 * n + 1]), c2, n0);
                         const float2 xb = ffma2(make_float2(s[4 * n + 2], s[4 * n + 3]), c2, n1);
                         const float2 pa = make_float2(ex2_approx(xa.x), ex2_approx(xa.y));
-                        const float2 pb = make_float2(ex2_approx(xb.x), ex2_fma(xb.y));
+                        const float2 pb = make_float2(ex2_approx(xb.x), FP8 ? ex2_approx(xb.y) : ex2_fma(xb.y));
                         sum0 = fadd2(sum0, pa);
                         sum1 = fadd2(sum1, pb);
                         if constexpr (FP8) {
