@@ -185,7 +185,9 @@ def oracle_sample(w, heads: int, seed: int):
     t0 = time.perf_counter()
     oracle.attn_fwd(q, k, v, w.scale, w.causal)
     if w.backward:
-        oracle.attn_bwd(q, k, v, do, w.scale, w.causal)
+        # the oracle's one-head backward spreads a head's rows over the threads
+        for h in range(heads):
+            oracle.attn_bwd_head(q[0, h], k[0, h], v[0, h], do[0, h], w.scale, w.causal)
     dt = time.perf_counter() - t0
     per_head = (w.flops_fwd() + (w.flops_bwd() if w.backward else 0.0)) / (w.B * w.H)
     return dt, per_head * heads, oracle.num_threads()
