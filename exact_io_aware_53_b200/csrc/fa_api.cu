@@ -761,6 +761,60 @@ size_t fa_attention_host_arena_bytes(int B, int H, int N, int d)
     return 5 * up(E * 2) + 3 * up(E * 4) + up(R * 4) + up(fa_bwd_workspace_bytes(B, H, N, d));
 }
 
+}  // extern "C"
+
+namespace {
+
+// fa_attention_host splits the heads into chunks and runs three stages on three
+// streams: host-to-device copies of chunk c on a copy-in stream, the forward and
+// backward of chunk c on the caller's stream, device-to-host copies of chunk c on
+// a copy-out stream.  Heads are independent in both passes, so the copies of one
+// chunk overlap the compute of the next and, on a full-duplex link, the two copy
+// directions overlap each other.  The two copy streams and the events that order
+// the stages are created once per device and kept until the process exits.
+constexpr int kHostMaxChunks = 8;
+constexpr int kHostMaxDevices = 64;
+
+struct HostPipe {
+    cudaStream_t in = nullptr;
+    cudaStream_t out = nullptr;
+    cudaEvent_t start = nullptr, end = nullptr;
+    cudaEvent_t in_done[kHostMaxChunks] = {};
+    cudaEvent_t comp_done[kHostMaxChunks] = {};
+    bool ready = false;
+};
+
+std::mutex g_pipe_mu;  // held while a call enqueues: the streams and events are shared
+HostPipe g_pipe[kHostMaxDevices];
+
+// The current device's pipe, created on first use; call with g_pipe_mu held.
+int host_pipe(HostPipe** out)
+{
+    int dev = 0;
+    int st = cuda_status(cudaGetDevice(&dev));
+    if (st != FA_OK) return st;
+    if (dev < 0 || dev >= kHostMaxDevices) return FA_ERR_UNSUPPORTED;
+    HostPipe& hp = g_pipe[dev];
+    if (!hp.ready) {
+        if ((st = cuda_status(cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking))) != FA_OK ||
+            (st = cuda_status(cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking))) != FA_OK ||
+            (st = cuda_status(cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming))) != FA_OK ||
+            (st = cuda_status(cudaEventCreateWithFlags(&hp.end, cudaEventDisableTiming))) != FA_OK)
+            return st;
+        for (int c = 0; c < kHostMaxChunks; ++c)
+            if ((st = cuda_status(cudaEventCreateWithFlags(&hp.in_done[c], cudaEventDisableTiming))) != FA_OK ||
+                (st = cuda_status(cudaEventCreateWithFlags(&hp.comp_done[c], cudaEventDisableTiming))) != FA_OK)
+                return st;
+        hp.ready = true;
+    }
+    *out = &hp;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const void* h_dO, void* h_o, float* h_lse,
                       float* h_dq, float* h_dk, float* h_dv, void* arena, size_t arena_bytes, int B, int H, int N,
                       int d, float scale, int causal, void* stream)
@@ -776,43 +830,94 @@ int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const v
     const size_t R = static_cast<size_t>(B) * H * N;
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     char* a = static_cast<char*>(arena);
-    void* q = a;
+    char* q = a;
     a += up(E * 2);
-    void* k = a;
+    char* k = a;
     a += up(E * 2);
-    void* v = a;
+    char* v = a;
     a += up(E * 2);
-    void* dO = a;
+    char* dO = a;
     a += up(E * 2);
-    void* o = a;
+    char* o = a;
     a += up(E * 2);
-    float* dq = reinterpret_cast<float*>(a);
+    char* dq = a;
     a += up(E * 4);
-    float* dk = reinterpret_cast<float*>(a);
+    char* dk = a;
     a += up(E * 4);
-    float* dv = reinterpret_cast<float*>(a);
+    char* dv = a;
     a += up(E * 4);
-    float* lse = reinterpret_cast<float*>(a);
+    char* lse = a;
     a += up(R * 4);
     void* ws = a;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const void* srcs[4] = {h_q, h_k, h_v, h_dO};
-    void* dsts[4] = {q, k, v, dO};
-    for (int i = 0; i < 4; ++i)
-        if ((st = cuda_status(cudaMemcpyAsync(dsts[i], srcs[i], E * 2, cudaMemcpyHostToDevice, s))) != FA_OK) return st;
-    if ((st = fa_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, stream)) != FA_OK) return st;
-    const int n_fwd = g_last_launches;
-    if ((st = fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, ws, B, H, N, d, scale, causal, stream)) != FA_OK) return st;
-    const int n_bwd = g_last_launches;
-    struct {
-        void* dst;
-        const void* src;
-        size_t bytes;
-    } back[5] = {{h_o, o, E * 2}, {h_lse, lse, R * 4}, {h_dq, dq, E * 4}, {h_dk, dk, E * 4}, {h_dv, dv, E * 4}};
-    for (auto& b : back)
-        if (b.dst && (st = cuda_status(cudaMemcpyAsync(b.dst, b.src, b.bytes, cudaMemcpyDeviceToHost, s))) != FA_OK)
+
+    // chunks of G heads, G a multiple of 4 so that every chunk's LSE slice
+    // starts on a 16-byte boundary (the bf16 and fp32 rows always do)
+    const int BH = B * H;
+    int G = (BH + kHostMaxChunks - 1) / kHostMaxChunks;
+    G = (G + 3) / 4 * 4;
+    const int n_chunks = (BH + G - 1) / G;
+
+    std::lock_guard<std::mutex> lk(g_pipe_mu);
+    HostPipe* hp = nullptr;
+    if ((st = host_pipe(&hp)) != FA_OK) return st;
+    // both copy streams start after the work already on the caller's stream
+    if ((st = cuda_status(cudaEventRecord(hp->start, s))) != FA_OK ||
+        (st = cuda_status(cudaStreamWaitEvent(hp->in, hp->start, 0))) != FA_OK ||
+        (st = cuda_status(cudaStreamWaitEvent(hp->out, hp->start, 0))) != FA_OK)
+        return st;
+    const char* hsrc[4] = {static_cast<const char*>(h_q), static_cast<const char*>(h_k),
+                           static_cast<const char*>(h_v), static_cast<const char*>(h_dO)};
+    char* dsrc[4] = {q, k, v, dO};
+    for (int c = 0; c < n_chunks; ++c) {
+        const size_t h0 = static_cast<size_t>(c) * G;
+        const size_t gh = std::min<size_t>(G, BH - h0);
+        const size_t off = h0 * N * d * 2, bytes = gh * N * d * 2;
+        for (int i = 0; i < 4; ++i)
+            if ((st = cuda_status(cudaMemcpyAsync(dsrc[i] + off, hsrc[i] + off, bytes, cudaMemcpyHostToDevice,
+                                                  hp->in))) != FA_OK)
+                return st;
+        if ((st = cuda_status(cudaEventRecord(hp->in_done[c], hp->in))) != FA_OK) return st;
+    }
+    int launches = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+        const size_t h0 = static_cast<size_t>(c) * G;
+        const int gh = static_cast<int>(std::min<size_t>(G, BH - h0));
+        const size_t e2 = h0 * N * d * 2, e4 = h0 * N * d * 4, r4 = h0 * N * 4;
+        if ((st = cuda_status(cudaStreamWaitEvent(s, hp->in_done[c], 0))) != FA_OK) return st;
+        // the chunk is gh heads of one batch: heads are independent in both passes
+        if ((st = fa_fwd(q + e2, k + e2, v + e2, o + e2, reinterpret_cast<float*>(lse + r4), 1, gh, N, d, scale,
+                         causal, stream)) != FA_OK)
             return st;
-    g_last_launches = n_fwd + n_bwd;
+        launches += g_last_launches;
+        if ((st = fa_bwd(q + e2, k + e2, v + e2, o + e2, reinterpret_cast<const float*>(lse + r4), dO + e2,
+                         reinterpret_cast<float*>(dq + e4), reinterpret_cast<float*>(dk + e4),
+                         reinterpret_cast<float*>(dv + e4), ws, 1, gh, N, d, scale, causal, stream)) != FA_OK)
+            return st;
+        launches += g_last_launches;
+        if ((st = cuda_status(cudaEventRecord(hp->comp_done[c], s))) != FA_OK ||
+            (st = cuda_status(cudaStreamWaitEvent(hp->out, hp->comp_done[c], 0))) != FA_OK)
+            return st;
+        const size_t n2 = static_cast<size_t>(gh) * N * d * 2, n4 = n2 * 2, nr = static_cast<size_t>(gh) * N * 4;
+        struct {
+            void* dst;
+            const char* src;
+            size_t bytes;
+        } back[5] = {{h_o ? static_cast<char*>(h_o) + e2 : nullptr, o + e2, n2},
+                     {h_lse ? reinterpret_cast<char*>(h_lse) + r4 : nullptr, lse + r4, nr},
+                     {h_dq ? reinterpret_cast<char*>(h_dq) + e4 : nullptr, dq + e4, n4},
+                     {h_dk ? reinterpret_cast<char*>(h_dk) + e4 : nullptr, dk + e4, n4},
+                     {h_dv ? reinterpret_cast<char*>(h_dv) + e4 : nullptr, dv + e4, n4}};
+        for (auto& bk : back)
+            if (bk.dst &&
+                (st = cuda_status(cudaMemcpyAsync(bk.dst, bk.src, bk.bytes, cudaMemcpyDeviceToHost, hp->out))) != FA_OK)
+                return st;
+    }
+    // the caller's stream completes after the last copy back
+    if ((st = cuda_status(cudaEventRecord(hp->end, hp->out))) != FA_OK ||
+        (st = cuda_status(cudaStreamWaitEvent(s, hp->end, 0))) != FA_OK)
+        return st;
+    g_last_launches = launches;
     return FA_OK;
 }
 

@@ -156,9 +156,19 @@ size_t fa_attention_host_arena_bytes(int B, int H, int N, int d);
  * (bf16, host memory -- pinned for asynchronous copies) into `arena` (device,
  * fa_attention_host_arena_bytes bytes, 256-byte aligned), runs fa_fwd and
  * fa_bwd there, and copies o (bf16), lse, dq, dk, dv (fp32) back to the host
- * buffers, all on `stream`.  Returns after enqueueing; the host buffers are
- * valid once the stream is synchronised.  Any output pointer may be NULL to
- * skip that copy back.
+ * buffers.  The heads are processed in up to 8 chunks (a multiple of 4 heads
+ * each; heads are independent in both passes): chunk c is copied in on a
+ * library-owned copy-in stream, computed on `stream`, and copied back on a
+ * library-owned copy-out stream, ordered by events, so that the copies of one
+ * chunk overlap the compute and the copies of the others.  The two copy
+ * streams and their events are created on the first call on a device and kept
+ * until the process exits; calls from several host threads are serialised
+ * while they enqueue.  The copies start after the work already enqueued on
+ * `stream`, and `stream` waits for the last copy back, so the host buffers
+ * are valid once `stream` is synchronised.  Returns after enqueueing.  Any
+ * output pointer may be NULL to skip that copy back.  The results equal those
+ * of fa_fwd and fa_bwd on the whole tensors (dq up to the order of its fp32
+ * additions).
  */
 int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const void* h_dO, void* h_o,
                       float* h_lse, float* h_dq, float* h_dk, float* h_dv, void* arena, size_t arena_bytes, int B,
