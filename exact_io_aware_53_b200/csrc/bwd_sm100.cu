@@ -9,9 +9,15 @@
 //   dS^T = P^T o (dP^T - D_t)                        D_t = <dO, O> per query row
 //   dV += P^T dO_t,  dK += dS^T Q_t,  dQ_t = dS K_j   (dK, dQ times scale)
 //
-// One CTA owns 128 keys (K_j, V_j stay in shared memory) and walks the
-// 128-row query tiles t that see them, so every tensor-core instruction is
-// 128 rows by 128 (or by d) columns.
+// One CTA owns 128 keys at a time (K_j, V_j stay in shared memory) and walks
+// the 128-row query tiles t that see them, so every tensor-core instruction is
+// 128 rows by 128 (or by d) columns.  For d = 64 the CTAs are persistent: each
+// takes several (head, key tile) items in turn, with two K, V buffers, and the
+// query-tile pipeline runs on from one item's last tile into the next item's
+// first (barrier phases, Q stages and TMEM regions follow the CTA's running
+// tile count T); the dQ warps write an item's dV and dK (TMEM -> swizzled
+// shared boxes -> TMA tile stores) while the other warps start the next item.
+// For d = 128 shared memory holds one K, V buffer and a CTA runs one item.
 //
 // TMEM (512 columns): two 128-column regions R0, R1, then dV and dK (d columns
 // each) and, for d = 64, dQ (64 columns).  Tile t uses X = R[t & 1] for
@@ -78,11 +84,16 @@ constexpr int BOX = 128 * 128;  // 128 rows x 128 B (64 bf16)
 
 template <int D>
 struct Cfg {
+    // d = 64: persistent CTAs (one per SM) walk several (head, key tile) items,
+    // with two K, V buffers so that the next item's keys load during this one;
+    // d = 128 fills shared memory with one buffer and runs one CTA per item
+    static constexpr bool PERSIST = D == 64;
+    static constexpr int KV_BUFS = PERSIST ? 2 : 1;
     static constexpr int NDC = D / 64;  // 128-byte column boxes per row
     static constexpr int TILE = NDC * BOX;
-    static constexpr int K_OFF = 0;
+    static constexpr int K_OFF = 0;                        // buffer b: K at K_OFF + 2 b TILE, V after it
     static constexpr int V_OFF = K_OFF + TILE;
-    static constexpr int Q_OFF = V_OFF + TILE;             // Q_t, 2 stages
+    static constexpr int Q_OFF = KV_BUFS * 2 * TILE;       // Q_t, 2 stages
     static constexpr int DO_OFF = Q_OFF + QSTAGES * TILE;  // dO_t, 1 stage
     static constexpr int DS_OFF = DO_OFF + TILE;           // dS^T: 2 boxes of 64 query columns
     static constexpr int STG_OFF = DS_OFF + 2 * BOX;       // dQ staging
@@ -90,9 +101,12 @@ struct Cfg {
     // (64 of the d columns at a time)
     static constexpr int STG_ROWS = 128;
     static constexpr int STG_CHUNK = STG_ROWS * 128;
-    static constexpr int VEC_OFF = STG_OFF + 2 * STG_CHUNK;  // [stage][lse2 128 | delta 128]
+    // persistent: the dV epilogue's staging boxes ([128 keys][32 d] fp32, 128-byte swizzled)
+    static constexpr int EPI_OFF = STG_OFF + 2 * STG_CHUNK;
+    static constexpr int EPI_BYTES = PERSIST ? (D / 32) * BKV * 128 : 0;
+    static constexpr int VEC_OFF = EPI_OFF + EPI_BYTES;  // [stage][lse2 128 | delta 128]
     static constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
-    static constexpr int NBARS = 19;
+    static constexpr int NBARS = 24;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t DV_COL = 256;
@@ -194,19 +208,38 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     uint64_t* dqw_bar = bars + 15;  // the 4 dQ warps (128 threads)
     uint64_t* dp_read = bars + 16;  // the softmax warps hold dP^T of the tile in registers (Y is free)
     uint64_t* ds_free = bars + 17;  // the reduce-add staged in the dS^T buffer has read it
+    // persistent (d = 64): per K, V buffer full / free, and the previous item's dV,
+    // dK read out of TMEM by the dQ warps (their regions may then be overwritten)
+    uint64_t* kv_full_b[2] = {bars + 0, bars + 18};
+    uint64_t* kv_empty_b[2] = {bars + 19, bars + 20};
+    uint64_t* dv_free = bars + 21;
+    uint64_t* dk_free = bars + 22;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
 
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
-    // grouped longest-first order over (key tile, head): key tile 0 sees the
-    // most query tiles under the causal mask; a group's Q, dO and dQ share L2
-    int bh, j;
-    grouped_order(static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x), p.BH, p.n_kv_tiles, p.group_heads, bh, j);
     const int N = p.N;
     const int n_pad = p.n_kv_tiles * BKV;
     const int n_q = (N + BQ - 1) / BQ;
-    const int i_first = CAUSAL ? j : 0;
-    const int n_it = n_q - i_first;  // >= 1
+    // Items are (head, 128-key tile) pairs in the grouped longest-first order:
+    // key tile 0 sees the most query tiles under the causal mask, and a group's
+    // Q, dO and dQ share L2.  A persistent CTA takes items item0, item0 + stride,
+    // ...; otherwise the CTA has the one item of its grid position.
+    const int n_items = p.BH * p.n_kv_tiles;
+    const int item0 = C::PERSIST ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x);
+    const int stride = C::PERSIST ? static_cast<int>(gridDim.x) : n_items;
+    struct ItemInfo {
+        int bh, j;    // head, key tile
+        int i_first;  // first query tile that sees the keys
+        int n_it;     // query tiles walked (>= 1)
+    };
+    auto item_info = [&](int item) {
+        ItemInfo w;
+        grouped_order(item, p.BH, p.n_kv_tiles, p.group_heads, w.bh, w.j);
+        w.i_first = CAUSAL ? w.j : 0;
+        w.n_it = n_q - w.i_first;
+        return w;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
@@ -227,6 +260,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         mbar_init(drain, 1);
         mbar_init(dqw_bar, 128);
         mbar_init(ds_free, 1);
+        mbar_init(kv_full_b[1], 1);
+        mbar_init(kv_empty_b[0], 1);
+        mbar_init(kv_empty_b[1], 1);
+        mbar_init(dv_free, 128);
+        mbar_init(dk_free, 128);
         fence_mbar_init();
     }
     if (warp == MMA_WARP) {
@@ -253,7 +291,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     // with the lanes along a row, so that each store covers whole rows (512 bytes
     // at d = 128) instead of 16 bytes of 32 rows.  No other warp touches those
     // rows, and the stores need no shared memory once issued.
-    auto store_rows = [&](int which, uint32_t lane_off, int row0, float f) {
+    auto store_rows = [&](int which, uint32_t lane_off, int row0, float f, int bh, int j) {
         uint8_t* stg = which == 0 ? sK : sQ;
         const uint32_t col = which == 0 ? C::DV_COL : C::DK_COL;
         const uint32_t l = static_cast<uint32_t>(row0 + lane);
@@ -287,32 +325,42 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     if (warp == LOAD_WARP) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
-            for (int c = 0; c < C::NDC; ++c) {
-                tma_load_3d(sK + c * BOX, &p.tm_k, kv_full, c * 64, j * BKV, bh);
-                tma_load_3d(sV + c * BOX, &p.tm_v, kv_full, c * 64, j * BKV, bh);
-            }
-            const float* lse2_h = p.lse2 + static_cast<size_t>(bh) * n_pad;
-            const float* delta_h = p.delta + static_cast<size_t>(bh) * n_pad;
-            int nq = 0, ndo = 0;  // tiles issued: Q (with its row vectors), dO
+            int T = 0;                     // query tiles issued over all items
+            int nq = 0, ndo = 0, nkv = 0;  // loads issued: Q (with its row vectors), dO, K+V
             bool ok = true;
-            for (int t = 0; t < n_it && ok; ++t) {
-                const int s = t & 1;
-                const int i = i_first + t;
-                if (!(ok = mbar_wait(&q_empty[s], ((t >> 1) & 1) ^ 1, p.ctl))) break;
-                mbar_arrive_expect_tx(&q_full[s], C::TILE + 2 * BQ * 4);
-                for (int c = 0; c < C::NDC; ++c)
-                    tma_load_3d(sQ + s * C::TILE + c * BOX, &p.tm_q, &q_full[s], c * 64, i * BQ, bh);
-                bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &q_full[s]);
-                bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &q_full[s]);
-                ++nq;
-                if (!(ok = mbar_wait(do_empty, (t & 1) ^ 1, p.ctl))) break;
-                mbar_arrive_expect_tx(do_full, C::TILE);
-                for (int c = 0; c < C::NDC; ++c) tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, bh);
-                ++ndo;
+            for (int k = 0, item = item0; item < n_items && ok; ++k, item += stride) {
+                const ItemInfo w = item_info(item);
+                const int b = k & (C::KV_BUFS - 1);
+                // the buffer's previous item (k - 2) has been read and its dV stored
+                if (C::PERSIST && !(ok = mbar_wait(kv_empty_b[b], ((k >> 1) & 1) ^ 1, p.ctl))) break;
+                mbar_arrive_expect_tx(kv_full_b[b], 2 * C::TILE);
+                for (int c = 0; c < C::NDC; ++c) {
+                    tma_load_3d(sK + 2 * b * C::TILE + c * BOX, &p.tm_k, kv_full_b[b], c * 64, w.j * BKV, w.bh);
+                    tma_load_3d(sV + 2 * b * C::TILE + c * BOX, &p.tm_v, kv_full_b[b], c * 64, w.j * BKV, w.bh);
+                }
+                ++nkv;
+                const float* lse2_h = p.lse2 + static_cast<size_t>(w.bh) * n_pad;
+                const float* delta_h = p.delta + static_cast<size_t>(w.bh) * n_pad;
+                for (int t = 0; t < w.n_it; ++t, ++T) {
+                    const int s = T & 1;
+                    const int i = w.i_first + t;
+                    if (!(ok = mbar_wait(&q_empty[s], ((T >> 1) & 1) ^ 1, p.ctl))) break;
+                    mbar_arrive_expect_tx(&q_full[s], C::TILE + 2 * BQ * 4);
+                    for (int c = 0; c < C::NDC; ++c)
+                        tma_load_3d(sQ + s * C::TILE + c * BOX, &p.tm_q, &q_full[s], c * 64, i * BQ, w.bh);
+                    bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &q_full[s]);
+                    bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &q_full[s]);
+                    ++nq;
+                    if (!(ok = mbar_wait(do_empty, (T & 1) ^ 1, p.ctl))) break;
+                    mbar_arrive_expect_tx(do_full, C::TILE);
+                    for (int c = 0; c < C::NDC; ++c) tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, w.bh);
+                    ++ndo;
+                }
             }
             if (!ok) {
-                mbar_wait_drain(kv_full, 0, p.ctl.limit_ns);
+                // let every copy already issued land before the CTA exits
+                for (int u = max(0, nkv - C::KV_BUFS); u < nkv; ++u)
+                    mbar_wait_drain(kv_full_b[u & (C::KV_BUFS - 1)], (C::PERSIST ? (u >> 1) : u) & 1, p.ctl.limit_ns);
                 for (int u = max(0, nq - QSTAGES); u < nq; ++u)
                     mbar_wait_drain(&q_full[u & 1], (u >> 1) & 1, p.ctl.limit_ns);
                 if (ndo > 0) mbar_wait_drain(do_full, (ndo - 1) & 1, p.ctl.limit_ns);
@@ -357,67 +405,93 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             };
             // dQ = dS (shared dS^T read MN-major: 64 contiguous queries per 128-byte
             // row) x K (MN-major over d), walking the 128 keys
-            auto issue_dq = [&](uint32_t d_col) {
+            auto issue_dq = [&](uint32_t d_col, uint32_t k_base) {
 #pragma unroll
                 for (int kk = 0; kk < BKV / 16; ++kk)
                     mma_ss_elect(tmem + d_col, sdesc_sw128(aDS + kk * 2048, BOX, 1024),
-                                 sdesc_sw128(aK + kk * 2048, BOX, 1024), idesc_dq, kk > 0 ? 1u : 0u);
+                                 sdesc_sw128(k_base + kk * 2048, BOX, 1024), idesc_dq, kk > 0 ? 1u : 0u);
             };
+            // K of item k's buffer (V lies one tile after it)
+            auto kbase = [&](int k) { return aK + 2u * static_cast<uint32_t>(k & (C::KV_BUFS - 1)) * C::TILE; };
 
-            bool ok = warp_wait(kv_full, 0, p.ctl) && warp_wait(&q_full[0], 0, p.ctl);
+            bool ok = item0 < n_items && warp_wait(kv_full_b[0], 0, p.ctl) && warp_wait(&q_full[0], 0, p.ctl);
             if (ok) {
                 tc_fence_after();
-                issue_kk(rcol(0), aK, q_base(0));
+                issue_kk(rcol(0), kbase(0), q_base(0));
                 mma_commit_elect(s_full);
                 ok = warp_wait(do_full, 0, p.ctl);
                 if (ok) {
                     tc_fence_after();
-                    issue_kk(rcol(1), aV, aDO);
+                    issue_kk(rcol(1), kbase(0) + C::TILE, aDO);
                     mma_commit_elect(dp_full);
                 }
             }
-            for (int t = 0; t < n_it && ok; ++t) {
-                const uint32_t X = rcol(t), Y = rcol(t + 1);
-                if (!(ok = warp_wait(p_ready, t & 1, p.ctl))) break;
-                tc_fence_after();
-                issue_dv(X, t > 0);
-                mma_commit_elect(do_empty);
-                if (!(ok = warp_wait(EARLY_DP ? dp_read : ds_ready, t & 1, p.ctl))) break;
-                tc_fence_after();
-                if (t + 1 < n_it) {
-                    // Y held dP^T of tile t, already read by the softmax
-                    if (!(ok = warp_wait(&q_full[(t + 1) & 1], ((t + 1) >> 1) & 1, p.ctl))) break;
+            // T counts query tiles over all of the CTA's items: the barrier phases,
+            // Q stages and TMEM regions follow it, so the pipeline runs on from one
+            // item's last tile into the next item's first (whose S^T and dP^T are
+            // issued, as any next tile's, from the current tile's step)
+            int T = 0;
+            for (int k = 0, item = item0; item < n_items && ok; ++k, item += stride) {
+                const ItemInfo w = item_info(item);
+                const bool has_next = item + stride < n_items;
+                const uint32_t aKc = kbase(k), aKn = kbase(k + 1);
+                for (int t = 0; t < w.n_it && ok; ++t, ++T) {
+                    const uint32_t X = rcol(T), Y = rcol(T + 1);
+                    const bool cross = t + 1 == w.n_it;    // the next tile is the next item's first
+                    const bool more = !cross || has_next;  // there is a next tile
+                    if (!(ok = warp_wait(p_ready, T & 1, p.ctl))) break;
+                    // an item's first dV overwrites the region: the previous item's dV
+                    // must have been read out
+                    if (C::PERSIST && t == 0 && k > 0 && !(ok = warp_wait(dv_free, (k - 1) & 1, p.ctl))) break;
                     tc_fence_after();
-                    issue_kk(Y, aK, q_base(t + 1));
-                    mma_commit_elect(s_full);
-                }
-                if constexpr (EARLY_DP) {
-                    if (!(ok = warp_wait(ds_ready, t & 1, p.ctl))) break;
+                    issue_dv(X, t > 0);
+                    mma_commit_elect(do_empty);
+                    if (!(ok = warp_wait(EARLY_DP ? dp_read : ds_ready, T & 1, p.ctl))) break;
                     tc_fence_after();
-                }
-                issue_dk(q_base(t), t > 0);
-                mma_commit_elect(&q_empty[t & 1]);
-                if constexpr (D == 128) {
-                    issue_dq(X);
-                } else {
-                    // the dQ warps must have read the previous tile's dQ out
-                    if (t > 0 && !(ok = warp_wait(dq_empty, (t - 1) & 1, p.ctl))) break;
-                    tc_fence_after();
-                    issue_dq(C::DQ_COL);
-                }
-                mma_commit_elect(dq_full);
-                if (t + 1 < n_it) {
-                    if (!(ok = warp_wait(do_full, (t + 1) & 1, p.ctl))) break;
-                    if constexpr (D == 128) {
-                        // X holds dQ of tile t until the dQ warps have read it
-                        if (!(ok = warp_wait(dq_empty, t & 1, p.ctl))) break;
+                    if (more) {
+                        // Y held dP^T of this tile, already read by the softmax
+                        if (cross && !(ok = warp_wait(kv_full_b[(k + 1) & 1], ((k + 1) >> 1) & 1, p.ctl))) break;
+                        if (!(ok = warp_wait(&q_full[(T + 1) & 1], ((T + 1) >> 1) & 1, p.ctl))) break;
+                        tc_fence_after();
+                        issue_kk(Y, cross ? aKn : aKc, q_base(T + 1));
+                        mma_commit_elect(s_full);
                     }
-                    tc_fence_after();
-                    issue_kk(X, aV, aDO);
-                    mma_commit_elect(dp_full);
+                    if constexpr (EARLY_DP) {
+                        if (!(ok = warp_wait(ds_ready, T & 1, p.ctl))) break;
+                        tc_fence_after();
+                    }
+                    if (C::PERSIST && t == 0 && k > 0) {
+                        if (!(ok = warp_wait(dk_free, (k - 1) & 1, p.ctl))) break;
+                        tc_fence_after();
+                    }
+                    issue_dk(q_base(T), t > 0);
+                    mma_commit_elect(&q_empty[T & 1]);
+                    if constexpr (D == 128) {
+                        issue_dq(X, aKc);
+                    } else {
+                        // the dQ warps must have read the previous tile's dQ out
+                        if (T > 0 && !(ok = warp_wait(dq_empty, (T - 1) & 1, p.ctl))) break;
+                        tc_fence_after();
+                        issue_dq(C::DQ_COL, aKc);
+                    }
+                    mma_commit_elect(dq_full);
+                    if (cross) {
+                        mma_commit_elect(dkdv_done);  // the item's dV, dK are complete
+                        // and no MMA reads its K, V any more: the producer may refill them
+                        if (C::PERSIST) mma_commit_elect(kv_empty_b[k & 1]);
+                    }
+                    if (more) {
+                        if (!(ok = warp_wait(do_full, (T + 1) & 1, p.ctl))) break;
+                        if constexpr (D == 128) {
+                            // X holds dQ of tile T until the dQ warps have read it
+                            if (!(ok = warp_wait(dq_empty, T & 1, p.ctl))) break;
+                        }
+                        tc_fence_after();
+                        issue_kk(X, (cross ? aKn : aKc) + C::TILE, aDO);
+                        mma_commit_elect(dp_full);
+                    }
                 }
             }
-            if (ok) mma_commit_elect(dkdv_done);
             mma_commit_elect(drain);
             mbar_wait_drain(drain, 0, p.ctl.limit_ns);
         }
@@ -427,17 +501,21 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         const int quad = warp & 3;
         const int h0 = (SMW == 8) ? (warp >> 2) : 0;  // first query half of this warp
         const int r = quad * 32 + lane;
-        const int key = j * BKV + r;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const float cl2 = p.scale_log2;
         bool ok = true;
-        for (int t = 0; t < n_it && ok; ++t) {
-            const int s = t & 1;
-            const int i = i_first + t;
+        int T = 0;  // query tiles over all of the CTA's items
+        for (int item = item0; item < n_items && ok; item += stride) {
+        const ItemInfo w = item_info(item);
+        const int j = w.j, bh = w.bh;
+        const int key = j * BKV + r;
+        for (int t = 0; t < w.n_it && ok; ++t, ++T) {
+            const int s = T & 1;
+            const int i = w.i_first + t;
             const float* lse2 = sVec + s * 2 * BQ;
             const float* delta = lse2 + BQ;
-            const uint32_t xa = tmem + lane_off + rcol(t);
-            const uint32_t ya = tmem + lane_off + rcol(t + 1);
+            const uint32_t xa = tmem + lane_off + rcol(T);
+            const uint32_t ya = tmem + lane_off + rcol(T + 1);
             // keep bits of this key row for the warp's query quarters (bit c of
             // zq[q]: query 32 (2 h0 + q) + c), drawn while S^T is being computed
             uint32_t zq[DROPOUT ? 2 * HALVES : 1];
@@ -450,8 +528,8 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                                   static_cast<uint64_t>(bh), p.keep_t, p.seed, p.offset),
                         lane);
             }
-            if (!(ok = warp_wait(s_full, t & 1, p.ctl))) break;
-            if (!(ok = warp_wait(&q_full[s], (t >> 1) & 1, p.ctl))) break;
+            if (!(ok = warp_wait(s_full, T & 1, p.ctl))) break;
+            if (!(ok = warp_wait(&q_full[s], (T >> 1) & 1, p.ctl))) break;
             tc_fence_after();
             // causal: query (t-th tile, column c) sees this key iff key <= query; only
             // the first (diagonal) tile has such pairs.  Keys past N carry no weight.
@@ -508,7 +586,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
 
             // dP^T of this tile was issued after the dK and dQ MMAs of the previous
             // one, so once it is complete they have read the old dS^T
-            if (!(ok = warp_wait(dp_full, t & 1, p.ctl))) break;
+            if (!(ok = warp_wait(dp_full, T & 1, p.ctl))) break;
             tc_fence_after();
             // dS^T = P^T (dP^T - D), with the bf16 P^T read back from TMEM (it stays in
             // X until this tile's dS^T is written), to shared memory: row r, query
@@ -569,7 +647,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 // the previous tile's first dQ half was staged in the dS^T buffer: its
                 // reduce-add must have read it before dS^T is written there (dS^T is
                 // formed in registers meanwhile)
-                if (t > 0 && !(ok = warp_wait(ds_free, (t - 1) & 1, p.ctl))) break;
+                if (T > 0 && !(ok = warp_wait(ds_free, (T - 1) & 1, p.ctl))) break;
                 uint8_t* chunk = sDS + h0 * BOX;
 #pragma unroll
                 for (int qq = 0; qq < 2; ++qq)
@@ -582,13 +660,17 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             tc_fence_before();
             mbar_arrive(ds_ready);
         }
-        // epilogue: dV rows (times 256 / keep_t under dropout); with 8 warps the
-        // warps of query half 1 stage the dK rows (times scale) at the same time,
-        // while the dQ warps finish the last dQ
-        if (ok && warp_wait(dkdv_done, 0, p.ctl)) {
+        }
+        // epilogue (one item per CTA): dV rows (times 256 / keep_t under dropout);
+        // with 8 warps the warps of query half 1 stage the dK rows (times scale) at
+        // the same time, while the dQ warps finish the last dQ.  Persistent CTAs
+        // leave the epilogue to the dQ warps and go on to the next item.
+        if (!C::PERSIST && ok && item0 < n_items && warp_wait(dkdv_done, 0, p.ctl)) {
             tc_fence_after();
+            const ItemInfo w = item_info(item0);
             const bool dk_rows = SMW == 8 && h0 == 1;
-            store_rows(dk_rows ? 1 : 0, lane_off, quad * 32, dk_rows ? p.scale : (DROPOUT ? p.keep_scale : 1.f));
+            store_rows(dk_rows ? 1 : 0, lane_off, quad * 32, dk_rows ? p.scale : (DROPOUT ? p.keep_scale : 1.f), w.bh,
+                       w.j);
         }
     } else {
         // ------------------------------------------------------------ dQ (4 warps)
@@ -603,15 +685,19 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             return warp_wait(dqw_bar, (bar_uses++) & 1, p.ctl);
         };
         bool ok = true;
-        for (int t = 0; t < n_it && ok; ++t) {
-            const int i = i_first + t;
-            if (!(ok = warp_wait(dq_full, t & 1, p.ctl))) break;
+        int T = 0;  // query tiles over all of the CTA's items
+        for (int k = 0, item = item0; item < n_items && ok; ++k, item += stride) {
+        const ItemInfo w = item_info(item);
+        const int bh = w.bh;
+        for (int t = 0; t < w.n_it && ok; ++t, ++T) {
+            const int i = w.i_first + t;
+            if (!(ok = warp_wait(dq_full, T & 1, p.ctl))) break;
             tc_fence_after();
             // thread = query row qr (TMEM lane of dQ), D head-dim columns in halves of
             // 64; row qr of the [128][64] staging tile: 32-column chunk, 16-byte
             // piece swizzled with qr % 8
             const int qr = wq * 32 + lane;
-            const uint32_t qa = tmem + lane_off + (D == 128 ? rcol(t) : C::DQ_COL);
+            const uint32_t qa = tmem + lane_off + (D == 128 ? rcol(T) : C::DQ_COL);
             // with 4 softmax warps (168 registers) all of dQ is read before the region
             // is released; with 8 (128 registers) the second half is read after the
             // first has been staged
@@ -671,15 +757,64 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 bulk_wait_group_read1();
                 mbar_arrive(ds_free);
             }
-
+        }
+        if constexpr (C::PERSIST) {
+            if (!ok) break;
+            // epilogue of item k, while the other warps run the next item: dV and dK
+            // out of TMEM (lanes = key rows, times 256 / keep_t and scale) into
+            // 128-byte-swizzled [128 rows][32 columns] fp32 boxes -- dV in its own
+            // staging boxes, dK in the dQ staging tile -- once the previous item's
+            // stores and the last dQ reduce-add have read them, then TMA tile stores
+            // (rows past N are clipped).  The TMEM regions are released as soon as
+            // they are read.
+            if (issuer) bulk_wait_group_read0();
+            if (!(ok = sync_dq())) break;
+            if (!(ok = warp_wait(dkdv_done, k & 1, p.ctl))) break;
+            tc_fence_after();
+            const uint32_t l = static_cast<uint32_t>(wq * 32 + lane);  // key row
+            uint8_t* sEPI = smem + C::EPI_OFF;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                uint8_t* stg = which == 0 ? sEPI : sSTG;
+                const uint32_t col = which == 0 ? C::DV_COL : C::DK_COL;
+                const float f = which == 0 ? (DROPOUT ? p.keep_scale : 1.f) : p.scale;
+#pragma unroll
+                for (int cc = 0; cc < D; cc += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_off + col + cc, v);
+                    tmem_wait_ld();
+                    uint8_t* box = stg + (cc / 32) * (BKV * 128);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        *reinterpret_cast<uint4*>(box + sw128_offset(l, kk)) =
+                            make_uint4(__float_as_uint(__uint_as_float(v[4 * kk]) * f),
+                                       __float_as_uint(__uint_as_float(v[4 * kk + 1]) * f),
+                                       __float_as_uint(__uint_as_float(v[4 * kk + 2]) * f),
+                                       __float_as_uint(__uint_as_float(v[4 * kk + 3]) * f));
+                }
+                tc_fence_before();
+                mbar_arrive(which == 0 ? dv_free : dk_free);
+            }
+            fence_proxy_async_smem();
+            if (!(ok = sync_dq())) break;
+            if (issuer) {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    tma_store_3d(&p.tm_dv, sEPI + c * (BKV * 128), c * 32, w.j * BKV, w.bh);
+                    tma_store_3d(&p.tm_dk, sSTG + c * (BKV * 128), c * 32, w.j * BKV, w.bh);
+                }
+                bulk_commit_group();
+            }
+        }
         }
         // the staging buffers are read: the reduce-adds themselves complete in L2
         // before the grid does
         if (issuer) bulk_wait_group_read0();
-        // epilogue (4 softmax warps): dK rows (lanes = key rows)
-        if (SMW == 4 && ok && warp_wait(dkdv_done, 0, p.ctl)) {
+        // epilogue (one item per CTA, 4 softmax warps): dK rows (lanes = key rows)
+        if (!C::PERSIST && SMW == 4 && ok && item0 < n_items && warp_wait(dkdv_done, 0, p.ctl)) {
             tc_fence_after();
-            store_rows(1, lane_off, wq * 32, p.scale);
+            const ItemInfo w = item_info(item0);
+            store_rows(1, lane_off, wq * 32, p.scale, w.bh, w.j);
         }
     }
 
@@ -697,7 +832,8 @@ cudaError_t launch(const BwdParams& p, cudaStream_t stream)
     auto kern = bwd_kernel<D, CAUSAL, DROPOUT, SMW>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid(p.n_kv_tiles, p.BH);
+    // persistent: one CTA per SM (p.n_ctas, at most the item count); otherwise one per item
+    const dim3 grid = Cfg<D>::PERSIST ? dim3(static_cast<unsigned>(p.n_ctas)) : dim3(p.n_kv_tiles, p.BH);
     kern<<<grid, Roles<SMW>::NTHREADS, Cfg<D>::SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
 }

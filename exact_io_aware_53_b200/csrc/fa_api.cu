@@ -596,7 +596,11 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, f
         (st = encode_3d(&p.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, v, d, N, BH, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
         (st = encode_3d(&p.tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq, d, N, BH, 32,
-                        static_cast<uint32_t>(bwd_dq_tile_rows(d)), CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
+                        static_cast<uint32_t>(bwd_dq_tile_rows(d)), CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_dk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, d, N, BH, 32, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK ||
+        (st = encode_3d(&p.tm_dv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dv, d, N, BH, 32, 128,
+                        CU_TENSOR_MAP_SWIZZLE_128B)) != FA_OK)
         return st;
     if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
     p.delta = static_cast<const float*>(workspace);
@@ -623,6 +627,16 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, f
     p.offset = offset;
     const int smw = g_bwd_softmax_warps.load();
     p.softmax_warps = smw != 0 ? smw : 8;
+    {
+        // the persistent (d = 64) kernel runs one CTA per SM, at most one per item
+        int dev = 0, n_sm = 0;
+        if ((st = cuda_status(cudaGetDevice(&dev))) != FA_OK ||
+            (st = cuda_status(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev))) != FA_OK)
+            return st;
+        const long long items = static_cast<long long>(p.BH) * p.n_kv_tiles;
+        if (items > (1ll << 30)) return FA_ERR_UNSUPPORTED;
+        p.n_ctas = static_cast<int>(std::min<long long>(items, std::max(n_sm, 1)));
+    }
     st = cuda_status(launch_bwd_sm100(p, d, causal != 0, dropout, static_cast<cudaStream_t>(stream)));
     if (st == FA_OK) g_last_launches = 1;
     return st;

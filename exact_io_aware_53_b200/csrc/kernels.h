@@ -107,6 +107,8 @@ struct BwdParams {
     CUtensorMap tm_k;    // {d, N, B*H}, box {64, 128, 1}
     CUtensorMap tm_v;    // {d, N, B*H}, box {64, 128, 1}
     CUtensorMap tm_dq;   // fp32 {d, N, B*H}, box {32, bwd_dq_tile_rows(d), 1}, 128-byte swizzle, reduce-add target
+    CUtensorMap tm_dk;   // fp32 {d, N, B*H}, box {32, 128, 1}, 128-byte swizzle (persistent kernel's dK stores)
+    CUtensorMap tm_dv;   // as tm_dk, for dV
     const float* lse2;   // [B*H][n_kv_tiles * 128]; +inf past N
     const float* delta;  // [B*H][n_kv_tiles * 128]; 0 past N
     float* dq;           // [B*H][N][d], accumulated into (zeroed by the pre-pass)
@@ -124,6 +126,7 @@ struct BwdParams {
     uint64_t seed;     // Philox key (seed, offset)
     uint64_t offset;
     int softmax_warps;  // 4 or 8 softmax warps per CTA
+    int n_ctas;         // CTAs of the persistent (d = 64) kernel: min(items, SMs)
     WaitCtl ctl;
 };
 cudaError_t launch_bwd_sm100(const BwdParams& p, int d, bool causal, bool dropout, cudaStream_t stream);
