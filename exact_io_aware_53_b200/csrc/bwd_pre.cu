@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(WARPS * 32) bwd_pre_kernel(const BwdPreParams 
 {
     using S = Shape<D>;
     const int lane = threadIdx.x & 31;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.queue = 0u;  // the main kernel claims items from it
     const long long rows = static_cast<long long>(p.BH) * p.n_pad;
     const long long prow0 = (static_cast<long long>(blockIdx.x) * WARPS + (threadIdx.x >> 5)) * S::RPW;
     if (prow0 >= rows) return;

@@ -106,8 +106,8 @@ struct Cfg {
     static constexpr int EPI_BYTES = PERSIST ? (D / 32) * BKV * 128 : 0;
     static constexpr int VEC_OFF = EPI_OFF + EPI_BYTES;  // [stage][lse2 128 | delta 128]
     static constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
-    static constexpr int NBARS = 24;
-    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;
+    static constexpr int NBARS = 28;
+    static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;  // + TMEM slot, item ring
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t DV_COL = 256;
     static constexpr uint32_t DK_COL = 256 + D;
@@ -214,7 +214,12 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     uint64_t* kv_empty_b[2] = {bars + 19, bars + 20};
     uint64_t* dv_free = bars + 21;
     uint64_t* dk_free = bars + 22;
+    // persistent: the producer hands each claimed item to the other warps
+    // through a two-slot ring (item_buf, -1 when none is left)
+    uint64_t* item_full = bars + 23;   // [2]
+    uint64_t* item_empty = bars + 25;  // [2]: MMA warp, softmax warps, dQ warps
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+    int* item_buf = reinterpret_cast<int*>(tmem_slot + 1);  // [2]
 
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
@@ -223,11 +228,29 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     const int n_q = (N + BQ - 1) / BQ;
     // Items are (head, 128-key tile) pairs in the grouped longest-first order:
     // key tile 0 sees the most query tiles under the causal mask, and a group's
-    // Q, dO and dQ share L2.  A persistent CTA takes items item0, item0 + stride,
-    // ...; otherwise the CTA has the one item of its grid position.
+    // Q, dO and dQ share L2.  A persistent CTA's first item is its index; the
+    // producer claims each later one from the launch's counter in the workspace
+    // (zeroed by the pre-pass) and hands it on, so CTAs that finish early take
+    // more.  Otherwise the CTA has the one item of its grid position.
     const int n_items = p.BH * p.n_kv_tiles;
     const int item0 = C::PERSIST ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x);
-    const int stride = C::PERSIST ? static_cast<int>(gridDim.x) : n_items;
+    // item k of this CTA as the producer published it: -1 when there is none,
+    // -2 when the wait gave up (then the device error word is set)
+    auto read_item = [&](int k) -> int {
+        if constexpr (!C::PERSIST) {
+            return k == 0 && item0 < n_items ? item0 : -1;
+        } else {
+            if (!warp_wait(&item_full[k & 1], (k >> 1) & 1, p.ctl)) return -2;
+            return *reinterpret_cast<volatile int*>(&item_buf[k & 1]);
+        }
+    };
+    // this warp no longer needs item k's slot
+    auto release_item = [&](int k) {
+        if constexpr (C::PERSIST) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&item_empty[k & 1]);
+        }
+    };
     struct ItemInfo {
         int bh, j;    // head, key tile
         int i_first;  // first query tile that sees the keys
@@ -265,6 +288,10 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         mbar_init(kv_empty_b[1], 1);
         mbar_init(dv_free, 128);
         mbar_init(dk_free, 128);
+        for (int u = 0; u < 2; ++u) {
+            mbar_init(&item_full[u], 1);
+            mbar_init(&item_empty[u], SMW + 5);
+        }
         fence_mbar_init();
     }
     if (warp == MMA_WARP) {
@@ -328,7 +355,17 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             int T = 0;                     // query tiles issued over all items
             int nq = 0, ndo = 0, nkv = 0;  // loads issued: Q (with its row vectors), dO, K+V
             bool ok = true;
-            for (int k = 0, item = item0; item < n_items && ok; ++k, item += stride) {
+            for (int k = 0; ok; ++k) {
+                int item = k == 0 ? item0 : -1;
+                if constexpr (C::PERSIST) {
+                    if (k > 0) item = static_cast<int>(atomicAdd(p.queue, 1u)) + static_cast<int>(gridDim.x);
+                    if (item >= n_items) item = -1;
+                    // publish it once every warp has let go of item k - 2's slot
+                    if (!(ok = mbar_wait(&item_empty[k & 1], ((k >> 1) & 1) ^ 1, p.ctl))) break;
+                    item_buf[k & 1] = item;
+                    mbar_arrive(&item_full[k & 1]);
+                }
+                if (item < 0 || item >= n_items) break;
                 const ItemInfo w = item_info(item);
                 const int b = k & (C::KV_BUFS - 1);
                 // the buffer's previous item (k - 2) has been read and its dV stored
@@ -414,7 +451,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             // K of item k's buffer (V lies one tile after it)
             auto kbase = [&](int k) { return aK + 2u * static_cast<uint32_t>(k & (C::KV_BUFS - 1)) * C::TILE; };
 
-            bool ok = item0 < n_items && warp_wait(kv_full_b[0], 0, p.ctl) && warp_wait(&q_full[0], 0, p.ctl);
+            bool ok = warp_wait(kv_full_b[0], 0, p.ctl) && warp_wait(&q_full[0], 0, p.ctl);
             if (ok) {
                 tc_fence_after();
                 issue_kk(rcol(0), kbase(0), q_base(0));
@@ -431,14 +468,23 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             // item's last tile into the next item's first (whose S^T and dP^T are
             // issued, as any next tile's, from the current tile's step)
             int T = 0;
-            for (int k = 0, item = item0; item < n_items && ok; ++k, item += stride) {
+            for (int k = 0; ok; ++k) {
+                const int item = read_item(k);
+                if (item < 0) {
+                    ok = item == -1;
+                    break;
+                }
                 const ItemInfo w = item_info(item);
-                const bool has_next = item + stride < n_items;
                 const uint32_t aKc = kbase(k), aKn = kbase(k + 1);
                 for (int t = 0; t < w.n_it && ok; ++t, ++T) {
                     const uint32_t X = rcol(T), Y = rcol(T + 1);
-                    const bool cross = t + 1 == w.n_it;    // the next tile is the next item's first
-                    const bool more = !cross || has_next;  // there is a next tile
+                    const bool cross = t + 1 == w.n_it;  // the next tile is the next item's first
+                    bool more = !cross;                  // there is a next tile
+                    if (cross) {
+                        const int nxt = read_item(k + 1);
+                        if (!(ok = nxt != -2)) break;
+                        more = nxt >= 0;
+                    }
                     if (!(ok = warp_wait(p_ready, T & 1, p.ctl))) break;
                     // an item's first dV overwrites the region: the previous item's dV
                     // must have been read out
@@ -491,6 +537,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                         mma_commit_elect(dp_full);
                     }
                 }
+                release_item(k);
             }
             mma_commit_elect(drain);
             mbar_wait_drain(drain, 0, p.ctl.limit_ns);
@@ -505,7 +552,12 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         const float cl2 = p.scale_log2;
         bool ok = true;
         int T = 0;  // query tiles over all of the CTA's items
-        for (int item = item0; item < n_items && ok; item += stride) {
+        for (int k = 0; ok; ++k) {
+        const int item = read_item(k);
+        if (item < 0) {
+            ok = item == -1;
+            break;
+        }
         const ItemInfo w = item_info(item);
         const int j = w.j, bh = w.bh;
         const int key = j * BKV + r;
@@ -660,6 +712,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             tc_fence_before();
             mbar_arrive(ds_ready);
         }
+        release_item(k);
         }
         // epilogue (one item per CTA): dV rows (times 256 / keep_t under dropout);
         // with 8 warps the warps of query half 1 stage the dK rows (times scale) at
@@ -686,7 +739,12 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         };
         bool ok = true;
         int T = 0;  // query tiles over all of the CTA's items
-        for (int k = 0, item = item0; item < n_items && ok; ++k, item += stride) {
+        for (int k = 0; ok; ++k) {
+        const int item = read_item(k);
+        if (item < 0) {
+            ok = item == -1;
+            break;
+        }
         const ItemInfo w = item_info(item);
         const int bh = w.bh;
         for (int t = 0; t < w.n_it && ok; ++t, ++T) {
@@ -806,6 +864,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 bulk_commit_group();
             }
         }
+        release_item(k);
         }
         // the staging buffers are read: the reduce-adds themselves complete in L2
         // before the grid does

@@ -530,7 +530,8 @@ size_t fa_bwd_workspace_bytes(int B, int H, int N, int d)
 {
     if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
     const size_t rows = static_cast<size_t>(B) * H * (static_cast<size_t>(N + 127) / 128 * 128);
-    return 2 * ((rows * sizeof(float) + 255) & ~size_t(255));
+    // D and lse2, then one 256-byte slot for the main kernel's work counter
+    return 2 * ((rows * sizeof(float) + 255) & ~size_t(255)) + 256;
 }
 
 int fa_bwd_prep(const void* o, const float* lse, const void* dO, float* dq, void* workspace, int B, int H, int N,
@@ -552,6 +553,7 @@ int fa_bwd_prep(const void* o, const float* lse, const void* dO, float* dq, void
     pp.lse = lse;
     pp.delta = static_cast<float*>(workspace);
     pp.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + vec_bytes);
+    pp.queue = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + 2 * vec_bytes);
     pp.dq = dq;
     pp.BH = static_cast<int>(BH);
     pp.N = N;
@@ -568,7 +570,7 @@ namespace {
 
 // The tensor-core backward proper (fa_bwd_main), plain or with dropout.
 int bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, float* dq, float* dk, float* dv,
-                  const void* workspace, int B, int H, int N, int d, float scale, int causal, bool dropout, int keep_t,
+                  void* workspace, int B, int H, int N, int d, float scale, int causal, bool dropout, int keep_t,
                   unsigned long long seed, unsigned long long offset, void* stream)
 {
     g_last_launches = 0;
@@ -605,6 +607,7 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, f
     if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
     p.delta = static_cast<const float*>(workspace);
     p.lse2 = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + vec_bytes);
+    p.queue = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + 2 * vec_bytes);
     p.dq = dq;
     p.dk = dk;
     p.dv = dv;
@@ -647,7 +650,7 @@ int bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, f
 extern "C" {
 
 int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, float* dq, float* dk, float* dv,
-                const void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream)
+                void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream)
 {
     return bwd_main_impl(q, k, v, dO, dq, dk, dv, workspace, B, H, N, d, scale, causal, false, 256, 0, 0, stream);
 }

@@ -13,8 +13,8 @@
 // Every GPU that loads the library holds it until the process exits, every
 // call on a device shares it, and it keeps the last call's contents.  Nothing
 // in it has to start at zero: the pre-pass writes every entry the main kernel
-// reads (the row terms D and the base-2 log-sum-exp, padding rows included)
-// before the main kernel runs.  Two calls whose work overlaps on the GPU (two
+// reads (the row terms D and the base-2 log-sum-exp, padding rows included, and
+// the main kernel's work counter) before the main kernel runs.  Two calls whose work overlaps on the GPU (two
 // streams, or two host threads without ordering) race on the array.
 #include <mutex>
 

@@ -94,6 +94,7 @@ struct BwdPreParams {
     float* delta;  // D_i = <dO_i, O_i>            [B*H][n_pad]
     float* lse2;   // lse_i * log2(e)              [B*H][n_pad]
     float* dq;     // zeroed                       [B*H][N][d]
+    unsigned int* queue;  // the main kernel's work counter: set to 0
     int BH;
     int N;
     int n_pad;     // rows per head in delta / lse2 (N rounded up to 128)
@@ -114,6 +115,7 @@ struct BwdParams {
     float* dq;           // [B*H][N][d], accumulated into (zeroed by the pre-pass)
     float* dk;           // [B*H][N][d]
     float* dv;           // [B*H][N][d]
+    unsigned int* queue; // persistent kernel's item counter in the workspace (0 on entry)
     int BH;
     int N;
     int n_kv_tiles;

@@ -69,7 +69,9 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 /*
  * Bytes of device workspace fa_bwd needs: the row terms D_i = <dO_i, O_i> and
  * the log-sum-exp in base 2, both fp32 [B][H][N rounded up to 128] (O(N),
- * never O(N^2)).  Returns 0 for non-positive sizes.
+ * never O(N^2)), and one 256-byte slot holding the work counter from which the
+ * head-dimension-64 kernel's CTAs claim (head, key tile) items.  Returns 0 for
+ * non-positive sizes.
  */
 size_t fa_bwd_workspace_bytes(int B, int H, int N, int d);
 
@@ -88,15 +90,16 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 /*
  * The two stages of fa_bwd, for callers that time or schedule them apart.
  * fa_bwd_prep: from o, dO (bf16) and lse, writes the row terms D_i = <dO_i, O_i>
- * and lse_i * log2(e) into `workspace` and zeroes dq.  fa_bwd_main: the
- * tensor-core backward proper; it reads that workspace, so it must follow
+ * and lse_i * log2(e) into `workspace`, zeroes its work counter, and zeroes dq.
+ * fa_bwd_main: the tensor-core backward proper; it reads that workspace and
+ * advances its work counter, so each fa_bwd_main must follow its own
  * fa_bwd_prep for the same tensors on the same stream.  Arguments and errors
  * as fa_bwd.
  */
 int fa_bwd_prep(const void* o, const float* lse, const void* dO, float* dq, void* workspace, int B, int H, int N,
                 int d, void* stream);
 int fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, float* dq, float* dk, float* dv,
-                const void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream);
+                void* workspace, int B, int H, int N, int d, float scale, int causal, void* stream);
 
 /*
  * Size of the scratch area built into the library for fa_bwd_noalloc.
