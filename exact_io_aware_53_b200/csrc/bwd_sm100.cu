@@ -11,13 +11,18 @@
 //
 // One CTA owns 128 keys at a time (K_j, V_j stay in shared memory) and walks
 // the 128-row query tiles t that see them, so every tensor-core instruction is
-// 128 rows by 128 (or by d) columns.  For d = 64 the CTAs are persistent: each
-// takes several (head, key tile) items in turn, with two K, V buffers, and the
-// query-tile pipeline runs on from one item's last tile into the next item's
-// first (barrier phases, Q stages and TMEM regions follow the CTA's running
-// tile count T); the dQ warps write an item's dV and dK (TMEM -> swizzled
-// shared boxes -> TMA tile stores) while the other warps start the next item.
-// For d = 128 shared memory holds one K, V buffer and a CTA runs one item.
+// 128 rows by 128 (or by d) columns.  The CTAs are persistent (one per SM):
+// each takes (head, key tile) items in turn -- the first by its index, the
+// rest claimed from a counter in the workspace -- and the query-tile pipeline
+// runs on from one item's last tile into the next item's first (barrier
+// phases, Q stages and TMEM regions follow the CTA's running tile count T).
+//   d = 64:  two K, V buffers, so the next item's keys load during this one;
+//            the dQ warps write an item's dV and dK (TMEM -> swizzled shared
+//            boxes -> TMA tile stores) while the other warps start the next.
+//   d = 128: one K, V buffer, refilled once the item's last MMA is complete
+//            (the next item's first query tile loads ahead of it); the
+//            softmax warps write dV, then dK, through the dS^T buffer and the
+//            dQ staging tile while the next item's first S^T and dP^T run.
 //
 // TMEM (512 columns): two 128-column regions R0, R1, then dV and dK (d columns
 // each) and, for d = 64, dQ (64 columns).  Tile t uses X = R[t & 1] for
@@ -84,11 +89,15 @@ constexpr int BOX = 128 * 128;  // 128 rows x 128 B (64 bf16)
 
 template <int D>
 struct Cfg {
-    // d = 64: persistent CTAs (one per SM) walk several (head, key tile) items,
-    // with two K, V buffers so that the next item's keys load during this one;
-    // d = 128 fills shared memory with one buffer and runs one CTA per item
-    static constexpr bool PERSIST = D == 64;
-    static constexpr int KV_BUFS = PERSIST ? 2 : 1;
+    // Persistent CTAs (one per SM) walk several (head, key tile) items.  d = 64
+    // has room for two K, V buffers, so the next item's keys load during this
+    // one, and a separate dV staging area: its dQ warps write an item's dV and
+    // dK.  d = 128 has one K, V buffer (the next item's keys load once this
+    // item's MMAs are complete) and its softmax warps write dV and dK through
+    // the dS^T buffer and the dQ staging tile (64 KB together).
+    static constexpr bool PERSIST = true;
+    static constexpr int KV_BUFS = D == 64 ? 2 : 1;
+    static constexpr bool EPI_SOFTMAX = D == 128;
     static constexpr int NDC = D / 64;  // 128-byte column boxes per row
     static constexpr int TILE = NDC * BOX;
     static constexpr int K_OFF = 0;                        // buffer b: K at K_OFF + 2 b TILE, V after it
@@ -103,10 +112,10 @@ struct Cfg {
     static constexpr int STG_CHUNK = STG_ROWS * 128;
     // persistent: the dV epilogue's staging boxes ([128 keys][32 d] fp32, 128-byte swizzled)
     static constexpr int EPI_OFF = STG_OFF + 2 * STG_CHUNK;
-    static constexpr int EPI_BYTES = PERSIST ? (D / 32) * BKV * 128 : 0;
+    static constexpr int EPI_BYTES = (PERSIST && !EPI_SOFTMAX) ? (D / 32) * BKV * 128 : 0;
     static constexpr int VEC_OFF = EPI_OFF + EPI_BYTES;  // [stage][lse2 128 | delta 128]
     static constexpr int BAR_OFF = VEC_OFF + QSTAGES * 2 * BQ * 4;
-    static constexpr int NBARS = 28;
+    static constexpr int NBARS = 32;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16;  // + TMEM slot, item ring
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t DV_COL = 256;
@@ -177,6 +186,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     // buffer (free between this tile's dQ MMA and the next tile's dS^T), so the
     // region dQ occupies is released without waiting for the staging tile
     constexpr bool DQ_IN_DS = (D == 128 && SMW == 8);
+    // persistent CTAs (Cfg) except for d = 128 with dropout, whose generator
+    // state leaves no registers for the item bookkeeping: there it measured
+    // slower (1.31 against 1.19 ms, 4x16x4096x128 causal) and runs one CTA per item
+    constexpr bool PERSIST = C::PERSIST && !(D == 128 && DROPOUT);
+    constexpr bool EPI_SOFTMAX = PERSIST && C::EPI_SOFTMAX;
     extern __shared__ __align__(1024) uint8_t smem[];
     // the 128-byte-swizzled tiles need a 1024-byte aligned base; the layout
     // leaves no slack, so a misaligned base is reported instead of used
@@ -220,6 +234,13 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     uint64_t* item_empty = bars + 25;  // [2]: MMA warp, softmax warps, dQ warps
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
     int* item_buf = reinterpret_cast<int*>(tmem_slot + 1);  // [2]
+    // d = 128 epilogue by the softmax warps: the dQ warps' last reduce-adds of the
+    // item have read their staging (dS^T buffer, staging tile); the softmax warps
+    // have staged a round (dV, then dK); a round's stores have read the staging
+    uint64_t* dq_stg_free = bars + 27;
+    uint64_t* epi_sync = bars + 28;
+    uint64_t* epi_round = bars + 29;
+    uint64_t* epi_free = bars + 30;
 
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
@@ -233,11 +254,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     // (zeroed by the pre-pass) and hands it on, so CTAs that finish early take
     // more.  Otherwise the CTA has the one item of its grid position.
     const int n_items = p.BH * p.n_kv_tiles;
-    const int item0 = C::PERSIST ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x);
+    const int item0 = PERSIST ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.y * gridDim.x + blockIdx.x);
     // item k of this CTA as the producer published it: -1 when there is none,
     // -2 when the wait gave up (then the device error word is set)
     auto read_item = [&](int k) -> int {
-        if constexpr (!C::PERSIST) {
+        if constexpr (!PERSIST) {
             return k == 0 && item0 < n_items ? item0 : -1;
         } else {
             if (!warp_wait(&item_full[k & 1], (k >> 1) & 1, p.ctl)) return -2;
@@ -246,7 +267,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     };
     // this warp no longer needs item k's slot
     auto release_item = [&](int k) {
-        if constexpr (C::PERSIST) {
+        if constexpr (PERSIST) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&item_empty[k & 1]);
         }
@@ -286,8 +307,12 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         mbar_init(kv_full_b[1], 1);
         mbar_init(kv_empty_b[0], 1);
         mbar_init(kv_empty_b[1], 1);
-        mbar_init(dv_free, 128);
-        mbar_init(dk_free, 128);
+        mbar_init(dv_free, EPI_SOFTMAX ? 32 * SMW : 128);
+        mbar_init(dk_free, EPI_SOFTMAX ? 32 * SMW : 128);
+        mbar_init(dq_stg_free, 1);
+        mbar_init(epi_sync, 32 * SMW);
+        mbar_init(epi_round, 1);
+        mbar_init(epi_free, 1);
         for (int u = 0; u < 2; ++u) {
             mbar_init(&item_full[u], 1);
             mbar_init(&item_empty[u], SMW + 5);
@@ -357,7 +382,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             bool ok = true;
             for (int k = 0; ok; ++k) {
                 int item = k == 0 ? item0 : -1;
-                if constexpr (C::PERSIST) {
+                if constexpr (PERSIST) {
                     if (k > 0) item = static_cast<int>(atomicAdd(p.queue, 1u)) + static_cast<int>(gridDim.x);
                     if (item >= n_items) item = -1;
                     // publish it once every warp has let go of item k - 2's slot
@@ -368,36 +393,48 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 if (item < 0 || item >= n_items) break;
                 const ItemInfo w = item_info(item);
                 const int b = k & (C::KV_BUFS - 1);
-                // the buffer's previous item (k - 2) has been read and its dV stored
-                if (C::PERSIST && !(ok = mbar_wait(kv_empty_b[b], ((k >> 1) & 1) ^ 1, p.ctl))) break;
-                mbar_arrive_expect_tx(kv_full_b[b], 2 * C::TILE);
-                for (int c = 0; c < C::NDC; ++c) {
-                    tma_load_3d(sK + 2 * b * C::TILE + c * BOX, &p.tm_k, kv_full_b[b], c * 64, w.j * BKV, w.bh);
-                    tma_load_3d(sV + 2 * b * C::TILE + c * BOX, &p.tm_v, kv_full_b[b], c * 64, w.j * BKV, w.bh);
-                }
-                ++nkv;
+                auto load_kv = [&]() -> bool {
+                    // the buffer's previous item has no MMA left that reads it
+                    if (!mbar_wait(kv_empty_b[b], ((k / C::KV_BUFS) & 1) ^ 1, p.ctl)) return false;
+                    mbar_arrive_expect_tx(kv_full_b[b], 2 * C::TILE);
+                    for (int c = 0; c < C::NDC; ++c) {
+                        tma_load_3d(sK + 2 * b * C::TILE + c * BOX, &p.tm_k, kv_full_b[b], c * 64, w.j * BKV, w.bh);
+                        tma_load_3d(sV + 2 * b * C::TILE + c * BOX, &p.tm_v, kv_full_b[b], c * 64, w.j * BKV, w.bh);
+                    }
+                    ++nkv;
+                    return true;
+                };
                 const float* lse2_h = p.lse2 + static_cast<size_t>(w.bh) * n_pad;
                 const float* delta_h = p.delta + static_cast<size_t>(w.bh) * n_pad;
-                for (int t = 0; t < w.n_it; ++t, ++T) {
+                auto load_tile = [&](int t) -> bool {
                     const int s = T & 1;
                     const int i = w.i_first + t;
-                    if (!(ok = mbar_wait(&q_empty[s], ((T >> 1) & 1) ^ 1, p.ctl))) break;
+                    if (!mbar_wait(&q_empty[s], ((T >> 1) & 1) ^ 1, p.ctl)) return false;
                     mbar_arrive_expect_tx(&q_full[s], C::TILE + 2 * BQ * 4);
                     for (int c = 0; c < C::NDC; ++c)
                         tma_load_3d(sQ + s * C::TILE + c * BOX, &p.tm_q, &q_full[s], c * 64, i * BQ, w.bh);
                     bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &q_full[s]);
                     bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &q_full[s]);
                     ++nq;
-                    if (!(ok = mbar_wait(do_empty, (T & 1) ^ 1, p.ctl))) break;
+                    if (!mbar_wait(do_empty, (T & 1) ^ 1, p.ctl)) return false;
                     mbar_arrive_expect_tx(do_full, C::TILE);
                     for (int c = 0; c < C::NDC; ++c) tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, w.bh);
                     ++ndo;
-                }
+                    ++T;
+                    return true;
+                };
+                // with one K, V buffer the keys wait for the previous item's last MMA,
+                // so the first query tile is loaded ahead of them
+                const bool q_first = C::KV_BUFS == 1 && k > 0;
+                if (q_first && !(ok = load_tile(0))) break;
+                if (!(ok = load_kv())) break;
+                for (int t = q_first ? 1 : 0; t < w.n_it; ++t)
+                    if (!(ok = load_tile(t))) break;
             }
             if (!ok) {
                 // let every copy already issued land before the CTA exits
                 for (int u = max(0, nkv - C::KV_BUFS); u < nkv; ++u)
-                    mbar_wait_drain(kv_full_b[u & (C::KV_BUFS - 1)], (C::PERSIST ? (u >> 1) : u) & 1, p.ctl.limit_ns);
+                    mbar_wait_drain(kv_full_b[u & (C::KV_BUFS - 1)], (u / C::KV_BUFS) & 1, p.ctl.limit_ns);
                 for (int u = max(0, nq - QSTAGES); u < nq; ++u)
                     mbar_wait_drain(&q_full[u & 1], (u >> 1) & 1, p.ctl.limit_ns);
                 if (ndo > 0) mbar_wait_drain(do_full, (ndo - 1) & 1, p.ctl.limit_ns);
@@ -488,25 +525,32 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     if (!(ok = warp_wait(p_ready, T & 1, p.ctl))) break;
                     // an item's first dV overwrites the region: the previous item's dV
                     // must have been read out
-                    if (C::PERSIST && t == 0 && k > 0 && !(ok = warp_wait(dv_free, (k - 1) & 1, p.ctl))) break;
+                    if (PERSIST && t == 0 && k > 0 && !(ok = warp_wait(dv_free, (k - 1) & 1, p.ctl))) break;
                     tc_fence_after();
                     issue_dv(X, t > 0);
                     mma_commit_elect(do_empty);
                     if (!(ok = warp_wait(EARLY_DP ? dp_read : ds_ready, T & 1, p.ctl))) break;
                     tc_fence_after();
-                    if (more) {
-                        // Y held dP^T of this tile, already read by the softmax
-                        if (cross && !(ok = warp_wait(kv_full_b[(k + 1) & 1], ((k + 1) >> 1) & 1, p.ctl))) break;
-                        if (!(ok = warp_wait(&q_full[(T + 1) & 1], ((T + 1) >> 1) & 1, p.ctl))) break;
+                    // S^T of the next tile into Y (which held dP^T of this tile, already
+                    // read by the softmax), ahead of this tile's dK and dQ -- except,
+                    // with one K, V buffer, when the next tile is the next item's: its
+                    // keys load only after this item's last MMA
+                    auto issue_next_s = [&]() -> bool {
+                        if (cross && !warp_wait(kv_full_b[(k + 1) & (C::KV_BUFS - 1)], ((k + 1) / C::KV_BUFS) & 1, p.ctl))
+                            return false;
+                        if (!warp_wait(&q_full[(T + 1) & 1], ((T + 1) >> 1) & 1, p.ctl)) return false;
                         tc_fence_after();
                         issue_kk(Y, cross ? aKn : aKc, q_base(T + 1));
                         mma_commit_elect(s_full);
-                    }
+                        return true;
+                    };
+                    const bool early_next = more && !(cross && C::KV_BUFS == 1);
+                    if (early_next && !(ok = issue_next_s())) break;
                     if constexpr (EARLY_DP) {
                         if (!(ok = warp_wait(ds_ready, T & 1, p.ctl))) break;
                         tc_fence_after();
                     }
-                    if (C::PERSIST && t == 0 && k > 0) {
+                    if (PERSIST && t == 0 && k > 0) {
                         if (!(ok = warp_wait(dk_free, (k - 1) & 1, p.ctl))) break;
                         tc_fence_after();
                     }
@@ -524,8 +568,9 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     if (cross) {
                         mma_commit_elect(dkdv_done);  // the item's dV, dK are complete
                         // and no MMA reads its K, V any more: the producer may refill them
-                        if (C::PERSIST) mma_commit_elect(kv_empty_b[k & 1]);
+                        if (PERSIST) mma_commit_elect(kv_empty_b[k & (C::KV_BUFS - 1)]);
                     }
+                    if (more && !early_next && !(ok = issue_next_s())) break;
                     if (more) {
                         if (!(ok = warp_wait(do_full, (T + 1) & 1, p.ctl))) break;
                         if constexpr (D == 128) {
@@ -712,13 +757,67 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             tc_fence_before();
             mbar_arrive(ds_ready);
         }
+        if constexpr (EPI_SOFTMAX) {
+            if (!ok) break;
+            // epilogue of item k (d = 128): dV, then dK, out of TMEM (lanes = key
+            // rows; with 8 warps each takes half of the columns) into four
+            // 128-byte-swizzled [128 rows][32 columns] fp32 boxes over the dS^T
+            // buffer and the dQ staging tile, which the item's last dK, dQ MMAs and
+            // reduce-adds have read; warp 0's first thread issues the TMA tile
+            // stores of a round once every warp has staged it (rows past N are
+            // clipped) and releases the boxes when the stores have read them.
+            // Meanwhile the next item's keys and first query tile load and its
+            // first S^T and dP^T run.
+            if (!(ok = warp_wait(dkdv_done, k & 1, p.ctl))) break;
+            if (!(ok = warp_wait(dq_stg_free, k & 1, p.ctl))) break;
+            tc_fence_after();
+            const bool epi_issuer = warp == 0 && lane == 0;
+            const int c0 = SMW == 8 ? h0 * (D / 2) : 0;
+            const int c1 = SMW == 8 ? c0 + D / 2 : D;
+            const uint32_t l = static_cast<uint32_t>(r);  // key row
+#pragma unroll
+            for (int which = 0; which < 2 && ok; ++which) {
+                const uint32_t col = which == 0 ? C::DV_COL : C::DK_COL;
+                const float f = which == 0 ? (DROPOUT ? p.keep_scale : 1.f) : p.scale;
+                for (int cc = c0; cc < c1; cc += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(tmem + lane_off + col + static_cast<uint32_t>(cc), v);
+                    tmem_wait_ld();
+                    uint8_t* box = sDS + (cc / 32) * (BKV * 128);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        *reinterpret_cast<uint4*>(box + sw128_offset(l, kk)) =
+                            make_uint4(__float_as_uint(__uint_as_float(v[4 * kk]) * f),
+                                       __float_as_uint(__uint_as_float(v[4 * kk + 1]) * f),
+                                       __float_as_uint(__uint_as_float(v[4 * kk + 2]) * f),
+                                       __float_as_uint(__uint_as_float(v[4 * kk + 3]) * f));
+                }
+                // this thread has read its dV (dK) rows out of TMEM
+                tc_fence_before();
+                mbar_arrive(which == 0 ? dv_free : dk_free);
+                fence_proxy_async_smem();
+                mbar_arrive(epi_sync);
+                if (epi_issuer) {
+                    if ((ok = mbar_wait(epi_sync, static_cast<uint32_t>(which), p.ctl))) {
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c)
+                            tma_store_3d(which == 0 ? &p.tm_dv : &p.tm_dk, sDS + c * (BKV * 128), c * 32, j * BKV, bh);
+                        bulk_commit_group();
+                        bulk_wait_group_read0();
+                        mbar_arrive(which == 0 ? epi_round : epi_free);
+                    }
+                }
+                ok = __all_sync(0xffffffffu, ok) && warp_wait(which == 0 ? epi_round : epi_free, k & 1, p.ctl);
+            }
+            if (!ok) break;
+        }
         release_item(k);
         }
         // epilogue (one item per CTA): dV rows (times 256 / keep_t under dropout);
         // with 8 warps the warps of query half 1 stage the dK rows (times scale) at
         // the same time, while the dQ warps finish the last dQ.  Persistent CTAs
         // leave the epilogue to the dQ warps and go on to the next item.
-        if (!C::PERSIST && ok && item0 < n_items && warp_wait(dkdv_done, 0, p.ctl)) {
+        if (!PERSIST && ok && item0 < n_items && warp_wait(dkdv_done, 0, p.ctl)) {
             tc_fence_after();
             const ItemInfo w = item_info(item0);
             const bool dk_rows = SMW == 8 && h0 == 1;
@@ -815,8 +914,14 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 bulk_wait_group_read1();
                 mbar_arrive(ds_free);
             }
+            if (EPI_SOFTMAX && issuer && t + 1 == w.n_it) {
+                // the item's last reduce-adds have read the dS^T buffer and the
+                // staging tile: the softmax warps' epilogue may stage there
+                bulk_wait_group_read0();
+                mbar_arrive(dq_stg_free);
+            }
         }
-        if constexpr (C::PERSIST) {
+        if constexpr (PERSIST && !EPI_SOFTMAX) {
             if (!ok) break;
             // epilogue of item k, while the other warps run the next item: dV and dK
             // out of TMEM (lanes = key rows, times 256 / keep_t and scale) into
@@ -870,7 +975,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         // before the grid does
         if (issuer) bulk_wait_group_read0();
         // epilogue (one item per CTA, 4 softmax warps): dK rows (lanes = key rows)
-        if (!C::PERSIST && SMW == 4 && ok && item0 < n_items && warp_wait(dkdv_done, 0, p.ctl)) {
+        if (!PERSIST && SMW == 4 && ok && item0 < n_items && warp_wait(dkdv_done, 0, p.ctl)) {
             tc_fence_after();
             const ItemInfo w = item_info(item0);
             store_rows(1, lane_off, wq * 32, p.scale, w.bh, w.j);
@@ -892,7 +997,8 @@ cudaError_t launch(const BwdParams& p, cudaStream_t stream)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (p.n_ctas, at most the item count); otherwise one per item
-    const dim3 grid = Cfg<D>::PERSIST ? dim3(static_cast<unsigned>(p.n_ctas)) : dim3(p.n_kv_tiles, p.BH);
+    constexpr bool persist = Cfg<D>::PERSIST && !(D == 128 && DROPOUT);
+    const dim3 grid = persist ? dim3(static_cast<unsigned>(p.n_ctas)) : dim3(p.n_kv_tiles, p.BH);
     kern<<<grid, Roles<SMW>::NTHREADS, Cfg<D>::SMEM_BYTES, stream>>>(p);
     return cudaGetLastError();
 }
