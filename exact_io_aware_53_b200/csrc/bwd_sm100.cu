@@ -238,9 +238,9 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     // item have read their staging (dS^T buffer, staging tile); the softmax warps
     // have staged a round (dV, then dK); a round's stores have read the staging
     uint64_t* dq_stg_free = bars + 27;
-    uint64_t* epi_sync = bars + 28;
-    uint64_t* epi_round = bars + 29;
-    uint64_t* epi_free = bars + 30;
+    uint64_t* dv_staged = bars + 28;  // every softmax thread has staged its dV rows
+    uint64_t* dk_staged = bars + 29;  // ... its dK rows
+    uint64_t* epi_free = bars + 30;   // the dK stores have read the dS^T buffer and staging tile
 
     const int warp = static_cast<int>(warp_id());
     const int lane = static_cast<int>(lane_id());
@@ -310,8 +310,8 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         mbar_init(dv_free, EPI_SOFTMAX ? 32 * SMW : 128);
         mbar_init(dk_free, EPI_SOFTMAX ? 32 * SMW : 128);
         mbar_init(dq_stg_free, 1);
-        mbar_init(epi_sync, 32 * SMW);
-        mbar_init(epi_round, 1);
+        mbar_init(dv_staged, 32 * SMW);
+        mbar_init(dk_staged, 32 * SMW);
         mbar_init(epi_free, 1);
         for (int u = 0; u < 2; ++u) {
             mbar_init(&item_full[u], 1);
@@ -568,7 +568,8 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     if (cross) {
                         mma_commit_elect(dkdv_done);  // the item's dV, dK are complete
                         // and no MMA reads its K, V any more: the producer may refill them
-                        if (PERSIST) mma_commit_elect(kv_empty_b[k & (C::KV_BUFS - 1)]);
+                        // (d = 128: the epilogue stages dV there first and releases it)
+                        if (PERSIST && !EPI_SOFTMAX) mma_commit_elect(kv_empty_b[k & (C::KV_BUFS - 1)]);
                     }
                     if (more && !early_next && !(ok = issue_next_s())) break;
                     if (more) {
@@ -759,17 +760,16 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
         }
         if constexpr (EPI_SOFTMAX) {
             if (!ok) break;
-            // epilogue of item k (d = 128): dV, then dK, out of TMEM (lanes = key
-            // rows; with 8 warps each takes half of the columns) into four
-            // 128-byte-swizzled [128 rows][32 columns] fp32 boxes over the dS^T
-            // buffer and the dQ staging tile, which the item's last dK, dQ MMAs and
-            // reduce-adds have read; warp 0's first thread issues the TMA tile
-            // stores of a round once every warp has staged it (rows past N are
-            // clipped) and releases the boxes when the stores have read them.
-            // Meanwhile the next item's keys and first query tile load and its
-            // first S^T and dP^T run.
+            // epilogue of item k (d = 128): dV and dK out of TMEM (lanes = key rows;
+            // with 8 warps each takes half of the columns) into 128-byte-swizzled
+            // [128 rows][32 columns] fp32 boxes: dV over the K, V buffer, free once
+            // the item's MMAs are complete, and dK over the dS^T buffer and the dQ
+            // staging tile once the dQ warps' last reduce-adds have read them.
+            // Warp 0's first thread issues each half's TMA tile stores when every
+            // warp has staged it (rows past N are clipped); once the dV stores have
+            // read the K, V buffer it releases it to the producer, which loads the
+            // next item's keys while the dK half is staged and stored.
             if (!(ok = warp_wait(dkdv_done, k & 1, p.ctl))) break;
-            if (!(ok = warp_wait(dq_stg_free, k & 1, p.ctl))) break;
             tc_fence_after();
             const bool epi_issuer = warp == 0 && lane == 0;
             const int c0 = SMW == 8 ? h0 * (D / 2) : 0;
@@ -777,13 +777,15 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             const uint32_t l = static_cast<uint32_t>(r);  // key row
 #pragma unroll
             for (int which = 0; which < 2 && ok; ++which) {
+                if (which == 1 && !(ok = warp_wait(dq_stg_free, k & 1, p.ctl))) break;
+                uint8_t* area = which == 0 ? sK : sDS;
                 const uint32_t col = which == 0 ? C::DV_COL : C::DK_COL;
                 const float f = which == 0 ? (DROPOUT ? p.keep_scale : 1.f) : p.scale;
                 for (int cc = c0; cc < c1; cc += 32) {
                     uint32_t v[32];
                     tmem_ld32(tmem + lane_off + col + static_cast<uint32_t>(cc), v);
                     tmem_wait_ld();
-                    uint8_t* box = sDS + (cc / 32) * (BKV * 128);
+                    uint8_t* box = area + (cc / 32) * (BKV * 128);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
                         *reinterpret_cast<uint4*>(box + sw128_offset(l, kk)) =
@@ -796,19 +798,21 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 tc_fence_before();
                 mbar_arrive(which == 0 ? dv_free : dk_free);
                 fence_proxy_async_smem();
-                mbar_arrive(epi_sync);
+                mbar_arrive(which == 0 ? dv_staged : dk_staged);
                 if (epi_issuer) {
-                    if ((ok = mbar_wait(epi_sync, static_cast<uint32_t>(which), p.ctl))) {
+                    if ((ok = mbar_wait(which == 0 ? dv_staged : dk_staged, static_cast<uint32_t>(k & 1), p.ctl))) {
 #pragma unroll
                         for (int c = 0; c < D / 32; ++c)
-                            tma_store_3d(which == 0 ? &p.tm_dv : &p.tm_dk, sDS + c * (BKV * 128), c * 32, j * BKV, bh);
+                            tma_store_3d(which == 0 ? &p.tm_dv : &p.tm_dk, area + c * (BKV * 128), c * 32, j * BKV, bh);
                         bulk_commit_group();
                         bulk_wait_group_read0();
-                        mbar_arrive(which == 0 ? epi_round : epi_free);
+                        mbar_arrive(which == 0 ? kv_empty_b[0] : epi_free);
                     }
                 }
-                ok = __all_sync(0xffffffffu, ok) && warp_wait(which == 0 ? epi_round : epi_free, k & 1, p.ctl);
+                ok = __all_sync(0xffffffffu, ok);
             }
+            // the dS^T buffer and the staging tile are read before the next item's dS^T
+            ok = ok && warp_wait(epi_free, k & 1, p.ctl);
             if (!ok) break;
         }
         release_item(k);
