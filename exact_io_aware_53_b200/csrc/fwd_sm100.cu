@@ -651,9 +651,21 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                 ++pc;
             }
             if (ok && nk == 0) {
-                // tile 1 past N: pass the staging tile on
+                // tile 1 past N: pass the staging tile on, as the last of the tile's
+                // 8 warps to have seen it free -- not as soon as one warp has, which
+                // would let a slower warp of this tile miss the phase and wait for
+                // the next one (the next item's tile 0), while that item's tile 1
+                // needs this warp
                 ok = warp_wait(stg_free, 0u, p.ctl);
-                if (ok && warp == 8 && lane == 0) mbar_arrive(stg_free);
+                if (ok) {
+                    __syncwarp();
+                    if (lane == 0 && atomicAdd(stg_count, 1u) == 7u) {
+                        __threadfence_block();
+                        *stg_count = 0u;
+                        mbar_arrive(stg_free);
+                    }
+                    __syncwarp();
+                }
             }
             if (ok && nk > 0) {
                 ok = warp_wait(&o_full[t], oc & 1, p.ctl);
