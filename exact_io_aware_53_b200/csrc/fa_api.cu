@@ -789,7 +789,7 @@ namespace {
 // chunk overlap the compute of the next and, on a full-duplex link, the two copy
 // directions overlap each other.  The two copy streams and the events that order
 // the stages are created once per device and kept until the process exits.
-constexpr int kHostMaxChunks = 8;
+constexpr int kHostMaxChunks = 9;
 constexpr int kHostMaxDevices = 64;
 
 struct HostPipe {
@@ -868,12 +868,17 @@ int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const v
     void* ws = a;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    // chunks of G heads, G a multiple of 4 so that every chunk's LSE slice
-    // starts on a 16-byte boundary (the bf16 and fp32 rows always do)
+    // Chunks of whole heads, each a multiple of 4 heads so that every chunk's LSE
+    // slice starts on a 16-byte boundary (the bf16 and fp32 rows always do): a
+    // first chunk of 4, so that the copy-out stream (the slowest stage) starts
+    // early, then up to 8 chunks of G heads.
     const int BH = B * H;
-    int G = (BH + kHostMaxChunks - 1) / kHostMaxChunks;
-    G = (G + 3) / 4 * 4;
-    const int n_chunks = (BH + G - 1) / G;
+    const int G0 = std::min(BH, 4);
+    int G = (BH - G0 + (kHostMaxChunks - 1) - 1) / (kHostMaxChunks - 1);
+    G = std::max(4, (G + 3) / 4 * 4);
+    const int n_chunks = 1 + (BH - G0 + G - 1) / G;
+    auto chunk_h0 = [&](int c) { return c == 0 ? 0 : G0 + (c - 1) * G; };
+    auto chunk_gh = [&](int c) { return std::min(c == 0 ? G0 : G, BH - chunk_h0(c)); };
 
     std::lock_guard<std::mutex> lk(g_pipe_mu);
     HostPipe* hp = nullptr;
@@ -887,8 +892,8 @@ int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const v
                            static_cast<const char*>(h_v), static_cast<const char*>(h_dO)};
     char* dsrc[4] = {q, k, v, dO};
     for (int c = 0; c < n_chunks; ++c) {
-        const size_t h0 = static_cast<size_t>(c) * G;
-        const size_t gh = std::min<size_t>(G, BH - h0);
+        const size_t h0 = static_cast<size_t>(chunk_h0(c));
+        const size_t gh = static_cast<size_t>(chunk_gh(c));
         const size_t off = h0 * N * d * 2, bytes = gh * N * d * 2;
         for (int i = 0; i < 4; ++i)
             if ((st = cuda_status(cudaMemcpyAsync(dsrc[i] + off, hsrc[i] + off, bytes, cudaMemcpyHostToDevice,
@@ -898,8 +903,8 @@ int fa_attention_host(const void* h_q, const void* h_k, const void* h_v, const v
     }
     int launches = 0;
     for (int c = 0; c < n_chunks; ++c) {
-        const size_t h0 = static_cast<size_t>(c) * G;
-        const int gh = static_cast<int>(std::min<size_t>(G, BH - h0));
+        const size_t h0 = static_cast<size_t>(chunk_h0(c));
+        const int gh = chunk_gh(c);
         const size_t e2 = h0 * N * d * 2, e4 = h0 * N * d * 4, r4 = h0 * N * 4;
         if ((st = cuda_status(cudaStreamWaitEvent(s, hp->in_done[c], 0))) != FA_OK) return st;
         // the chunk is gh heads of one batch: heads are independent in both passes

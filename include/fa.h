@@ -159,8 +159,9 @@ size_t fa_attention_host_arena_bytes(int B, int H, int N, int d);
  * (bf16, host memory -- pinned for asynchronous copies) into `arena` (device,
  * fa_attention_host_arena_bytes bytes, 256-byte aligned), runs fa_fwd and
  * fa_bwd there, and copies o (bf16), lse, dq, dk, dv (fp32) back to the host
- * buffers.  The heads are processed in up to 8 chunks (a multiple of 4 heads
- * each; heads are independent in both passes): chunk c is copied in on a
+ * buffers.  The heads are processed in chunks (heads are independent in both
+ * passes): a first chunk of 4 heads, then up to 8 of equal size, each a
+ * multiple of 4 heads except the last: chunk c is copied in on a
  * library-owned copy-in stream, computed on `stream`, and copied back on a
  * library-owned copy-out stream, ordered by events, so that the copies of one
  * chunk overlap the compute and the copies of the others.  The two copy

@@ -21,10 +21,10 @@ from tests._parity import BF16_TOL, LSE_TOL, max_abs
 pytestmark = pytest.mark.gpu
 
 SHAPES = [
-    # (B, H, N, d, causal): chunks of G heads, G = 4 * ceil(ceil(B*H / 8) / 4)
+    # (B, H, N, d, causal): a first chunk of 4 heads, then chunks of G heads
     (1, 3, 200, 128, False),   # one chunk
     (2, 9, 333, 64, True),     # 18 heads: chunks 4, 4, 4, 4, 2; N odd
-    (4, 16, 1024, 128, True),  # 64 heads: 8 chunks of 8
+    (4, 16, 1024, 128, True),  # 64 heads: 4, then 8 chunks of 8 (the last 4)
     (3, 5, 130, 64, False),    # 15 heads: chunks 4, 4, 4, 3
 ]
 
@@ -56,8 +56,10 @@ def test_host_step_equals_device_calls(fa_lib, shape):
     o, lse = fa.fwd(xc["q"], xc["k"], xc["v"], causal=causal, scale=scale)
     dq, dk, dv = fa.bwd(xc["q"], xc["k"], xc["v"], o, lse, xc["do"], causal=causal, scale=scale)
     torch.cuda.synchronize()
-    G = 4 * math.ceil(math.ceil(B * H / 8) / 4)
-    assert launches == 3 * math.ceil(B * H / G)  # forward, pre-pass and main kernel per chunk
+    BH = B * H  # a first chunk of min(BH, 4) heads, then chunks of G (a multiple of 4) heads
+    G0 = min(BH, 4)
+    G = max(4, 4 * math.ceil(math.ceil((BH - G0) / 8) / 4))
+    assert launches == 3 * (1 + math.ceil((BH - G0) / G))  # forward, pre-pass and main kernel per chunk
     assert torch.equal(outs["o"], o.cpu())
     assert torch.equal(outs["lse"], lse.cpu())
     assert torch.equal(outs["dk"], dk.cpu())
