@@ -194,8 +194,8 @@ struct Cfg {
     static constexpr int STG_OFF = KV_OFF + STAGES * TILE_BYTES;  // O staging tile (bf16)
     static constexpr int BAR_OFF = STG_OFF + STG_BYTES;
     // q_full, q_empty, kv_full/empty[S], s_full, p_full, o_full, o_free [2],
-    // item_full, item_empty [2], drain, stg_free
-    static constexpr int NBARS = 2 + 2 * STAGES + 4 * 2 + 2 * 2 + 1 + 1;
+    // item_full, item_empty [2], drain, stg_done [2]
+    static constexpr int NBARS = 2 + 2 * STAGES + 4 * 2 + 2 * 2 + 1 + 2;
     static constexpr int SMEM_BYTES = BAR_OFF + NBARS * 8 + 16 + 1024;  // + TMEM slot, item ring, staging count
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static constexpr uint32_t TMEM_COLS = 512;
@@ -267,9 +267,11 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
     uint64_t* item_full = o_free + 2;         // [2]
     uint64_t* item_empty = item_full + 2;     // [2]
     uint64_t* drain = item_empty + 2;
-    uint64_t* stg_free = drain + 1;  // the TMA store has read the staging tile
+    // [2]: Q tile t's turn at the staging tile is over (its TMA store has read
+    // the tile, or a tile past N has passed its turn on)
+    uint64_t* stg_done = drain + 1;
     uint8_t* sSTG = smem + C::STG_OFF;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
     unsigned int* stg_count = tmem_slot + 3;  // warps of a Q tile done writing the staging tile
     int* item_buf = reinterpret_cast<int*>(tmem_slot + 1);  // [2]
 
@@ -295,7 +297,8 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
             mbar_init(&item_empty[t], 1 + 16);  // the MMA warp and the 16 softmax warps
         }
         mbar_init(drain, 1);
-        mbar_init(stg_free, 1);
+        mbar_init(&stg_done[0], 1);
+        mbar_init(&stg_done[1], 1);
         *stg_count = 0u;
         fence_mbar_init();
     }
@@ -490,9 +493,16 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
         int ring0 = 0;    // K/V ring slots used by earlier items
         // O leaves through one staging tile that the two Q tiles take in turn, in
         // the order their O is complete: tile 0 then tile 1 within an item (tile 0
-        // never has more key tiles), item after item.  Use 2 n + t therefore waits
-        // for the staging tile's free phase of parity t ^ 1; an item whose tile 1
-        // lies past N still takes its turn, without writing anything.
+        // never has more key tiles), item after item.  Each tile ends its turn with
+        // one arrival on its own barrier stg_done[t], so a turn waits for phase n of
+        // the other tile's barrier (tile 1 of item n: tile 0's turn of item n; tile 0:
+        // tile 1's turn of item n - 1).  A tile's warps thus wait on consecutive
+        // phases, one per item, and no warp can run two phases ahead of the barrier
+        // it waits on: with one barrier for both tiles a warp waited on every other
+        // phase, and a fast warp whose previous turn was not yet stored saw the
+        // phase two before its own as complete (a wait by parity cannot tell them
+        // apart) and wrote the staging tile while that store still read it.  An
+        // item whose tile 1 lies past N still takes its turn, without writing.
         bool ok = true;
         for (int n = 0; ok; ++n) {
             const int slot = n & 1;
@@ -650,19 +660,19 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                 mbar_arrive(&p_full[t]);
                 ++pc;
             }
+            // this tile's turn waits for the other tile's turn before it (above)
+            const uint32_t turn_parity = static_cast<uint32_t>((n & 1) ^ t ^ 1);
             if (ok && nk == 0) {
-                // tile 1 past N: pass the staging tile on, as the last of the tile's
-                // 8 warps to have seen it free -- not as soon as one warp has, which
-                // would let a slower warp of this tile miss the phase and wait for
-                // the next one (the next item's tile 0), while that item's tile 1
-                // needs this warp
-                ok = warp_wait(stg_free, 0u, p.ctl);
+                // tile 1 past N: pass the turn on, as the last of the tile's 8 warps
+                // to have seen tile 0's turn end -- every warp waits for that phase,
+                // so that none of them is left a phase behind at the next item
+                ok = warp_wait(&stg_done[0], turn_parity, p.ctl);
                 if (ok) {
                     __syncwarp();
                     if (lane == 0 && atomicAdd(stg_count, 1u) == 7u) {
                         __threadfence_block();
                         *stg_count = 0u;
-                        mbar_arrive(stg_free);
+                        mbar_arrive(&stg_done[1]);
                     }
                     __syncwarp();
                 }
@@ -670,7 +680,7 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
             if (ok && nk > 0) {
                 ok = warp_wait(&o_full[t], oc & 1, p.ctl);
                 ++oc;
-                if (ok) ok = warp_wait(stg_free, static_cast<uint32_t>(t ^ 1), p.ctl);
+                if (ok) ok = warp_wait(&stg_done[t ^ 1], turn_parity, p.ctl);
                 if (ok) {
                     tc_fence_after();
                     // each row's sum is split over its four threads
@@ -732,7 +742,7 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                                 tma_store_3d(&p.tm_o, sSTG + c * C::BOX_BYTES, c * 64, w.q0 + t * BM, w.bh);
                             bulk_commit_group();
                             bulk_wait_group_read0();
-                            mbar_arrive(stg_free);
+                            mbar_arrive(&stg_done[t]);
                         }
                     }
                     __syncwarp();
