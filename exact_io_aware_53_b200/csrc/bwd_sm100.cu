@@ -398,8 +398,8 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     if (!mbar_wait(kv_empty_b[b], ((k / C::KV_BUFS) & 1) ^ 1, p.ctl)) return false;
                     mbar_arrive_expect_tx(kv_full_b[b], 2 * C::TILE);
                     for (int c = 0; c < C::NDC; ++c) {
-                        tma_load_3d(sK + 2 * b * C::TILE + c * BOX, &p.tm_k, kv_full_b[b], c * 64, w.j * BKV, w.bh);
-                        tma_load_3d(sV + 2 * b * C::TILE + c * BOX, &p.tm_v, kv_full_b[b], c * 64, w.j * BKV, w.bh);
+                        tma_load_3d(sK + 2 * b * C::TILE + c * BOX, &p.tm_k, kv_full_b[b], c * 64, w.j * BKV, w.bh, &p.ctl);
+                        tma_load_3d(sV + 2 * b * C::TILE + c * BOX, &p.tm_v, kv_full_b[b], c * 64, w.j * BKV, w.bh, &p.ctl);
                     }
                     ++nkv;
                     return true;
@@ -412,13 +412,13 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     if (!mbar_wait(&q_empty[s], ((T >> 1) & 1) ^ 1, p.ctl)) return false;
                     mbar_arrive_expect_tx(&q_full[s], C::TILE + 2 * BQ * 4);
                     for (int c = 0; c < C::NDC; ++c)
-                        tma_load_3d(sQ + s * C::TILE + c * BOX, &p.tm_q, &q_full[s], c * 64, i * BQ, w.bh);
-                    bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &q_full[s]);
-                    bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &q_full[s]);
+                        tma_load_3d(sQ + s * C::TILE + c * BOX, &p.tm_q, &q_full[s], c * 64, i * BQ, w.bh, &p.ctl);
+                    bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &q_full[s], &p.ctl);
+                    bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &q_full[s], &p.ctl);
                     ++nq;
                     if (!mbar_wait(do_empty, (T & 1) ^ 1, p.ctl)) return false;
                     mbar_arrive_expect_tx(do_full, C::TILE);
-                    for (int c = 0; c < C::NDC; ++c) tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, w.bh);
+                    for (int c = 0; c < C::NDC; ++c) tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, w.bh, &p.ctl);
                     ++ndo;
                     ++T;
                     return true;
@@ -803,7 +803,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     if ((ok = mbar_wait(which == 0 ? dv_staged : dk_staged, static_cast<uint32_t>(k & 1), p.ctl))) {
 #pragma unroll
                         for (int c = 0; c < D / 32; ++c)
-                            tma_store_3d(which == 0 ? &p.tm_dv : &p.tm_dk, area + c * (BKV * 128), c * 32, j * BKV, bh);
+                            tma_store_3d(which == 0 ? &p.tm_dv : &p.tm_dk, area + c * (BKV * 128), c * 32, j * BKV, bh, &p.ctl);
                         bulk_commit_group();
                         bulk_wait_group_read0();
                         mbar_arrive(which == 0 ? kv_empty_b[0] : epi_free);
@@ -908,8 +908,8 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 fence_proxy_async_smem();
                 if (!(ok = sync_dq())) break;
                 if (issuer) {
-                    tma_reduce_add_3d(&p.tm_dq, stg, hd * 64, i * BQ, bh);
-                    tma_reduce_add_3d(&p.tm_dq, stg + C::STG_CHUNK, hd * 64 + 32, i * BQ, bh);
+                    tma_reduce_add_3d(&p.tm_dq, stg, hd * 64, i * BQ, bh, &p.ctl);
+                    tma_reduce_add_3d(&p.tm_dq, stg + C::STG_CHUNK, hd * 64 + 32, i * BQ, bh, &p.ctl);
                     bulk_commit_group();
                 }
             }
@@ -967,8 +967,8 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             if (issuer) {
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    tma_store_3d(&p.tm_dv, sEPI + c * (BKV * 128), c * 32, w.j * BKV, w.bh);
-                    tma_store_3d(&p.tm_dk, sSTG + c * (BKV * 128), c * 32, w.j * BKV, w.bh);
+                    tma_store_3d(&p.tm_dv, sEPI + c * (BKV * 128), c * 32, w.j * BKV, w.bh, &p.ctl);
+                    tma_store_3d(&p.tm_dk, sSTG + c * (BKV * 128), c * 32, w.j * BKV, w.bh, &p.ctl);
                 }
                 bulk_commit_group();
             }

@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
         if (lane == 0) {
             mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
             for (int c = 0; c < C::NDC; ++c)
-                tma_load_3d(sQ + c * C::BOX_BYTES, &p.tm_q, q_full, c * 64, qt * BM, bh);
+                tma_load_3d(sQ + c * C::BOX_BYTES, &p.tm_q, q_full, c * 64, qt * BM, bh, &p.ctl);
             int it = 0;
             bool ok = true;
             for (int jj = 0; jj < nj && ok; ++jj) {
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(NTHREADS, 2) decode_partial_kernel(const __gri
                     const int krow = tile_of(jj) * BN;
                     for (int c = 0; c < C::NDC; ++c)
                         tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64, krow,
-                                    bh);
+                                    bh, &p.ctl);
                     ++it;
                 }
             }

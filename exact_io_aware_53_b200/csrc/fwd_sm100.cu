@@ -345,7 +345,7 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                     if (w.n_kv[t] > 0)
                         for (int c = 0; c < C::NDC; ++c)
                             tma_load_3d(sQ + t * C::TILE_BYTES + c * C::BOX_BYTES, &p.tm_q, q_full, c * 64,
-                                        w.q0 + t * BM, w.bh);
+                                        w.q0 + t * BM, w.bh, &p.ctl);
                 ++nq;
                 for (int j = 0; j < w.n_kv_max && ok; ++j) {
                     for (int kind = 0; kind < 2; ++kind) {
@@ -361,11 +361,11 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                             // box order f, q, h, b): shared-memory row 16 b + 8 h + 2 q + f holds
                             // key 16 b + 4 q + 2 h + f, so a thread's S columns pair up into
                             // P words (N is a multiple of 16: blocks never straddle heads)
-                            tma_load_5d(sKV + s * C::TILE_BYTES, map, &kv_full[s], 0, 0, 0, 0, (w.bh * N + j * BN) / 16);
+                            tma_load_5d(sKV + s * C::TILE_BYTES, map, &kv_full[s], 0, 0, 0, 0, (w.bh * N + j * BN) / 16, &p.ctl);
                         } else {
                             for (int c = 0; c < C::NDC; ++c)
                                 tma_load_3d(sKV + s * C::TILE_BYTES + c * C::BOX_BYTES, map, &kv_full[s], c * 64,
-                                            j * BN, w.bh);
+                                            j * BN, w.bh, &p.ctl);
                         }
                         ++it;
                     }
@@ -739,7 +739,7 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
                             *stg_count = 0u;
                             fence_proxy_async_smem();
                             for (int c = 0; c < C::OUT_NDC; ++c)
-                                tma_store_3d(&p.tm_o, sSTG + c * C::BOX_BYTES, c * 64, w.q0 + t * BM, w.bh);
+                                tma_store_3d(&p.tm_o, sSTG + c * C::BOX_BYTES, c * 64, w.q0 + t * BM, w.bh, &p.ctl);
                             bulk_commit_group();
                             bulk_wait_group_read0();
                             mbar_arrive(&stg_done[t]);

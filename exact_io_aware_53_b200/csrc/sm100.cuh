@@ -133,11 +133,36 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
     }
 }
 
+#ifdef FA_CHECK_BUILD
+// Check build (libfa_sm100_check.so, for tests): one bounded wait in four sleeps
+// a pseudo-random 0 .. 2047 ns once it has succeeded, so that warps reach their
+// next synchronisation in orders that normal timing does not produce.  A race
+// between them (a barrier phase read as complete too early or too late, a
+// buffer reused before its reader is done) then shows up in the parity tests
+// as a wrong result or an expired wait instead of staying hidden.
+__device__ __forceinline__ void check_build_jitter()
+{
+    uint32_t h;
+    asm volatile("mov.u32 %0, %%clock;" : "=r"(h));
+    h = h * 2654435761u ^ threadIdx.x * 40503u ^ blockIdx.x * 9973u ^ blockIdx.y * 7919u;
+    h ^= h >> 13;
+    h *= 0x5bd1e995u;
+    h ^= h >> 15;
+    if ((h & 3u) == 0u) __nanosleep((h >> 8) & 2047u);
+}
+#endif
+
 // Bounded wait for the phase of `bar` with the given parity.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c)
 {
+#ifdef FA_CHECK_BUILD
+    const bool done = mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, c);
+    check_build_jitter();
+    return done;
+#else
     if (mbar_try_wait(bar, parity)) return true;
     return mbar_wait_slow(bar, parity, c);
+#endif
 }
 
 // Bounded wait used on error paths: ignores the device error word (so copies
@@ -158,11 +183,33 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Every tile copy below takes the kernel's WaitCtl (or null).  In the check
+// build each copy's coordinates are tested first: the innermost one must be a
+// non-negative multiple of 32 elements (every copy in this library starts on
+// a 64- or 32-element box boundary, which keeps it 16-byte aligned for 8-, 16-
+// and 32-bit elements) and the others non-negative (no copy starts before a
+// tensor; one that ends past it is clipped, as rows past N are).  A copy that
+// fails is not issued and FA_DEV_BAD_TILE is raised in the device error word;
+// its barrier then never completes and the bounded wait on it gives up.  The
+// untiled bulk copies are tested for 16-byte aligned addresses and sizes.
+__device__ __forceinline__ bool tile_coords_ok(const WaitCtl* chk, bool ok)
+{
+#ifdef FA_CHECK_BUILD
+    if (!ok && chk != nullptr) raise_status(*chk, FA_DEV_BAD_TILE);
+    return ok;
+#else
+    (void)chk;
+    (void)ok;
+    return true;
+#endif
+}
+
 // 3-D tiled load, completion counted in bytes on `bar`.  x is the innermost
 // coordinate and must be a multiple of 16 bytes / element size.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
-                                            int z)
+                                            int z, const WaitCtl* chk = nullptr)
 {
+    if (!tile_coords_ok(chk, x >= 0 && (x & 31) == 0 && y >= 0 && z >= 0)) return;
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
@@ -171,8 +218,9 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 }
 
 __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
-                                            int c2, int c3, int c4)
+                                            int c2, int c3, int c4, const WaitCtl* chk = nullptr)
 {
+    if (!tile_coords_ok(chk, c0 >= 0 && (c0 & 31) == 0 && c1 >= 0 && c2 >= 0 && c3 >= 0 && c4 >= 0)) return;
     asm volatile(
         "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
@@ -180,8 +228,10 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y)
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            const WaitCtl* chk = nullptr)
 {
+    if (!tile_coords_ok(chk, x >= 0 && (x & 31) == 0 && y >= 0)) return;
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
@@ -190,8 +240,11 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
 }
 
 // Untiled bulk copy global -> shared (16-byte aligned addresses, size multiple of 16).
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          const WaitCtl* chk = nullptr)
 {
+    if (!tile_coords_ok(chk, ((smem_u32(dst) | static_cast<uint32_t>(reinterpret_cast<uintptr_t>(src)) | bytes) & 15u) == 0u))
+        return;
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
             smem_u32(dst)),
@@ -200,8 +253,10 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 
 // 3-D tiled store shared -> global (rows outside the tensor are clipped).
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z)
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z,
+                                             const WaitCtl* chk = nullptr)
 {
+    if (!tile_coords_ok(chk, x >= 0 && (x & 31) == 0 && y >= 0 && z >= 0)) return;
     asm volatile(
         "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
             reinterpret_cast<uint64_t>(map)),
@@ -210,8 +265,10 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
 }
 
 // 3-D tiled reduce-add shared -> global (fp32 add; clipped like a store).
-__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int x, int y, int z)
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int x, int y, int z,
+                                                  const WaitCtl* chk = nullptr)
 {
+    if (!tile_coords_ok(chk, x >= 0 && (x & 31) == 0 && y >= 0 && z >= 0)) return;
     asm volatile(
         "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
             reinterpret_cast<uint64_t>(map)),

@@ -4,6 +4,10 @@ Every step of attention runs in the CUDA library ``libfa_sm100.so``; this
 module checks torch tensors, passes their device pointers and the current
 stream, and turns status codes into exceptions.  Importing it fails loudly if
 the library has not been built: there is no fallback path.
+
+``check_build()`` returns the same binding over ``libfa_sm100_check.so``, the
+build with jittered barrier waits and tested tile coordinates that the
+race-stress tests run.
 """
 from __future__ import annotations
 
@@ -14,11 +18,15 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libfa_sm100.so")
+# "check" when this module object was made by check_build() (set before the
+# module's code runs); the ordinary import binds the release library
+VARIANT = globals().get("VARIANT", "")
+LIB_PATH = os.path.join(_PKG, "libfa_sm100_check.so" if VARIANT == "check" else "libfa_sm100.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError("libfa_sm100.so is not built; run `python -m exact_io_aware_53_b200.build` "
-                      "(or __graft_entry__.build()) first")
+    raise ImportError("%s is not built; run `python -m exact_io_aware_53_b200.build%s` "
+                      "(or __graft_entry__.build()) first" % (os.path.basename(LIB_PATH),
+                                                               " --check" if VARIANT == "check" else ""))
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -99,6 +107,29 @@ def _ptr(t):
 
 def exported_symbols():
     return list(_SIGS)
+
+
+_check_module = None
+
+
+def check_build():
+    """This binding over the check build (libfa_sm100_check.so): the same kernels
+    compiled with FA_CHECK_BUILD, whose bounded waits sleep a pseudo-random
+    0-2 us once in four after they succeed and whose tile copies test their
+    coordinates first (a bad one raises the device error word instead of being
+    issued).  A separate module object with the same functions; loaded once."""
+    global _check_module
+    if VARIANT == "check":
+        return globals()["__check_self__"]
+    if _check_module is None:
+        import importlib.util
+        spec = importlib.util.spec_from_file_location(__name__ + "_check", __file__)
+        mod = importlib.util.module_from_spec(spec)
+        mod.VARIANT = "check"
+        mod.__check_self__ = mod
+        spec.loader.exec_module(mod)
+        _check_module = mod
+    return _check_module
 
 
 def status_string(status: int) -> str:

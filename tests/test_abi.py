@@ -36,6 +36,20 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(names) == set(lib.exported_symbols())
 
 
+def test_check_build_exports_the_same_entry_points(lib):
+    """The check build (jittered waits, tested tile coordinates) is the same
+    interface: every declared symbol, loaded as a second binding."""
+    from exact_io_aware_53_b200 import build
+    build.build(check=True)
+    chk = lib.check_build()
+    assert chk is not lib and chk.LIB_PATH != lib.LIB_PATH
+    assert chk.LIB_PATH.endswith("libfa_sm100_check.so")
+    so = ctypes.CDLL(chk.LIB_PATH)
+    for n in _declared():
+        assert hasattr(so, n), n
+    assert chk.status_string(5) == lib.status_string(5)
+
+
 def test_status_strings(lib):
     assert lib.status_string(0) == "FA_OK"
     assert lib.status_string(5) == "FA_ERR_TIMEOUT"
