@@ -103,8 +103,12 @@ struct Cfg {
     static constexpr int K_OFF = 0;                        // buffer b: K at K_OFF + 2 b TILE, V after it
     static constexpr int V_OFF = K_OFF + TILE;
     static constexpr int Q_OFF = KV_BUFS * 2 * TILE;       // Q_t, 2 stages
-    static constexpr int DO_OFF = Q_OFF + QSTAGES * TILE;  // dO_t, 1 stage
-    static constexpr int DS_OFF = DO_OFF + TILE;           // dS^T: 2 boxes of 64 query columns
+    // dO_t: at d = 64 one stage per Q stage, loaded with Q_t under its barrier
+    // (its readers, dP^T of the tile and its dV, come before the tile's dK, whose
+    // commit frees the Q stage); at d = 128 one stage with its own barriers
+    static constexpr int DO_STAGES = D == 64 ? QSTAGES : 1;
+    static constexpr int DO_OFF = Q_OFF + QSTAGES * TILE;
+    static constexpr int DS_OFF = DO_OFF + DO_STAGES * TILE;  // dS^T: 2 boxes of 64 query columns
     static constexpr int STG_OFF = DS_OFF + 2 * BOX;       // dQ staging
     // fp32 staging tile: 2 chunks of [STG_ROWS query rows][32 d], 128-byte swizzled
     // (64 of the d columns at a time)
@@ -191,6 +195,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
     // slower (1.31 against 1.19 ms, 4x16x4096x128 causal) and runs one CTA per item
     constexpr bool PERSIST = C::PERSIST && !(D == 128 && DROPOUT);
     constexpr bool EPI_SOFTMAX = PERSIST && C::EPI_SOFTMAX;
+    constexpr bool DO_WITH_Q = C::DO_STAGES == QSTAGES;  // dO_t shares Q_t's stage and barriers
     extern __shared__ __align__(1024) uint8_t smem[];
     // the 128-byte-swizzled tiles need a 1024-byte aligned base; the layout
     // leaves no slack, so a misaligned base is reported instead of used
@@ -410,16 +415,22 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     const int s = T & 1;
                     const int i = w.i_first + t;
                     if (!mbar_wait(&q_empty[s], ((T >> 1) & 1) ^ 1, p.ctl)) return false;
-                    mbar_arrive_expect_tx(&q_full[s], C::TILE + 2 * BQ * 4);
+                    mbar_arrive_expect_tx(&q_full[s], C::TILE + 2 * BQ * 4 + (DO_WITH_Q ? C::TILE : 0));
                     for (int c = 0; c < C::NDC; ++c)
                         tma_load_3d(sQ + s * C::TILE + c * BOX, &p.tm_q, &q_full[s], c * 64, i * BQ, w.bh, &p.ctl);
                     bulk_load(sVec + s * 2 * BQ, lse2_h + i * BQ, BQ * 4, &q_full[s], &p.ctl);
                     bulk_load(sVec + s * 2 * BQ + BQ, delta_h + i * BQ, BQ * 4, &q_full[s], &p.ctl);
                     ++nq;
-                    if (!mbar_wait(do_empty, (T & 1) ^ 1, p.ctl)) return false;
-                    mbar_arrive_expect_tx(do_full, C::TILE);
-                    for (int c = 0; c < C::NDC; ++c) tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, w.bh, &p.ctl);
-                    ++ndo;
+                    if constexpr (DO_WITH_Q) {
+                        for (int c = 0; c < C::NDC; ++c)
+                            tma_load_3d(sDO + s * C::TILE + c * BOX, &p.tm_do, &q_full[s], c * 64, i * BQ, w.bh, &p.ctl);
+                    } else {
+                        if (!mbar_wait(do_empty, (T & 1) ^ 1, p.ctl)) return false;
+                        mbar_arrive_expect_tx(do_full, C::TILE);
+                        for (int c = 0; c < C::NDC; ++c)
+                            tma_load_3d(sDO + c * BOX, &p.tm_do, do_full, c * 64, i * BQ, w.bh, &p.ctl);
+                        ++ndo;
+                    }
                     ++T;
                     return true;
                 };
@@ -454,6 +465,7 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
             const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
                            aDS = smem_u32(sDS);
             auto q_base = [&](int t) { return aQ + (t & 1) * C::TILE; };
+            auto do_base = [&](int t) { return aDO + (DO_WITH_Q ? (t & 1) : 0) * C::TILE; };
             // (K or V) x (Q or dO)^T, both K-major over the head dimension
             auto issue_kk = [&](uint32_t d_col, uint32_t a_base, uint32_t b_base) {
 #pragma unroll
@@ -464,11 +476,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 }
             };
             // dV += P^T (TMEM: queries 16 kk .. 16 kk + 15 in half kk / 4) x dO (MN-major over d)
-            auto issue_dv = [&](uint32_t a_col, bool acc0) {
+            auto issue_dv = [&](uint32_t a_col, uint32_t b_base, bool acc0) {
 #pragma unroll
                 for (int kk = 0; kk < BQ / 16; ++kk)
                     mma_ts_elect(tmem + C::DV_COL, tmem + a_col + (kk >> 2) * 64 + (kk & 3) * 8,
-                           sdesc_sw128(aDO + kk * 2048, BOX, 1024), idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
+                           sdesc_sw128(b_base + kk * 2048, BOX, 1024), idesc_tm, (acc0 || kk > 0) ? 1u : 0u);
             };
             // dK += dS^T (shared, K-major) x Q (MN-major over d)
             auto issue_dk = [&](uint32_t b_base, bool acc0) {
@@ -493,10 +505,11 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                 tc_fence_after();
                 issue_kk(rcol(0), kbase(0), q_base(0));
                 mma_commit_elect(s_full);
-                ok = warp_wait(do_full, 0, p.ctl);
+                // dO_0 came with Q_0 (waited above) or has its own barrier
+                ok = DO_WITH_Q || warp_wait(do_full, 0, p.ctl);
                 if (ok) {
                     tc_fence_after();
-                    issue_kk(rcol(1), kbase(0) + C::TILE, aDO);
+                    issue_kk(rcol(1), kbase(0) + C::TILE, do_base(0));
                     mma_commit_elect(dp_full);
                 }
             }
@@ -527,8 +540,8 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     // must have been read out
                     if (PERSIST && t == 0 && k > 0 && !(ok = warp_wait(dv_free, (k - 1) & 1, p.ctl))) break;
                     tc_fence_after();
-                    issue_dv(X, t > 0);
-                    mma_commit_elect(do_empty);
+                    issue_dv(X, do_base(T), t > 0);
+                    if constexpr (!DO_WITH_Q) mma_commit_elect(do_empty);
                     if (!(ok = warp_wait(EARLY_DP ? dp_read : ds_ready, T & 1, p.ctl))) break;
                     tc_fence_after();
                     // S^T of the next tile into Y (which held dP^T of this tile, already
@@ -573,13 +586,16 @@ __global__ void __launch_bounds__(Roles<SMW>::NTHREADS, 1) __maxnreg__(Roles<SMW
                     }
                     if (more && !early_next && !(ok = issue_next_s())) break;
                     if (more) {
-                        if (!(ok = warp_wait(do_full, (T + 1) & 1, p.ctl))) break;
+                        // with DO_WITH_Q, dO of tile T + 1 came with its Q, whose barrier
+                        // phase issue_next_s (above, on every path with a next tile) has
+                        // already waited for
+                        if (!DO_WITH_Q && !(ok = warp_wait(do_full, (T + 1) & 1, p.ctl))) break;
                         if constexpr (D == 128) {
                             // X holds dQ of tile T until the dQ warps have read it
                             if (!(ok = warp_wait(dq_empty, T & 1, p.ctl))) break;
                         }
                         tc_fence_after();
-                        issue_kk(X, (cross ? aKn : aKc) + C::TILE, aDO);
+                        issue_kk(X, (cross ? aKn : aKc) + C::TILE, do_base(T + 1));
                         mma_commit_elect(dp_full);
                     }
                 }
