@@ -228,7 +228,7 @@ int fa_set_fwd_queue_words(int n)
 
 // Persistent grid, work queue and dispatch grouping of the square forward
 // (bf16 or e4m3 inputs, bytes_per_elem of each).
-static int fwd_grid(FwdParams& p, uint64_t BH, int N, int d, int causal, size_t bytes_per_elem)
+static int fwd_grid(FwdParams& p, uint64_t BH, int N, int d, int causal, size_t bytes_per_elem, cudaStream_t stream)
 {
     int st = FA_OK;
     p.BH = static_cast<int>(BH);
@@ -249,6 +249,17 @@ static int fwd_grid(FwdParams& p, uint64_t BH, int N, int d, int causal, size_t 
         const unsigned int t = g_fwd_tickets[dev].fetch_add(1u);
         p.ticket = t & 0xFFFFu;
         p.queue_slot = static_cast<int>(t % static_cast<unsigned int>(g_fwd_queue_slots.load()));
+        // A launch recorded into a CUDA graph keeps its ticket in every replay,
+        // and two executables of one capture could run at once with the same
+        // ticket and join each other's hand-out: captured launches take the
+        // fixed item order instead and leave the queue alone.  (If the query
+        // itself fails, the fixed order is the safe choice.)
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) {
+            (void)cudaGetLastError();
+            cap = cudaStreamCaptureStatusActive;
+        }
+        p.fixed_order = cap != cudaStreamCaptureStatusNone ? 1 : 0;
     }
     p.group_heads = 1;
     if (causal) {
@@ -288,7 +299,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
         return st;
     if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
     p.lse = lse;
-    if ((st = fwd_grid(p, BH, N, d, causal, 2)) != FA_OK) return st;
+    if ((st = fwd_grid(p, BH, N, d, causal, 2, static_cast<cudaStream_t>(stream))) != FA_OK) return st;
     p.scale_log2 = scale * kLog2e;
     p.o_scale = 1.f;
     st = cuda_status(launch_fwd_sm100(p, d, causal != 0, false, static_cast<cudaStream_t>(stream)));
@@ -493,7 +504,7 @@ int fa_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
             return st;
         if ((st = get_ctl(&p.ctl)) != FA_OK) return st;
         p.lse = lse;
-        if ((st = fwd_grid(p, BH, N, d, causal, 1)) != FA_OK) return st;
+        if ((st = fwd_grid(p, BH, N, d, causal, 1, static_cast<cudaStream_t>(stream))) != FA_OK) return st;
         p.scale_log2 = scale * q_descale * k_descale * kLog2e;
         p.o_scale = v_descale;
         st = cuda_status(launch_fwd_sm100(p, d, causal != 0, true, static_cast<cudaStream_t>(stream)));

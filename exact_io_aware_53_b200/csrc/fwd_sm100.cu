@@ -77,12 +77,15 @@ constexpr float LN2 = 0.6931471805599453f;
 // draws exactly the item count sets DONE, and each leaves (-1 taker) after its
 // first draw past the end.  While a CTA takes items the word cannot be freed,
 // so no draw lands in another launch's counter.  A CTA that finds the word held
-// by another launch (more than QUEUE_SLOTS launches in flight, or replays of
-// one captured launch on two streams) takes items blockIdx.x + s * gridDim.x
-// instead, so every item is processed, some twice with identical results.  A
-// free word with the launch's own ticket is what an earlier run of the same
-// launch left (a graph replay) when it equals what the CTA read at its start,
-// else the end of this run's own hand-out.  Nothing is ever reset.
+// by another launch (more than QUEUE_SLOTS launches in flight) takes items
+// blockIdx.x + s * gridDim.x instead, so every item is processed, some twice
+// with identical results.  A free word with the launch's own ticket is what an
+// earlier launch with that ticket left (tickets repeat every 65536 launches)
+// when it equals what the CTA read at its start, else the end of this launch's
+// own hand-out.  Nothing is ever reset.  Launches recorded into a CUDA graph do
+// not use the queue at all (FwdParams::fixed_order): every replay carries the
+// capture's ticket, and two executables of one capture running at once could
+// not be told apart by it.
 constexpr int QUEUE_SLOTS = 64;
 constexpr unsigned long long Q_COUNT = (1ull << 30) - 1;
 constexpr unsigned long long Q_TAKER = 1ull << 30;
@@ -323,9 +326,9 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
             int it = 0, nq = 0;  // K/V ring slots and Q tiles issued so far
             bool ok = true;
             QueueCursor qc;
-            qc.snap = queue_read(queue);
-            qc.mode = Q_UNDECIDED;  // the first access decides
-            qc.next_fixed = 0;
+            qc.snap = p.fixed_order ? 0ull : queue_read(queue);
+            qc.mode = p.fixed_order ? Q_FIXED : Q_UNDECIDED;  // else the first access decides
+            qc.next_fixed = static_cast<int>(blockIdx.x + gridDim.x);
             for (int n = 0; ok; ++n) {
                 const int slot = n & 1;
                 const int item = (n == 0) ? static_cast<int>(blockIdx.x)

@@ -188,10 +188,12 @@ def test_forward_on_concurrent_streams_with_shared_queue_words(fa_lib, words):
 
 
 def test_forward_replayed_from_a_captured_graph(fa_lib):
-    """A captured forward keeps its launch ticket, so each replay finds the
-    queue word as the previous replay left it; every replay must still process
-    every item (inputs change between replays, outputs must follow)."""
-    x = to_cuda(_inputs((2, 3, 1100, 128), seed=4321))
+    """A forward recorded into a CUDA graph takes the fixed item order (CTA b:
+    items b, b + grid, ...) and leaves the work queue alone, since every replay
+    would carry the capture's ticket.  Every replay must process every item
+    (inputs change between replays, outputs must follow); 4 x 40 heads of 600
+    rows give 480 items, more than one per CTA."""
+    x = to_cuda(_inputs((4, 40, 600, 128), seed=4321))
     scale = 1 / math.sqrt(128)
     o = torch.empty_like(x["q"])
     lse = torch.empty(x["q"].shape[:3], dtype=torch.float32, device="cuda")
@@ -201,7 +203,7 @@ def test_forward_replayed_from_a_captured_graph(fa_lib):
     with torch.cuda.graph(g, capture_error_mode="relaxed"):
         fa_lib.fwd(x["q"], x["k"], x["v"], causal=True, scale=scale, out=o, lse=lse)
     for rep in range(4):
-        fresh = _inputs((2, 3, 1100, 128), seed=5000 + rep)
+        fresh = _inputs((4, 40, 600, 128), seed=5000 + rep)
         for n in ("q", "k", "v"):
             x[n].copy_(fresh[n])
         o.fill_(float("nan"))
