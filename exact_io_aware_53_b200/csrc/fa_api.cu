@@ -30,10 +30,14 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 unsigned int* g_status_ptr[kMaxDevices] = {};
 std::atomic<unsigned long long> g_limit_ns{2000000000ull};
-// forward launches per device (work-queue tickets) and the number of queue
-// words in use (64; fewer only to exercise shared words in tests)
+// forward launches per device (their numbers pick a work-queue word and give
+// the launch's identity there), the number of queue words in use (64; fewer
+// only to exercise shared words in tests), and per device and word the
+// identity of the last launch that used the queue on it (guarded by g_mu)
 std::atomic<unsigned int> g_fwd_tickets[kMaxDevices];
 std::atomic<int> g_fwd_queue_slots{64};
+unsigned int g_fwd_last_queue_id[kMaxDevices][64];
+bool g_fwd_last_queue_id_set[kMaxDevices][64] = {};
 // softmax warps per backward CTA (4 or 8; 0: the library's choice)
 std::atomic<int> g_bwd_softmax_warps{0};
 thread_local int g_last_launches = 0;
@@ -236,8 +240,8 @@ static int fwd_grid(FwdParams& p, uint64_t BH, int N, int d, int causal, size_t 
     p.n_pairs = (N + 255) / 256;
     {
         // persistent grid: one CTA per SM, no more than there are work items;
-        // each launch gets a ticket (its number on this device, 16 bits kept)
-        // and the work-queue word ticket % 64
+        // each launch gets a number on this device, which picks its work-queue
+        // word (number % words) and, in 24 bits, its identity there
         int dev = 0, n_sm = 0;
         if ((st = cuda_status(cudaGetDevice(&dev))) != FA_OK) return st;
         if (dev < 0 || dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
@@ -246,12 +250,9 @@ static int fwd_grid(FwdParams& p, uint64_t BH, int N, int d, int causal, size_t 
         if (items >= (1ll << 29)) return FA_ERR_UNSUPPORTED;  // the queue counter has 30 bits
         p.n_ctas = static_cast<int>(std::max<long long>(1, std::min<long long>(n_sm, items)));
         if (p.n_ctas > 511) return FA_ERR_UNSUPPORTED;  // the queue word counts takers in 9 bits
-        const unsigned int t = g_fwd_tickets[dev].fetch_add(1u);
-        p.ticket = t & 0xFFFFu;
-        p.queue_slot = static_cast<int>(t % static_cast<unsigned int>(g_fwd_queue_slots.load()));
-        // A launch recorded into a CUDA graph keeps its ticket in every replay,
+        // A launch recorded into a CUDA graph keeps its identity in every replay,
         // and two executables of one capture could run at once with the same
-        // ticket and join each other's hand-out: captured launches take the
+        // identity and join each other's hand-out: captured launches take the
         // fixed item order instead and leave the queue alone.  (If the query
         // itself fails, the fixed order is the safe choice.)
         cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
@@ -260,6 +261,25 @@ static int fwd_grid(FwdParams& p, uint64_t BH, int N, int d, int causal, size_t 
             cap = cudaStreamCaptureStatusActive;
         }
         p.fixed_order = cap != cudaStreamCaptureStatusNone ? 1 : 0;
+        // A launch that uses the queue never gets the identity of the last
+        // launch that used its word (possible only across the 24-bit wrap): a
+        // finished word with its own identity must be its own hand-out.
+        const bool uses_queue = p.fixed_order == 0 && items > p.n_ctas;
+        const unsigned int words = static_cast<unsigned int>(g_fwd_queue_slots.load());
+        for (;;) {
+            const unsigned int t = g_fwd_tickets[dev].fetch_add(1u);
+            p.queue_slot = static_cast<int>(t % words);
+            p.queue_id = t & 0xFFFFFFu;
+            if (!uses_queue) break;
+            std::lock_guard<std::mutex> lk(g_mu);
+            unsigned int& last = g_fwd_last_queue_id[dev][p.queue_slot];
+            bool& seen = g_fwd_last_queue_id_set[dev][p.queue_slot];
+            if (!seen || last != p.queue_id) {
+                last = p.queue_id;
+                seen = true;
+                break;
+            }
+        }
     }
     p.group_heads = 1;
     if (causal) {

@@ -65,27 +65,28 @@ constexpr float LN2 = 0.6931471805599453f;
 // Work queue.  Each CTA's first item is item blockIdx.x (the first gridDim.x
 // items are the longest, so that is what a queue would hand out anyway); the
 // rest come from a counter in one of QUEUE_SLOTS 64-bit words, picked by the
-// launch's ticket (a per-device launch number).  A word holds
-//   [63:48] ticket of the launch that claimed it   [47:40] claim epoch
+// launch's number on the device.  A word holds
+//   [63:40] identity of the launch that claimed it (24 bits of its number)
 //   [39]    DONE: every item has been handed out   [38:30] CTAs taking items
 //   [29:0]  counter of the next item
 // and is free when it is zero or DONE with no CTA taking items.  The first CTA
-// of a launch to want a second item claims a free word (compare and swap:
-// ticket, epoch + 1, one taker, counter gridDim.x + 1, taking item gridDim.x);
-// the launch's other CTAs join it (+1 taker, checked afterwards) and then take
-// items by atomic add until the counter passes the last item; the one that
-// draws exactly the item count sets DONE, and each leaves (-1 taker) after its
-// first draw past the end.  While a CTA takes items the word cannot be freed,
-// so no draw lands in another launch's counter.  A CTA that finds the word held
-// by another launch (more than QUEUE_SLOTS launches in flight) takes items
-// blockIdx.x + s * gridDim.x instead, so every item is processed, some twice
-// with identical results.  A free word with the launch's own ticket is what an
-// earlier launch with that ticket left (tickets repeat every 65536 launches)
-// when it equals what the CTA read at its start, else the end of this launch's
-// own hand-out.  Nothing is ever reset.  Launches recorded into a CUDA graph do
-// not use the queue at all (FwdParams::fixed_order): every replay carries the
-// capture's ticket, and two executables of one capture running at once could
-// not be told apart by it.
+// of a launch to want a second item claims a free word that is not its own
+// (compare and swap: identity, one taker, counter gridDim.x + 1, taking item
+// gridDim.x); the launch's other CTAs join it (+1 taker, checked afterwards)
+// and then take items by atomic add until the counter passes the last item;
+// the one that draws exactly the item count sets DONE, and each leaves (-1
+// taker) after its first draw past the end.  While a CTA takes items the word
+// cannot be freed, so no draw lands in another launch's counter.  A free word
+// with the launch's own identity is the end of its own hand-out: a CTA that
+// starts late (its SM was busy) stops after its first item instead of handing
+// the items out again.  The host never gives a launch that uses the queue the
+// identity of the last launch that used its word, so no older word can pass for
+// its own.  A CTA that finds the word held by another launch (more than
+// QUEUE_SLOTS launches in flight) takes items blockIdx.x + s * gridDim.x
+// instead, so every item is processed, some twice with identical results.
+// Nothing is ever reset.  Launches recorded into a CUDA graph do not use the
+// queue at all (FwdParams::fixed_order): every replay would carry the
+// capture's identity.
 constexpr int QUEUE_SLOTS = 64;
 constexpr unsigned long long Q_COUNT = (1ull << 30) - 1;
 constexpr unsigned long long Q_TAKER = 1ull << 30;
@@ -96,7 +97,6 @@ __device__ unsigned long long g_queue[QUEUE_SLOTS];
 enum QueueMode { Q_UNDECIDED = 0, Q_TAKING = 1, Q_FIXED = 2, Q_FINISHED = 3 };
 
 struct QueueCursor {
-    unsigned long long snap;  // the word as this CTA first read it
     int mode;                 // QueueMode
     int next_fixed;           // next item of the fixed sequence (Q_FIXED)
 };
@@ -116,8 +116,8 @@ __device__ __forceinline__ bool queue_free(unsigned long long w)
 __device__ __forceinline__ void queue_leave(unsigned long long* word) { atomicAdd(word, ~Q_TAKER + 1ull); }
 
 // Next work item of this CTA, or -1 when the launch has none left for it.
-// `ticket` is the launch's 16-bit ticket; total > gridDim.x.
-__device__ int queue_next(unsigned long long* word, unsigned int ticket, int total, QueueCursor& qc,
+// `ident` is the launch's 24-bit identity; total > gridDim.x.
+__device__ int queue_next(unsigned long long* word, unsigned int ident, int total, QueueCursor& qc,
                           const WaitCtl& ctl)
 {
     const unsigned int P = gridDim.x;
@@ -128,16 +128,15 @@ __device__ int queue_next(unsigned long long* word, unsigned int ticket, int tot
             break;
         }
         const unsigned long long w = queue_read(word);
-        const bool own = w != 0ull && static_cast<unsigned int>(w >> 48) == ticket;
+        const bool own = w != 0ull && static_cast<unsigned int>(w >> 40) == ident;
         if (queue_free(w)) {
-            if (own && w != qc.snap) {
-                qc.mode = Q_FINISHED;  // this run's own hand-out is over
+            if (own) {
+                qc.mode = Q_FINISHED;  // this launch's own hand-out is over
                 break;
             }
-            // claim it for this run and take item P
-            const unsigned long long ep = ((w >> 40) + 1ull) & 0xFFull;
+            // claim it for this launch and take item P
             const unsigned long long want =
-                (static_cast<unsigned long long>(ticket) << 48) | (ep << 40) | Q_TAKER | static_cast<unsigned long long>(P + 1u);
+                (static_cast<unsigned long long>(ident) << 40) | Q_TAKER | static_cast<unsigned long long>(P + 1u);
             if (atomicCAS(word, w, want) != w) continue;
             qc.mode = Q_TAKING;
             if (P + 1u >= static_cast<unsigned int>(total)) {
@@ -155,7 +154,7 @@ __device__ int queue_next(unsigned long long* word, unsigned int ticket, int tot
             }
             // join; while this CTA counts as a taker the word stays this run's
             const unsigned long long old = atomicAdd(word, Q_TAKER);
-            if (old != 0ull && static_cast<unsigned int>(old >> 48) == ticket && (old & Q_DONE) == 0ull) {
+            if (old != 0ull && static_cast<unsigned int>(old >> 40) == ident && (old & Q_DONE) == 0ull) {
                 qc.mode = Q_TAKING;
             } else {
                 queue_leave(word);  // it changed under us: undo and look again
@@ -326,13 +325,12 @@ __global__ void __maxnreg__(MAX_REGS) fwd_kernel(const __grid_constant__ FwdPara
             int it = 0, nq = 0;  // K/V ring slots and Q tiles issued so far
             bool ok = true;
             QueueCursor qc;
-            qc.snap = p.fixed_order ? 0ull : queue_read(queue);
             qc.mode = p.fixed_order ? Q_FIXED : Q_UNDECIDED;  // else the first access decides
             qc.next_fixed = static_cast<int>(blockIdx.x + gridDim.x);
             for (int n = 0; ok; ++n) {
                 const int slot = n & 1;
                 const int item = (n == 0) ? static_cast<int>(blockIdx.x)
-                                          : (total > static_cast<int>(gridDim.x) ? queue_next(queue, p.ticket, total, qc, p.ctl)
+                                          : (total > static_cast<int>(gridDim.x) ? queue_next(queue, p.queue_id, total, qc, p.ctl)
                                                                                  : -1);
                 if (!(ok = mbar_wait(&item_empty[slot], ((n >> 1) & 1) ^ 1, p.ctl))) break;
                 item_buf[slot] = item;

@@ -32,7 +32,7 @@ struct FwdParams {
     int group_heads;   // grouping of the (pair, head) work items, >= 1 (grouped_order)
     int n_ctas;        // persistent CTAs, <= min(SMs, B*H*n_pairs)
     int queue_slot;    // work queue word of this launch, < 64
-    unsigned int ticket;  // launch number on this device, low 16 bits
+    unsigned int queue_id;  // identity in the queue word: the launch's number on this device, low 24 bits
     int fixed_order;   // 1: CTA b takes items b, b + n_ctas, ... and never touches the queue
     float scale_log2;  // scale * log2(e) (e4m3: times the q and k descales)
     float o_scale;     // factor on O / l: 1, or the v descale for e4m3

@@ -56,12 +56,13 @@ typedef enum {
  * not overlap any input.
  * The kernel is persistent: one CTA per SM takes work items (256 query rows
  * of one head) from a queue.  The queue is one of 64 counter words in the
- * library's device memory, claimed per launch with a launch ticket and never
- * reset; a launch that finds its word held by another launch in flight takes
- * its items in a fixed order instead.  So launches may run concurrently on any
- * number of streams, and a captured launch may be replayed, with every output
- * element written by this launch's own arithmetic (at worst some items twice,
- * with identical results).
+ * library's device memory, claimed per launch with the launch's number on the
+ * device (24 bits) and never reset; a launch that finds its word held by
+ * another launch in flight takes its items in a fixed order instead, and so
+ * does every launch recorded into a CUDA graph (it leaves the queue alone).
+ * So launches may run concurrently on any number of streams, and a captured
+ * launch may be replayed, with every output element written by this launch's
+ * own arithmetic (at worst some items twice, with identical results).
  */
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
            float scale, int causal, void* stream);
