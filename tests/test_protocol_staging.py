@@ -206,3 +206,140 @@ def test_per_tile_protocol_on_fixed_item_mixes(items):
         violation, stored = simulate("per_tile", items, seed=seed)
         assert violation is None, (seed, violation)
         assert stored == [(n, t) for n in range(len(items)) for t in (0, 1)]
+
+
+# ---------------------------------------------------------------------------
+# Exhaustive search over small scopes: every interleaving of W warps per tile
+# and the stores, for short item sequences (the random runs above sample the
+# 8-warp case).  A state is (warp states, barrier phases, turn count, writers,
+# stores reading, warps done writing per item, turns passed on); every enabled
+# step of every warp or store is explored.  Checked in every reachable state:
+# no warp enters or stays in a turn's writes, and no store starts, while
+# another turn's writes or store are in flight; a state with no enabled step
+# is the end (every turn stored or passed on once, in order) and not a
+# deadlock.
+
+def explore(protocol, items, W=2):
+    per_tile = protocol.startswith("per_tile")
+    first_passes = protocol == "per_tile_first_passes"
+    nbar = 2 if per_tile else 1
+    M = len(items)
+    OFREE, WAIT, WRITE, INC, END = range(5)
+
+    def bar_of(t):
+        return t if per_tile else 0
+
+    def wait_of(t, n, rows):
+        if per_tile:
+            return t ^ 1, (n & 1) ^ t ^ 1
+        return 0, (t ^ 1) if rows else 0
+
+    # state: warps (tuple of (n, phase) per warp, t = i // W), phases, count,
+    # writers (tuple of (turn, k)), reading (frozenset of turns), done (tuple per
+    # tile of per-item counts), passed (frozenset), stored (tuple of turns)
+    start = (tuple((0, OFREE) for _ in range(2 * W)), (0,) * nbar, 0, (), frozenset(),
+             ((0,) * M, (0,) * M), frozenset(), ())
+    seen, stack = {start}, [start]
+    while stack:
+        st = stack.pop()
+        warps, phases, count, writers, reading, done, passed, stored = st
+        wr = dict(writers)
+        succ = []
+
+        def other_active(turn):
+            return any(k > 0 and u != turn for u, k in wr.items()) or any(u != turn for u in reading)
+
+        for i, (n, ph) in enumerate(warps):
+            t = i // W
+            if ph == END:
+                continue
+            rows = items[n][t]
+            turn = (n, t)
+            nxt = (n + 1, OFREE) if n + 1 < M else (n + 1, END)
+            if ph == OFREE:
+                prev = [m for m in range(n) if items[m][t]]
+                if rows and prev and done[t][prev[-1]] < W:
+                    continue
+                succ.append((i, (n, WAIT), phases, count, wr, reading, done, passed, stored))
+            elif ph == WAIT:
+                b, parity = wait_of(t, n, rows)
+                if parity == (phases[b] & 1):
+                    continue  # that phase is not complete
+                if not rows and first_passes:
+                    if turn in passed:
+                        succ.append((i, nxt, phases, count, wr, reading, done, passed, stored))
+                    else:
+                        ph2 = list(phases)
+                        ph2[bar_of(t)] += 1
+                        succ.append((i, nxt, tuple(ph2), count, wr, reading, done, passed | {turn},
+                                     stored + (turn,)))
+                    continue
+                if rows:
+                    if other_active(turn):
+                        return "turn %s writes while another turn is in flight" % (turn,)
+                    w2 = dict(wr)
+                    w2[turn] = w2.get(turn, 0) + 1
+                    succ.append((i, (n, WRITE), phases, count, w2, reading, done, passed, stored))
+                else:
+                    succ.append((i, (n, INC), phases, count, wr, reading, done, passed, stored))
+            elif ph == WRITE:
+                if other_active(turn):
+                    return "turn %s writes while another turn is in flight" % (turn,)
+                w2 = dict(wr)
+                w2[turn] -= 1
+                d2 = [list(done[0]), list(done[1])]
+                d2[t][n] += 1
+                succ.append((i, (n, INC), phases, count, w2, reading, (tuple(d2[0]), tuple(d2[1])), passed, stored))
+            elif ph == INC:
+                c = count + 1
+                if c < W:
+                    succ.append((i, nxt, phases, c, wr, reading, done, passed, stored))
+                elif rows:
+                    if any(k > 0 and u != turn for u, k in wr.items()):
+                        return "turn %s's store starts while another turn writes" % (turn,)
+                    succ.append((i, nxt, phases, 0, wr, reading | {turn}, done, passed, stored))
+                else:
+                    ph2 = list(phases)
+                    ph2[bar_of(t)] += 1
+                    succ.append((i, nxt, tuple(ph2), 0, wr, reading, done, passed, stored + (turn,)))
+        for turn in reading:  # a store finishes reading: its turn ends
+            ph2 = list(phases)
+            ph2[bar_of(turn[1])] += 1
+            succ.append((None, None, tuple(ph2), count, wr, reading - {turn}, done, passed, stored + (turn,)))
+        if not succ:
+            if all(ph == END for _, ph in warps) and not reading:
+                if list(stored) != [(n, t) for n in range(M) for t in (0, 1)]:
+                    return "turns ended out of order: %s" % (stored,)
+                continue
+            return "deadlock"
+        for i, w_new, ph2, c2, w2, r2, d2, p2, s2 in succ:
+            ws = list(warps)
+            if i is not None:
+                ws[i] = w_new
+            ns = (tuple(ws), ph2, c2, tuple(sorted((u, k) for u, k in w2.items() if k)), r2, d2, p2, s2)
+            if ns not in seen:
+                seen.add(ns)
+                stack.append(ns)
+    return None
+
+
+def _mixes(max_items):
+    import itertools
+    for m in range(1, max_items + 1):
+        for rows1 in itertools.product((True, False), repeat=m):
+            yield [(True, r) for r in rows1]
+
+
+def test_per_tile_protocol_holds_in_every_interleaving_of_small_scopes():
+    for items in _mixes(4):
+        assert explore("per_tile", items) is None, items
+
+
+def test_every_interleaving_search_finds_both_earlier_forms_wrong():
+    shared = [explore("shared", items) for items in _mixes(3)]
+    # the one-barrier form: from two items on, some interleaving overlaps a turn's
+    # writes with another turn's store
+    assert all((r is not None) == (len(items) > 1) for r, items in zip(shared, _mixes(3)))
+    assert any(r and ("in flight" in r or "store starts" in r) for r in shared)
+    first = [explore("per_tile_first_passes", items) for items in _mixes(4)]
+    assert any(r == "deadlock" for r in first)
