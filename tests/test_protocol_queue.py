@@ -277,3 +277,159 @@ def test_many_launches_in_sequence_and_overlapping():
                 launches.append((host.launch(True)[1], total, grid, rng.randint(0, 20)))
             recs, word = run(launches, seed * 10 + rnd, word)
             check(launches, recs, word)
+
+
+# ---------------------------------------------------------------------------
+# Exhaustive search over small scopes.  Each CTA is a small state machine over
+# the same steps as `cta` above (each atomic access of the word one step; a
+# CTA's start -- when it takes its first item and, in the earlier form, reads
+# its snapshot of the word -- is a step too, so every start order, late starts
+# included, is explored).  Every interleaving of the CTAs of one or two
+# launches on one word is visited.  Checked in every terminal state: each
+# launch processed every item; a launch none of whose CTAs fell back to the
+# fixed order processed no item twice; no draw came from another launch's
+# counter; the word is free.  (With two launches on one word, a CTA that starts
+# after its own launch's hand-out AND another launch's later hand-out on the
+# same word are both over finds a free word of another identity and hands its
+# launch's items out again: identical results, only repeated work.  With 64
+# words the other launch is 64 launches later, so this is checked for single
+# launches only.)  The earlier form ("snapshot": a 16-bit ticket
+# and a claim epoch, a free word with the launch's own ticket taken for its own
+# only if it differs from the CTA's snapshot) is kept as a mutant: the search
+# must find its late-start double hand-out.
+
+def explore(launches, protocol="identity", word0=0, allow_repeats=False):
+    """launches: list of (identity, total, grid).  Returns None or a failure."""
+    (START, READ, DECIDE, CAS, JOIN_ADD, JOIN_UNDO, DRAW, OR_DONE_LAST, LEAVE_LAST,
+     OR_DONE_CLAIM, LEAVE_CLAIM, FIXED, END) = range(13)
+    snapshot = protocol == "snapshot"
+    shift = 48 if snapshot else 40
+    ctas = [(li, b) for li, (_, _, grid) in enumerate(launches) for b in range(grid)]
+    # CTA: (pc, next_fixed, w (value read / old value), snap, items, n_items, draws_ok, fixed)
+    init = (word0, tuple((START, 0, 0, 0, frozenset(), 0, True, False) for _ in ctas))
+    seen, stack = {init}, [init]
+    terminal = 0
+    while stack:
+        word, cs = stack.pop()
+        moved = False
+        for k, (li, b) in enumerate(ctas):
+            ident, total, grid = launches[li]
+            pc, nf, w, snap, items, n_items, ok, fixed = cs[k]
+            if pc == END:
+                continue
+            nw = word
+            npc, nnf, nwv, nsnap, nitems, nn, nok, nfixed = pc, nf, w, snap, items, n_items, ok, fixed
+
+            def take(item):
+                return items | {item}, n_items + 1
+
+            if pc == START:
+                nsnap = word
+                nitems, nn = take(b)
+                npc = READ
+            elif pc == READ:
+                nwv, npc = word, DECIDE
+            elif pc == DECIDE:
+                own = w != 0 and (w >> shift) == ident
+                if is_free(w):
+                    if own and (not snapshot or w != snap):
+                        npc = END
+                    else:
+                        npc = CAS
+                elif own:
+                    npc = END if (w & DONE) else JOIN_ADD
+                else:
+                    npc, nnf, nfixed = FIXED, b + grid, True
+            elif pc == CAS:
+                if word != w:
+                    npc = READ
+                else:
+                    ep = (((w >> 40) + 1) & 0xFF) << 40 if snapshot else 0
+                    nw = (ident << shift) | ep | TAKER | (grid + 1)
+                    nitems, nn = take(grid)
+                    npc = OR_DONE_CLAIM if grid + 1 >= total else DRAW
+            elif pc == OR_DONE_CLAIM:
+                nw, npc = word | DONE, LEAVE_CLAIM
+            elif pc == LEAVE_CLAIM:
+                nw, npc = (word - TAKER) & M64, END
+            elif pc == JOIN_ADD:
+                old = word
+                nw = (old + TAKER) & M64
+                if old != 0 and (old >> shift) == ident and not (old & DONE):
+                    npc = DRAW
+                else:
+                    npc = JOIN_UNDO
+            elif pc == JOIN_UNDO:
+                nw, npc = (word - TAKER) & M64, READ
+            elif pc == DRAW:
+                old = word
+                nw = (old + 1) & M64
+                if (old >> shift) != ident:
+                    nok = False
+                c = old & COUNT
+                if c < total:
+                    nitems, nn = take(c)
+                elif c == total:
+                    npc = OR_DONE_LAST
+                else:
+                    npc = LEAVE_LAST
+            elif pc == OR_DONE_LAST:
+                nw, npc = word | DONE, LEAVE_LAST
+            elif pc == LEAVE_LAST:
+                nw, npc = (word - TAKER) & M64, END
+            elif pc == FIXED:
+                if nf < total:
+                    nitems, nn = take(nf)
+                    nnf = nf + grid
+                else:
+                    npc = END
+            ncs = list(cs)
+            ncs[k] = (npc, nnf, nwv, nsnap, nitems, nn, nok, nfixed)
+            ns = (nw, tuple(ncs))
+            moved = True
+            if ns not in seen:
+                seen.add(ns)
+                stack.append(ns)
+        if not moved:
+            terminal += 1
+            for li, (ident, total, grid) in enumerate(launches):
+                mine = [cs[k] for k, (lj, _) in enumerate(ctas) if lj == li]
+                got = set().union(*(c[4] for c in mine))
+                if got != set(range(total)):
+                    return "launch %d missed items %s" % (li, sorted(set(range(total)) - got))
+                if not allow_repeats and not any(c[7] for c in mine) and sum(c[5] for c in mine) != total:
+                    return "launch %d handed items out twice (%d for %d)" % (li, sum(c[5] for c in mine), total)
+                if not all(c[6] for c in mine):
+                    return "launch %d drew from another launch's counter" % li
+            if not is_free(word):
+                return "word left held: %x" % word
+    return None if terminal else "no terminal state"
+
+
+SMALL_SCOPES = [[(1, 2, 1)], [(1, 3, 2)], [(1, 4, 2)], [(1, 5, 3)], [(1, 6, 3)]]
+TWO_LAUNCHES = [[(1, 2, 1), (2, 2, 1)], [(1, 3, 2), (2, 2, 1)], [(1, 3, 1), (2, 3, 1)], [(1, 2, 1), (2, 4, 2)]]
+
+
+@pytest.mark.parametrize("launches", SMALL_SCOPES)
+def test_every_interleaving_of_one_launch_hands_each_item_out_once(launches):
+    assert explore(launches) is None, launches
+
+
+@pytest.mark.parametrize("launches", TWO_LAUNCHES)
+def test_every_interleaving_of_two_launches_on_one_word(launches):
+    assert explore(launches, allow_repeats=True) is None, launches
+
+
+@pytest.mark.parametrize("launches", SMALL_SCOPES[:4])
+def test_every_interleaving_from_a_word_an_older_launch_left(launches):
+    """The word starts as an older launch left it: free (DONE, no takers) with
+    another identity, or with the same low 16 bits of identity."""
+    for word0 in ((9 << 40) | DONE | 7, ((launches[0][0] | (1 << 16)) << 40) | DONE | 3):
+        assert explore(launches, word0=word0) is None, (launches, hex(word0))
+
+
+def test_the_snapshot_form_hands_items_out_twice_after_a_late_start():
+    """The earlier form: some interleaving (a CTA starting after its launch's
+    hand-out is over) hands items out a second time."""
+    found = [explore(launches, protocol="snapshot") for launches in SMALL_SCOPES]
+    assert any(r and "twice" in r for r in found), found
