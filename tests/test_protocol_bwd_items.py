@@ -338,3 +338,237 @@ def test_dv_dk_free_are_implied_at_d128(drop):
     for items in ITEM_MIXES:
         for seed in range(60):
             assert simulate(items, seed, drop=drop) is None, (items, seed)
+
+
+# ---------------------------------------------------------------------------
+# d = 64: two K, V buffers (item k in buffer k % 2, released by an MMA commit
+# after the item's last product), dQ in its own TMEM region, the whole dQ
+# staged in the staging tile, and the dQ warps writing an item's dV (into the
+# dV staging area) and dK (into the staging tile) while the other warps run
+# the next item.
+
+def simulate64(item_tiles, seed, drop=None, max_idle=800):
+    rng = random.Random(seed)
+    K = len(item_tiles)
+    tiles = [(k, t) for k in range(K) for t in range(item_tiles[k])]
+    NT = len(tiles)
+    SMW = 2
+    B = {n: Bar() for n in ("kv_full0", "kv_full1", "kv_empty0", "kv_empty1", "s_full", "dp_full", "dq_full",
+                            "dq_empty", "dkdv_done", "dv_free", "dk_free")}
+    for n in ("p_ready", "dp_read", "ds_ready"):
+        B[n] = Bar(SMW)
+    inflight = {b: [] for b in ("KV0", "KV1", "DS", "STG", "EPI", "DV", "DK", "DQ")}
+    problems, pipe, tma, groups, ran = [], [], [], [], set()
+
+    def touch(agent, buf, kind):
+        for a, k in inflight[buf]:
+            if a != agent and (kind == "w" or k == "w") and not problems:
+                problems.append("%s %ss %s while %s has a %s in flight" % (agent, "write" if kind == "w" else "read", buf, a, k))
+        inflight[buf].append((agent, kind))
+
+    def release(agent, buf, kind):
+        inflight[buf].remove((agent, kind))
+
+    def wait(bar, parity):
+        while not B[bar].done(parity):
+            yield "blocked"
+
+    def issue(reads, writes, tag):
+        for b in reads:
+            touch("mma", b, "r")
+        for b in writes:
+            touch("mma", b, "w")
+        pipe.append(("mma", reads, writes, tag))
+
+    def commit(bar):
+        pipe.append(("commit", bar))
+
+    def tensor_pipe():
+        while True:
+            if not pipe:
+                yield "idle"
+                continue
+            op = pipe[0]
+            if op[0] == "mma":
+                for _ in range(rng.randint(1, 6)):
+                    yield "work"
+                for b in op[1]:
+                    release("mma", b, "r")
+                for b in op[2]:
+                    release("mma", b, "w")
+                ran.add(op[3])
+            else:
+                B[op[1]].arrive()
+            pipe.pop(0)
+            yield "work"
+
+    def tma_engine():
+        while True:
+            if not tma:
+                yield "idle"
+                continue
+            op = rng.choice(tma)
+            op["left"] -= 1
+            if op["left"] <= 0:
+                tma.remove(op)
+                release(op["agent"], op["buf"], op["kind"])
+                op["done"] = True
+                if op.get("bar"):
+                    B[op["bar"]].arrive()
+            yield "work"
+
+    def tma_op(agent, buf, kind, bar=None):
+        touch(agent, buf, kind)
+        op = {"agent": agent, "buf": buf, "kind": kind, "left": rng.randint(1, 40), "bar": bar, "done": False}
+        tma.append(op)
+        return op
+
+    def wait_groups(keep):
+        while any(not op["done"] for g in groups[: max(0, len(groups) - keep)] for op in g):
+            yield "blocked"
+
+    def kv(k):
+        return "KV%d" % (k & 1)
+
+    def producer():
+        for k in range(K):
+            b = k & 1
+            if drop != "kv_empty":
+                yield from wait("kv_empty%d" % b, ((k >> 1) & 1) ^ 1)
+            tma_op("load", kv(k), "w", bar="kv_full%d" % b)
+            yield "work"
+
+    def mma():
+        yield from wait("kv_full0", 0)
+        issue([kv(0)], [], "S0")
+        commit("s_full")
+        issue([kv(0)], [], "dP0")
+        commit("dp_full")
+        for T, (k, t) in enumerate(tiles):
+            cross = t + 1 == item_tiles[k]
+            more = T + 1 < NT
+            nk = k + 1 if cross else k
+            yield from wait("p_ready", T & 1)
+            if t == 0 and k > 0 and drop != "dv_free":
+                yield from wait("dv_free", (k - 1) & 1)
+            issue([], ["DV"], "dV%d" % T)
+            yield from wait("dp_read", T & 1)
+            if more:
+                if cross:
+                    yield from wait("kv_full%d" % (nk & 1), (nk >> 1) & 1)
+                issue([kv(nk)], [], "S%d" % (T + 1))
+                commit("s_full")
+            yield from wait("ds_ready", T & 1)
+            if t == 0 and k > 0 and drop != "dk_free":
+                yield from wait("dk_free", (k - 1) & 1)
+            issue(["DS"], ["DK"], "dK%d" % T)
+            if T > 0:
+                yield from wait("dq_empty", (T - 1) & 1)
+            issue(["DS", kv(k)], ["DQ"], "dQ%d" % T)
+            commit("dq_full")
+            if cross:
+                commit("dkdv_done")
+                commit("kv_empty%d" % (k & 1))
+            if more:
+                issue([kv(nk)], [], "dP%d" % (T + 1))
+                commit("dp_full")
+            yield "work"
+
+    def softmax(w):
+        for T, (k, t) in enumerate(tiles):
+            yield from wait("s_full", T & 1)
+            for _ in range(rng.randint(0, 5)):
+                yield "work"
+            B["p_ready"].arrive()
+            yield from wait("dp_full", T & 1)
+            B["dp_read"].arrive()
+            touch("soft", "DS", "w")
+            for _ in range(rng.randint(1, 4)):
+                yield "write"
+            release("soft", "DS", "w")
+            B["ds_ready"].arrive()
+
+    def dq_warps():
+        agent = "dq"
+        for T, (k, t) in enumerate(tiles):
+            last = t + 1 == item_tiles[k]
+            yield from wait("dq_full", T & 1)
+            touch(agent, "DQ", "r")
+            yield "read"
+            release(agent, "DQ", "r")
+            B["dq_empty"].arrive()
+            if drop != "stg_wait":
+                yield from wait_groups(0)  # the previous reduce-add (or epilogue store) has read its staging
+            touch(agent, "STG", "w")
+            yield "write"
+            release(agent, "STG", "w")
+            groups.append([tma_op("reduce", "STG", "r")])
+            if not last:
+                continue
+            # epilogue of item k, while the other warps run the next item
+            if drop != "epi_wait":
+                yield from wait_groups(0)
+            yield from wait("dkdv_done", k & 1)
+            for acc, area, bar in (("DV", "EPI", "dv_free"), ("DK", "STG", "dk_free")):
+                touch(agent, acc, "r")
+                touch(agent, area, "w")
+                yield "write"
+                release(agent, acc, "r")
+                release(agent, area, "w")
+                B[bar].arrive()
+            groups.append([tma_op("store", "EPI", "r"), tma_op("store", "STG", "r")])
+
+    workers = [producer(), mma(), softmax(0), softmax(1), dq_warps()]
+    daemons = [tensor_pipe(), tma_engine()]
+    asleep, idle, tick = {}, 0, 0
+    while workers:
+        tick += 1
+        progressed = False
+        order = workers + daemons
+        rng.shuffle(order)
+        for g in order:
+            if asleep.get(id(g), 0) > tick or rng.random() < 0.3:
+                continue
+            if g in workers and rng.random() < 0.003:
+                asleep[id(g)] = tick + rng.randint(20, 200)
+                continue
+            try:
+                progressed |= next(g) not in ("blocked", "idle")
+            except StopIteration:
+                workers.remove(g)
+                progressed = True
+        if problems:
+            return problems[0]
+        idle = 0 if progressed else idle + 1
+        if idle > max_idle:
+            return "deadlock"
+    for _ in range(5000):
+        if not pipe and not tma:
+            break
+        for g in daemons:
+            next(g)
+    if problems:
+        return problems[0]
+    missing = [tag for T in range(NT) for tag in ("dV%d" % T, "dK%d" % T, "dQ%d" % T) if tag not in ran]
+    return "products never ran: %s" % missing[:4] if missing else None
+
+
+@pytest.mark.parametrize("items", ITEM_MIXES)
+def test_d64_buffer_protocol_holds_under_random_interleavings(items):
+    for seed in range(120):
+        r = simulate64(items, seed)
+        assert r is None, (items, seed, r)
+
+
+@pytest.mark.parametrize("drop", ["kv_empty", "dv_free", "dk_free", "stg_wait", "epi_wait"])
+def test_d64_each_protocol_step_is_needed(drop):
+    found = None
+    for items in ITEM_MIXES:
+        for seed in range(150):
+            r = simulate64(items, seed, drop=drop)
+            if r is not None and r != "deadlock":
+                found = r
+                break
+        if found:
+            break
+    assert found, drop
