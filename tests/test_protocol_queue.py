@@ -176,7 +176,7 @@ def check(launches, recs, word):
 
 
 @pytest.mark.parametrize("grid,total", [(1, 2), (3, 4), (3, 10), (8, 9), (8, 45), (16, 200)])
-def test_one_launch_hands_every_item_out_once(grid, total):  # noqa: D103
+def test_one_launch_hands_every_item_out_once(grid, total):
     for seed in range(150):
         launches = [(5, total, grid, 0)]
         recs, word = run(launches, seed)
